@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the rank-r W4A4 linear layer (H-SVDQuant forward) on B200.
+
+One step = one pass of the hot path over one batch: for every linear of the
+workload, the fused activation step (hsq_quantize_act) followed by the INT4
+GEMM + low-rank/bias epilogue (hsq_linear_forward), weights pre-packed (packing
+is offline).  Default workload: the FLUX.1 double-stream block linears
+(M = 4608 tokens; QKV 3072->9216, MLP up 3072->12288, MLP down 12288->3072;
+rank 4; group-64 INT4), synthetic seeded inputs.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the whole workload on
+its own batch (token-parallel replicas, no data-path collective); the step time
+is the max over ranks and ``value`` aggregates all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from w4a4_rank_assisted_b200.synth import WORKLOADS, make_layer  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+INT8_OVER_BF16_NOMINAL = 2.0  # dense INT8 (4.5 POPS) over dense BF16 (2.25 PFLOP/s), nominal
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def layer_ops(spec):
+    """Algorithmic operations of one layer call: the INT4 product (2MNK) plus the
+    rank-r branch (2MKr down-projection, 2MNr up-projection)."""
+    return 2 * spec.M * spec.N * spec.K + 2 * spec.M * spec.K * spec.r + 2 * spec.M * spec.N * spec.r
+
+
+def layer_gemm_bytes(spec):
+    """Algorithmic HBM bytes of one hsq_linear_forward call (each operand once)."""
+    M, N, K, r = spec.M, spec.N, spec.K, spec.r
+    G = -(-K // 64)
+    Kp = 64 * G
+    return (M * Kp // 2 + 4 * M * G + 4 * M * r      # x codes, scales, U
+            + N * Kp // 2 + 4 * N * G + 2 * r * N    # w codes, scales, L2
+            + 2 * M * N)                             # Y (bf16)
+
+
+def layer_act_bytes(spec):
+    M, K, r = spec.M, spec.K, spec.r
+    G = -(-K // 64)
+    return 2 * M * K + M * 64 * G // 2 + 4 * M * G + 4 * M * r + 4 * K + 2 * K * r
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def oracle_timing(specs, budget_s: float = 12.0, seed_rows: int = 4):
+    """Time the CPU oracle (as it stands) on a bounded row sample of every layer
+    with pre-packed weights; returns (ops/s, cores, sample description)."""
+    from oracle import hsq_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    packed = []
+    for spec in specs:
+        lay = make_layer(spec)
+        Wn, sn = lay.W.float().numpy(), lay.s.numpy()
+        L1n = lay.L1.float().numpy() if spec.r else None
+        L2n = lay.L2.float().numpy() if spec.r else None
+        wc, ws = O.pack_weights(Wn, sn, L1n, L2n)
+        packed.append((spec, lay.X.float().numpy(), sn, L1n, L2n, wc, ws))
+
+    def run(rows):
+        t0 = time.perf_counter()
+        ops = 0
+        for spec, X, sn, L1n, L2n, wc, ws in packed:
+            m = min(rows, spec.M)
+            xc, xs, U = O.quantize_act(X[:m], sn, L1n)
+            O.linear_forward(xc, xs, U, wc, ws, L2n, None)
+            ops += layer_ops(spec) * m / spec.M
+        return time.perf_counter() - t0, ops
+
+    dt, _ = run(seed_rows)
+    rows = max(seed_rows, int(seed_rows * budget_s / max(dt, 1e-3)))
+    rows = min(rows, min(s.M for s in specs))
+    dt, ops = run(rows)
+    return ops / dt, cores, f"first {rows} token rows of each layer, weights pre-packed ({dt:.1f} s of CPU work)", dt
+
+
+def run_reference(args, specs, wl_name, rank, world):
+    if rank != 0:
+        return
+    per_step = []
+    sample = None
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        v, cores, sample, dt = oracle_timing(specs, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+        if i >= args.warmup:
+            per_step.append((v, dt))
+    v = statistics.median([p[0] for p in per_step])
+    tops = v / 1e12
+    line = {
+        "impl": "reference", "metric": "W4A4 rank-4 linear TOPS (FLUX block linears)", "value": tops,
+        "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.median([p[1] for p in per_step]) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; layer shapes of the pages' backbones)",
+        "config": {"workload": wl_name, "layers": [s.name for s in specs]},
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU leg
+def run_gpu(args, specs, wl_name, rank, world, local):
+    from w4a4_rank_assisted_b200 import hsq
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    layers = []
+    for spec in specs:
+        lay = make_layer(spec)
+        d = lambda t: None if t is None else t.to(dev).contiguous()
+        pl = hsq.PackedLinear(d(lay.W), d(lay.s), d(lay.L1) if spec.r else None,
+                              d(lay.L2) if spec.r else None, None)
+        X = d(lay.X)
+        act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev)
+        Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
+        ws = pl.workspace(spec.M)
+        X_host = lay.X.pin_memory()
+        Y_host = torch.empty((spec.M, spec.N), dtype=torch.bfloat16).pin_memory()
+        layers.append(dict(spec=spec, pl=pl, X=X, act=act, Y=Y, ws=ws, X_host=X_host, Y_host=Y_host))
+    torch.cuda.synchronize()
+    if hsq.hsq_get_device_status() != hsq.HSQ_OK:
+        raise RuntimeError("device status not clean after packing")
+
+    n_ev = 2 * len(layers)
+
+    def step(evs=None):
+        for i, L in enumerate(layers):
+            s = L["spec"]
+            if evs is not None:
+                evs[4 * i].record(stream)
+            hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
+                                 L["act"].x_scales, L["act"].U, stream=stream)
+            if evs is not None:
+                evs[4 * i + 1].record(stream)
+            hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
+                                   L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
+                                   workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
+                                   stream=stream)
+            if evs is not None:
+                evs[4 * i + 2].record(stream)
+
+    def step_e2e():
+        for L in layers:
+            s = L["spec"]
+            L["X"].copy_(L["X_host"], non_blocking=True)
+            hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
+            L["Y_host"].copy_(L["Y"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps, per-kernel events recorded on the launching stream
+    ev_steps = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * len(layers))] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(ev_steps[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_total = _max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    if hsq.hsq_get_device_status() != hsq.HSQ_OK:
+        raise RuntimeError("a kernel reported a timeout during the timed region")
+
+    # per-kernel device time (averaged over the timed steps)
+    gemm_ms = [statistics.mean(ev[4 * i + 1].elapsed_time(ev[4 * i + 2]) for ev in ev_steps)
+               for i in range(len(layers))]
+    act_ms = [statistics.mean(ev[4 * i].elapsed_time(ev[4 * i + 1]) for ev in ev_steps)
+              for i in range(len(layers))]
+
+    # ---- end to end through the public API with host buffers
+    for _ in range(max(1, args.warmup // 2)):
+        step_e2e()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step_e2e()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+
+    ops_step = sum(layer_ops(L["spec"]) for L in layers)
+    tokens_step = specs[0].M
+    tops = ops_step * world / (ms_step * 1e-3) / 1e12
+    tops_e2e = ops_step * world / (ms_e2e * 1e-3) / 1e12
+    h2d = sum(L["X_host"].numel() * 2 for L in layers)
+    d2h = sum(L["Y_host"].numel() * 2 for L in layers)
+
+    peaks = _peaks()
+    int8_peak = peaks["bf16_sustained"] * INT8_OVER_BF16_NOMINAL
+    gemm_ops = sum(2 * L["spec"].M * L["spec"].N * L["spec"].K + 2 * L["spec"].M * L["spec"].N * L["spec"].r
+                   for L in layers)
+    gemm_time = sum(gemm_ms) * 1e-3
+    achieved = gemm_ops / gemm_time / 1e12
+    roofline = {
+        "bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": achieved, "peak": int8_peak,
+        "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": None,
+        "peak_source": f"{peaks['source']}: bf16 sustained {peaks['bf16_sustained']} TFLOP/s x nominal INT8/BF16 "
+                       f"ratio {INT8_OVER_BF16_NOMINAL}",
+        "frac_of_spec_4500": achieved / 4500.0,
+    }
+    layer_detail = []
+    for L, g, a in zip(layers, gemm_ms, act_ms):
+        s = L["spec"]
+        gops = 2 * s.M * s.N * s.K + 2 * s.M * s.N * s.r
+        layer_detail.append({"layer": s.name, "M": s.M, "K": s.K, "N": s.N, "r": s.r,
+                             "gemm_us": g * 1e3, "act_us": a * 1e3,
+                             "gemm_tops": gops / (g * 1e-3) / 1e12,
+                             "gemm_gbs": layer_gemm_bytes(s) / (g * 1e-3) / 1e9,
+                             "act_gbs": layer_act_bytes(s) / (a * 1e-3) / 1e9})
+    ws_bytes = sum(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in layers)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, _ = oracle_timing(specs)
+        cpu = {"value": v / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": "W4A4 rank-4 linear TOPS (FLUX block linears)", "value": tops, "unit": "TOPS",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4xint4->int32/f32",
+            "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",
+            "config": {"workload": wl_name, "layers": [s.name for s in specs], "tokens_per_step": tokens_step,
+                       "r": specs[0].r, "group": 64, "parallelism": f"replicas x{world}",
+                       "l2": f"no flush; per-step working set {ws_bytes / 2**20:.0f} MiB > 126 MiB L2"},
+            "tokens_per_s": tokens_step * world / (ms_step * 1e-3),
+            "e2e": {"value": tops_e2e, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": ms_e2e},
+            "gpu_launches": 2 * len(layers) * args.steps,
+            "roofline": roofline,
+            "layers": layer_detail,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hsq", choices=["hsq", "reference"])
+    ap.add_argument("--workload", default="flux_block_r4", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl != "reference":
+        args.warmup = 3
+    rank, world, local = _dist_init()
+    specs = WORKLOADS[args.workload]
+    try:
+        if args.impl == "reference":
+            run_reference(args, specs, args.workload, rank, world)
+        else:
+            run_gpu(args, specs, args.workload, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,153 @@
+/*
+ * hsq.h -- C ABI of libhsq, a B200 (sm_100a) implementation of the
+ * low-rank-assisted W4A4 linear layer
+ *
+ *     Y = Q4(X_hat) Q4(R)^T + (X_hat L1) L2 + b,
+ *     X_hat = X diag(s)^-1,     R = W diag(s) - (L1 L2)^T,
+ *
+ * from "Deflating the Hessian: Rank-4 W4A4 Quantization for Multimodal
+ * Diffusion Transformers" (H-SVDQuant, arXiv 2610.11315):
+ *   - Abstract: every weight is a low-bit residual plus a high-precision
+ *     low-rank component; weights and activations are both 4-bit (W4A4).
+ *   - Table 1 and Table 8 captions: quantization groups of 64 along K.
+ *   - rit.work blog, diagonal-scaling paragraph: the smoothing vector s moves
+ *     range between activations and weights without changing the layer's
+ *     full-precision map (X_hat R^T + X_hat L1 L2 = X W^T before quantizing).
+ *
+ * Quantizer (symmetric signed INT4, one fp32 scale per 64 values along K):
+ *   scale = fp32(absmax / 7); code = clamp(round_half_even(fp32(v / scale)), -7, 7);
+ *   an all-zero group has scale 0 and codes 0.  K is zero-padded to
+ *   Kp = 64 * ceil(K / 64).
+ *
+ * Conventions shared by every call
+ *   - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *     allocates no device memory.  Every pointer must be 16-byte aligned.
+ *   - bf16 tensors are row-major __nv_bfloat16 (passed as void*).
+ *   - Packed codes: row-major [rows][Kp/2] bytes; byte j of a row holds code
+ *     2j in bits 0-3 and code 2j+1 in bits 4-7, 4-bit two's complement.
+ *     Padded codes (k >= K) are 0.
+ *   - Scales: group-major fp32 [G][ld] with G = ceil(K/64) and
+ *     ld = hsq_scales_ld(rows) = rows rounded up to a multiple of 4; entry
+ *     [g][i] is the scale of group g of row i; entries i >= rows are written 0.
+ *   - Calls are asynchronous on `stream`.  Arguments are validated on the host
+ *     before anything is launched; a rejected call launches nothing.
+ *   - Every wait inside a kernel is bounded; a kernel that gives up records
+ *     HSQ_ERR_TIMEOUT in a device status word, which hsq_get_device_status()
+ *     reports.
+ *   - Supported: group == 64, 0 <= r <= 32, K % 8 == 0, N % 8 == 0,
+ *     1 <= M, N, K <= 2^20.
+ */
+#ifndef HSQ_H_
+#define HSQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSQ_OK = 0,
+  HSQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, L1/L2 null with r > 0, ws too small */
+  HSQ_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned */
+  HSQ_ERR_UNSUPPORTED = 3,   /* group != 64, r > 32, K or N not a multiple of 8 */
+  HSQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+  HSQ_ERR_TIMEOUT = 5        /* a kernel gave up waiting (reported by hsq_get_device_status) */
+} hsq_status;
+
+typedef enum { HSQ_OUT_BF16 = 0, HSQ_OUT_F32 = 1 } hsq_out_dtype;
+
+/* Number of 64-wide groups along K: ceil(K / group).  Returns 0 if group <= 0. */
+int hsq_num_groups(int K, int group);
+
+/* Bytes of a packed code matrix with `rows` rows: rows * Kp / 2. */
+size_t hsq_codes_bytes(int rows, int K, int group);
+
+/* Leading dimension (in floats) of a group-major scale matrix: rows rounded up to 4. */
+int hsq_scales_ld(int rows);
+
+/* Bytes of a scale matrix: ceil(K/group) * hsq_scales_ld(rows) * 4. */
+size_t hsq_scales_bytes(int rows, int K, int group);
+
+/*
+ * Bytes of split-K scratch that hsq_linear_forward needs for this shape on the
+ * current device (0 when the shape runs without split-K).  The caller zero-fills
+ * the workspace once before its first use; every completed call leaves it
+ * zero-filled again.
+ */
+size_t hsq_workspace_bytes(int M, int N, int K, int r);
+
+/*
+ * Offline weight packing (Abstract: low-bit residual + high-precision
+ * low-rank part).  R[n,k] = fp32(W[n,k]*s[k] - sum_{j<r} L1[k,j]*L2[j,n]),
+ * formed in fp64 with the sum taken for j = 0..r-1, each multiply and add
+ * rounded separately; R is then quantized per 64-group of each row.
+ *   W_bf16   [N][K] bf16        s   [K] fp32 (all > 0)
+ *   L1_bf16  [K][r] bf16        L2_bf16 [r][N] bf16   (both NULL iff r == 0)
+ *   w_codes  out [N][Kp/2] u8   w_scales out [G][hsq_scales_ld(N)] fp32
+ */
+hsq_status hsq_pack_weights(const void* W_bf16, const float* s, const void* L1_bf16,
+                            const void* L2_bf16, int N, int K, int r, int group,
+                            uint8_t* w_codes, float* w_scales, cudaStream_t stream);
+
+/*
+ * Per-forward activation step (one fused kernel): X_hat = fp32(fp32(X)/s_k)
+ * (rit.work blog: smoothing), its group-64 INT4 codes and scales, and the
+ * low-rank down-projection U = X_hat L1 accumulated in fp32.
+ *   X_bf16  [M][K] bf16          s [K] fp32        L1_bf16 [K][r] bf16 (NULL iff r == 0)
+ *   x_codes out [M][Kp/2] u8     x_scales out [G][hsq_scales_ld(M)] fp32
+ *   U       out [M][r] fp32 (may be NULL iff r == 0)
+ */
+hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_bf16,
+                            int M, int K, int r, int group, uint8_t* x_codes,
+                            float* x_scales, float* U, cudaStream_t stream);
+
+/*
+ * The layer's forward (Abstract: 4-bit residual product plus the 16-bit
+ * low-rank branch):
+ *   Y[m,n] = sum_g sx[g][m] * sw[g][n] * P_g[m,n] + sum_j U[m,j] * L2[j,n] + b[n],
+ * with P_g the exact integer dot product of group g's codes.  The INT4 codes are
+ * multiplied on the tensor cores (tcgen05, kind::i8) one group at a time into
+ * Tensor Memory and each group's int32 partial is rescaled into an fp32
+ * accumulator; the low-rank branch and bias are added in the epilogue.
+ *   x_codes/x_scales/U   as written by hsq_quantize_act (U NULL iff r == 0)
+ *   w_codes/w_scales     as written by hsq_pack_weights
+ *   L2_bf16 [r][N] (NULL iff r == 0), bias_bf16 [N] or NULL for no bias
+ *   Y out [M][N], bf16 (HSQ_OUT_BF16, round-to-nearest-even) or fp32 (HSQ_OUT_F32)
+ *   workspace / ws_bytes: scratch of at least hsq_workspace_bytes(M,N,K,r) bytes
+ *     (may be NULL when that is 0); calls that share a workspace must not run
+ *     concurrently.
+ */
+hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, const float* U,
+                              const uint8_t* w_codes, const float* w_scales,
+                              const void* L2_bf16, const void* bias_bf16,
+                              int M, int N, int K, int r, int group,
+                              void* Y, hsq_out_dtype out,
+                              void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* hsq_status_string(hsq_status status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word of the
+ * current device: HSQ_ERR_TIMEOUT if any kernel since the last read gave up
+ * waiting, HSQ_ERR_CUDA if the synchronization itself failed, else HSQ_OK.
+ */
+hsq_status hsq_get_device_status(cudaStream_t stream);
+
+/*
+ * Test hook: when `flags` is nonzero, the next hsq_linear_forward call on this
+ * host thread runs with a deliberately unreachable wait and a wait limit of
+ * about `limit_ms` milliseconds, so that its kernel exits through the timeout
+ * path (no data movement is issued).  Used to check that a kernel that gives
+ * up returns cleanly and reports HSQ_ERR_TIMEOUT.
+ */
+void hsq_debug_force_timeout(int flags, int limit_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSQ_H_ */

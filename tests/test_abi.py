@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds, loads and
+exports every symbol that include/hsq.h declares; size helpers; argument
+validation that rejects a call before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w4a4_rank_assisted_b200 import hsq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hsq.h")
+
+# fake, non-null device addresses: the calls below must fail validation before
+# touching them
+A = 1 << 20          # 16-byte aligned
+MIS = (1 << 20) + 4  # misaligned
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hsq_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = hsq.load()
+    declared = _declared()
+    assert declared, "no declarations parsed"
+    assert set(declared) == set(hsq.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_size_helpers():
+    assert hsq.hsq_num_groups(64) == 1
+    assert hsq.hsq_num_groups(96) == 2
+    assert hsq.hsq_num_groups(5600) == 88
+    assert hsq.hsq_codes_bytes(3, 96) == 3 * 64
+    assert hsq.hsq_codes_bytes(4608, 3072) == 4608 * 1536
+    assert hsq.hsq_scales_ld(1) == 4 and hsq.hsq_scales_ld(4) == 4 and hsq.hsq_scales_ld(5) == 8
+    assert hsq.hsq_scales_bytes(5, 128) == 2 * 8 * 4
+    assert hsq.load().hsq_num_groups(10, 0) == 0
+
+
+def test_status_strings():
+    names = [hsq.status_string(i) for i in range(6)]
+    assert names == ["HSQ_OK", "HSQ_ERR_INVALID_ARG", "HSQ_ERR_ALIGNMENT", "HSQ_ERR_UNSUPPORTED",
+                     "HSQ_ERR_CUDA", "HSQ_ERR_TIMEOUT"]
+
+
+def _fwd(lib, **kw):
+    a = dict(xc=A, xs=A, U=A, wc=A, ws=A, L2=A, b=None, M=16, N=64, K=64, r=4, g=64, Y=A, out=0,
+             wsp=None, wsb=0)
+    a.update(kw)
+    return lib.hsq_linear_forward(a["xc"], a["xs"], a["U"], a["wc"], a["ws"], a["L2"], a["b"], a["M"],
+                                  a["N"], a["K"], a["r"], a["g"], a["Y"], a["out"], a["wsp"], a["wsb"],
+                                  None)
+
+
+def test_forward_argument_validation():
+    lib = hsq.load()
+    assert _fwd(lib, g=128) == hsq.HSQ_ERR_UNSUPPORTED
+    assert _fwd(lib, r=33) == hsq.HSQ_ERR_UNSUPPORTED
+    assert _fwd(lib, r=-1) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, K=100) == hsq.HSQ_ERR_UNSUPPORTED
+    assert _fwd(lib, N=60) == hsq.HSQ_ERR_UNSUPPORTED
+    assert _fwd(lib, M=0) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, N=0) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, K=(1 << 20) + 8) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, out=7) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, xc=None) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, Y=None) == hsq.HSQ_ERR_INVALID_ARG
+    assert _fwd(lib, L2=None) == hsq.HSQ_ERR_INVALID_ARG          # r > 0 needs L2
+    assert _fwd(lib, r=0) == hsq.HSQ_ERR_INVALID_ARG              # r == 0 wants L2 == U == NULL
+    assert _fwd(lib, xs=MIS) == hsq.HSQ_ERR_ALIGNMENT
+    assert _fwd(lib, b=MIS) == hsq.HSQ_ERR_ALIGNMENT
+
+
+def test_pack_and_act_argument_validation():
+    lib = hsq.load()
+    pk = lib.hsq_pack_weights
+    assert pk(A, A, A, A, 64, 64, 4, 32, A, A, None) == hsq.HSQ_ERR_UNSUPPORTED
+    assert pk(A, A, None, A, 64, 64, 4, 64, A, A, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert pk(A, A, A, A, 64, 66, 4, 64, A, A, None) == hsq.HSQ_ERR_UNSUPPORTED
+    assert pk(A, A, A, A, 64, 64, 4, 64, MIS, A, None) == hsq.HSQ_ERR_ALIGNMENT
+    assert pk(None, A, A, A, 64, 64, 4, 64, A, A, None) == hsq.HSQ_ERR_INVALID_ARG
+    qa = lib.hsq_quantize_act
+    assert qa(A, A, A, 8, 64, 4, 64, A, A, None, None) == hsq.HSQ_ERR_INVALID_ARG  # U missing
+    assert qa(A, A, A, 8, 64, 40, 64, A, A, A, None) == hsq.HSQ_ERR_UNSUPPORTED
+    assert qa(MIS, A, A, 8, 64, 4, 64, A, A, A, None) == hsq.HSQ_ERR_ALIGNMENT
+    assert qa(A, A, A, 0, 64, 4, 64, A, A, A, None) == hsq.HSQ_ERR_INVALID_ARG
+
+
+def test_workspace_needs_are_consistent():
+    # split-K is used only when the output tiles cannot fill the device
+    assert hsq.hsq_workspace_bytes(4608, 12288, 3072, 4) == 0
+    assert hsq.hsq_workspace_bytes(1, 4096, 12288, 4) > 0
+    assert hsq.hsq_workspace_bytes(0, 4096, 12288, 4) == 0

@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Codes, packed bytes and scales must match bit for bit; outputs must meet the
+layer's tolerance (see tests/_helpers.py).  Small shapes are compared element
+by element; shapes span several tiles and ragged tails in M, N and K.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hsq_oracle as O
+from w4a4_rank_assisted_b200 import hsq
+from w4a4_rank_assisted_b200.synth import LayerSpec, make_layer
+
+from _helpers import check_y, oracle_layer, pad_scales, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _run_gpu(layer, out=hsq.HSQ_OUT_F32, X=None):
+    X = layer.X if X is None else X
+    M, K = X.shape
+    N = layer.W.shape[0]
+    r = layer.spec.r
+    d = lambda t: None if t is None else t.to(DEV).contiguous()
+    pl = hsq.PackedLinear(d(layer.W), d(layer.s), d(layer.L1) if r else None,
+                          d(layer.L2) if r else None, d(layer.bias))
+    act = hsq.ActBuffers(M, K, r, DEV)
+    Y = torch.empty((M, N), dtype=torch.float32 if out == hsq.HSQ_OUT_F32 else torch.bfloat16, device=DEV)
+    ws = pl.workspace(M)
+    hsq.forward(pl, d(X), act, Y, workspace=ws, out=out)
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    torch.cuda.synchronize()
+    return pl, act, Y, ws
+
+
+def _spec(M, K, N, r, seed=0, bias=True, act="outlier"):
+    return LayerSpec(f"t{M}x{K}x{N}r{r}", M, K, N, r, act=act, outlier_frac=0.01, outlier_mult=30.0,
+                     seed=seed, bias=bias)
+
+
+def _check_all(layer, pl, act, Y, out_f32, where):
+    ref = oracle_layer(layer.X, layer.W, layer.s, layer.L1 if layer.spec.r else None,
+                       layer.L2 if layer.spec.r else None, layer.bias)
+    M, N = Y.shape
+    # weights: bit-exact codes and scales (with the zero padding of the layout)
+    assert np.array_equal(to_np(pl.w_codes), ref["w_codes"]), f"{where}: weight codes differ"
+    assert np.array_equal(to_np(pl.w_scales), pad_scales(ref["w_scales"], hsq.hsq_scales_ld(N))), \
+        f"{where}: weight scales differ"
+    # activations: bit-exact codes and scales; U within fp32 accumulation error
+    assert np.array_equal(to_np(act.x_codes), ref["x_codes"]), f"{where}: activation codes differ"
+    assert np.array_equal(to_np(act.x_scales), pad_scales(ref["x_scales"], hsq.hsq_scales_ld(M))), \
+        f"{where}: activation scales differ"
+    if layer.spec.r:
+        U = to_np(act.U).astype(np.float64)
+        scale = np.abs(ref["U"]).max() + 1e-30
+        assert np.max(np.abs(U - ref["U"])) <= 1e-5 * scale, f"{where}: U differs"
+    return check_y(to_np(Y), ref["Y"], out_f32, where)
+
+
+SMALL_SHAPES = [
+    # (M, K, N, r)   -- decode tiles, split-K, ragged M/N/K tails, large-M tiles
+    (1, 64, 128, 4),
+    (5, 96, 136, 1),
+    (16, 1152, 1152, 4),
+    (17, 256, 264, 4),
+    (33, 320, 128, 0),
+    (64, 512, 384, 32),
+    (65, 192, 520, 4),
+    (128, 1152, 256, 4),
+    (200, 224, 1160, 4),
+    (256, 1152, 1152, 4),
+    (300, 640, 512, 32),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r", SMALL_SHAPES)
+@pytest.mark.parametrize("out", [hsq.HSQ_OUT_F32, hsq.HSQ_OUT_BF16])
+def test_layer_matches_oracle(M, K, N, r, out):
+    layer = make_layer(_spec(M, K, N, r, seed=M + K + N + r))
+    pl, act, Y, _ = _run_gpu(layer, out)
+    _check_all(layer, pl, act, Y, out == hsq.HSQ_OUT_F32, f"{M}x{K}x{N} r{r}")
+
+
+def test_strong_low_rank_branch_and_zero_bias():
+    """Scale up L1, L2 so that the branch carries a large share of Y: a dropped
+    or transposed branch would fail the tolerance by a wide margin."""
+    layer = make_layer(_spec(96, 256, 192, 4, seed=5, bias=False))
+    layer.L1 = (layer.L1.float() * 40).to(torch.bfloat16)
+    layer.L2 = (layer.L2.float() * 40).to(torch.bfloat16)
+    pl, act, Y, _ = _run_gpu(layer)
+    ratio, r = _check_all(layer, pl, act, Y, True, "strong branch")
+    ref = oracle_layer(layer.X, layer.W, layer.s, layer.L1, layer.L2, None)
+    branch = ref["U"] @ to_np(layer.L2).astype(np.float64)
+    assert np.sqrt(np.mean(branch ** 2)) > 0.2 * r
+
+
+def test_zero_rows_and_zero_groups():
+    layer = make_layer(_spec(40, 192, 128, 4, seed=9))
+    X = layer.X.clone()
+    X[3] = 0           # an all-zero token: every group scale is 0
+    X[7, 64:128] = 0   # one all-zero group
+    layer.X = X
+    pl, act, Y, _ = _run_gpu(layer)
+    _check_all(layer, pl, act, Y, True, "zero rows")
+    assert np.all(to_np(act.x_scales)[:, 3] == 0)
+
+
+def test_unit_smoothing_lossless_grid_matches_dense_product():
+    """s = 1, r = 0, both operands on their INT4 grids: the layer is exact, so
+    the GPU output equals the fp64 X W^T up to fp32 accumulation."""
+    rng = np.random.default_rng(4)
+    M, K, N = 130, 256, 264
+    def grid(rows):
+        q = rng.integers(-7, 8, size=(rows, K))
+        q[:, ::64] = 7
+        sc = 2.0 ** rng.integers(-6, 2, size=(rows, K // 64))
+        return (q.reshape(rows, -1, 64) * sc[:, :, None]).reshape(rows, K)
+    X = torch.tensor(grid(M), dtype=torch.bfloat16)
+    W = torch.tensor(grid(N), dtype=torch.bfloat16)
+    grid_x = to_np(X)  # exact: every value is q * 2^e with |q| <= 7
+    pl = hsq.PackedLinear(W.to(DEV), torch.ones(K, device=DEV), None, None)
+    act = hsq.ActBuffers(M, K, 0, DEV)
+    Y = torch.empty((M, N), dtype=torch.float32, device=DEV)
+    hsq.forward(pl, X.to(DEV), act, Y, workspace=pl.workspace(M), out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    dense = O.dense_forward(grid_x, to_np(W), None)
+    assert np.max(np.abs(to_np(Y) - dense)) <= 1e-6 * np.abs(dense).max()
+
+
+def test_repeated_calls_are_deterministic_and_reuse_workspace():
+    layer = make_layer(_spec(3, 2048, 512, 4, seed=2))
+    pl, act, Y, ws = _run_gpu(layer)
+    assert ws is not None  # split-K path
+    assert int(ws[:16].view(torch.int32).abs().sum()) == 0  # counters back at zero
+    Y0 = Y.clone()
+    for _ in range(3):
+        hsq.forward(pl, layer.X.to(DEV), act, Y, workspace=ws, out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y0)
+
+
+def test_forced_timeout_reports_status_and_library_recovers():
+    layer = make_layer(_spec(16, 256, 256, 4, seed=3))
+    pl, act, Y, ws = _run_gpu(layer)
+    Y_ok = Y.clone()
+    hsq.hsq_debug_force_timeout(1, 30)
+    hsq.forward(pl, layer.X.to(DEV), act, Y, workspace=ws, out=hsq.HSQ_OUT_F32)
+    assert hsq.hsq_get_device_status() == hsq.HSQ_ERR_TIMEOUT
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK  # the word is cleared by the read
+    if ws is not None:
+        ws.zero_()  # an aborted call may leave split-K counters behind
+    hsq.forward(pl, layer.X.to(DEV), act, Y, workspace=ws, out=hsq.HSQ_OUT_F32)
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    assert torch.equal(Y, Y_ok)
+
+
+def test_invalid_arguments_launch_nothing():
+    layer = make_layer(_spec(8, 128, 64, 4, seed=1))
+    pl, act, Y, ws = _run_gpu(layer)
+    with pytest.raises(hsq.HsqError) as e:
+        hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, None,
+                               8, 64, 128, 4, Y, group=128)
+    assert e.value.status == hsq.HSQ_ERR_UNSUPPORTED
+    big = hsq.hsq_workspace_bytes(1, 4096, 12288, 4)
+    with pytest.raises(hsq.HsqError) as e:
+        hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, None,
+                               1, 4096, 12288, 4, Y, workspace=None)
+    assert big > 0 and e.value.status == hsq.HSQ_ERR_INVALID_ARG

@@ -1,0 +1,333 @@
+// hsq_lib.cu -- the C ABI of libhsq (declared in include/hsq.h): argument
+// validation, launch planning, tensor-map construction and kernel launches.
+//
+// Everything numeric happens in the kernels of hsq_quant.cuh and hsq_gemm.cuh;
+// this file only checks arguments (synchronously, before any launch) and
+// launches them.  It allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/hsq.h"
+#include "hsq_device.cuh"
+#include "hsq_gemm.cuh"
+#include "hsq_quant.cuh"
+
+namespace {
+
+constexpr int kGroup = 64;
+constexpr int kMaxDim = 1 << 20;
+constexpr int kMaxRank = 32;
+
+// Kernel configurations (see hsq_gemm.cuh).
+using CfgLarge = hsq::GemmCfg<256, 2, 8, false>;  // M > 64: 128 tokens x 256 outputs per tile
+using CfgDec16 = hsq::GemmCfg<16, 1, 16, true>;   // M <= 16: 128 outputs x 16 tokens
+using CfgDec32 = hsq::GemmCfg<32, 1, 12, true>;   // M <= 32
+using CfgDec64 = hsq::GemmCfg<64, 1, 10, true>;   // M <= 64
+
+thread_local int t_debug_flags = 0;
+thread_local int t_debug_limit_ms = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int groups_of(int K) { return (K + kGroup - 1) / kGroup; }
+int scales_ld(int rows) { return (rows + 3) & ~3; }
+
+uint64_t wait_limit_ns() {
+  static uint64_t v = [] {
+    const char* e = std::getenv("HSQ_WAIT_LIMIT_MS");
+    long ms = e ? std::strtol(e, nullptr, 10) : 4000;
+    if (ms <= 0) ms = 4000;
+    return static_cast<uint64_t>(ms) * 1000000ull;
+  }();
+  return v;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+// ------------------------------------------------------------------ planning
+enum Kind { kLarge = 0, kDec16, kDec32, kDec64 };
+
+struct Plan {
+  Kind kind;
+  int BN;
+  bool swap;
+  int drain_warps;
+  int tiles_r, tiles_c, splits, gps, units, grid;
+  size_t counters_bytes, partial_bytes;
+  size_t ws_bytes() const { return splits > 1 ? counters_bytes + partial_bytes : 0; }
+};
+
+Plan make_plan(int M, int N, int K, int nsm) {
+  Plan p{};
+  const int G = groups_of(K);
+  if (M <= 64) {
+    p.swap = true;
+    p.kind = M <= 16 ? kDec16 : M <= 32 ? kDec32 : kDec64;
+    p.BN = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+    p.drain_warps = 4;
+    p.tiles_r = (N + 127) / 128;
+    p.tiles_c = (M + p.BN - 1) / p.BN;
+  } else {
+    p.swap = false;
+    p.kind = kLarge;
+    p.BN = 256;
+    p.drain_warps = 8;
+    p.tiles_r = (M + 127) / 128;
+    p.tiles_c = (N + 255) / 256;
+  }
+  const int tiles = p.tiles_r * p.tiles_c;
+  // choose the split count that minimises the critical path (work units of the
+  // busiest CTA times groups per unit), preferring fewer splits on ties
+  int best_s = 1;
+  double best_cost = 1e30;
+  const int max_s = tiles >= nsm ? 1 : std::min(16, std::max(1, G / 4));
+  for (int s = 1; s <= max_s; ++s) {
+    const int gps = (G + s - 1) / s;
+    const int s_eff = (G + gps - 1) / gps;
+    const long units = static_cast<long>(tiles) * s_eff;
+    const double waves = static_cast<double>((units + nsm - 1) / nsm);
+    const double cost = waves * gps + (s_eff > 1 ? 2.0 : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best_s = s_eff;
+    }
+  }
+  p.gps = (G + best_s - 1) / best_s;
+  p.splits = (G + p.gps - 1) / p.gps;
+  p.units = tiles * p.splits;
+  p.grid = std::min(p.units, nsm);
+  p.counters_bytes = ((static_cast<size_t>(tiles) * p.drain_warps * 4 + 255) / 256) * 256;
+  p.partial_bytes = static_cast<size_t>(tiles) * p.splits * p.BN * 128 * 4;
+  return p;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// 2-D map over packed codes [rows][Kp/2] bytes, box = one 64-group (32 bytes) x box_rows.
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Kp / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Kp / 2)};
+  const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class Cfg>
+hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& tc, const hsq::GemmArgs& a,
+                       cudaStream_t st) {
+  static std::mutex mu;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      if (cudaFuncSetAttribute(hsq::w4a4_gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::SMEM_BYTES) != cudaSuccess)
+        return HSQ_ERR_CUDA;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
+  hsq::w4a4_gemm_kernel<Cfg><<<p.grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(tr, tc, a);
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hsq_num_groups(int K, int group) {
+  if (group <= 0 || K < 0) return 0;
+  return (K + group - 1) / group;
+}
+
+size_t hsq_codes_bytes(int rows, int K, int group) {
+  if (rows < 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(hsq_num_groups(K, group)) * group / 2;
+}
+
+int hsq_scales_ld(int rows) { return rows < 0 ? 0 : scales_ld(rows); }
+
+size_t hsq_scales_bytes(int rows, int K, int group) {
+  return static_cast<size_t>(hsq_num_groups(K, group)) * hsq_scales_ld(rows) * 4;
+}
+
+size_t hsq_workspace_bytes(int M, int N, int K, int r) {
+  (void)r;
+  if (M < 1 || N < 1 || K < 1) return 0;
+  return make_plan(M, N, K, device_sm_count()).ws_bytes();
+}
+
+const char* hsq_status_string(hsq_status s) {
+  switch (s) {
+    case HSQ_OK: return "HSQ_OK";
+    case HSQ_ERR_INVALID_ARG: return "HSQ_ERR_INVALID_ARG";
+    case HSQ_ERR_ALIGNMENT: return "HSQ_ERR_ALIGNMENT";
+    case HSQ_ERR_UNSUPPORTED: return "HSQ_ERR_UNSUPPORTED";
+    case HSQ_ERR_CUDA: return "HSQ_ERR_CUDA";
+    case HSQ_ERR_TIMEOUT: return "HSQ_ERR_TIMEOUT";
+  }
+  return "HSQ_UNKNOWN_STATUS";
+}
+
+void hsq_debug_force_timeout(int flags, int limit_ms) {
+  t_debug_flags = flags;
+  t_debug_limit_ms = limit_ms;
+}
+
+hsq_status hsq_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HSQ_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, hsq::g_status, sizeof(v)) != cudaSuccess) return HSQ_ERR_CUDA;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(hsq::g_status, &zero, sizeof(zero)) != cudaSuccess) return HSQ_ERR_CUDA;
+    return HSQ_ERR_TIMEOUT;
+  }
+  return HSQ_OK;
+}
+
+static hsq_status check_common(int rows, int K, int r, int group) {
+  if (group != kGroup) return HSQ_ERR_UNSUPPORTED;
+  if (rows < 1 || K < 1 || rows > kMaxDim || K > kMaxDim || r < 0) return HSQ_ERR_INVALID_ARG;
+  if (r > kMaxRank || (K % 8) != 0) return HSQ_ERR_UNSUPPORTED;
+  return HSQ_OK;
+}
+
+hsq_status hsq_pack_weights(const void* W_bf16, const float* s, const void* L1_bf16, const void* L2_bf16, int N,
+                            int K, int r, int group, uint8_t* w_codes, float* w_scales, cudaStream_t stream) {
+  hsq_status st = check_common(N, K, r, group);
+  if (st != HSQ_OK) return st;
+  if (!W_bf16 || !s || !w_codes || !w_scales) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1_bf16 != nullptr) || (r > 0) != (L2_bf16 != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      (L1_bf16 && !aligned16(L1_bf16)) || (L2_bf16 && !aligned16(L2_bf16)))
+    return HSQ_ERR_ALIGNMENT;
+  const int G = groups_of(K), Kp = G * kGroup, ld = scales_ld(N);
+  const int blocks = (N + 7) / 8;
+  hsq::pack_weights_kernel<<<blocks, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(W_bf16), s, static_cast<const __nv_bfloat16*>(L1_bf16),
+      static_cast<const __nv_bfloat16*>(L2_bf16), N, K, r, Kp, ld, w_codes, w_scales);
+  if (cudaGetLastError() != cudaSuccess) return HSQ_ERR_CUDA;
+  if (ld > N) {
+    const int n = (ld - N) * G;
+    hsq::zero_scale_pad_kernel<<<(n + 255) / 256, 256, 0, stream>>>(w_scales, N, ld, G);
+    if (cudaGetLastError() != cudaSuccess) return HSQ_ERR_CUDA;
+  }
+  return HSQ_OK;
+}
+
+hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_bf16, int M, int K, int r,
+                            int group, uint8_t* x_codes, float* x_scales, float* U, cudaStream_t stream) {
+  hsq_status st = check_common(M, K, r, group);
+  if (st != HSQ_OK) return st;
+  if (!X_bf16 || !s || !x_codes || !x_scales) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1_bf16 != nullptr) || (r > 0 && !U)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(x_codes) || !aligned16(x_scales) ||
+      (L1_bf16 && !aligned16(L1_bf16)) || (U && !aligned16(U)))
+    return HSQ_ERR_ALIGNMENT;
+  const int G = groups_of(K), Kp = G * kGroup, ld = scales_ld(M);
+  const dim3 grid((M + 7) / 8);
+  const auto* X = static_cast<const __nv_bfloat16*>(X_bf16);
+  const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
+  if (r == 0) hsq::quantize_act_kernel<0><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
+  else if (r <= 4) hsq::quantize_act_kernel<4><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
+  else if (r <= 8) hsq::quantize_act_kernel<8><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
+  else if (r <= 16) hsq::quantize_act_kernel<16><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
+  else hsq::quantize_act_kernel<32><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
+hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, const float* U, const uint8_t* w_codes,
+                              const float* w_scales, const void* L2_bf16, const void* bias_bf16, int M, int N, int K,
+                              int r, int group, void* Y, hsq_out_dtype out, void* workspace, size_t ws_bytes,
+                              cudaStream_t stream) {
+  hsq_status st = check_common(M, K, r, group);
+  if (st != HSQ_OK) return st;
+  if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return HSQ_ERR_UNSUPPORTED;
+  if (out != HSQ_OUT_BF16 && out != HSQ_OUT_F32) return HSQ_ERR_INVALID_ARG;
+  if (!x_codes || !x_scales || !w_codes || !w_scales || !Y) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L2_bf16 != nullptr) || (r > 0) != (U != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(Y) || (U && !aligned16(U)) || (L2_bf16 && !aligned16(L2_bf16)) ||
+      (bias_bf16 && !aligned16(bias_bf16)) || (workspace && !aligned16(workspace)))
+    return HSQ_ERR_ALIGNMENT;
+
+  const int G = groups_of(K), Kp = G * kGroup;
+  const Plan p = make_plan(M, N, K, device_sm_count());
+  if (p.ws_bytes() > 0 && (!workspace || ws_bytes < p.ws_bytes())) return HSQ_ERR_INVALID_ARG;
+
+  hsq::GemmArgs a{};
+  const int ldx = scales_ld(M), ldw = scales_ld(N);
+  CUtensorMap tm_row, tm_col;
+  bool ok;
+  if (!p.swap) {
+    a.scales_r = x_scales; a.ld_r = ldx; a.rows_r = M;
+    a.scales_c = w_scales; a.ld_c = ldw; a.rows_c = N;
+    ok = make_codes_map(&tm_row, x_codes, M, Kp, 128) && make_codes_map(&tm_col, w_codes, N, Kp, p.BN);
+  } else {
+    a.scales_r = w_scales; a.ld_r = ldw; a.rows_r = N;
+    a.scales_c = x_scales; a.ld_c = ldx; a.rows_c = M;
+    ok = make_codes_map(&tm_row, w_codes, N, Kp, 128) && make_codes_map(&tm_col, x_codes, M, Kp, p.BN);
+  }
+  if (!ok) return HSQ_ERR_CUDA;
+  a.U = U;
+  a.L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
+  a.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+  a.Y = Y;
+  a.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
+  a.M = M; a.N = N; a.G = G; a.r = r;
+  a.tiles_r = p.tiles_r; a.tiles_c = p.tiles_c; a.splits = p.splits; a.groups_per_split = p.gps;
+  if (p.splits > 1) {
+    a.ws_counters = static_cast<unsigned*>(workspace);
+    a.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.counters_bytes);
+  }
+  a.limit_ns = wait_limit_ns();
+  if (t_debug_flags) {
+    a.debug_flags = t_debug_flags;
+    a.limit_ns = static_cast<uint64_t>(t_debug_limit_ms > 0 ? t_debug_limit_ms : 50) * 1000000ull;
+    t_debug_flags = 0;
+  }
+  switch (p.kind) {
+    case kLarge: return launch_gemm<CfgLarge>(p, tm_row, tm_col, a, stream);
+    case kDec16: return launch_gemm<CfgDec16>(p, tm_row, tm_col, a, stream);
+    case kDec32: return launch_gemm<CfgDec32>(p, tm_row, tm_col, a, stream);
+    case kDec64: return launch_gemm<CfgDec64>(p, tm_row, tm_col, a, stream);
+  }
+  return HSQ_ERR_INVALID_ARG;
+}
+
+}  // extern "C"

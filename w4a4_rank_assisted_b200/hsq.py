@@ -1,0 +1,215 @@
+"""Python binding of libhsq's C ABI (include/hsq.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libhsq.so``.  Tensors are torch CUDA tensors (torch supplies device memory and
+streams); their ``data_ptr()`` values are handed to the C functions of the
+same names.  There is no CPU fallback: if the library is missing or a call
+fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+GROUP = 64
+
+HSQ_OK = 0
+HSQ_ERR_INVALID_ARG = 1
+HSQ_ERR_ALIGNMENT = 2
+HSQ_ERR_UNSUPPORTED = 3
+HSQ_ERR_CUDA = 4
+HSQ_ERR_TIMEOUT = 5
+HSQ_OUT_BF16 = 0
+HSQ_OUT_F32 = 1
+
+#: Every symbol that include/hsq.h declares.
+EXPORTED = (
+    "hsq_num_groups", "hsq_codes_bytes", "hsq_scales_ld", "hsq_scales_bytes",
+    "hsq_workspace_bytes", "hsq_pack_weights", "hsq_quantize_act",
+    "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
+    "hsq_debug_force_timeout",
+)
+
+
+class HsqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what} failed: {status_string(status)}")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libhsq.so (building it first if it is absent and nvcc is available)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        if not build_if_missing:
+            raise RuntimeError(f"libhsq.so not built at {path}")
+        _build.build()
+    lib = ctypes.CDLL(path)
+    c = ctypes
+    vp, i, sz = c.c_void_p, c.c_int, c.c_size_t
+    lib.hsq_num_groups.argtypes = [i, i]; lib.hsq_num_groups.restype = i
+    lib.hsq_codes_bytes.argtypes = [i, i, i]; lib.hsq_codes_bytes.restype = sz
+    lib.hsq_scales_ld.argtypes = [i]; lib.hsq_scales_ld.restype = i
+    lib.hsq_scales_bytes.argtypes = [i, i, i]; lib.hsq_scales_bytes.restype = sz
+    lib.hsq_workspace_bytes.argtypes = [i, i, i, i]; lib.hsq_workspace_bytes.restype = sz
+    lib.hsq_pack_weights.argtypes = [vp, vp, vp, vp, i, i, i, i, vp, vp, vp]
+    lib.hsq_pack_weights.restype = i
+    lib.hsq_quantize_act.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, vp]
+    lib.hsq_quantize_act.restype = i
+    lib.hsq_linear_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, sz, vp]
+    lib.hsq_linear_forward.restype = i
+    lib.hsq_status_string.argtypes = [i]; lib.hsq_status_string.restype = c.c_char_p
+    lib.hsq_get_device_status.argtypes = [vp]; lib.hsq_get_device_status.restype = i
+    lib.hsq_debug_force_timeout.argtypes = [i, i]; lib.hsq_debug_force_timeout.restype = None
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().hsq_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhsq takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libhsq takes contiguous tensors only")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != HSQ_OK:
+        raise HsqError(status, what)
+
+
+# ---------------------------------------------------------------- sizes
+def hsq_num_groups(K: int, group: int = GROUP) -> int:
+    return load().hsq_num_groups(K, group)
+
+
+def hsq_codes_bytes(rows: int, K: int, group: int = GROUP) -> int:
+    return load().hsq_codes_bytes(rows, K, group)
+
+
+def hsq_scales_ld(rows: int) -> int:
+    return load().hsq_scales_ld(rows)
+
+
+def hsq_scales_bytes(rows: int, K: int, group: int = GROUP) -> int:
+    return load().hsq_scales_bytes(rows, K, group)
+
+
+def hsq_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return load().hsq_workspace_bytes(M, N, K, r)
+
+
+# ---------------------------------------------------------------- the three calls
+def hsq_pack_weights(W, s, L1, L2, N, K, r, w_codes, w_scales, group=GROUP, stream=None) -> None:
+    _check(load().hsq_pack_weights(_ptr(W), _ptr(s), _ptr(L1), _ptr(L2), N, K, r, group,
+                                   _ptr(w_codes), _ptr(w_scales), _stream(stream)), "hsq_pack_weights")
+
+
+def hsq_quantize_act(X, s, L1, M, K, r, x_codes, x_scales, U, group=GROUP, stream=None) -> None:
+    _check(load().hsq_quantize_act(_ptr(X), _ptr(s), _ptr(L1), M, K, r, group,
+                                   _ptr(x_codes), _ptr(x_scales), _ptr(U), _stream(stream)),
+           "hsq_quantize_act")
+
+
+def hsq_linear_forward(x_codes, x_scales, U, w_codes, w_scales, L2, bias, M, N, K, r, Y,
+                       out: int = HSQ_OUT_BF16, workspace=None, ws_bytes: int = 0,
+                       group=GROUP, stream=None) -> None:
+    _check(load().hsq_linear_forward(_ptr(x_codes), _ptr(x_scales), _ptr(U), _ptr(w_codes),
+                                     _ptr(w_scales), _ptr(L2), _ptr(bias), M, N, K, r, group,
+                                     _ptr(Y), int(out), _ptr(workspace), int(ws_bytes),
+                                     _stream(stream)), "hsq_linear_forward")
+
+
+def hsq_get_device_status(stream=None) -> int:
+    return load().hsq_get_device_status(_stream(stream))
+
+
+def hsq_debug_force_timeout(flags: int, limit_ms: int) -> None:
+    load().hsq_debug_force_timeout(int(flags), int(limit_ms))
+
+
+# ---------------------------------------------------------------- buffers
+def alloc_codes(rows: int, K: int, device) -> torch.Tensor:
+    Kp = hsq_num_groups(K) * GROUP
+    return torch.empty((rows, Kp // 2), dtype=torch.uint8, device=device)
+
+
+def alloc_scales(rows: int, K: int, device) -> torch.Tensor:
+    return torch.empty((hsq_num_groups(K), hsq_scales_ld(rows)), dtype=torch.float32, device=device)
+
+
+class PackedLinear:
+    """A packed layer: INT4 residual codes and scales plus the low-rank pair,
+    the smoothing vector and the bias, all resident on one device."""
+
+    def __init__(self, W, s, L1, L2, bias=None, stream=None):
+        N, K = W.shape
+        r = 0 if L1 is None else int(L1.shape[1])
+        dev = W.device
+        self.N, self.K, self.r = N, K, r
+        self.s = s.contiguous()
+        self.L1 = None if r == 0 else L1.contiguous()
+        self.L2 = None if r == 0 else L2.contiguous()
+        self.bias = None if bias is None else bias.contiguous()
+        self.w_codes = alloc_codes(N, K, dev)
+        self.w_scales = alloc_scales(N, K, dev)
+        hsq_pack_weights(W.contiguous(), self.s, self.L1, self.L2, N, K, r,
+                         self.w_codes, self.w_scales, stream=stream)
+
+    def workspace(self, M: int) -> Optional[torch.Tensor]:
+        n = hsq_workspace_bytes(M, self.N, self.K, self.r)
+        if n == 0:
+            return None
+        return torch.zeros(n, dtype=torch.uint8, device=self.w_codes.device)
+
+
+class ActBuffers:
+    """Per-forward buffers of the activation step for M tokens."""
+
+    def __init__(self, M: int, K: int, r: int, device):
+        self.M, self.K, self.r = M, K, r
+        self.x_codes = alloc_codes(M, K, device)
+        self.x_scales = alloc_scales(M, K, device)
+        self.U = torch.empty((M, r), dtype=torch.float32, device=device) if r > 0 else None
+
+
+def forward(layer: PackedLinear, X: torch.Tensor, act: ActBuffers, Y: torch.Tensor,
+            workspace: Optional[torch.Tensor] = None, out: int = HSQ_OUT_BF16, stream=None) -> torch.Tensor:
+    """One forward of the layer: the activation step, then the GEMM + epilogue."""
+    M = X.shape[0]
+    hsq_quantize_act(X, layer.s, layer.L1, M, layer.K, layer.r, act.x_codes, act.x_scales, act.U,
+                     stream=stream)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    hsq_linear_forward(act.x_codes, act.x_scales, act.U, layer.w_codes, layer.w_scales, layer.L2,
+                       layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace,
+                       ws_bytes=ws_bytes, stream=stream)
+    return Y
