@@ -187,10 +187,12 @@ def oracle_timing(specs, budget_s: float = 12.0, seed_rows: int = 4):
             ops += layer_ops(spec) * m / spec.M
         return time.perf_counter() - t0, ops
 
-    dt, _ = run(seed_rows)
-    rows = max(seed_rows, int(seed_rows * budget_s / max(dt, 1e-3)))
-    rows = min(rows, min(s.M for s in specs))
+    rows = seed_rows
+    max_rows = min(s.M for s in specs)
     dt, ops = run(rows)
+    while dt < budget_s / 2 and rows < max_rows:
+        rows = min(max_rows, rows * 2)
+        dt, ops = run(rows)
     return ops / dt, cores, f"first {rows} token rows of each layer, weights pre-packed ({dt:.1f} s of CPU work)", dt
 
 

@@ -60,14 +60,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Test a phase; if it is not complete the hardware may park the thread (no
+// issue slots used) until it completes or about HSQ_SUSPEND_NS nanoseconds pass.
+#ifndef HSQ_SUSPEND_NS
+#define HSQ_SUSPEND_NS 20000
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(static_cast<uint32_t>(HSQ_SUSPEND_NS))
       : "memory");
   return ok != 0;
 }
@@ -93,7 +98,7 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, const W
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 31u) == 0) {
+    if ((spin & 3u) == 0) {
       if (*w.abort) return false;
       if (global_timer_ns() - t0 > w.limit_ns) {
         raise_timeout(w);
@@ -103,15 +108,18 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, const W
   }
 }
 
-// Whole-warp bounded wait with warp-uniform control flow: every lane polls the
-// barrier (so every lane acquires the phase), lane 0 alone decides a timeout.
+#ifndef HSQ_WAIT_ALL_LANES
+#define HSQ_WAIT_ALL_LANES 1
+#endif
+#if HSQ_WAIT_ALL_LANES
+// Whole-warp bounded wait: every lane polls; lane 0 alone decides a timeout.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitPolicy& w) {
   uint64_t t0 = 0;
   if (lane_id() == 0) t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     const bool done = mbar_try_wait(bar, parity);
     if (__all_sync(0xffffffffu, done)) return true;
-    if ((spin & 31u) == 0) {
+    if ((spin & 3u) == 0) {
       int give_up = 0;
       if (lane_id() == 0) {
         if (*w.abort) {
@@ -125,6 +133,37 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const 
     }
   }
 }
+#else
+// Whole-warp bounded wait with warp-uniform control flow.  Lane 0 alone polls
+// (and decides a timeout); once it sees the phase complete, every lane tests
+// the barrier once more, so that every lane acquires the phase itself.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitPolicy& w) {
+  int state = 0;  // 1 = phase complete, 2 = give up
+  if (lane_id() == 0) {
+    if (mbar_try_wait(bar, parity)) {
+      state = 1;
+    } else {
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(bar, parity)) { state = 1; break; }
+        if ((spin & 3u) == 0) {
+          if (*w.abort) { state = 2; break; }
+          if (global_timer_ns() - t0 > w.limit_ns) { raise_timeout(w); state = 2; break; }
+        }
+      }
+    }
+  }
+  state = __shfl_sync(0xffffffffu, state, 0);
+  if (state != 1) return false;
+  // the phase is complete and cannot advance without this warp, so this succeeds at once
+  bool ok = mbar_try_wait(bar, parity);
+  for (uint32_t i = 0; !ok && i < (1u << 16); ++i) ok = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, ok)) return true;
+  if (lane_id() == 0) raise_timeout(w);
+  return false;
+}
+
+#endif
 
 // ---------------------------------------------------------------- TMA / bulk copy
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
@@ -201,6 +240,41 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32-bit, 16 consecutive columns per thread, every value = `v`.
+__device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Packed fp32 pairs (sm_100 f32x2 instructions): d = a*b + c, d = a*b, d = a + b.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 
 // Shared-memory matrix descriptor for a K-major operand in the canonical
 // no-swizzle layout: 8-row x 16-byte core matrices, `lbo` bytes between the two

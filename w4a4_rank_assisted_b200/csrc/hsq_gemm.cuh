@@ -37,6 +37,19 @@
 
 namespace hsq {
 
+// Canonical no-swizzle K-major layout of an operand with `rows` rows and one
+// 64-wide group: core matrix (row/8, kc) (kc = 16-byte K chunk 0..3) at
+// (row/8)*SBO + kc*LBO bytes, its 8 rows 16 bytes apart; the second K=32 MMA
+// starts 2*LBO bytes in.  LBO = 160 (not 128) staggers the four K chunks of a
+// row block across shared-memory banks, so that the unpack warps' 16-byte
+// stores of 8 consecutive threads (4 rows x 2 halves) hit 8 distinct bank groups;
+// SBO = 3*LBO + 128.
+#ifndef HSQ_PAD_LAYOUT
+#define HSQ_PAD_LAYOUT 1
+#endif
+constexpr uint32_t kLBO = HSQ_PAD_LAYOUT ? 160 : 128;
+constexpr uint32_t kSBO = 3 * kLBO + 128;
+
 struct GemmArgs {
   const float* scales_r;  // row operand scales   [G][ld_r]
   const float* scales_c;  // col operand scales   [G][ld_c]
@@ -55,7 +68,18 @@ struct GemmArgs {
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
 };
 
-template <int BN_, int DH_, int STAGES_, bool SWAP_>
+// DRAIN_ selects how a group's int32 partial becomes fp32 in the drain; all
+// three give bit-identical results:
+//   0: cvt.rn.f32.s32 per value, scalar fmul/fma
+//   1: cvt.rn.f32.s32 per value, packed f32x2 mul/fma
+//   2: the TMEM partial starts each group at the bit pattern of 1.5*2^23, so the
+//      MMA leaves 1.5*2^23 + P (exact, |P| < 2^22) as an fp32 bit pattern; one
+//      packed f32x2 subtract recovers P exactly (no int->float conversion), and
+//      the drain re-fills the buffer with the pattern after reading it.
+#ifndef HSQ_DRAIN_MODE
+#define HSQ_DRAIN_MODE 1
+#endif
+template <int BN_, int DH_, int STAGES_, bool SWAP_, int DRAIN_ = HSQ_DRAIN_MODE>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -63,16 +87,25 @@ struct GemmCfg {
   static constexpr int CW = BN / DH;           // columns per drain thread
   static constexpr int STAGES = STAGES_;
   static constexpr bool SWAP = SWAP_;
+  static constexpr int DRAIN = DRAIN_;
   static constexpr int NUM_UNPACK_WARPS = 6;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
-  static constexpr bool REALLOC = CW > 64;     // drain needs > 128 registers
+  // Register split (setmaxnreg): producer/MMA/unpack warpgroups give registers
+  // to the drain warpgroups, which hold CW fp32 accumulators per thread.
+  static constexpr bool REALLOC = CW >= 64;
+#ifndef HSQ_REGS_LOW
+#define HSQ_REGS_LOW 64
+#endif
+  static constexpr int REGS_LOW = HSQ_REGS_LOW;
+  static constexpr int REGS_HIGH_RAW = ((65536 - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
+  static constexpr int REGS_HIGH = REGS_HIGH_RAW > 232 ? 232 : REGS_HIGH_RAW;
   static constexpr int A_PACK = BM * 32;       // packed bytes per group
   static constexpr int B_PACK = BN * 32;
   static constexpr int CS_BYTES = BN * 4;
   static constexpr int STAGE_BYTES = ((A_PACK + B_PACK + CS_BYTES + 1023) / 1024) * 1024;
-  static constexpr int A_I8 = BM * 64;
-  static constexpr int B_I8 = BN * 64;
+  static constexpr int A_I8 = (BM / 8) * kSBO;  // int8 operand bytes per group
+  static constexpr int B_I8 = (BN / 8) * kSBO;
   static constexpr int I8_BYTES = ((A_I8 + B_I8 + 1023) / 1024) * 1024;
   static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                  : (2 * BN <= 256) ? 256 : 512;
@@ -83,16 +116,17 @@ struct GemmCfg {
   static_assert(2 * BN <= 512, "TMEM");
 };
 
-// Canonical no-swizzle K-major layout of an operand with `rows` rows and one
-// 64-wide group: core matrix (row/8, kc) (kc = 16-byte K chunk 0..3) at
-// ((row/8)*4 + kc)*128 bytes, its 8 rows 16 bytes apart.  LBO = 128 (next K
-// chunk), SBO = 512 (next 8-row block); the second K=32 MMA starts 256 bytes in.
-constexpr uint32_t kLBO = 128, kSBO = 512;
 
-__device__ __forceinline__ void unpack_task(const uint8_t* src_stage, uint8_t* dst, int rows, int t) {
-  const int half = t / rows;      // which 16 packed bytes (K 0-31 or 32-63)
-  const int row = t - half * rows;
-  const uint4 p = *reinterpret_cast<const uint4*>(src_stage + row * 32 + half * 16);
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;
+
+// One unpack task: 16 packed bytes (32 codes) of one row -> two 16-byte core
+// matrix rows (even codes, odd codes).  Task t reads row t/2, half t%2, so 8
+// consecutive threads read 128 contiguous bytes.
+__device__ __forceinline__ void unpack_task(const uint8_t* src_stage, uint8_t* dst, int t) {
+  const int row = t >> 1;
+  const int half = t & 1;  // which 16 packed bytes (K 0-31 or 32-63)
+  const uint4 p = *reinterpret_cast<const uint4*>(src_stage + t * 16);
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint4 lo, hi;
   uint32_t* lo_w = reinterpret_cast<uint32_t*>(&lo);
@@ -102,9 +136,9 @@ __device__ __forceinline__ void unpack_task(const uint8_t* src_stage, uint8_t* d
     lo_w[i] = (w[i] << 4) & 0xF0F0F0F0u;  // even codes, 16*q as int8
     hi_w[i] = w[i] & 0xF0F0F0F0u;         // odd codes,  16*q as int8
   }
-  uint8_t* base = dst + ((row >> 3) * 4 + 2 * half) * 128 + (row & 7) * 16;
+  uint8_t* base = dst + (row >> 3) * kSBO + (2 * half) * kLBO + (row & 7) * 16;
   *reinterpret_cast<uint4*>(base) = lo;
-  *reinterpret_cast<uint4*>(base + 128) = hi;
+  *reinterpret_cast<uint4*>(base + kLBO) = hi;
 }
 
 template <class Cfg>
@@ -166,7 +200,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (Cfg::REALLOC) regs_dealloc<64>();
+    if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
     if (lane == 0 && !(args.debug_flags & 1)) {
       uint32_t it = 0;
       bool ok = true;
@@ -193,7 +227,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (Cfg::REALLOC) regs_dealloc<64>();
+    if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(BM, BN);
       uint32_t it = 0;
@@ -206,13 +240,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const int b = it & 1;
           const uint32_t ph = (it >> 1) & 1;
           if (!wait_one(&full8[b], ph, wp)) { ok = false; break; }
-          if (!wait_one(&tempty[b], ph ^ 1, wp)) { ok = false; break; }
+          // DRAIN 2: the drain pre-fills both buffers once and so completes phase 0 itself
+          if (!wait_one(&tempty[b], Cfg::DRAIN == 2 ? ph : ph ^ 1, wp)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(i8_base + b * Cfg::I8_BYTES);
           const uint32_t b_addr = a_addr + Cfg::A_I8;
           const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
-          mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
-          mma_i8(d, smem_desc_kmajor(a_addr + 256, kLBO, kSBO), smem_desc_kmajor(b_addr + 256, kLBO, kSBO),
+          mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc,
+                 Cfg::DRAIN == 2 ? 1u : 0u);
+          mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO), smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO),
                  idesc, 1u);
           mma_commit(&empty8[b]);
           mma_commit(&tfull[b]);
@@ -221,7 +257,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp < 2 + Cfg::NUM_UNPACK_WARPS) {
     // ------------------------------------------------------------ unpack
-    if (Cfg::REALLOC) regs_dealloc<64>();
+    if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
     const int ut = (warp - 2) * 32 + lane;
     constexpr int NT = 32 * Cfg::NUM_UNPACK_WARPS;
     uint32_t it = 0;
@@ -237,8 +273,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (!wait_warp(&empty8[b], ((it >> 1) & 1) ^ 1, wp)) { ok = false; break; }
         const uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
         uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
-        for (int t = ut; t < 2 * BM; t += NT) unpack_task(st, dst, BM, t);
-        for (int t = ut; t < 2 * BN; t += NT) unpack_task(st + Cfg::A_PACK, dst + Cfg::A_I8, BN, t);
+        for (int t = ut; t < 2 * BM; t += NT) unpack_task(st, dst, t);
+        for (int t = ut; t < 2 * BN; t += NT) unpack_task(st + Cfg::A_PACK, dst + Cfg::A_I8, t);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -249,7 +285,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ drain + epilogue
-    if (Cfg::REALLOC) regs_alloc<192>();
+    if (Cfg::REALLOC) regs_alloc<Cfg::REGS_HIGH>();
     const int dw = warp - (2 + Cfg::NUM_UNPACK_WARPS);
     const int q = warp & 3;            // TMEM lane quadrant
     const int h = dw >> 2;             // column slice
@@ -257,6 +293,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
+    if (Cfg::DRAIN == 2) {
+      // pre-fill this warp's lanes/columns of both TMEM buffers with the pattern
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int c = 0; c < CW / 16; ++c) tmem_st16_fill(t_lane + static_cast<uint32_t>(b * BN + h * CW + c * 16), kMagicBits);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[0]);
+        mbar_arrive(&tempty[1]);
+      }
+    }
     for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
       const int split = u % args.splits;
       const int tile = u / args.splits;
@@ -282,20 +332,37 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < CW / 16; ++c) {
           uint32_t v[16];
-          tmem_ld16(t_lane + static_cast<uint32_t>(b * BN + h * CW + c * 16), v);
+          const uint32_t taddr = t_lane + static_cast<uint32_t>(b * BN + h * CW + c * 16);
+          tmem_ld16(taddr, v);
           tmem_ld_wait();
+          if (Cfg::DRAIN == 2) tmem_st16_fill(taddr, kMagicBits);
 #pragma unroll
           for (int j4 = 0; j4 < 4; ++j4) {
             const float4 sc = *reinterpret_cast<const float4*>(cs + c * 16 + j4 * 4);
             const float scv[4] = {sc.x, sc.y, sc.z, sc.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 4; e += 2) {
               const int j = j4 * 4 + e;
-              const float t = scv[e] * __int2float_rn(static_cast<int>(v[j]));
-              acc[c * 16 + j] = fmaf(s_row, t, acc[c * 16 + j]);
+              float& a0 = acc[c * 16 + j];
+              float& a1 = acc[c * 16 + j + 1];
+              if (Cfg::DRAIN == 0) {
+                a0 = fmaf(s_row, scv[e] * __int2float_rn(static_cast<int>(v[j])), a0);
+                a1 = fmaf(s_row, scv[e + 1] * __int2float_rn(static_cast<int>(v[j + 1])), a1);
+              } else {
+                float p0, p1, t0, t1;
+                if (Cfg::DRAIN == 1) {
+                  p0 = __int2float_rn(static_cast<int>(v[j]));
+                  p1 = __int2float_rn(static_cast<int>(v[j + 1]));
+                } else {
+                  fadd2(p0, p1, __uint_as_float(v[j]), __uint_as_float(v[j + 1]), -kMagic, -kMagic);
+                }
+                fmul2(t0, t1, p0, p1, scv[e], scv[e + 1]);
+                ffma2(a0, a1, s_row, s_row, t0, t1, a0, a1);
+              }
             }
           }
         }
+        if (Cfg::DRAIN == 2) tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {

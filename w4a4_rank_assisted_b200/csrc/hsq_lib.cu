@@ -259,14 +259,31 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
       (L1_bf16 && !aligned16(L1_bf16)) || (U && !aligned16(U)))
     return HSQ_ERR_ALIGNMENT;
   const int G = groups_of(K), Kp = G * kGroup, ld = scales_ld(M);
-  const dim3 grid((M + 7) / 8);
   const auto* X = static_cast<const __nv_bfloat16*>(X_bf16);
   const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
-  if (r == 0) hsq::quantize_act_kernel<0><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
-  else if (r <= 4) hsq::quantize_act_kernel<4><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
-  else if (r <= 8) hsq::quantize_act_kernel<8><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
-  else if (r <= 16) hsq::quantize_act_kernel<16><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
-  else hsq::quantize_act_kernel<32><<<grid, 256, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U);
+#define HSQ_ACT_LAUNCH(RV, SM)                                                                     \
+  hsq::quantize_act_kernel<RV, SM><<<(M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB,      \
+                                     hsq::ActCfg<RV, SM>::NW * 32, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, \
+                                                                                x_codes, x_scales, U)
+#define HSQ_ACT_RANKS(SM)                   \
+  switch (r) {                              \
+    case 0: HSQ_ACT_LAUNCH(0, SM); break;   \
+    case 1: HSQ_ACT_LAUNCH(1, SM); break;   \
+    case 2: HSQ_ACT_LAUNCH(2, SM); break;   \
+    case 4: HSQ_ACT_LAUNCH(4, SM); break;   \
+    case 8: HSQ_ACT_LAUNCH(8, SM); break;   \
+    case 16: HSQ_ACT_LAUNCH(16, SM); break; \
+    case 32: HSQ_ACT_LAUNCH(32, SM); break; \
+    default: HSQ_ACT_LAUNCH(-1, SM); break; \
+  }
+  // few rows: one block per sub-block with 32 warps spread over K; else 8 warps x 2 sub-blocks
+  if (M <= 64) {
+    HSQ_ACT_RANKS(true)
+  } else {
+    HSQ_ACT_RANKS(false)
+  }
+#undef HSQ_ACT_RANKS
+#undef HSQ_ACT_LAUNCH
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 

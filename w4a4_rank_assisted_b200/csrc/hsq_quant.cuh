@@ -92,69 +92,151 @@ __global__ void zero_scale_pad_kernel(float* scales, int rows, int ld, int G) {
 
 // ---------------------------------------------------------------------------
 // Fused activation step: X_hat = fp32(X)/s (IEEE division), its group codes and
-// scales, and U = X_hat L1 in fp32.  One warp per token row, 8 rows per block;
-// each lane loads 8 bf16 (one 16-byte load) per 256-wide chunk of K.
-// RT is a compile-time upper bound on r (the loops are unrolled and predicated).
+// scales, and U = X_hat L1 accumulated in fp32.
+//
+// A block of NW warps owns RB consecutive token rows, split into sub-blocks of
+// SUB rows.  Warp w works on sub-block w % (RB/SUB) and on the 256-wide K chunks
+// w / (RB/SUB), + NW/(RB/SUB), ...  Per chunk a lane loads the smoothing factors
+// and the L1 rows of its 8 channels once (16-byte loads) and reuses them for the
+// SUB rows, whose X loads are issued together.  U is reduced across lanes with
+// shuffles and across warps through shared memory in a fixed order, so the
+// result does not depend on scheduling.  Small M uses NW = 32 warps on one
+// sub-block so that K is spread over the whole block.
+//
+// R is the rank as a compile-time constant (1, 2, 4, 8, 16, 32, or 0 for no
+// branch); R = -1 is the generic path for any other r <= 32 (scalar L1 loads).
 // ---------------------------------------------------------------------------
-template <int RT>
-__global__ void __launch_bounds__(256) quantize_act_kernel(const __nv_bfloat16* __restrict__ X,
-                                                           const float* __restrict__ s,
-                                                           const __nv_bfloat16* __restrict__ L1, int M,
-                                                           int K, int r, int Kp, int ld,
-                                                           uint8_t* __restrict__ codes,
-                                                           float* __restrict__ scales,
-                                                           float* __restrict__ U) {
-  const int m = static_cast<int>(blockIdx.x * 8 + (threadIdx.x >> 5));
-  const int lane = lane_id();
-  if (m >= M) return;  // warp-uniform
-  float u[RT > 0 ? RT : 1];
-#pragma unroll
-  for (int j = 0; j < (RT > 0 ? RT : 1); ++j) u[j] = 0.f;
+template <int R, bool SMALL>
+struct ActCfg {
+  static constexpr int RMAX = R < 0 ? 32 : R;  // accumulator width
+  static constexpr int SUB = (SMALL || R < 0 || R == 32) ? 2 : 4;
+  static constexpr int NW = SMALL ? 16 : 8;
+  static constexpr int RB = SMALL ? SUB : 2 * SUB;
+  static constexpr int NSUB = RB / SUB;
+};
 
-  for (int c0 = 0; c0 < Kp; c0 += 256) {
-    const int k0 = c0 + lane * 8;
-    float xh[8];
-    if (k0 < K) {
-      const uint4 xraw = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k0));
+template <int R, bool SMALL>
+__global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
+    quantize_act_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
+                        const __nv_bfloat16* __restrict__ L1, int M, int K, int r, int Kp, int ld,
+                        uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U) {
+  using C = ActCfg<R, SMALL>;
+  constexpr int SUB = C::SUB, NW = C::NW, RB = C::RB, NSUB = C::NSUB;
+  constexpr int RA = C::RMAX > 0 ? C::RMAX : 1;
+  __shared__ float upart[R != 0 ? NW : 1][SUB][RA];
+  const int warp = threadIdx.x >> 5;
+  const int lane = lane_id();
+  const int sb = warp % NSUB;
+  const int mb = blockIdx.x * RB + sb * SUB;  // first row of this warp's sub-block
+  const int nchunks = (Kp + 255) / 256;
+
+  float u[SUB][RA];
+#pragma unroll
+  for (int i = 0; i < SUB; ++i)
+#pragma unroll
+    for (int j = 0; j < RA; ++j) u[i][j] = 0.f;
+
+  for (int c = warp / NSUB; c < nchunks; c += NW / NSUB) {
+    const int k0 = c * 256 + lane * 8;
+    const bool real = k0 < K;  // K % 8 == 0: a lane's 8 channels are all real or all padding
+    const bool in_k = k0 < Kp;
+    float sv[8];
+    if (real) {
       const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + k0));
       const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + k0 + 4));
-      float x[8];
-      bf16x8_to_f32(xraw, x);
-      const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) xh[e] = __fdiv_rn(x[e], sv[e]);
-      if (RT > 0) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const __nv_bfloat16* l1row = L1 + static_cast<size_t>(k0 + e) * r;
-#pragma unroll
-          for (int j = 0; j < RT; ++j)
-            if (j < r) u[j] = fmaf(xh[e], __bfloat162float(__ldg(l1row + j)), u[j]);
-        }
-      }
+      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+      sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xh[e] = 0.f;
+      for (int e = 0; e < 8; ++e) sv[e] = 1.f;
     }
-    float sc;
-    const uint32_t packed = quantize8(xh, sc);
-    if (k0 < Kp) {
-      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
-      if ((lane & 7) == 0) {
-        float* srow = scales + static_cast<size_t>(k0 / 64) * ld;
-        srow[m] = sc;
-        if (m == M - 1)
-          for (int p = M; p < ld; ++p) srow[p] = 0.f;  // padding of the group-major layout
+    // small ranks: the 8 channels' L1 rows (8*R bf16, contiguous) stay in registers
+    float l1s[8][(R > 0 && R <= 4) ? R : 1];
+    if constexpr (R > 0 && R <= 4) {
+      const uint4* src = reinterpret_cast<const uint4*>(L1 + static_cast<size_t>(k0) * R);
+#pragma unroll
+      for (int v = 0; v < R; ++v) {
+        float f[8];
+        bf16x8_to_f32(real ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u), f);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) l1s[(v * 8 + t) / R][(v * 8 + t) % R] = f[t];
+      }
+    }
+    uint4 xr[SUB];
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      const int m = mb + i;
+      xr[i] = (real && m < M) ? __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k0))
+                              : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      const int m = mb + i;
+      if (m >= M) break;  // warp-uniform
+      float x[8], xh[8];
+      bf16x8_to_f32(xr[i], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xh[e] = real ? __fdiv_rn(x[e], sv[e]) : 0.f;
+      if constexpr (R > 0 && R <= 4) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+          for (int j = 0; j < R; ++j) u[i][j] = fmaf(xh[e], l1s[e][j], u[i][j]);
+      } else if constexpr (R >= 8) {
+        // L1 row of channel k0+e, 8 ranks at a time (16-byte loads; L1-cache hits after the first row)
+        if (real) {
+#pragma unroll
+          for (int jc = 0; jc < R; jc += 8)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float f[8];
+              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(L1 + static_cast<size_t>(k0 + e) * R + jc)), f);
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) u[i][jc + jj] = fmaf(xh[e], f[jj], u[i][jc + jj]);
+            }
+        }
+      } else if constexpr (R < 0) {
+        if (real) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const __nv_bfloat16* row = L1 + static_cast<size_t>(k0 + e) * r;
+#pragma unroll
+            for (int j = 0; j < RA; ++j)
+              if (j < r) u[i][j] = fmaf(xh[e], __bfloat162float(__ldg(row + j)), u[i][j]);
+          }
+        }
+      }
+      float sc;
+      const uint32_t packed = quantize8(xh, sc);
+      if (in_k) {
+        *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
+        if ((lane & 7) == 0) {
+          float* srow = scales + static_cast<size_t>(k0 / 64) * ld;
+          srow[m] = sc;
+          if (m == M - 1)
+            for (int p = M; p < ld; ++p) srow[p] = 0.f;  // padding of the group-major layout
+        }
       }
     }
   }
-  if (RT > 0) {
+  if constexpr (R != 0) {
 #pragma unroll
-    for (int j = 0; j < RT; ++j) {
-      float v = u[j];
+    for (int i = 0; i < SUB; ++i)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && j < r) U[static_cast<size_t>(m) * r + j] = v;
+      for (int j = 0; j < RA; ++j) {
+        float v = u[i][j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) upart[warp][i][j] = v;
+      }
+    __syncthreads();
+    const int rows = min(RB, M - static_cast<int>(blockIdx.x) * RB);
+    for (int t = threadIdx.x; t < rows * r; t += blockDim.x) {
+      const int row = t / r, j = t - (t / r) * r;
+      const int tsb = row / SUB, i = row - tsb * SUB;
+      float v = 0.f;
+      for (int w = tsb; w < NW; w += NSUB) v += upart[w][i][j];  // fixed order
+      U[(static_cast<size_t>(blockIdx.x) * RB + row) * r + j] = v;
     }
   }
 }
