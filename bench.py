@@ -245,37 +245,70 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     if hsq.hsq_get_device_status() != hsq.HSQ_OK:
         raise RuntimeError("device status not clean after packing")
 
-    n_ev = 2 * len(layers)
+    def launch_act(L, st):
+        s = L["spec"]
+        hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
+                             L["act"].x_scales, L["act"].U, stream=st)
 
-    def step(evs=None):
-        for i, L in enumerate(layers):
-            s = L["spec"]
-            if evs is not None:
-                evs[4 * i].record(stream)
-            hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
-                                 L["act"].x_scales, L["act"].U, stream=stream)
-            if evs is not None:
-                evs[4 * i + 1].record(stream)
-            hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
-                                   L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
-                                   workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
-                                   stream=stream)
-            if evs is not None:
-                evs[4 * i + 2].record(stream)
+    def launch_gemm(L, st):
+        s = L["spec"]
+        hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
+                               L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
+                               workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
+                               stream=st)
+
+    def step(st):
+        for L in layers:
+            launch_act(L, st)
+            launch_gemm(L, st)
 
     def step_e2e():
         for L in layers:
-            s = L["spec"]
             L["X"].copy_(L["X_host"], non_blocking=True)
             hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
             L["Y_host"].copy_(L["Y"], non_blocking=True)
 
+    # Working sets smaller than L2 (decode sizes) are timed with L2 flushed before
+    # every step: a 256 MiB write, captured with the step, whose own time is
+    # measured alone and subtracted.
+    ws_bytes = sum(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in layers)
+    flush = ws_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if flush else None
+
+    # One step is captured once into a CUDA graph and replayed: at decode sizes a
+    # kernel runs for a few microseconds, less than its host-side launch.
+    gstream = torch.cuda.Stream(device=dev)
+    gstream.wait_stream(stream)
+    with torch.cuda.stream(gstream):
+        for _ in range(2):
+            step(gstream)
+    torch.cuda.synchronize()
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gstream):
+            fn(gstream)
+        return g
+
+    def do_flush(st):
+        if flush:
+            flush_buf.fill_(1)
+
+    g_step = capture(lambda st: (do_flush(st), step(st)))
+    g_flush = capture(do_flush) if flush else None
     for _ in range(args.warmup):
-        step()
+        g_step.replay()
     torch.cuda.synchronize()
 
-    # ---- timed region: exactly K steps, per-kernel events recorded on the launching stream
-    ev_steps = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * len(layers))] for _ in range(args.steps)]
+    def replay_ms(g, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(gstream)
+        for _ in range(n):
+            g.replay()
+        b.record(gstream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    # ---- timed region: exactly K steps
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -283,26 +316,40 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for k in range(args.steps):
-        step(ev_steps[k])
-    t1.record(stream)
+    t0.record(gstream)
+    for _ in range(args.steps):
+        g_step.replay()
+    t1.record(gstream)
     torch.cuda.synchronize()
     _barrier(world)
     clk = clocks.stop()
     ms_total = t0.elapsed_time(t1)
+    if flush:
+        ms_total -= replay_ms(g_flush, args.steps)
     ms_total = _max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
     if hsq.hsq_get_device_status() != hsq.HSQ_OK:
         raise RuntimeError("a kernel reported a timeout during the timed region")
 
-    # per-kernel device time (averaged over the timed steps)
-    gemm_ms = [statistics.mean(ev[4 * i + 1].elapsed_time(ev[4 * i + 2]) for ev in ev_steps)
-               for i in range(len(layers))]
-    act_ms = [statistics.mean(ev[4 * i].elapsed_time(ev[4 * i + 1]) for ev in ev_steps)
-              for i in range(len(layers))]
+    # ---- per-kernel device time: each kernel alone, REPS launches per graph,
+    # CUDA events on the replaying stream
+    def kernel_us(fn):
+        reps = 20
+        if flush:  # (flush + kernel) minus (flush alone), per launch
+            g = capture(lambda st: [(do_flush(st), fn(st)) for _ in range(reps)])
+            g0 = capture(lambda st: [do_flush(st) for _ in range(reps)])
+            g.replay(); g0.replay()
+            torch.cuda.synchronize()
+            return (replay_ms(g, 3) - replay_ms(g0, 3)) * 1e3 / (3 * reps)
+        g = capture(lambda st: [fn(st) for _ in range(reps)])
+        g.replay()
+        torch.cuda.synchronize()
+        return replay_ms(g, 3) * 1e3 / (3 * reps)
 
-    # ---- end to end through the public API with host buffers
+    gemm_us = [kernel_us(lambda st, L=L: launch_gemm(L, st)) for L in layers]
+    act_us = [kernel_us(lambda st, L=L: launch_act(L, st)) for L in layers]
+
+    # ---- end to end through the public API with host buffers (no graph)
     for _ in range(max(1, args.warmup // 2)):
         step_e2e()
     torch.cuda.synchronize()
@@ -322,29 +369,38 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     h2d = sum(L["X_host"].numel() * 2 for L in layers)
     d2h = sum(L["Y_host"].numel() * 2 for L in layers)
 
+    # ---- roofline of the dominant kernel (the GEMM, all layers of the step):
+    # tensor-bound when its INT8 time floor exceeds its HBM floor, else HBM-bound
     peaks = _peaks()
     int8_peak = peaks["bf16_sustained"] * INT8_OVER_BF16_NOMINAL
     gemm_ops = sum(2 * L["spec"].M * L["spec"].N * L["spec"].K + 2 * L["spec"].M * L["spec"].N * L["spec"].r
                    for L in layers)
-    gemm_time = sum(gemm_ms) * 1e-3
-    achieved = gemm_ops / gemm_time / 1e12
-    roofline = {
-        "bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": achieved, "peak": int8_peak,
-        "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": None,
-        "peak_source": f"{peaks['source']}: bf16 sustained {peaks['bf16_sustained']} TFLOP/s x nominal INT8/BF16 "
-                       f"ratio {INT8_OVER_BF16_NOMINAL}",
-        "frac_of_spec_4500": achieved / 4500.0,
-    }
+    gemm_bytes = sum(layer_gemm_bytes(L["spec"]) for L in layers)
+    gemm_time = sum(gemm_us) * 1e-6
+    t_tensor = gemm_ops / (int8_peak * 1e12)
+    t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        achieved = gemm_ops / gemm_time / 1e12
+        roofline = {"bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": achieved, "peak": int8_peak,
+                    "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": None,
+                    "peak_source": f"{peaks['source']}: bf16 sustained {peaks['bf16_sustained']} TFLOP/s x nominal "
+                                   f"INT8/BF16 ratio {INT8_OVER_BF16_NOMINAL}",
+                    "frac_of_spec_4500": achieved / 4500.0}
+    else:
+        achieved = gemm_bytes / gemm_time / 1e9
+        roofline = {"bound": "hbm", "kernel": "w4a4_gemm_kernel", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "peak_source": f"{peaks['source']} copy bandwidth", "frac_of_spec_8000": achieved / 8000.0}
+    roofline["algorithmic_per_launch"] = {"ops": gemm_ops / len(layers), "bytes": gemm_bytes / len(layers)}
     layer_detail = []
-    for L, g, a in zip(layers, gemm_ms, act_ms):
+    for L, g, a in zip(layers, gemm_us, act_us):
         s = L["spec"]
         gops = 2 * s.M * s.N * s.K + 2 * s.M * s.N * s.r
         layer_detail.append({"layer": s.name, "M": s.M, "K": s.K, "N": s.N, "r": s.r,
-                             "gemm_us": g * 1e3, "act_us": a * 1e3,
-                             "gemm_tops": gops / (g * 1e-3) / 1e12,
-                             "gemm_gbs": layer_gemm_bytes(s) / (g * 1e-3) / 1e9,
-                             "act_gbs": layer_act_bytes(s) / (a * 1e-3) / 1e9})
-    ws_bytes = sum(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in layers)
+                             "gemm_us": g, "act_us": a,
+                             "gemm_tops": gops / (g * 1e-6) / 1e12,
+                             "gemm_gbs": layer_gemm_bytes(s) / (g * 1e-6) / 1e9,
+                             "act_gbs": layer_act_bytes(s) / (a * 1e-6) / 1e9})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -359,11 +415,15 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",
             "config": {"workload": wl_name, "layers": [s.name for s in specs], "tokens_per_step": tokens_step,
                        "r": specs[0].r, "group": 64, "parallelism": f"replicas x{world}",
-                       "l2": f"no flush; per-step working set {ws_bytes / 2**20:.0f} MiB > 126 MiB L2"},
+                       "l2": (f"L2 flushed (256 MiB write) before every step and every timed kernel; flush "
+                              f"time measured alone and subtracted; working set {ws_bytes / 2**20:.0f} MiB"
+                              if flush else
+                              f"no flush; per-step working set {ws_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2")},
             "tokens_per_s": tokens_step * world / (ms_step * 1e-3),
             "e2e": {"value": tops_e2e, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": ms_e2e},
             "gpu_launches": 2 * len(layers) * args.steps,
+            "graph": "one step captured in a CUDA graph, replayed K times",
             "roofline": roofline,
             "layers": layer_detail,
             "cpu_baseline": cpu,
@@ -375,7 +435,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hsq", choices=["hsq", "reference"])
     ap.add_argument("--workload", default="flux_block_r4", choices=sorted(WORKLOADS))

@@ -73,6 +73,8 @@ SMALL_SHAPES = [
     (200, 224, 1160, 4),
     (256, 1152, 1152, 4),
     (300, 640, 512, 32),
+    (16, 4096, 2048, 4),     # stream-K, decode tile
+    (128, 2048, 1024, 4),    # stream-K, large tile
 ]
 
 
@@ -131,9 +133,9 @@ def test_unit_smoothing_lossless_grid_matches_dense_product():
 
 
 def test_repeated_calls_are_deterministic_and_reuse_workspace():
-    layer = make_layer(_spec(3, 2048, 512, 4, seed=2))
+    layer = make_layer(_spec(3, 4096, 2048, 4, seed=2))
     pl, act, Y, ws = _run_gpu(layer)
-    assert ws is not None  # split-K path
+    assert ws is not None  # stream-K path (tiles cut between CTAs)
     assert int(ws[:16].view(torch.int32).abs().sum()) == 0  # counters back at zero
     Y0 = Y.clone()
     for _ in range(3):

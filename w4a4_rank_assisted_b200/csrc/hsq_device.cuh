@@ -65,8 +65,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 #ifndef HSQ_SUSPEND_NS
 #define HSQ_SUSPEND_NS 20000
 #endif
+#ifndef HSQ_SPIN
+#define HSQ_SPIN 0
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
+#if HSQ_SPIN
+  // non-blocking test: the caller's loop spins
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+#elif HSQ_SUSPEND_NS > 0
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -74,8 +87,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity), "r"(static_cast<uint32_t>(HSQ_SUSPEND_NS))
       : "memory");
+#else
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+#endif
   return ok != 0;
 }
+
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// How often a polling loop checks the clock and the abort flag.
+#define HSQ_CHECK_MASK (HSQ_SPIN ? 255u : 3u)
 
 // Per-CTA wait policy: a time limit and a shared abort flag.
 struct WaitPolicy {
@@ -94,11 +132,11 @@ __device__ __forceinline__ void raise_timeout(const WaitPolicy& w) {
 //
 // Single-thread bounded wait.  Returns false on timeout or abort.
 __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, const WaitPolicy& w) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 3u) == 0) {
+    if ((spin & HSQ_CHECK_MASK) == 0) {
       if (*w.abort) return false;
       if (global_timer_ns() - t0 > w.limit_ns) {
         raise_timeout(w);
@@ -108,62 +146,16 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, const W
   }
 }
 
-#ifndef HSQ_WAIT_ALL_LANES
-#define HSQ_WAIT_ALL_LANES 1
-#endif
-#if HSQ_WAIT_ALL_LANES
-// Whole-warp bounded wait: every lane polls; lane 0 alone decides a timeout.
+// Whole-warp bounded wait: lane 0 tests the barrier (and decides a timeout),
+// then __syncwarp orders every other lane's later accesses after lane 0's
+// acquire of the phase.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitPolicy& w) {
-  uint64_t t0 = 0;
-  if (lane_id() == 0) t0 = global_timer_ns();
-  for (uint32_t spin = 1;; ++spin) {
-    const bool done = mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, done)) return true;
-    if ((spin & 3u) == 0) {
-      int give_up = 0;
-      if (lane_id() == 0) {
-        if (*w.abort) {
-          give_up = 1;
-        } else if (global_timer_ns() - t0 > w.limit_ns) {
-          raise_timeout(w);
-          give_up = 1;
-        }
-      }
-      if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
-    }
-  }
+  int ok = 1;
+  if (lane_id() == 0) ok = wait_one(bar, parity, w) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);  // also a warp barrier with memory ordering
+  __syncwarp();
+  return ok != 0;
 }
-#else
-// Whole-warp bounded wait with warp-uniform control flow.  Lane 0 alone polls
-// (and decides a timeout); once it sees the phase complete, every lane tests
-// the barrier once more, so that every lane acquires the phase itself.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitPolicy& w) {
-  int state = 0;  // 1 = phase complete, 2 = give up
-  if (lane_id() == 0) {
-    if (mbar_try_wait(bar, parity)) {
-      state = 1;
-    } else {
-      const uint64_t t0 = global_timer_ns();
-      for (uint32_t spin = 1;; ++spin) {
-        if (mbar_try_wait(bar, parity)) { state = 1; break; }
-        if ((spin & 3u) == 0) {
-          if (*w.abort) { state = 2; break; }
-          if (global_timer_ns() - t0 > w.limit_ns) { raise_timeout(w); state = 2; break; }
-        }
-      }
-    }
-  }
-  state = __shfl_sync(0xffffffffu, state, 0);
-  if (state != 1) return false;
-  // the phase is complete and cannot advance without this warp, so this succeeds at once
-  bool ok = mbar_try_wait(bar, parity);
-  for (uint32_t i = 0; !ok && i < (1u << 16); ++i) ok = mbar_try_wait(bar, parity);
-  if (__all_sync(0xffffffffu, ok)) return true;
-  if (lane_id() == 0) raise_timeout(w);
-  return false;
-}
-
-#endif
 
 // ---------------------------------------------------------------- TMA / bulk copy
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
@@ -240,6 +232,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Wait for this thread's TMEM loads; the 16 destination registers are passed
+// through the asm so that the compiler cannot read them before the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
+               :
+               : "memory");
+}
 
 // 32 lanes x 32-bit, 16 consecutive columns per thread, every value = `v`.
 __device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t v) {

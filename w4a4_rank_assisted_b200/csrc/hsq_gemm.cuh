@@ -8,8 +8,8 @@
 //
 // Blackwell has no INT4 tensor-core mode, so each 64-wide group is unpacked in
 // shared memory to INT8 and multiplied with two tcgen05.mma.kind::i8 (K = 32
-// each) into a Tensor Memory buffer; drain warps read the int32 partial with
-// tcgen05.ld and fold it into fp32 register accumulators with its two scales.
+// each) into its own Tensor Memory region; drain warps read the int32 partial
+// with tcgen05.ld and fold it into fp32 register accumulators with its scales.
 //
 // Operands are named by their role in the MMA:
 //   "row" operand  -> MMA A, 128 rows per tile, one TMEM lane per row;
@@ -21,34 +21,38 @@
 // Unpack: a packed byte holds two 4-bit two's-complement codes.  Masking a code
 // into the HIGH nibble of a byte gives the int8 value 16*q, so one AND (odd
 // codes) or one shift+AND (even codes) unpacks four codes; the MMA then sums
-// 256*q_x*q_w, and the drain folds 1/256 into the per-row scale (a power-of-two,
+// 256*q_x*q_w, and the drain folds 1/256 into the per-row scale (a power of two,
 // so the fp32 result is unchanged).  The even/odd split permutes K inside a
 // group identically for both operands, which leaves every P_g unchanged.
 //
-// Warp roles (one CTA per SM, persistent over work units):
-//   warp 0      TMA producer: packed row/col tiles + the col scales of one group
+// Pipeline (one CTA per SM, persistent over work units).  One pipeline step
+// ("stage") carries GPS consecutive 64-groups, so that the fixed cost of each
+// hand-off is shared by GPS groups:
+//   warp 0      TMA producer: packed row/col tiles (GPS groups wide) + the row
+//               and col scales of each group, into a STAGES-deep ring
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2-7   unpack packed -> INT8 canonical K-major smem layout
-//   warps 8..   drain / epilogue; warp w reads TMEM lanes 32*(w%4)..+31
-// Pipelines: packed ring (STAGES) -> int8 double buffer -> TMEM double buffer.
+//   warps 2-7   unpack packed -> int8 canonical K-major layout, NI8 buffers
+//   warps 8..   drain / epilogue; warp w reads TMEM lanes 32*(w%4)..+31; NTM
+//               TMEM buffers of GPS x BN columns
 #pragma once
 
 #include "hsq_device.cuh"
 
 namespace hsq {
 
-// Canonical no-swizzle K-major layout of an operand with `rows` rows and one
-// 64-wide group: core matrix (row/8, kc) (kc = 16-byte K chunk 0..3) at
-// (row/8)*SBO + kc*LBO bytes, its 8 rows 16 bytes apart; the second K=32 MMA
-// starts 2*LBO bytes in.  LBO = 160 (not 128) staggers the four K chunks of a
-// row block across shared-memory banks, so that the unpack warps' 16-byte
-// stores of 8 consecutive threads (4 rows x 2 halves) hit 8 distinct bank groups;
-// SBO = 3*LBO + 128.
-#ifndef HSQ_PAD_LAYOUT
-#define HSQ_PAD_LAYOUT 1
-#endif
-constexpr uint32_t kLBO = HSQ_PAD_LAYOUT ? 160 : 128;
+// Canonical no-swizzle K-major layout of one operand and one 64-wide group:
+// core matrix (row/8, kc) (kc = 16-byte K chunk 0..3) at (row/8)*SBO + kc*LBO
+// bytes, its 8 rows 16 bytes apart; the second K=32 MMA starts 2*LBO bytes in.
+// LBO = 160 (not 128) staggers the four K chunks of a row block across shared-
+// memory banks so the unpack's 16-byte stores are conflict free; SBO = 3*LBO+128.
+constexpr uint32_t kLBO = 160;
 constexpr uint32_t kSBO = 3 * kLBO + 128;
+
+// Bytes of one group's int8 operand with `rows` rows, padded so that
+// consecutive groups start 16 bytes apart modulo 128 (another bank stagger).
+__host__ __device__ constexpr int i8_group_stride(int rows) {
+  return (rows / 8) * static_cast<int>(kSBO) + ((16 - ((rows / 8) * static_cast<int>(kSBO)) % 128) + 128) % 128;
+}
 
 struct GemmArgs {
   const float* scales_r;  // row operand scales   [G][ld_r]
@@ -61,25 +65,16 @@ struct GemmArgs {
   void* Y;                // [M][N]
   int out_f32;
   int M, N, G, r;
-  int tiles_r, tiles_c, splits, groups_per_split;
-  float* ws_partials;     // split-K partial tiles
-  unsigned* ws_counters;  // split-K arrival counters (zero between calls)
+  int tiles_r, tiles_c;   // output tiles along the row / col operand
+  int stages_per_tile;    // ceil(G / GPS)
+  int stream_len;         // 0: whole tiles per CTA; else stages per CTA (stream-K)
+  float* ws_partials;     // stream-K partial tiles, [CTA][2][BN][128]
+  unsigned* ws_counters;  // stream-K arrival counters per (tile, drain warp), zero between calls
   uint64_t limit_ns;      // wait limit
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
 };
 
-// DRAIN_ selects how a group's int32 partial becomes fp32 in the drain; all
-// three give bit-identical results:
-//   0: cvt.rn.f32.s32 per value, scalar fmul/fma
-//   1: cvt.rn.f32.s32 per value, packed f32x2 mul/fma
-//   2: the TMEM partial starts each group at the bit pattern of 1.5*2^23, so the
-//      MMA leaves 1.5*2^23 + P (exact, |P| < 2^22) as an fp32 bit pattern; one
-//      packed f32x2 subtract recovers P exactly (no int->float conversion), and
-//      the drain re-fills the buffer with the pattern after reading it.
-#ifndef HSQ_DRAIN_MODE
-#define HSQ_DRAIN_MODE 1
-#endif
-template <int BN_, int DH_, int STAGES_, bool SWAP_, int DRAIN_ = HSQ_DRAIN_MODE>
+template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -87,46 +82,47 @@ struct GemmCfg {
   static constexpr int CW = BN / DH;           // columns per drain thread
   static constexpr int STAGES = STAGES_;
   static constexpr bool SWAP = SWAP_;
-  static constexpr int DRAIN = DRAIN_;
+  static constexpr int GPS = GPS_;             // 64-groups per pipeline stage
+  static constexpr int NI8 = NI8_;             // int8 operand buffers
+  static constexpr int NTM = NTM_;             // TMEM partial buffers
   static constexpr int NUM_UNPACK_WARPS = 6;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
   // Register split (setmaxnreg): producer/MMA/unpack warpgroups give registers
   // to the drain warpgroups, which hold CW fp32 accumulators per thread.
-  static constexpr bool REALLOC = CW >= 64;
-#ifndef HSQ_REGS_LOW
-#define HSQ_REGS_LOW 64
-#endif
-  static constexpr int REGS_LOW = HSQ_REGS_LOW;
-  static constexpr int REGS_HIGH_RAW = ((65536 - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
-  static constexpr int REGS_HIGH = REGS_HIGH_RAW > 232 ? 232 : REGS_HIGH_RAW;
-  static constexpr int A_PACK = BM * 32;       // packed bytes per group
-  static constexpr int B_PACK = BN * 32;
-  static constexpr int CS_BYTES = BN * 4;
-  static constexpr int STAGE_BYTES = ((A_PACK + B_PACK + CS_BYTES + 1023) / 1024) * 1024;
-  static constexpr int A_I8 = (BM / 8) * kSBO;  // int8 operand bytes per group
-  static constexpr int B_I8 = (BN / 8) * kSBO;
-  static constexpr int I8_BYTES = ((A_I8 + B_I8 + 1023) / 1024) * 1024;
-  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                 : (2 * BN <= 256) ? 256 : 512;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 + 2 + 1;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 2 * I8_BYTES + NUM_BARS * 8 + 64;
+  static constexpr bool REALLOC = CW >= 128;
+  static constexpr int REGS_LOW = 64;
+  static constexpr int REGS_HIGH = ((65536 - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8 > 232
+                                       ? 232
+                                       : ((65536 - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
+  static constexpr int A_PACK = BM * 32 * GPS;  // packed bytes per stage (row operand)
+  static constexpr int B_PACK = BN * 32 * GPS;  // packed bytes per stage (col operand)
+  static constexpr int CS_BYTES = BN * 4;       // col scales of one group
+  static constexpr int RS_BYTES = BM * 4;       // row scales of one group
+  static constexpr int CS_OFF = A_PACK + B_PACK;                 // stage layout: packed row tile,
+  static constexpr int RS_OFF = CS_OFF + GPS * CS_BYTES;         // packed col tile, col scales,
+  static constexpr int STAGE_BYTES = ((RS_OFF + GPS * RS_BYTES + 1023) / 1024) * 1024;  // row scales
+  static constexpr int SA = i8_group_stride(BM);  // int8 bytes of one group, row operand
+  static constexpr int SB = i8_group_stride(BN);  // int8 bytes of one group, col operand
+  static constexpr int I8_BYTES = ((GPS * (SA + SB) + 1023) / 1024) * 1024;
+  static constexpr int TMEM_NEED = NTM * GPS * BN;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                 : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NI8 + 2 * NTM + 1;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8 * I8_BYTES + NUM_BARS * 8 + 64;
+  // unpack tasks (16 packed bytes each) per stage, and per unpack thread
+  static constexpr int TASKS = 2 * GPS * (BM + BN);
+  static constexpr int TPT = (TASKS + 32 * NUM_UNPACK_WARPS - 1) / (32 * NUM_UNPACK_WARPS);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-  static_assert(CW % 16 == 0, "drain chunks of 16 columns");
-  static_assert(2 * BN <= 512, "TMEM");
+  static_assert(CW % 16 == 0, "drain chunks");
+  static_assert(TMEM_NEED <= 512, "TMEM");
+  static_assert(32 * GPS <= 256, "TMA box width");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-
-constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
-constexpr float kMagic = 12582912.0f;
-
-// One unpack task: 16 packed bytes (32 codes) of one row -> two 16-byte core
-// matrix rows (even codes, odd codes).  Task t reads row t/2, half t%2, so 8
-// consecutive threads read 128 contiguous bytes.
-__device__ __forceinline__ void unpack_task(const uint8_t* src_stage, uint8_t* dst, int t) {
-  const int row = t >> 1;
-  const int half = t & 1;  // which 16 packed bytes (K 0-31 or 32-63)
-  const uint4 p = *reinterpret_cast<const uint4*>(src_stage + t * 16);
+// Unpack 16 packed bytes (32 codes) into two 16-byte int8 core-matrix rows
+// (even codes, odd codes).
+__device__ __forceinline__ void unpack16(const uint4& p, uint8_t* dst) {
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint4 lo, hi;
   uint32_t* lo_w = reinterpret_cast<uint32_t*>(&lo);
@@ -136,28 +132,71 @@ __device__ __forceinline__ void unpack_task(const uint8_t* src_stage, uint8_t* d
     lo_w[i] = (w[i] << 4) & 0xF0F0F0F0u;  // even codes, 16*q as int8
     hi_w[i] = w[i] & 0xF0F0F0F0u;         // odd codes,  16*q as int8
   }
-  uint8_t* base = dst + (row >> 3) * kSBO + (2 * half) * kLBO + (row & 7) * 16;
-  *reinterpret_cast<uint4*>(base) = lo;
-  *reinterpret_cast<uint4*>(base + kLBO) = hi;
+  *reinterpret_cast<uint4*>(dst) = lo;
+  *reinterpret_cast<uint4*>(dst + kLBO) = hi;
+}
+
+// One unit of a CTA's work: groups [g0, g1) of one output tile.
+struct Unit {
+  int tile, g0, g1;
+  int nslots;  // CTAs contributing to this tile (1: this CTA owns it whole)
+  int slot;    // 0 if this is the CTA's first unit, 1 if its last (stream-K partials)
+  int first;   // first contributing CTA
+};
+
+// Work decomposition.  Whole-tile mode: CTA b takes tiles b, b + grid, ...
+// Stream-K mode: the tiles' pipeline stages, laid end to end, are cut into
+// equal ranges of stream_len stages, one per CTA, so every CTA streams the same
+// amount of operand data; a range splits at tile boundaries into units, and a
+// tile cut between CTAs is finished by whichever of them arrives last.
+// All stage arithmetic is 32-bit: the host uses stream-K only when the total
+// stage count is below 2^30 (64-bit division would expand into a long call-like
+// sequence inside warps running with a reduced register budget).
+template <int GPS>
+__device__ __forceinline__ bool next_unit(const GemmArgs& a, int k, Unit& u) {
+  const int tiles = a.tiles_r * a.tiles_c;
+  if (a.stream_len == 0) {
+    const int t = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+    if (t >= tiles) return false;
+    u.tile = t; u.g0 = 0; u.g1 = a.G; u.nslots = 1; u.slot = 0; u.first = static_cast<int>(blockIdx.x);
+    return true;
+  }
+  const unsigned S = static_cast<unsigned>(a.stages_per_tile), L = static_cast<unsigned>(a.stream_len);
+  const unsigned begin = blockIdx.x * L;
+  const unsigned end = min(begin + L, static_cast<unsigned>(tiles) * S);
+  unsigned pos = begin;
+  for (int i = 0; i < k && pos < end; ++i) pos = (pos / S + 1) * S;
+  if (pos >= end) return false;
+  const unsigned t = pos / S;
+  const unsigned uend = min(end, (t + 1) * S);
+  u.tile = static_cast<int>(t);
+  u.g0 = static_cast<int>((pos - t * S) * GPS);
+  u.g1 = min(a.G, static_cast<int>((uend - t * S) * GPS));
+  u.first = static_cast<int>((t * S) / L);
+  const int last = static_cast<int>(((t + 1) * S - 1) / L);
+  u.nslots = last - u.first + 1;
+  u.slot = (begin >= t * S) ? 0 : 1;
+  return true;
 }
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_row, const __grid_constant__ CUtensorMap tm_col,
                      const GemmArgs args) {
-  constexpr int BM = Cfg::BM, BN = Cfg::BN, CW = Cfg::CW, STAGES = Cfg::STAGES;
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, CW = Cfg::CW, STAGES = Cfg::STAGES, GPS = Cfg::GPS;
+  constexpr int NI8 = Cfg::NI8, NTM = Cfg::NTM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* i8_base = smem + STAGES * Cfg::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(i8_base + 2 * Cfg::I8_BYTES);
-  uint64_t* full = bars;                 // [STAGES] packed stage landed
-  uint64_t* empty = bars + STAGES;       // [STAGES] packed stage free
-  uint64_t* full8 = bars + 2 * STAGES;   // [2] int8 operands ready
-  uint64_t* empty8 = full8 + 2;          // [2] int8 operands consumed by the MMA
-  uint64_t* tfull = empty8 + 2;          // [2] TMEM partial ready
-  uint64_t* tempty = tfull + 2;          // [2] TMEM partial drained
-  uint64_t* final_bar = tempty + 2;      // teardown: all MMAs done
+  uint64_t* bars = reinterpret_cast<uint64_t*>(i8_base + NI8 * Cfg::I8_BYTES);
+  uint64_t* full = bars;                   // [STAGES] packed stage landed
+  uint64_t* empty = bars + STAGES;         // [STAGES] packed stage free
+  uint64_t* full8 = bars + 2 * STAGES;     // [NI8] int8 operands ready
+  uint64_t* empty8 = full8 + NI8;          // [NI8] int8 operands consumed by the MMA
+  uint64_t* tfull = empty8 + NI8;          // [NTM] TMEM partials ready
+  uint64_t* tempty = tfull + NTM;          // [NTM] TMEM partials drained
+  uint64_t* final_bar = tempty + NTM;      // teardown: all MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* tail_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -171,9 +210,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], Cfg::NUM_UNPACK_WARPS + Cfg::NUM_DRAIN_WARPS);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NI8; ++b) {
       mbar_init(&full8[b], Cfg::NUM_UNPACK_WARPS);
       mbar_init(&empty8[b], 1);
+    }
+    for (int b = 0; b < NTM; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], Cfg::NUM_DRAIN_WARPS);
     }
@@ -195,8 +236,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int units = args.tiles_r * args.tiles_c * args.splits;
-  uint32_t issued = 0;  // producer: loads issued (for the teardown drain)
+  uint32_t issued = 0;  // producer: stages issued (for the teardown drain)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -204,23 +244,28 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     if (lane == 0 && !(args.debug_flags & 1)) {
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-        const int split = u % args.splits;
-        const int tile = u / args.splits;
-        const int tr = tile % args.tiles_r, tc = tile / args.tiles_r;
-        const int g0 = split * args.groups_per_split;
-        const int g1 = min(args.G, g0 + args.groups_per_split);
+      Unit un;
+      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+        const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
+        const int g0 = un.g0, g1 = un.g1;
         const int c0 = tc * BN;
+        const int r0 = tr * BM;
         const uint32_t cs_bytes = static_cast<uint32_t>(min(BN, args.ld_c - c0)) * 4u;
-        for (int g = g0; g < g1; ++g, ++it) {
+        const uint32_t rs_bytes = static_cast<uint32_t>(min(BM, args.ld_r - r0)) * 4u;
+        for (int g = g0; g < g1; g += GPS, ++it) {
+          const int ng = min(GPS, g1 - g);
           const int s = it % STAGES;
           if (!wait_one(&empty[s], ((it / STAGES) & 1) ^ 1, wp)) { ok = false; break; }
           uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK + cs_bytes);
-          tma_load_2d(st, &tm_row, &full[s], g * 32, tr * BM);
+          mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK + ng * (cs_bytes + rs_bytes));
+          tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
           tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * 32, c0);
-          bulk_load(st + Cfg::A_PACK + Cfg::B_PACK, args.scales_c + static_cast<size_t>(g) * args.ld_c + c0,
-                    cs_bytes, &full[s]);
+          for (int j = 0; j < ng; ++j) {
+            bulk_load(st + Cfg::CS_OFF + j * Cfg::CS_BYTES,
+                      args.scales_c + static_cast<size_t>(g + j) * args.ld_c + c0, cs_bytes, &full[s]);
+            bulk_load(st + Cfg::RS_OFF + j * Cfg::RS_BYTES,
+                      args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, &full[s]);
+          }
           issued = it + 1;
         }
       }
@@ -232,49 +277,77 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       constexpr uint32_t idesc = idesc_i8(BM, BN);
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-        const int split = u % args.splits;
-        const int g0 = split * args.groups_per_split;
-        const int g1 = min(args.G, g0 + args.groups_per_split);
-        for (int g = g0; g < g1; ++g, ++it) {
-          const int b = it & 1;
-          const uint32_t ph = (it >> 1) & 1;
-          if (!wait_one(&full8[b], ph, wp)) { ok = false; break; }
-          // DRAIN 2: the drain pre-fills both buffers once and so completes phase 0 itself
-          if (!wait_one(&tempty[b], Cfg::DRAIN == 2 ? ph : ph ^ 1, wp)) { ok = false; break; }
+      Unit un;
+      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+        const int g0 = un.g0, g1 = un.g1;
+        for (int g = g0; g < g1; g += GPS, ++it) {
+          const int ng = min(GPS, g1 - g);
+          const int b = it % NI8;
+          const int tb = it % NTM;
+          if (!wait_one(&full8[b], (it / NI8) & 1, wp)) { ok = false; break; }
+          if (!wait_one(&tempty[tb], ((it / NTM) & 1) ^ 1, wp)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(i8_base + b * Cfg::I8_BYTES);
-          const uint32_t b_addr = a_addr + Cfg::A_I8;
-          const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
-          mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc,
-                 Cfg::DRAIN == 2 ? 1u : 0u);
-          mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO), smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO),
-                 idesc, 1u);
+          const uint32_t buf = smem_u32(i8_base + b * Cfg::I8_BYTES);
+          for (int j = 0; j < ng; ++j) {
+            const uint32_t a_addr = buf + j * Cfg::SA;
+            const uint32_t b_addr = buf + GPS * Cfg::SA + j * Cfg::SB;
+            const uint32_t d = tmem_base + static_cast<uint32_t>((tb * GPS + j) * BN);
+            mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
+            mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
+                   smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+          }
           mma_commit(&empty8[b]);
-          mma_commit(&tfull[b]);
+          mma_commit(&tfull[tb]);
         }
       }
     }
   } else if (warp < 2 + Cfg::NUM_UNPACK_WARPS) {
     // ------------------------------------------------------------ unpack
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
-    const int ut = (warp - 2) * 32 + lane;
     constexpr int NT = 32 * Cfg::NUM_UNPACK_WARPS;
+    // This thread's tasks are the same at every stage: precompute their offsets.
+    // Task t -> operand (row tasks first), row, 16-byte chunk c of the row's
+    // 32*GPS packed bytes (c fastest, so 8 consecutive threads read 128
+    // contiguous bytes); group j = c/2, half = c%2.
+    uint32_t src_off[Cfg::TPT], dst_off[Cfg::TPT];
+    int grp[Cfg::TPT];
+    const int ut = (warp - 2) * 32 + lane;
+#pragma unroll
+    for (int i = 0; i < Cfg::TPT; ++i) {
+      int t = ut + i * NT;
+      grp[i] = GPS;  // GPS = no task
+      src_off[i] = dst_off[i] = 0;
+      if (t < Cfg::TASKS) {
+        const bool colop = t >= 2 * GPS * BM;
+        if (colop) t -= 2 * GPS * BM;
+        const int row = t / (2 * GPS), c = t % (2 * GPS);
+        const int j = c >> 1, half = c & 1;
+        grp[i] = j;
+        src_off[i] = (colop ? Cfg::A_PACK : 0) + row * 32 * GPS + c * 16;
+        dst_off[i] = (colop ? GPS * Cfg::SA + j * Cfg::SB : j * Cfg::SA) + (row >> 3) * kSBO + 2 * half * kLBO +
+                     (row & 7) * 16;
+      }
+    }
     uint32_t it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-      const int split = u % args.splits;
-      const int g0 = split * args.groups_per_split;
-      const int g1 = min(args.G, g0 + args.groups_per_split);
-      for (int g = g0; g < g1; ++g, ++it) {
+    Unit un;
+    for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      const int g0 = un.g0, g1 = un.g1;
+      for (int g = g0; g < g1; g += GPS, ++it) {
+        const int ng = min(GPS, g1 - g);
         const int s = it % STAGES;
-        const int b = it & 1;
+        const int b = it % NI8;
         if (!wait_warp(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
-        if (!wait_warp(&empty8[b], ((it >> 1) & 1) ^ 1, wp)) { ok = false; break; }
+        if (!wait_warp(&empty8[b], ((it / NI8) & 1) ^ 1, wp)) { ok = false; break; }
         const uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
         uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
-        for (int t = ut; t < 2 * BM; t += NT) unpack_task(st, dst, t);
-        for (int t = ut; t < 2 * BN; t += NT) unpack_task(st + Cfg::A_PACK, dst + Cfg::A_I8, t);
+        uint4 pk[Cfg::TPT];
+#pragma unroll
+        for (int i = 0; i < Cfg::TPT; ++i)  // all loads first (always inside the stage)
+          pk[i] = *reinterpret_cast<const uint4*>(st + src_off[i]);
+#pragma unroll
+        for (int i = 0; i < Cfg::TPT; ++i)
+          if (grp[i] < ng) unpack16(pk[i], dst + dst_off[i]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -293,80 +366,70 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
-    if (Cfg::DRAIN == 2) {
-      // pre-fill this warp's lanes/columns of both TMEM buffers with the pattern
-#pragma unroll
-      for (int b = 0; b < 2; ++b)
-#pragma unroll
-        for (int c = 0; c < CW / 16; ++c) tmem_st16_fill(t_lane + static_cast<uint32_t>(b * BN + h * CW + c * 16), kMagicBits);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tempty[0]);
-        mbar_arrive(&tempty[1]);
-      }
-    }
-    for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-      const int split = u % args.splits;
-      const int tile = u / args.splits;
+    Unit un;
+    for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      const int tile = un.tile;
       const int tr = tile % args.tiles_r, tc = tile / args.tiles_r;
-      const int g0 = split * args.groups_per_split;
-      const int g1 = min(args.G, g0 + args.groups_per_split);
+      const int g0 = un.g0, g1 = un.g1;
       const int row = tr * BM + row_local;
       const bool row_ok = row < args.rows_r;
-      float acc[CW];
+      // fp32 accumulators as pairs, for the packed f32x2 multiply-add
+      float2 acc2[CW / 2];
 #pragma unroll
-      for (int j = 0; j < CW; ++j) acc[j] = 0.f;
-      float s_next = row_ok ? __ldg(args.scales_r + static_cast<size_t>(g0) * args.ld_r + row) : 0.f;
-      for (int g = g0; g < g1; ++g, ++it) {
+      for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.f, 0.f);
+#define ACC(j) (((j) & 1) ? acc2[(j) >> 1].y : acc2[(j) >> 1].x)
+      for (int g = g0; g < g1; g += GPS, ++it) {
+        const int ng = min(GPS, g1 - g);
         const int s = it % STAGES;
-        const int b = it & 1;
-        const float s_row = s_next * (1.0f / 256.0f);
-        if (g + 1 < g1 && row_ok) s_next = __ldg(args.scales_r + static_cast<size_t>(g + 1) * args.ld_r + row);
-        if (!wait_warp(&tfull[b], (it >> 1) & 1, wp)) { ok = false; break; }
+        const int tb = it % NTM;
+        if (!wait_warp(&tfull[tb], (it / NTM) & 1, wp)) { ok = false; break; }
         if (!wait_warp(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
         tc_fence_after();
-        const float* cs = reinterpret_cast<const float*>(stage_base + s * Cfg::STAGE_BYTES + Cfg::A_PACK +
-                                                         Cfg::B_PACK) + h * CW;
+        const float* cs_stage = reinterpret_cast<const float*>(stage_base + s * Cfg::STAGE_BYTES + Cfg::CS_OFF);
+        const float* rs_stage = reinterpret_cast<const float*>(stage_base + s * Cfg::STAGE_BYTES + Cfg::RS_OFF);
+        // Software pipeline over the stage's 16-column chunks: the TMEM load of
+        // chunk c+1 is in flight while chunk c is folded into the accumulators.
+        constexpr int NCH = CW / 16;  // chunks per group
+        uint32_t va[16], vb[16];
+        tmem_ld16(t_lane + static_cast<uint32_t>(tb * GPS * BN + h * CW), va);
+        tmem_ld_wait(va);
 #pragma unroll
-        for (int c = 0; c < CW / 16; ++c) {
-          uint32_t v[16];
-          const uint32_t taddr = t_lane + static_cast<uint32_t>(b * BN + h * CW + c * 16);
-          tmem_ld16(taddr, v);
-          tmem_ld_wait();
-          if (Cfg::DRAIN == 2) tmem_st16_fill(taddr, kMagicBits);
+        for (int j = 0; j < GPS; ++j) {
+          if (j >= ng) break;  // warp-uniform
+          const float* cs = cs_stage + j * BN + h * CW;
+          // this row's scale of group g+j; 1/256 undoes the 16*q encoding of both operands
+          const float rs = rs_stage[j * BM + row_local] * (1.0f / 256.0f);
+          const float2 rs2 = make_float2(rs, rs);
 #pragma unroll
-          for (int j4 = 0; j4 < 4; ++j4) {
-            const float4 sc = *reinterpret_cast<const float4*>(cs + c * 16 + j4 * 4);
-            const float scv[4] = {sc.x, sc.y, sc.z, sc.w};
+          for (int c = 0; c < NCH; ++c) {
+            const int k = j * NCH + c;  // running chunk index within the stage
+            uint32_t(&cur)[16] = (k & 1) ? vb : va;
+            uint32_t(&nxt)[16] = (k & 1) ? va : vb;
+            const bool more = (c + 1 < NCH) || (j + 1 < ng);
+            if (more) {
+              const int jn = (c + 1 < NCH) ? j : j + 1;
+              const int cn = (c + 1 < NCH) ? c + 1 : 0;
+              tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + jn) * BN + h * CW + cn * 16), nxt);
+            }
 #pragma unroll
-            for (int e = 0; e < 4; e += 2) {
-              const int j = j4 * 4 + e;
-              float& a0 = acc[c * 16 + j];
-              float& a1 = acc[c * 16 + j + 1];
-              if (Cfg::DRAIN == 0) {
-                a0 = fmaf(s_row, scv[e] * __int2float_rn(static_cast<int>(v[j])), a0);
-                a1 = fmaf(s_row, scv[e + 1] * __int2float_rn(static_cast<int>(v[j + 1])), a1);
-              } else {
-                float p0, p1, t0, t1;
-                if (Cfg::DRAIN == 1) {
-                  p0 = __int2float_rn(static_cast<int>(v[j]));
-                  p1 = __int2float_rn(static_cast<int>(v[j + 1]));
-                } else {
-                  fadd2(p0, p1, __uint_as_float(v[j]), __uint_as_float(v[j + 1]), -kMagic, -kMagic);
-                }
-                fmul2(t0, t1, p0, p1, scv[e], scv[e + 1]);
-                ffma2(a0, a1, s_row, s_row, t0, t1, a0, a1);
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 sc = *reinterpret_cast<const float4*>(cs + c * 16 + j4 * 4);
+#pragma unroll
+              for (int e = 0; e < 4; e += 2) {
+                const int jj = c * 16 + j4 * 4 + e;
+                const float2 p = make_float2(__int2float_rn(static_cast<int>(cur[j4 * 4 + e])),
+                                             __int2float_rn(static_cast<int>(cur[j4 * 4 + e + 1])));
+                const float2 t = __fmul2_rn(p, e == 0 ? make_float2(sc.x, sc.y) : make_float2(sc.z, sc.w));
+                acc2[jj >> 1] = __ffma2_rn(rs2, t, acc2[jj >> 1]);
               }
             }
+            if (more) tmem_ld_wait(nxt);
           }
         }
-        if (Cfg::DRAIN == 2) tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&tempty[b]);
+          mbar_arrive(&tempty[tb]);
           mbar_arrive(&empty[s]);
         }
       }
@@ -374,29 +437,34 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
       // ---------------------------------------------------------- epilogue
       const int col0 = tc * BN + h * CW;
-      if (args.splits > 1) {
-        // Split-K: every drain warp owns a 32-row x CW-column sub-tile.  It
-        // writes its fp32 partial, and the warp that arrives last for that
-        // sub-tile sums all splits in split order (deterministic), runs the
-        // epilogue and re-zeroes the counter.  No cross-warp barrier is used.
-        const size_t tile_base = static_cast<size_t>(tile) * args.splits;
-        float* part = args.ws_partials + ((tile_base + split) * BN + h * CW) * BM + row_local;
+      if (un.nslots > 1) {
+        // Stream-K: every drain warp owns a 32-row x CW-column sub-tile.  It
+        // writes its fp32 partial to this CTA's slot, and the warp that arrives
+        // last for that sub-tile sums the contributing CTAs' partials in CTA
+        // order (deterministic), runs the epilogue and re-zeroes the counter.
+        // No cross-warp or cross-CTA waiting.
+        float* part = args.ws_partials +
+                      ((static_cast<size_t>(blockIdx.x) * 2 + un.slot) * BN + h * CW) * BM + row_local;
 #pragma unroll
-        for (int j = 0; j < CW; ++j) part[static_cast<size_t>(j) * BM] = acc[j];
+        for (int j = 0; j < CW; ++j) part[static_cast<size_t>(j) * BM] = ACC(j);
         __threadfence();
         __syncwarp();
         unsigned* counter = args.ws_counters + static_cast<size_t>(tile) * Cfg::NUM_DRAIN_WARPS + dw;
         int last = 0;
-        if (lane == 0) last = (atomicAdd(counter, 1u) == static_cast<unsigned>(args.splits - 1)) ? 1 : 0;
+        if (lane == 0) last = (atomicAdd(counter, 1u) == static_cast<unsigned>(un.nslots - 1)) ? 1 : 0;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) continue;
         __threadfence();
 #pragma unroll
-        for (int j = 0; j < CW; ++j) acc[j] = 0.f;
-        for (int sp = 0; sp < args.splits; ++sp) {
-          const float* p = args.ws_partials + ((tile_base + sp) * BN + h * CW) * BM + row_local;
+        for (int j = 0; j < CW; ++j) ACC(j) = 0.f;
+        const unsigned S = static_cast<unsigned>(args.stages_per_tile);
+        const unsigned L = static_cast<unsigned>(args.stream_len);
+#pragma unroll 2
+        for (int c = un.first; c < un.first + un.nslots; ++c) {
+          const int cslot = (static_cast<unsigned>(c) * L >= static_cast<unsigned>(tile) * S) ? 0 : 1;
+          const float* p = args.ws_partials + ((static_cast<size_t>(c) * 2 + cslot) * BN + h * CW) * BM + row_local;
 #pragma unroll
-          for (int j = 0; j < CW; ++j) acc[j] += __ldcg(p + static_cast<size_t>(j) * BM);
+          for (int j = 0; j < CW; ++j) ACC(j) += __ldcg(p + static_cast<size_t>(j) * BM);
         }
         if (lane == 0) *counter = 0u;
       }
@@ -414,7 +482,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               float l[8];
               bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + n)), l);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) acc[j8 * 8 + e] = fmaf(um, l[e], acc[j8 * 8 + e]);
+              for (int e = 0; e < 8; ++e) ACC(j8 * 8 + e) = fmaf(um, l[e], ACC(j8 * 8 + e));
             }
           }
         }
@@ -424,7 +492,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (n < args.N) {
             float y[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = acc[j8 * 8 + e];
+            for (int e = 0; e < 8; ++e) y[e] = ACC(j8 * 8 + e);
             if (args.bias) {
               float bb[8];
               bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), bb);
@@ -454,14 +522,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
           for (int j = 0; j < CW; ++j) {
             const int m = col0 + j;
-            if (m < args.M) acc[j] = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + i), l2, acc[j]);
+            if (m < args.M) ACC(j) = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + i), l2, ACC(j));
           }
         }
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
           const int m = col0 + j;
           if (m < args.M) {
-            const float y = acc[j] + bn;
+            const float y = ACC(j) + bn;
             const size_t off = static_cast<size_t>(m) * args.N + n;
             if (args.out_f32) static_cast<float*>(args.Y)[off] = y;
             else static_cast<__nv_bfloat16*>(args.Y)[off] = __float2bfloat16_rn(y);
@@ -471,6 +539,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   }
 
+#undef ACC
   // ------------------------------------------------------------ teardown
   __syncthreads();
   if (*abort_flag) {

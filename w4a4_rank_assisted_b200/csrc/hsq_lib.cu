@@ -23,10 +23,18 @@ constexpr int kMaxDim = 1 << 20;
 constexpr int kMaxRank = 32;
 
 // Kernel configurations (see hsq_gemm.cuh).
-using CfgLarge = hsq::GemmCfg<256, 2, 8, false>;  // M > 64: 128 tokens x 256 outputs per tile
-using CfgDec16 = hsq::GemmCfg<16, 1, 16, true>;   // M <= 16: 128 outputs x 16 tokens
-using CfgDec32 = hsq::GemmCfg<32, 1, 12, true>;   // M <= 32
-using CfgDec64 = hsq::GemmCfg<64, 1, 10, true>;   // M <= 64
+//                           BN  DH STAGES SWAP  GPS NI8 NTM
+#ifndef HSQ_LARGE_BN
+#define HSQ_LARGE_BN 256
+#endif
+#if HSQ_LARGE_BN == 128
+using CfgLarge = hsq::GemmCfg<128, 2, 8, false, 1, 3, 4>;  // M > 64: 128 tokens x 128 outputs per tile
+#else
+using CfgLarge = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2>;  // M > 64: 128 tokens x 256 outputs per tile
+#endif
+using CfgDec16 = hsq::GemmCfg<16, 1, 5, true, 4, 2, 4>;    // M <= 16: 128 outputs x 16 tokens
+using CfgDec32 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2>;    // M <= 32
+using CfgDec64 = hsq::GemmCfg<64, 1, 6, true, 2, 2, 2>;    // M <= 64
 
 thread_local int t_debug_flags = 0;
 thread_local int t_debug_limit_ms = 0;
@@ -65,9 +73,10 @@ struct Plan {
   int BN;
   bool swap;
   int drain_warps;
-  int tiles_r, tiles_c, splits, gps, units, grid;
+  int gps_stage;  // 64-groups per pipeline stage of the chosen kernel
+  int tiles_r, tiles_c, stages_per_tile, stream_len, grid;
   size_t counters_bytes, partial_bytes;
-  size_t ws_bytes() const { return splits > 1 ? counters_bytes + partial_bytes : 0; }
+  size_t ws_bytes() const { return stream_len > 0 ? counters_bytes + partial_bytes : 0; }
 };
 
 Plan make_plan(int M, int N, int K, int nsm) {
@@ -76,41 +85,36 @@ Plan make_plan(int M, int N, int K, int nsm) {
   if (M <= 64) {
     p.swap = true;
     p.kind = M <= 16 ? kDec16 : M <= 32 ? kDec32 : kDec64;
-    p.BN = M <= 16 ? 16 : M <= 32 ? 32 : 64;
-    p.drain_warps = 4;
+    p.BN = M <= 16 ? CfgDec16::BN : M <= 32 ? CfgDec32::BN : CfgDec64::BN;
+    p.gps_stage = M <= 16 ? CfgDec16::GPS : M <= 32 ? CfgDec32::GPS : CfgDec64::GPS;
+    p.drain_warps = CfgDec16::NUM_DRAIN_WARPS;
     p.tiles_r = (N + 127) / 128;
     p.tiles_c = (M + p.BN - 1) / p.BN;
   } else {
     p.swap = false;
     p.kind = kLarge;
-    p.BN = 256;
-    p.drain_warps = 8;
+    p.BN = CfgLarge::BN;
+    p.gps_stage = CfgLarge::GPS;
+    p.drain_warps = CfgLarge::NUM_DRAIN_WARPS;
     p.tiles_r = (M + 127) / 128;
-    p.tiles_c = (N + 255) / 256;
+    p.tiles_c = (N + CfgLarge::BN - 1) / CfgLarge::BN;
   }
-  const int tiles = p.tiles_r * p.tiles_c;
-  // choose the split count that minimises the critical path (work units of the
-  // busiest CTA times groups per unit), preferring fewer splits on ties
-  int best_s = 1;
-  double best_cost = 1e30;
-  const int max_s = tiles >= nsm ? 1 : std::min(16, std::max(1, G / 4));
-  for (int s = 1; s <= max_s; ++s) {
-    const int gps = (G + s - 1) / s;
-    const int s_eff = (G + gps - 1) / gps;
-    const long units = static_cast<long>(tiles) * s_eff;
-    const double waves = static_cast<double>((units + nsm - 1) / nsm);
-    const double cost = waves * gps + (s_eff > 1 ? 2.0 : 0.0);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best_s = s_eff;
-    }
+  const long tiles = static_cast<long>(p.tiles_r) * p.tiles_c;
+  p.stages_per_tile = (G + p.gps_stage - 1) / p.gps_stage;
+  // Whole tiles per CTA when they fill the device in nearly full waves;
+  // otherwise stream-K: equal runs of stages per CTA across tile boundaries.
+  const long waves = (tiles + nsm - 1) / nsm;
+  const double fill = static_cast<double>(tiles) / static_cast<double>(waves * nsm);
+  const long total = tiles * p.stages_per_tile;
+  if ((tiles >= nsm && fill >= 0.9) || total <= nsm || total >= (1l << 30)) {
+    p.stream_len = 0;
+    p.grid = static_cast<int>(std::min<long>(tiles, nsm));
+  } else {
+    p.stream_len = static_cast<int>((total + nsm - 1) / nsm);
+    p.grid = static_cast<int>((total + p.stream_len - 1) / p.stream_len);
   }
-  p.gps = (G + best_s - 1) / best_s;
-  p.splits = (G + p.gps - 1) / p.gps;
-  p.units = tiles * p.splits;
-  p.grid = std::min(p.units, nsm);
   p.counters_bytes = ((static_cast<size_t>(tiles) * p.drain_warps * 4 + 255) / 256) * 256;
-  p.partial_bytes = static_cast<size_t>(tiles) * p.splits * p.BN * 128 * 4;
+  p.partial_bytes = static_cast<size_t>(p.grid) * 2 * p.BN * 128 * 4;
   return p;
 }
 
@@ -131,13 +135,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over packed codes [rows][Kp/2] bytes, box = one 64-group (32 bytes) x box_rows.
-bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, int box_rows) {
+// 2-D map over packed codes [rows][Kp/2] bytes, box = `groups` 64-groups (32 bytes each) x box_rows.
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, int box_rows, int groups) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Kp / 2), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Kp / 2)};
-  const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(32 * groups), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -314,11 +318,13 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   if (!p.swap) {
     a.scales_r = x_scales; a.ld_r = ldx; a.rows_r = M;
     a.scales_c = w_scales; a.ld_c = ldw; a.rows_c = N;
-    ok = make_codes_map(&tm_row, x_codes, M, Kp, 128) && make_codes_map(&tm_col, w_codes, N, Kp, p.BN);
+    ok = make_codes_map(&tm_row, x_codes, M, Kp, 128, p.gps_stage) &&
+         make_codes_map(&tm_col, w_codes, N, Kp, p.BN, p.gps_stage);
   } else {
     a.scales_r = w_scales; a.ld_r = ldw; a.rows_r = N;
     a.scales_c = x_scales; a.ld_c = ldx; a.rows_c = M;
-    ok = make_codes_map(&tm_row, w_codes, N, Kp, 128) && make_codes_map(&tm_col, x_codes, M, Kp, p.BN);
+    ok = make_codes_map(&tm_row, w_codes, N, Kp, 128, p.gps_stage) &&
+         make_codes_map(&tm_col, x_codes, M, Kp, p.BN, p.gps_stage);
   }
   if (!ok) return HSQ_ERR_CUDA;
   a.U = U;
@@ -327,8 +333,9 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   a.Y = Y;
   a.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
   a.M = M; a.N = N; a.G = G; a.r = r;
-  a.tiles_r = p.tiles_r; a.tiles_c = p.tiles_c; a.splits = p.splits; a.groups_per_split = p.gps;
-  if (p.splits > 1) {
+  a.tiles_r = p.tiles_r; a.tiles_c = p.tiles_c;
+  a.stages_per_tile = p.stages_per_tile; a.stream_len = p.stream_len;
+  if (p.stream_len > 0) {
     a.ws_counters = static_cast<unsigned*>(workspace);
     a.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.counters_bytes);
   }

@@ -36,6 +36,57 @@ __device__ __forceinline__ uint32_t quantize8(const float (&v)[8], float& scale)
   return packed;
 }
 
+// x / y rounded to nearest-even, given z = RN(1/y): one product and Markstein's
+// fused-multiply-add correction, q1 = RN(q + z (x - q y)) with the remainder
+// x - q y exact (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990).  The result
+// equals the IEEE quotient for normal x, y and a normal, finite quotient; very
+// small or very large inputs take the ordinary division.  The tests compare every code and scale it
+// decides against the oracle's IEEE division.
+__device__ __forceinline__ float div_by_recip(float x, float y, float z) {
+  const float ax = fabsf(x);
+  if (ax < 0x1p-100f || ax > 0x1p100f) return __fdiv_rn(x, y);
+  const float q = __fmul_rn(x, z);
+  const float r = __fmaf_rn(-q, y, x);
+  return __fmaf_rn(r, z, q);
+}
+
+// Round-half-even of |t| < 2^22 to an integer: add 1.5*2^23 (the sum's last
+// mantissa bit is then the units place) and read the integer from the bits.
+__device__ __forceinline__ int rint_small(float t) {
+  return __float_as_int(__fadd_rn(t, 12582912.0f)) - 0x4B400000;
+}
+
+// Same result as quantize8, with the per-element divisions by the group scale
+// done as div_by_recip (one reciprocal per group).
+__device__ __forceinline__ uint32_t quantize8_fast(const float (&v)[8], float& scale) {
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  scale = __fdiv_rn(amax, 7.0f);
+  uint32_t packed = 0;
+  if (scale >= 0x1p-100f && scale <= 0x1p100f) {
+    const float z = __frcp_rn(scale);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int q = rint_small(div_by_recip(v[e], scale, z));
+      q = max(-7, min(7, q));
+      packed |= static_cast<uint32_t>(q & 0xF) << (4 * e);
+    }
+  } else if (scale != 0.f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int q = __float2int_rn(__fdiv_rn(v[e], scale));
+      q = max(-7, min(7, q));
+      packed |= static_cast<uint32_t>(q & 0xF) << (4 * e);
+    }
+  }
+  return packed;
+}
+
 // ---------------------------------------------------------------------------
 // Weight packing (offline): R[n,k] = fp32(W[n,k]*s[k] - sum_j L1[k,j]*L2[j,n]),
 // the sum in fp64 for j = 0..r-1 with every multiply and add rounded on its own
@@ -140,7 +191,7 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
     const int k0 = c * 256 + lane * 8;
     const bool real = k0 < K;  // K % 8 == 0: a lane's 8 channels are all real or all padding
     const bool in_k = k0 < Kp;
-    float sv[8];
+    float sv[8], sz[8];
     if (real) {
       const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + k0));
       const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + k0 + 4));
@@ -150,6 +201,8 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
 #pragma unroll
       for (int e = 0; e < 8; ++e) sv[e] = 1.f;
     }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sz[e] = __frcp_rn(sv[e]);  // reused by the SUB rows
     // small ranks: the 8 channels' L1 rows (8*R bf16, contiguous) stay in registers
     float l1s[8][(R > 0 && R <= 4) ? R : 1];
     if constexpr (R > 0 && R <= 4) {
@@ -176,7 +229,7 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
       float x[8], xh[8];
       bf16x8_to_f32(xr[i], x);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xh[e] = real ? __fdiv_rn(x[e], sv[e]) : 0.f;
+      for (int e = 0; e < 8; ++e) xh[e] = real ? div_by_recip(x[e], sv[e], sz[e]) : 0.f;
       if constexpr (R > 0 && R <= 4) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -207,7 +260,7 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
         }
       }
       float sc;
-      const uint32_t packed = quantize8(xh, sc);
+      const uint32_t packed = quantize8_fast(xh, sc);
       if (in_k) {
         *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
         if ((lane & 7) == 0) {
