@@ -36,6 +36,7 @@ if ROOT not in sys.path:
 from w4a4_rank_assisted_b200.synth import WORKLOADS, make_layer  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
+METRIC = "W4A4 rank-4 linear TOPS & tokens/s at FLUX/SANA/Qwen3 shapes; % of roofline"
 INT8_OVER_BF16_NOMINAL = 2.0  # dense INT8 (4.5 POPS) over dense BF16 (2.25 PFLOP/s), nominal
 
 
@@ -209,7 +210,7 @@ def run_reference(args, specs, wl_name, rank, world):
     v = statistics.median([p[0] for p in per_step])
     tops = v / 1e12
     line = {
-        "impl": "reference", "metric": "W4A4 rank-4 linear TOPS (FLUX block linears)", "value": tops,
+        "impl": "reference", "metric": METRIC, "value": tops,
         "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": statistics.median([p[1] for p in per_step]) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -295,16 +296,19 @@ def run_gpu(args, specs, wl_name, rank, world, local):
 
     g_step = capture(lambda st: (do_flush(st), step(st)))
     g_flush = capture(do_flush) if flush else None
-    for _ in range(args.warmup):
-        g_step.replay()
+    with torch.cuda.stream(gstream):
+        for _ in range(args.warmup):
+            g_step.replay()
     torch.cuda.synchronize()
 
     def replay_ms(g, n):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(gstream)
-        for _ in range(n):
-            g.replay()
-        b.record(gstream)
+        # CUDAGraph.replay() launches on the current stream: make it gstream
+        with torch.cuda.stream(gstream):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(gstream)
+            for _ in range(n):
+                g.replay()
+            b.record(gstream)
         torch.cuda.synchronize()
         return a.elapsed_time(b)
 
@@ -316,10 +320,11 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(gstream)
-    for _ in range(args.steps):
-        g_step.replay()
-    t1.record(gstream)
+    with torch.cuda.stream(gstream):
+        t0.record(gstream)
+        for _ in range(args.steps):
+            g_step.replay()
+        t1.record(gstream)
     torch.cuda.synchronize()
     _barrier(world)
     clk = clocks.stop()
@@ -338,11 +343,13 @@ def run_gpu(args, specs, wl_name, rank, world, local):
         if flush:  # (flush + kernel) minus (flush alone), per launch
             g = capture(lambda st: [(do_flush(st), fn(st)) for _ in range(reps)])
             g0 = capture(lambda st: [do_flush(st) for _ in range(reps)])
-            g.replay(); g0.replay()
+            with torch.cuda.stream(gstream):
+                g.replay(); g0.replay()
             torch.cuda.synchronize()
             return (replay_ms(g, 3) - replay_ms(g0, 3)) * 1e3 / (3 * reps)
         g = capture(lambda st: [fn(st) for _ in range(reps)])
-        g.replay()
+        with torch.cuda.stream(gstream):
+            g.replay()
         torch.cuda.synchronize()
         return replay_ms(g, 3) * 1e3 / (3 * reps)
 
@@ -409,7 +416,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
 
     if rank == 0:
         line = {
-            "metric": "W4A4 rank-4 linear TOPS (FLUX block linears)", "value": tops, "unit": "TOPS",
+            "metric": METRIC, "value": tops, "unit": "TOPS",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4xint4->int32/f32",
             "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",

@@ -74,7 +74,7 @@ struct GemmArgs {
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
 };
 
-template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_>
+template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -85,16 +85,26 @@ struct GemmCfg {
   static constexpr int GPS = GPS_;             // 64-groups per pipeline stage
   static constexpr int NI8 = NI8_;             // int8 operand buffers
   static constexpr int NTM = NTM_;             // TMEM partial buffers
-  static constexpr int NUM_UNPACK_WARPS = 6;
+  static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
   // Register split (setmaxnreg): producer/MMA/unpack warpgroups give registers
   // to the drain warpgroups, which hold CW fp32 accumulators per thread.
-  static constexpr bool REALLOC = CW >= 128;
-  static constexpr int REGS_LOW = 64;
-  static constexpr int REGS_HIGH = ((65536 - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8 > 232
-                                       ? 232
-                                       : ((65536 - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
+  // setmaxnreg.inc draws only on the registers the block was launched with
+  // (THREADS x LAUNCH_REGS, LAUNCH_REGS being the __launch_bounds__ cap that
+  // ptxas allocates for kernels that reallocate), so the split is sized
+  // against that total; the host checks the kernel's actual register count
+  // against LAUNCH_REGS before the first launch.
+  static constexpr bool REALLOC = CW >= 128 || THREADS >= 768;
+  static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8 * 8) > 255 ? 248 : (65536 / THREADS) / 8 * 8;
+  static constexpr int REGS_LOW = THREADS >= 768 ? 40 : 64;
+  static constexpr int REGS_HIGH_RAW =
+      ((THREADS * LAUNCH_REGS - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
+  static constexpr int REGS_HIGH = REGS_HIGH_RAW > 232 ? 232 : REGS_HIGH_RAW;
+  static_assert(!REALLOC || 256 * REGS_LOW + 32 * NUM_DRAIN_WARPS * REGS_HIGH <= THREADS * LAUNCH_REGS,
+                "register split exceeds the block's launch allocation");
+  static_assert(!REALLOC || THREADS == 256 + 32 * NUM_DRAIN_WARPS, "two low warpgroups");
+  static_assert((2 + NUM_UNPACK_WARPS) % 4 == 0, "drain warps start on a warpgroup boundary");
   static constexpr int A_PACK = BM * 32 * GPS;  // packed bytes per stage (row operand)
   static constexpr int B_PACK = BN * 32 * GPS;  // packed bytes per stage (col operand)
   static constexpr int CS_BYTES = BN * 4;       // col scales of one group
@@ -113,6 +123,10 @@ struct GemmCfg {
   // unpack tasks (16 packed bytes each) per stage, and per unpack thread
   static constexpr int TASKS = 2 * GPS * (BM + BN);
   static constexpr int TPT = (TASKS + 32 * NUM_UNPACK_WARPS - 1) / (32 * NUM_UNPACK_WARPS);
+  // Drain software pipeline (next chunk's TMEM load in flight during the current
+  // chunk) when registers allow; with 4 drain warps per scheduler the warps
+  // themselves hide the load latency.
+  static constexpr bool PIPE = NUM_DRAIN_WARPS <= 8;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(CW % 16 == 0, "drain chunks");
   static_assert(TMEM_NEED <= 512, "TMEM");
@@ -390,9 +404,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         // Software pipeline over the stage's 16-column chunks: the TMEM load of
         // chunk c+1 is in flight while chunk c is folded into the accumulators.
         constexpr int NCH = CW / 16;  // chunks per group
-        uint32_t va[16], vb[16];
-        tmem_ld16(t_lane + static_cast<uint32_t>(tb * GPS * BN + h * CW), va);
-        tmem_ld_wait(va);
+        uint32_t va[16], vb[Cfg::PIPE ? 16 : 1];
+        if (Cfg::PIPE) {
+          tmem_ld16(t_lane + static_cast<uint32_t>(tb * GPS * BN + h * CW), va);
+          tmem_ld_wait(va);
+        }
 #pragma unroll
         for (int j = 0; j < GPS; ++j) {
           if (j >= ng) break;  // warp-uniform
@@ -403,13 +419,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < NCH; ++c) {
             const int k = j * NCH + c;  // running chunk index within the stage
-            uint32_t(&cur)[16] = (k & 1) ? vb : va;
-            uint32_t(&nxt)[16] = (k & 1) ? va : vb;
-            const bool more = (c + 1 < NCH) || (j + 1 < ng);
-            if (more) {
-              const int jn = (c + 1 < NCH) ? j : j + 1;
-              const int cn = (c + 1 < NCH) ? c + 1 : 0;
-              tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + jn) * BN + h * CW + cn * 16), nxt);
+            uint32_t* cur = va;
+            if constexpr (Cfg::PIPE) {
+              cur = (k & 1) ? vb : va;
+              uint32_t(&nxt)[16] = *reinterpret_cast<uint32_t(*)[16]>((k & 1) ? va : vb);
+              const bool more = (c + 1 < NCH) || (j + 1 < ng);
+              if (more) {
+                const int jn = (c + 1 < NCH) ? j : j + 1;
+                const int cn = (c + 1 < NCH) ? c + 1 : 0;
+                tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + jn) * BN + h * CW + cn * 16), nxt);
+              }
+            } else {
+              tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + c * 16), va);
+              tmem_ld_wait(va);
             }
 #pragma unroll
             for (int j4 = 0; j4 < 4; ++j4) {
@@ -423,7 +445,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 acc2[jj >> 1] = __ffma2_rn(rs2, t, acc2[jj >> 1]);
               }
             }
-            if (more) tmem_ld_wait(nxt);
+            if constexpr (Cfg::PIPE) {
+              const bool more = (c + 1 < NCH) || (j + 1 < ng);
+              if (more) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[16]>((k & 1) ? va : vb));
+            }
           }
         }
         tc_fence_before();

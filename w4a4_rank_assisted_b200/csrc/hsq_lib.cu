@@ -24,17 +24,19 @@ constexpr int kMaxRank = 32;
 
 // Kernel configurations (see hsq_gemm.cuh).
 //                           BN  DH STAGES SWAP  GPS NI8 NTM
-#ifndef HSQ_LARGE_BN
-#define HSQ_LARGE_BN 256
+#ifndef HSQ_LARGE_DH
+#define HSQ_LARGE_DH 2
 #endif
-#if HSQ_LARGE_BN == 128
-using CfgLarge = hsq::GemmCfg<128, 2, 8, false, 1, 3, 4>;  // M > 64: 128 tokens x 128 outputs per tile
-#else
-using CfgLarge = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2>;  // M > 64: 128 tokens x 256 outputs per tile
+// M > 64: 128 tokens x 256 outputs per tile; HSQ_LARGE_DH column slices of drain warps
+using CfgLarge = hsq::GemmCfg<256, HSQ_LARGE_DH, 6, false, 1, 3, 2>;
+#ifndef HSQ_DEC_UNPACK_WARPS
+#define HSQ_DEC_UNPACK_WARPS 10
 #endif
-using CfgDec16 = hsq::GemmCfg<16, 1, 5, true, 4, 2, 4>;    // M <= 16: 128 outputs x 16 tokens
-using CfgDec32 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2>;    // M <= 32
-using CfgDec64 = hsq::GemmCfg<64, 1, 6, true, 2, 2, 2>;    // M <= 64
+// M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; the drain is light,
+// so more warps unpack
+using CfgDec16 = hsq::GemmCfg<16, 1, 5, true, 4, 2, 4, HSQ_DEC_UNPACK_WARPS>;
+using CfgDec32 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, HSQ_DEC_UNPACK_WARPS>;
+using CfgDec64 = hsq::GemmCfg<64, 1, 6, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
 
 thread_local int t_debug_flags = 0;
 thread_local int t_debug_limit_ms = 0;
@@ -161,6 +163,13 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
       if (cudaFuncSetAttribute(hsq::w4a4_gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::SMEM_BYTES) != cudaSuccess)
         return HSQ_ERR_CUDA;
+      if (Cfg::REALLOC) {
+        // the warpgroup register split assumes the block launches with exactly
+        // LAUNCH_REGS registers per thread; refuse to launch otherwise
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, hsq::w4a4_gemm_kernel<Cfg>) != cudaSuccess) return HSQ_ERR_CUDA;
+        if (fa.numRegs != Cfg::LAUNCH_REGS) return HSQ_ERR_UNSUPPORTED;
+      }
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
   }
