@@ -157,6 +157,42 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const 
   return ok != 0;
 }
 
+// Whole-warp bounded wait for two phases at once: lane 0 tests barrier a, lane 1
+// barrier b, in the same instructions; one vote ends the wait.  __syncwarp
+// then orders every lane's later accesses after both lanes' acquires.  (The
+// common case, both phases already complete, costs one test and one vote.)
+__device__ __forceinline__ bool wait2_warp(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb,
+                                           const WaitPolicy& w) {
+  const int lane = lane_id();
+  uint64_t* bar = lane == 0 ? a : b;
+  const uint32_t par = lane == 0 ? pa : pb;
+  bool done = lane >= 2 || mbar_test_wait(bar, par);
+  if (__all_sync(0xffffffffu, done)) {
+    __syncwarp();
+    return true;
+  }
+  uint64_t t0 = 0;
+  if (lane == 0) t0 = global_timer_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    done = done || lane >= 2 || mbar_try_wait(bar, par);
+    if (__all_sync(0xffffffffu, done)) break;
+    if ((spin & HSQ_CHECK_MASK) == 0) {
+      int give_up = 0;
+      if (lane == 0) {
+        if (*w.abort) {
+          give_up = 1;
+        } else if (global_timer_ns() - t0 > w.limit_ns) {
+          raise_timeout(w);
+          give_up = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+    }
+  }
+  __syncwarp();
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA / bulk copy
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(

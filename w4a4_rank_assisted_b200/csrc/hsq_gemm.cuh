@@ -74,7 +74,8 @@ struct GemmArgs {
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
 };
 
-template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6>
+template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
+          int SSLOTS_ = STAGES_ + 4>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -85,6 +86,7 @@ struct GemmCfg {
   static constexpr int GPS = GPS_;             // 64-groups per pipeline stage
   static constexpr int NI8 = NI8_;             // int8 operand buffers
   static constexpr int NTM = NTM_;             // TMEM partial buffers
+  static constexpr int SSLOTS = SSLOTS_;       // scale ring slots (released by the drain)
   static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
@@ -109,17 +111,22 @@ struct GemmCfg {
   static constexpr int B_PACK = BN * 32 * GPS;  // packed bytes per stage (col operand)
   static constexpr int CS_BYTES = BN * 4;       // col scales of one group
   static constexpr int RS_BYTES = BM * 4;       // row scales of one group
-  static constexpr int CS_OFF = A_PACK + B_PACK;                 // stage layout: packed row tile,
-  static constexpr int RS_OFF = CS_OFF + GPS * CS_BYTES;         // packed col tile, col scales,
-  static constexpr int STAGE_BYTES = ((RS_OFF + GPS * RS_BYTES + 1023) / 1024) * 1024;  // row scales
+  // Packed stage: row tile then col tile (released by the unpack warps).  The
+  // scales of the same stage go to a separate, deeper ring (released by the
+  // drain), so a packed stage is free again as soon as it is unpacked.
+  static constexpr int STAGE_BYTES = ((A_PACK + B_PACK + 1023) / 1024) * 1024;
+  static constexpr int CS_OFF = 0;                        // scale slot: col scales,
+  static constexpr int RS_OFF = GPS * CS_BYTES;           // then row scales
+  static constexpr int SSLOT_BYTES = ((RS_OFF + GPS * RS_BYTES + 127) / 128) * 128;
   static constexpr int SA = i8_group_stride(BM);  // int8 bytes of one group, row operand
   static constexpr int SB = i8_group_stride(BN);  // int8 bytes of one group, col operand
   static constexpr int I8_BYTES = ((GPS * (SA + SB) + 1023) / 1024) * 1024;
   static constexpr int TMEM_NEED = NTM * GPS * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                  : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NI8 + 2 * NTM + 1;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8 * I8_BYTES + NUM_BARS * 8 + 64;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * SSLOTS + 2 * NI8 + 2 * NTM + 1;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8 * I8_BYTES +
+                                    SSLOTS * SSLOT_BYTES + NUM_BARS * 8 + 64;
   // unpack tasks (16 packed bytes each) per stage, and per unpack thread
   static constexpr int TASKS = 2 * GPS * (BM + BN);
   static constexpr int TPT = (TASKS + 32 * NUM_UNPACK_WARPS - 1) / (32 * NUM_UNPACK_WARPS);
@@ -203,10 +210,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* i8_base = smem + STAGES * Cfg::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(i8_base + NI8 * Cfg::I8_BYTES);
+  uint8_t* sc_base = i8_base + NI8 * Cfg::I8_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sc_base + Cfg::SSLOTS * Cfg::SSLOT_BYTES);
   uint64_t* full = bars;                   // [STAGES] packed stage landed
-  uint64_t* empty = bars + STAGES;         // [STAGES] packed stage free
-  uint64_t* full8 = bars + 2 * STAGES;     // [NI8] int8 operands ready
+  uint64_t* empty = bars + STAGES;         // [STAGES] packed stage unpacked
+  uint64_t* sfull = bars + 2 * STAGES;     // [SSLOTS] scales landed
+  uint64_t* sempty = sfull + Cfg::SSLOTS;  // [SSLOTS] scales drained
+  uint64_t* full8 = sempty + Cfg::SSLOTS;  // [NI8] int8 operands ready
   uint64_t* empty8 = full8 + NI8;          // [NI8] int8 operands consumed by the MMA
   uint64_t* tfull = empty8 + NI8;          // [NTM] TMEM partials ready
   uint64_t* tempty = tfull + NTM;          // [NTM] TMEM partials drained
@@ -222,7 +232,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], Cfg::NUM_UNPACK_WARPS + Cfg::NUM_DRAIN_WARPS);
+      mbar_init(&empty[s], Cfg::NUM_UNPACK_WARPS);
+    }
+    for (int s = 0; s < Cfg::SSLOTS; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], Cfg::NUM_DRAIN_WARPS);
     }
     for (int b = 0; b < NI8; ++b) {
       mbar_init(&full8[b], Cfg::NUM_UNPACK_WARPS);
@@ -269,16 +283,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int g = g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
           const int s = it % STAGES;
+          const int ss = it % Cfg::SSLOTS;
           if (!wait_one(&empty[s], ((it / STAGES) & 1) ^ 1, wp)) { ok = false; break; }
+          if (!wait_one(&sempty[ss], ((it / Cfg::SSLOTS) & 1) ^ 1, wp)) { ok = false; break; }
           uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK + ng * (cs_bytes + rs_bytes));
+          uint8_t* sc = sc_base + ss * Cfg::SSLOT_BYTES;
+          mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
           tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
           tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * 32, c0);
+          mbar_arrive_expect_tx(&sfull[ss], ng * (cs_bytes + rs_bytes));
           for (int j = 0; j < ng; ++j) {
-            bulk_load(st + Cfg::CS_OFF + j * Cfg::CS_BYTES,
-                      args.scales_c + static_cast<size_t>(g + j) * args.ld_c + c0, cs_bytes, &full[s]);
-            bulk_load(st + Cfg::RS_OFF + j * Cfg::RS_BYTES,
-                      args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, &full[s]);
+            bulk_load(sc + Cfg::CS_OFF + j * Cfg::CS_BYTES,
+                      args.scales_c + static_cast<size_t>(g + j) * args.ld_c + c0, cs_bytes, &sfull[ss]);
+            bulk_load(sc + Cfg::RS_OFF + j * Cfg::RS_BYTES,
+                      args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, &sfull[ss]);
           }
           issued = it + 1;
         }
@@ -351,8 +369,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int ng = min(GPS, g1 - g);
         const int s = it % STAGES;
         const int b = it % NI8;
-        if (!wait_warp(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
-        if (!wait_warp(&empty8[b], ((it / NI8) & 1) ^ 1, wp)) { ok = false; break; }
+        if (!wait2_warp(&full[s], (it / STAGES) & 1, &empty8[b], ((it / NI8) & 1) ^ 1, wp)) { ok = false; break; }
         const uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
         uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
         uint4 pk[Cfg::TPT];
@@ -392,15 +409,64 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
       for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.f, 0.f);
 #define ACC(j) (((j) & 1) ? acc2[(j) >> 1].y : acc2[(j) >> 1].x)
+      const int col0 = tc * BN + h * CW;
+      // The unit that holds the tile's first stage starts its accumulators at
+      // U L2 + b, so these loads overlap the pipeline instead of lengthening
+      // the epilogue's chain of dependent global accesses.
+      if (g0 == 0 && row_ok) {
+        if (!Cfg::SWAP) {
+          // rows are tokens m, columns are output features n
+          const int m = row;
+          if (args.bias) {
+#pragma unroll
+            for (int j8 = 0; j8 < CW / 8; ++j8) {
+              const int n = col0 + j8 * 8;
+              if (n < args.N) {
+                float bb[8];
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), bb);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ACC(j8 * 8 + e) = bb[e];
+              }
+            }
+          }
+          for (int i = 0; i < args.r; ++i) {
+            const float um = __ldg(args.U + static_cast<size_t>(m) * args.r + i);
+            const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(i) * args.N;
+#pragma unroll
+            for (int j8 = 0; j8 < CW / 8; ++j8) {
+              const int n = col0 + j8 * 8;
+              if (n < args.N) {
+                float l[8];
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + n)), l);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ACC(j8 * 8 + e) = fmaf(um, l[e], ACC(j8 * 8 + e));
+              }
+            }
+          }
+        } else {
+          // rows are output features n, columns are tokens m
+          const int n = row;
+          const float bn = args.bias ? __bfloat162float(args.bias[n]) : 0.f;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) ACC(j) = bn;
+          for (int i = 0; i < args.r; ++i) {
+            const float l2 = __bfloat162float(args.L2[static_cast<size_t>(i) * args.N + n]);
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+              const int m = col0 + j;
+              if (m < args.M) ACC(j) = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + i), l2, ACC(j));
+            }
+          }
+        }
+      }
       for (int g = g0; g < g1; g += GPS, ++it) {
         const int ng = min(GPS, g1 - g);
-        const int s = it % STAGES;
+        const int ss = it % Cfg::SSLOTS;
         const int tb = it % NTM;
-        if (!wait_warp(&tfull[tb], (it / NTM) & 1, wp)) { ok = false; break; }
-        if (!wait_warp(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
+        if (!wait2_warp(&tfull[tb], (it / NTM) & 1, &sfull[ss], (it / Cfg::SSLOTS) & 1, wp)) { ok = false; break; }
         tc_fence_after();
-        const float* cs_stage = reinterpret_cast<const float*>(stage_base + s * Cfg::STAGE_BYTES + Cfg::CS_OFF);
-        const float* rs_stage = reinterpret_cast<const float*>(stage_base + s * Cfg::STAGE_BYTES + Cfg::RS_OFF);
+        const float* cs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::CS_OFF);
+        const float* rs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::RS_OFF);
         // Software pipeline over the stage's 16-column chunks: the TMEM load of
         // chunk c+1 is in flight while chunk c is folded into the accumulators.
         constexpr int NCH = CW / 16;  // chunks per group
@@ -455,13 +521,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&tempty[tb]);
-          mbar_arrive(&empty[s]);
+          mbar_arrive(&sempty[ss]);
         }
       }
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue
-      const int col0 = tc * BN + h * CW;
       if (un.nslots > 1) {
         // Stream-K: every drain warp owns a 32-row x CW-column sub-tile.  It
         // writes its fp32 partial to this CTA's slot, and the warp that arrives
@@ -494,46 +559,24 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (lane == 0) *counter = 0u;
       }
       if (!row_ok) continue;
+      // the accumulators already hold U L2 + b (added by the tile's first unit)
       if (!Cfg::SWAP) {
         // rows are tokens m, columns are output features n
-        const int m = row;
-        for (int i = 0; i < args.r; ++i) {
-          const float um = __ldg(args.U + static_cast<size_t>(m) * args.r + i);
-          const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(i) * args.N;
-#pragma unroll
-          for (int j8 = 0; j8 < CW / 8; ++j8) {
-            const int n = col0 + j8 * 8;
-            if (n < args.N) {
-              float l[8];
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + n)), l);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) ACC(j8 * 8 + e) = fmaf(um, l[e], ACC(j8 * 8 + e));
-            }
-          }
-        }
+        const size_t rowoff = static_cast<size_t>(row) * args.N;
 #pragma unroll
         for (int j8 = 0; j8 < CW / 8; ++j8) {
           const int n = col0 + j8 * 8;
           if (n < args.N) {
-            float y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = ACC(j8 * 8 + e);
-            if (args.bias) {
-              float bb[8];
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), bb);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] += bb[e];
-            }
-            const size_t off = static_cast<size_t>(m) * args.N + n;
+            const size_t off = rowoff + n;
             if (args.out_f32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + off);
-              dst[0] = make_float4(y[0], y[1], y[2], y[3]);
-              dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+              dst[0] = make_float4(ACC(j8 * 8 + 0), ACC(j8 * 8 + 1), ACC(j8 * 8 + 2), ACC(j8 * 8 + 3));
+              dst[1] = make_float4(ACC(j8 * 8 + 4), ACC(j8 * 8 + 5), ACC(j8 * 8 + 6), ACC(j8 * 8 + 7));
             } else {
               uint4 o;
               __nv_bfloat162* ob = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) ob[e] = __floats2bfloat162_rn(y[2 * e], y[2 * e + 1]);
+              for (int e = 0; e < 4; ++e) ob[e] = __floats2bfloat162_rn(ACC(j8 * 8 + 2 * e), ACC(j8 * 8 + 2 * e + 1));
               *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off) = o;
             }
           }
@@ -541,23 +584,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       } else {
         // rows are output features n, columns are tokens m
         const int n = row;
-        const float bn = args.bias ? __bfloat162float(args.bias[n]) : 0.f;
-        for (int i = 0; i < args.r; ++i) {
-          const float l2 = __bfloat162float(args.L2[static_cast<size_t>(i) * args.N + n]);
-#pragma unroll
-          for (int j = 0; j < CW; ++j) {
-            const int m = col0 + j;
-            if (m < args.M) ACC(j) = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + i), l2, ACC(j));
-          }
-        }
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
           const int m = col0 + j;
           if (m < args.M) {
-            const float y = ACC(j) + bn;
             const size_t off = static_cast<size_t>(m) * args.N + n;
-            if (args.out_f32) static_cast<float*>(args.Y)[off] = y;
-            else static_cast<__nv_bfloat16*>(args.Y)[off] = __float2bfloat16_rn(y);
+            if (args.out_f32) static_cast<float*>(args.Y)[off] = ACC(j);
+            else static_cast<__nv_bfloat16*>(args.Y)[off] = __float2bfloat16_rn(ACC(j));
           }
         }
       }
@@ -573,6 +606,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // let every load still in flight land before the CTA's shared memory goes away
       const uint32_t first = issued > static_cast<uint32_t>(STAGES) ? issued - STAGES : 0u;
       for (uint32_t i = first; i < issued; ++i) wait_one(&full[i % STAGES], (i / STAGES) & 1, tail);
+      const uint32_t sfirst = issued > static_cast<uint32_t>(Cfg::SSLOTS) ? issued - Cfg::SSLOTS : 0u;
+      for (uint32_t i = sfirst; i < issued; ++i)
+        wait_one(&sfull[i % Cfg::SSLOTS], (i / Cfg::SSLOTS) & 1, tail);
     }
     if (warp == 1 && lane == 0) {
       mma_commit(final_bar);  // arrives once every MMA issued above has completed

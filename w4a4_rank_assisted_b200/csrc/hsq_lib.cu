@@ -28,15 +28,21 @@ constexpr int kMaxRank = 32;
 #define HSQ_LARGE_DH 2
 #endif
 // M > 64: 128 tokens x 256 outputs per tile; HSQ_LARGE_DH column slices of drain warps
-using CfgLarge = hsq::GemmCfg<256, HSQ_LARGE_DH, 6, false, 1, 3, 2>;
+#ifndef HSQ_LARGE_STAGES
+#define HSQ_LARGE_STAGES 6
+#endif
+using CfgLarge = hsq::GemmCfg<256, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, 1, 3, 2>;
 #ifndef HSQ_DEC_UNPACK_WARPS
 #define HSQ_DEC_UNPACK_WARPS 10
 #endif
 // M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; the drain is light,
 // so more warps unpack
-using CfgDec16 = hsq::GemmCfg<16, 1, 5, true, 4, 2, 4, HSQ_DEC_UNPACK_WARPS>;
+#ifndef HSQ_DEC_STAGES
+#define HSQ_DEC_STAGES 6
+#endif
+using CfgDec16 = hsq::GemmCfg<16, 1, HSQ_DEC_STAGES, true, 4, 2, 4, HSQ_DEC_UNPACK_WARPS>;
 using CfgDec32 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, HSQ_DEC_UNPACK_WARPS>;
-using CfgDec64 = hsq::GemmCfg<64, 1, 6, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
+using CfgDec64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
 
 thread_local int t_debug_flags = 0;
 thread_local int t_debug_limit_ms = 0;
