@@ -54,7 +54,8 @@ typedef enum {
   HSQ_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned */
   HSQ_ERR_UNSUPPORTED = 3,   /* group != 64, r > 32, K or N not a multiple of 8 */
   HSQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, tensor map) */
-  HSQ_ERR_TIMEOUT = 5        /* a kernel gave up waiting (reported by hsq_get_device_status) */
+  HSQ_ERR_TIMEOUT = 5,       /* a kernel gave up waiting (reported by hsq_get_device_status) */
+  HSQ_ERR_SCRATCH_LIMIT = 6  /* hsq_linear_forward_noalloc: shape needs more than HSQ_NOALLOC_SCRATCH_BYTES */
 } hsq_status;
 
 typedef enum { HSQ_OUT_BF16 = 0, HSQ_OUT_F32 = 1 } hsq_out_dtype;
@@ -111,7 +112,8 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
  * with P_g the exact integer dot product of group g's codes.  The INT4 codes are
  * multiplied on the tensor cores (tcgen05, kind::i8) one group at a time into
  * Tensor Memory and each group's int32 partial is rescaled into an fp32
- * accumulator; the low-rank branch and bias are added in the epilogue.
+ * accumulator, which also receives the low-rank branch and the bias before
+ * the single rounding to the output type.
  *   x_codes/x_scales/U   as written by hsq_quantize_act (U NULL iff r == 0)
  *   w_codes/w_scales     as written by hsq_pack_weights
  *   L2_bf16 [r][N] (NULL iff r == 0), bias_bf16 [N] or NULL for no bias
@@ -126,6 +128,47 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
                               int M, int N, int K, int r, int group,
                               void* Y, hsq_out_dtype out,
                               void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Bytes of the library's built-in scratch array used by
+ * hsq_linear_forward_noalloc (16 MiB).  Every GPU on which the library is
+ * loaded holds this array for the life of the process.
+ */
+#define HSQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * hsq_linear_forward without a caller-provided workspace.  The paper has no
+ * counterpart: this is a convenience of the library, not a step of the method.
+ *
+ * Some callers cannot hand the library scratch memory: a plain C host program
+ * that links only this library and has no device allocator of its own, or a
+ * serving loop that must not allocate once it is running (cudaMalloc and
+ * cudaFree synchronize the device and may fail under memory pressure).  For
+ * them this call takes the same arguments as hsq_linear_forward minus
+ * workspace/ws_bytes, and uses a file-scope device array of
+ * HSQ_NOALLOC_SCRATCH_BYTES bytes for the split-K counters and partial tiles.
+ * It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *
+ *   - Inputs and outputs are still caller-owned device pointers, exactly as
+ *     for hsq_linear_forward; the results are the same.
+ *   - Shapes whose scratch need, hsq_workspace_bytes(M,N,K,r), exceeds
+ *     HSQ_NOALLOC_SCRATCH_BYTES are rejected with HSQ_ERR_SCRATCH_LIMIT before
+ *     anything is launched (split-K shapes with 128x256 tiles can need up to
+ *     about 39 MB; the decode tiles, M <= 64, need at most about 10 MB).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Each call first clears, on `stream`, the part of the array that must
+ *     start at zero (the split-K counters).  All calls share the one array and
+ *     it keeps the last call's contents, so calls whose kernels overlap on the
+ *     GPU (different streams, no ordering between them) race and give wrong
+ *     results; order them on one stream or with events.
+ */
+hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_scales, const float* U,
+                                      const uint8_t* w_codes, const float* w_scales,
+                                      const void* L2_bf16, const void* bias_bf16,
+                                      int M, int N, int K, int r, int group,
+                                      void* Y, hsq_out_dtype out, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* hsq_status_string(hsq_status status);

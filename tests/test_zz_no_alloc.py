@@ -1,0 +1,92 @@
+"""hsq_linear_forward_noalloc: the forward that uses the library's built-in
+scratch array instead of a caller workspace.
+
+Checked through the C ABI against hsq_linear_forward (the regular entry point,
+with a workspace the test allocates) on the same inputs, on two calls in a row
+so that the second call starts from the scratch contents the first one left.
+Runs alone in a fresh process and after the other test files alike: it builds
+all of its own inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+from w4a4_rank_assisted_b200 import hsq
+from w4a4_rank_assisted_b200.synth import LayerSpec, make_layer
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+REL_TOL = 1e-2  # max |dY| <= 1e-2 * rms(Y), the layer tolerance used by every output check
+
+
+def _prepare(M, K, N, r, seed):
+    spec = LayerSpec(f"na{M}x{K}x{N}", M, K, N, r, act="outlier", outlier_frac=0.01, outlier_mult=30.0,
+                     seed=seed, bias=True)
+    lay = make_layer(spec)
+    d = lambda t: None if t is None else t.to(DEV).contiguous()
+    pl = hsq.PackedLinear(d(lay.W), d(lay.s), d(lay.L1) if r else None, d(lay.L2) if r else None, d(lay.bias))
+    act = hsq.ActBuffers(M, K, r, DEV)
+    hsq.hsq_quantize_act(d(lay.X), pl.s, pl.L1, M, K, r, act.x_codes, act.x_scales, act.U)
+    return pl, act
+
+
+def _regular(pl, act, M, K, N, r):
+    Y = torch.empty((M, N), dtype=torch.float32, device=DEV)
+    ws = pl.workspace(M)
+    hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, pl.bias,
+                           M, N, K, r, Y, out=hsq.HSQ_OUT_F32, workspace=ws,
+                           ws_bytes=0 if ws is None else ws.numel())
+    return Y
+
+
+def _noalloc(pl, act, M, K, N, r):
+    Y = torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
+    hsq.hsq_linear_forward_noalloc(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, pl.bias,
+                                   M, N, K, r, Y, out=hsq.HSQ_OUT_F32)
+    return Y
+
+
+@pytest.mark.parametrize("M,K,N,r", [
+    (16, 4096, 2048, 4),   # split-K decode tiles: uses the scratch array
+    (128, 2048, 1024, 4),  # split-K 128x256 tiles: uses the scratch array
+    (200, 224, 1160, 32),  # whole tiles: no scratch
+])
+def test_noalloc_matches_regular_entry_point_twice(M, K, N, r):
+    pl, act = _prepare(M, K, N, r, seed=M + N)
+    ref = _regular(pl, act, M, K, N, r)
+    torch.cuda.synchronize()
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    ref_np = ref.cpu().numpy().astype(np.float64)
+    rms = np.sqrt(np.mean(ref_np ** 2))
+    for call in range(2):
+        Y = _noalloc(pl, act, M, K, N, r)
+        torch.cuda.synchronize()
+        assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+        y = Y.cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(y)), f"call {call}: outputs left unwritten"
+        err = np.max(np.abs(y - ref_np))
+        assert err <= REL_TOL * rms, f"call {call}: max|dY| {err:.3e} > {REL_TOL} * rms {rms:.3e}"
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    # 256 tokens x 4096 outputs: 32 tiles of 128x256 cut between CTAs, whose
+    # partial tiles need more than the built-in array on a full-size GPU.
+    M, K, N, r = 256, 4096, 4096, 4
+    need = hsq.hsq_workspace_bytes(M, N, K, r)
+    if need <= hsq.HSQ_NOALLOC_SCRATCH_BYTES:
+        pytest.skip(f"this device needs only {need} bytes for the shape")
+    # full-size buffers, so that nothing could be read out of bounds even if a launch happened
+    x_codes = torch.zeros((M, K // 2), dtype=torch.uint8, device=DEV)
+    x_scales = torch.zeros((K // 64, hsq.hsq_scales_ld(M)), dtype=torch.float32, device=DEV)
+    U = torch.zeros((M, r), dtype=torch.float32, device=DEV)
+    w_codes = torch.zeros((N, K // 2), dtype=torch.uint8, device=DEV)
+    w_scales = torch.zeros((K // 64, hsq.hsq_scales_ld(N)), dtype=torch.float32, device=DEV)
+    L2 = torch.zeros((r, N), dtype=torch.bfloat16, device=DEV)
+    Y = torch.full((M, N), 7.0, dtype=torch.float32, device=DEV)
+    with pytest.raises(hsq.HsqError) as e:
+        hsq.hsq_linear_forward_noalloc(x_codes, x_scales, U, w_codes, w_scales, L2, None, M, N, K, r, Y,
+                                       out=hsq.HSQ_OUT_F32)
+    assert e.value.status == hsq.HSQ_ERR_SCRATCH_LIMIT
+    torch.cuda.synchronize()
+    assert bool(torch.all(Y == 7.0)), "a rejected call must launch nothing"

@@ -44,6 +44,33 @@ using CfgDec16 = hsq::GemmCfg<16, 1, HSQ_DEC_STAGES, true, 4, 2, 4, HSQ_DEC_UNPA
 using CfgDec32 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, HSQ_DEC_UNPACK_WARPS>;
 using CfgDec64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
 
+// Scratch of hsq_linear_forward_noalloc (split-K counters, then partial tiles),
+// for callers that cannot provide a workspace.  In host code this name only
+// stands in for the device array: its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+constexpr size_t kNoallocScratchBytes = HSQ_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+struct NoallocSlot {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoallocSlot g_noalloc_slots[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device (set-up on first use).
+hsq_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HSQ_ERR_UNSUPPORTED;
+  NoallocSlot& slot = g_noalloc_slots[dev];
+  std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch); });
+  if (slot.err != cudaSuccess || !slot.ptr) return HSQ_ERR_CUDA;
+  *out = slot.ptr;
+  return HSQ_OK;
+}
+
 thread_local int t_debug_flags = 0;
 thread_local int t_debug_limit_ms = 0;
 
@@ -217,6 +244,7 @@ const char* hsq_status_string(hsq_status s) {
     case HSQ_ERR_UNSUPPORTED: return "HSQ_ERR_UNSUPPORTED";
     case HSQ_ERR_CUDA: return "HSQ_ERR_CUDA";
     case HSQ_ERR_TIMEOUT: return "HSQ_ERR_TIMEOUT";
+    case HSQ_ERR_SCRATCH_LIMIT: return "HSQ_ERR_SCRATCH_LIMIT";
   }
   return "HSQ_UNKNOWN_STATUS";
 }
@@ -367,6 +395,36 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     case kDec64: return launch_gemm<CfgDec64>(p, tm_row, tm_col, a, stream);
   }
   return HSQ_ERR_INVALID_ARG;
+}
+
+hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_scales, const float* U,
+                                      const uint8_t* w_codes, const float* w_scales, const void* L2_bf16,
+                                      const void* bias_bf16, int M, int N, int K, int r, int group, void* Y,
+                                      hsq_out_dtype out, cudaStream_t stream) {
+  // The same argument checks as hsq_linear_forward, made before the scratch is touched,
+  // so that a rejected call launches nothing.
+  hsq_status st = check_common(M, K, r, group);
+  if (st != HSQ_OK) return st;
+  if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return HSQ_ERR_UNSUPPORTED;
+  if (out != HSQ_OUT_BF16 && out != HSQ_OUT_F32) return HSQ_ERR_INVALID_ARG;
+  if (!x_codes || !x_scales || !w_codes || !w_scales || !Y) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L2_bf16 != nullptr) || (r > 0) != (U != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(Y) || (U && !aligned16(U)) || (L2_bf16 && !aligned16(L2_bf16)) ||
+      (bias_bf16 && !aligned16(bias_bf16)))
+    return HSQ_ERR_ALIGNMENT;
+  const Plan p = make_plan(M, N, K, device_sm_count());
+  void* scratch = nullptr;
+  if (p.ws_bytes() > 0) {
+    if (p.ws_bytes() > kNoallocScratchBytes) return HSQ_ERR_SCRATCH_LIMIT;
+    st = noalloc_scratch(&scratch);
+    if (st != HSQ_OK) return st;
+    // the split-K counters must start at zero; the partial tiles are written before they are read
+    if (cudaMemsetAsync(scratch, 0, p.counters_bytes, stream) != cudaSuccess) return HSQ_ERR_CUDA;
+  }
+  return hsq_linear_forward(x_codes, x_scales, U, w_codes, w_scales, L2_bf16, bias_bf16, M, N, K, r, group, Y, out,
+                            scratch, scratch ? kNoallocScratchBytes : 0, stream);
 }
 
 }  // extern "C"

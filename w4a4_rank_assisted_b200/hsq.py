@@ -24,6 +24,9 @@ HSQ_ERR_ALIGNMENT = 2
 HSQ_ERR_UNSUPPORTED = 3
 HSQ_ERR_CUDA = 4
 HSQ_ERR_TIMEOUT = 5
+HSQ_ERR_SCRATCH_LIMIT = 6
+#: Size of the built-in scratch array of hsq_linear_forward_noalloc.
+HSQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 HSQ_OUT_BF16 = 0
 HSQ_OUT_F32 = 1
 
@@ -32,7 +35,7 @@ EXPORTED = (
     "hsq_num_groups", "hsq_codes_bytes", "hsq_scales_ld", "hsq_scales_bytes",
     "hsq_workspace_bytes", "hsq_pack_weights", "hsq_quantize_act",
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
-    "hsq_debug_force_timeout",
+    "hsq_debug_force_timeout", "hsq_linear_forward_noalloc",
 )
 
 
@@ -73,6 +76,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_quantize_act.restype = i
     lib.hsq_linear_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, sz, vp]
     lib.hsq_linear_forward.restype = i
+    lib.hsq_linear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
+    lib.hsq_linear_forward_noalloc.restype = i
     lib.hsq_status_string.argtypes = [i]; lib.hsq_status_string.restype = c.c_char_p
     lib.hsq_get_device_status.argtypes = [vp]; lib.hsq_get_device_status.restype = i
     lib.hsq_debug_force_timeout.argtypes = [i, i]; lib.hsq_debug_force_timeout.restype = None
@@ -147,6 +152,18 @@ def hsq_linear_forward(x_codes, x_scales, U, w_codes, w_scales, L2, bias, M, N, 
                                      _ptr(w_scales), _ptr(L2), _ptr(bias), M, N, K, r, group,
                                      _ptr(Y), int(out), _ptr(workspace), int(ws_bytes),
                                      _stream(stream)), "hsq_linear_forward")
+
+
+def hsq_linear_forward_noalloc(x_codes, x_scales, U, w_codes, w_scales, L2, bias, M, N, K, r, Y,
+                               out: int = HSQ_OUT_BF16, group=GROUP, stream=None) -> None:
+    """hsq_linear_forward with the library's own scratch array instead of a
+    workspace: for callers that must not allocate.  Calls that overlap on the
+    GPU share that array and race; the first call on a device must come
+    before any stream capture."""
+    _check(load().hsq_linear_forward_noalloc(_ptr(x_codes), _ptr(x_scales), _ptr(U), _ptr(w_codes),
+                                             _ptr(w_scales), _ptr(L2), _ptr(bias), M, N, K, r, group,
+                                             _ptr(Y), int(out), _stream(stream)),
+           "hsq_linear_forward_noalloc")
 
 
 def hsq_get_device_status(stream=None) -> int:
