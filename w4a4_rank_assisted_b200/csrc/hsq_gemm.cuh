@@ -72,10 +72,11 @@ struct GemmArgs {
   unsigned* ws_counters;  // stream-K arrival counters per (tile, drain warp), zero between calls
   uint64_t limit_ns;      // wait limit
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
+  int lr_mma;             // 1: a tile's first unit starts with the low-rank step (kernels with LR_MMA)
 };
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
-          int SSLOTS_ = STAGES_ + 4>
+          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int DRAIN_BATCH_ = 0, int PIPE_ = -1>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -87,8 +88,16 @@ struct GemmCfg {
   static constexpr int NI8 = NI8_;             // int8 operand buffers
   static constexpr int NTM = NTM_;             // TMEM partial buffers
   static constexpr int SSLOTS = SSLOTS_;       // scale ring slots (released by the drain)
+  // Operand encoding of the unpacked codes.  false: int8 16*q, kind::i8, int32
+  // group partials in TMEM (converted to fp32 by the drain).  true: E4M3
+  // subnormals q * 2^-9, kind::f8f6f4, fp32 group partials in TMEM; every
+  // product and every partial sum (|P| <= 64 * 49) is exact in both, so both
+  // give the same per-group partial P_g.
+  static constexpr bool F8 = F8_;
   static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
+  // DRAIN_BATCH: 16-column chunks per TMEM load batch of the drain (larger
+  // batches hide more load latency; each costs 16 more registers, twice).
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
   // Register split (setmaxnreg): producer/MMA/unpack warpgroups give registers
   // to the drain warpgroups, which hold CW fp32 accumulators per thread.
@@ -97,7 +106,8 @@ struct GemmCfg {
   // ptxas allocates for kernels that reallocate), so the split is sized
   // against that total; the host checks the kernel's actual register count
   // against LAUNCH_REGS before the first launch.
-  static constexpr bool REALLOC = CW >= 128 || THREADS >= 768;
+  static constexpr int DRAIN_BATCH = DRAIN_BATCH_ > 0 ? DRAIN_BATCH_ : (!SWAP && CW == 64 ? 2 : 1);
+  static constexpr bool REALLOC = CW >= 128 || THREADS >= 768 || DRAIN_BATCH >= 2;
   static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8 * 8) > 255 ? 248 : (65536 / THREADS) / 8 * 8;
   static constexpr int REGS_LOW = THREADS >= 768 ? 40 : 64;
   static constexpr int REGS_HIGH_RAW =
@@ -124,6 +134,15 @@ struct GemmCfg {
   static constexpr int TMEM_NEED = NTM * GPS * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                  : TMEM_NEED <= 256 ? 256 : 512;
+  // Low-rank step (tokens x outputs tiles with E4M3 operands): U L2 + b enters
+  // a tile's accumulators as one extra pipeline step ahead of its groups, a
+  // bf16 MMA over an augmented K of LR_K = 32 (hi and lo bf16 parts of U
+  // against L2 twice, then ones against the bias), so that r <= LR_MAX_RANK.
+  static constexpr bool LR_MMA = F8 && !SWAP && GPS == 1;
+  static constexpr int LR_K = 32;
+  static constexpr int LR_MAX_RANK = (LR_K - 2) / 2;
+  static constexpr int LR_SBO = LR_K / 8 * 128;  // bytes per 8-row group (4 K-chunks of 16 B)
+  static_assert(!LR_MMA || (BM + BN) / 8 * LR_SBO <= I8_BYTES, "low-rank operands fit an int8 buffer");
   static constexpr int NUM_BARS = 2 * STAGES + 2 * SSLOTS + 2 * NI8 + 2 * NTM + 1;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8 * I8_BYTES +
                                     SSLOTS * SSLOT_BYTES + NUM_BARS * 8 + 64;
@@ -133,9 +152,10 @@ struct GemmCfg {
   // Drain software pipeline (next chunk's TMEM load in flight during the current
   // chunk) when registers allow; with 4 drain warps per scheduler the warps
   // themselves hide the load latency.
-  static constexpr bool PIPE = NUM_DRAIN_WARPS <= 8;
+  static constexpr bool PIPE = PIPE_ >= 0 ? PIPE_ != 0 : NUM_DRAIN_WARPS <= 8;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(CW % 16 == 0, "drain chunks");
+  static_assert((CW / 16) % DRAIN_BATCH == 0, "drain batches");
   static_assert(TMEM_NEED <= 512, "TMEM");
   static_assert(32 * GPS <= 256, "TMA box width");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -143,6 +163,7 @@ struct GemmCfg {
 
 // Unpack 16 packed bytes (32 codes) into two 16-byte int8 core-matrix rows
 // (even codes, odd codes).
+template <bool F8>
 __device__ __forceinline__ void unpack16(const uint4& p, uint8_t* dst) {
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint4 lo, hi;
@@ -150,11 +171,72 @@ __device__ __forceinline__ void unpack16(const uint4& p, uint8_t* dst) {
   uint32_t* hi_w = reinterpret_cast<uint32_t*>(&hi);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    lo_w[i] = (w[i] << 4) & 0xF0F0F0F0u;  // even codes, 16*q as int8
-    hi_w[i] = w[i] & 0xF0F0F0F0u;         // odd codes,  16*q as int8
+    if constexpr (!F8) {
+      lo_w[i] = (w[i] << 4) & 0xF0F0F0F0u;  // even codes, 16*q as int8
+      hi_w[i] = w[i] & 0xF0F0F0F0u;         // odd codes,  16*q as int8
+    } else {
+      // Two's complement nibbles -> sign-magnitude nibbles (codes are never -8):
+      // for a negative nibble 8+j, (8+j) ^ 7 + 1 = 8 | (8-j) = sign | |q|.
+      const uint32_t sg = w[i] & 0x88888888u;
+      const uint32_t one = sg >> 3;
+      const uint32_t sm = (w[i] ^ (sg - one)) + one;
+      // E4M3 subnormal bytes: sign in bit 7, |q| in the mantissa, value q * 2^-9
+      lo_w[i] = (sm & 0x07070707u) | ((sm << 4) & 0x80808080u);  // even codes
+      hi_w[i] = ((sm >> 4) & 0x07070707u) | (sm & 0x80808080u);  // odd codes
+    }
   }
   *reinterpret_cast<uint4*>(dst) = lo;
   *reinterpret_cast<uint4*>(dst + kLBO) = hi;
+}
+
+// Operands of the low-rank step for one tile (rows r0.. of tokens, columns c0..
+// of outputs), written as bf16 K-major core matrices (8 rows x 16 bytes,
+// K-chunks 128 bytes apart, 8-row groups LR_SBO apart) into an int8 buffer:
+//   A[m][2i] = bf16(U[m][i]),  A[m][2i+1] = bf16(U[m][i] - A[m][2i]),  A[m][LR_K-2] = 1
+//   B[n][2i] = B[n][2i+1] = L2[i][n],                               B[n][LR_K-2] = bias[n]
+// so that A B^T = U L2 + b with U carried to about 16 significant bits.  Rows
+// outside the matrices and unused K are zero.  Threads t0, t0 + nt, ... each
+// build whole rows.
+template <class Cfg>
+__device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int c0, uint8_t* dst, int t0, int nt) {
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, K = Cfg::LR_K;
+  for (int t = t0; t < BM + BN; t += nt) {
+    const bool rowop = t < BM;
+    const int row = rowop ? t : t - BM;
+    const int idx = rowop ? r0 + row : c0 + row;  // token m or output n
+    const bool valid = idx < (rowop ? a.M : a.N);
+    uint8_t* base = dst + (rowop ? 0 : (BM / 8) * Cfg::LR_SBO) + (row >> 3) * Cfg::LR_SBO + (row & 7) * 16;
+#pragma unroll
+    for (int c = 0; c < K / 8; ++c) {  // one 16-byte K-chunk: ranks 4c .. 4c+3
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0.f;
+      if (valid) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * c + e;
+          if (i < a.r && i < Cfg::LR_MAX_RANK) {
+            if (rowop) {
+              const float v = __ldg(a.U + static_cast<size_t>(idx) * a.r + i);
+              f[2 * e] = __bfloat162float(__float2bfloat16_rn(v));
+              f[2 * e + 1] = v - f[2 * e];  // exact; rounded to bf16 below
+            } else {
+              const float l = __bfloat162float(a.L2[static_cast<size_t>(i) * a.N + idx]);
+              f[2 * e] = l;
+              f[2 * e + 1] = l;
+            }
+          }
+        }
+        if (c == K / 8 - 1)  // element K-2: ones against the bias
+          f[6] = rowop ? 1.f : (a.bias ? __bfloat162float(a.bias[idx]) : 0.f);
+      }
+      uint4 w;
+      __nv_bfloat162* wb = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) wb[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+      *reinterpret_cast<uint4*>(base + c * 128) = w;
+    }
+  }
 }
 
 // One unit of a CTA's work: groups [g0, g1) of one output tile.
@@ -280,12 +362,26 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int r0 = tr * BM;
         const uint32_t cs_bytes = static_cast<uint32_t>(min(BN, args.ld_c - c0)) * 4u;
         const uint32_t rs_bytes = static_cast<uint32_t>(min(BM, args.ld_r - r0)) * 4u;
-        for (int g = g0; g < g1; g += GPS, ++it) {
+        const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
+        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
           const int s = it % STAGES;
           const int ss = it % Cfg::SSLOTS;
           if (!wait_one(&empty[s], ((it / STAGES) & 1) ^ 1, wp)) { ok = false; break; }
           if (!wait_one(&sempty[ss], ((it / Cfg::SSLOTS) & 1) ^ 1, wp)) { ok = false; break; }
+          if (g < g0) {
+            // low-rank step: its operands are built by the unpack warps; its
+            // scales are 1 (columns) and 2^-18 (rows, undone by the drain's
+            // E4M3 factor), so the drain folds it in like any group
+            float4* scw = reinterpret_cast<float4*>(sc_base + ss * Cfg::SSLOT_BYTES);
+            for (int i = 0; i < BN / 4; ++i) scw[(Cfg::CS_OFF / 16) + i] = make_float4(1.f, 1.f, 1.f, 1.f);
+            const float lo = 1.0f / 262144.0f;
+            for (int i = 0; i < BM / 4; ++i) scw[(Cfg::RS_OFF / 16) + i] = make_float4(lo, lo, lo, lo);
+            mbar_arrive(&sfull[ss]);
+            mbar_arrive(&full[s]);
+            issued = it + 1;
+            continue;
+          }
           uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
           uint8_t* sc = sc_base + ss * Cfg::SSLOT_BYTES;
           mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
@@ -306,13 +402,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(BM, BN);
+      constexpr uint32_t idesc = Cfg::F8 ? idesc_f8(BM, BN) : idesc_i8(BM, BN);
       uint32_t it = 0;
       bool ok = true;
       Unit un;
       for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
-        for (int g = g0; g < g1; g += GPS, ++it) {
+        const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
+        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
           const int b = it % NI8;
           const int tb = it % NTM;
@@ -320,13 +417,32 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (!wait_one(&tempty[tb], ((it / NTM) & 1) ^ 1, wp)) { ok = false; break; }
           tc_fence_after();
           const uint32_t buf = smem_u32(i8_base + b * Cfg::I8_BYTES);
+          if (Cfg::LR_MMA && g < g0) {
+            // low-rank step: [U_hi U_lo 1] x [L2 L2 b] over K = LR_K, two K=16 bf16 MMAs
+            constexpr uint32_t idesc_lr = idesc_bf16(BM, BN);
+            const uint32_t d = tmem_base + static_cast<uint32_t>(tb * GPS * BN);
+            const uint32_t b_addr = buf + (BM / 8) * Cfg::LR_SBO;
+#pragma unroll
+            for (int q = 0; q < Cfg::LR_K / 16; ++q)
+              mma_bf16(d, smem_desc_kmajor(buf + q * 256, 128, Cfg::LR_SBO),
+                       smem_desc_kmajor(b_addr + q * 256, 128, Cfg::LR_SBO), idesc_lr, q > 0 ? 1u : 0u);
+            mma_commit(&empty8[b]);
+            mma_commit(&tfull[tb]);
+            continue;
+          }
           for (int j = 0; j < ng; ++j) {
             const uint32_t a_addr = buf + j * Cfg::SA;
             const uint32_t b_addr = buf + GPS * Cfg::SA + j * Cfg::SB;
             const uint32_t d = tmem_base + static_cast<uint32_t>((tb * GPS + j) * BN);
-            mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
-            mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
-                   smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+            if constexpr (Cfg::F8) {
+              mma_f8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
+              mma_f8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
+                     smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+            } else {
+              mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
+              mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
+                     smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+            }
           }
           mma_commit(&empty8[b]);
           mma_commit(&tfull[tb]);
@@ -365,20 +481,32 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     Unit un;
     for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
       const int g0 = un.g0, g1 = un.g1;
-      for (int g = g0; g < g1; g += GPS, ++it) {
+      const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
+      for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
         const int ng = min(GPS, g1 - g);
         const int s = it % STAGES;
         const int b = it % NI8;
         if (!wait2_warp(&full[s], (it / STAGES) & 1, &empty8[b], ((it / NI8) & 1) ^ 1, wp)) { ok = false; break; }
         const uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
         uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
+        if (Cfg::LR_MMA && g < g0) {
+          const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
+          build_lr_operands<Cfg>(args, tr * BM, tc * BN, dst, ut, NT);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&full8[b]);
+            mbar_arrive(&empty[s]);
+          }
+          continue;
+        }
         uint4 pk[Cfg::TPT];
 #pragma unroll
         for (int i = 0; i < Cfg::TPT; ++i)  // all loads first (always inside the stage)
           pk[i] = *reinterpret_cast<const uint4*>(st + src_off[i]);
 #pragma unroll
         for (int i = 0; i < Cfg::TPT; ++i)
-          if (grp[i] < ng) unpack16(pk[i], dst + dst_off[i]);
+          if (grp[i] < ng) unpack16<Cfg::F8>(pk[i], dst + dst_off[i]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -404,6 +532,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int g0 = un.g0, g1 = un.g1;
       const int row = tr * BM + row_local;
       const bool row_ok = row < args.rows_r;
+      const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
       // fp32 accumulators as pairs, for the packed f32x2 multiply-add
       float2 acc2[CW / 2];
 #pragma unroll
@@ -413,10 +542,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // The unit that holds the tile's first stage starts its accumulators at
       // U L2 + b, so these loads overlap the pipeline instead of lengthening
       // the epilogue's chain of dependent global accesses.
-      if (g0 == 0 && row_ok) {
-        if (!Cfg::SWAP) {
+      if constexpr (!Cfg::SWAP) {
+        if (g0 == 0 && row_ok && !lr_unit) {
           // rows are tokens m, columns are output features n
-          const int m = row;
+          const float* urow = args.U + static_cast<size_t>(row) * args.r;
           if (args.bias) {
 #pragma unroll
             for (int j8 = 0; j8 < CW / 8; ++j8) {
@@ -430,7 +559,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
           }
           for (int i = 0; i < args.r; ++i) {
-            const float um = __ldg(args.U + static_cast<size_t>(m) * args.r + i);
+            const float um = __ldg(urow + i);
             const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(i) * args.N;
 #pragma unroll
             for (int j8 = 0; j8 < CW / 8; ++j8) {
@@ -443,7 +572,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               }
             }
           }
-        } else {
+        }
+      } else if (g0 == 0 && row_ok) {
+        {
           // rows are output features n, columns are tokens m
           const int n = row;
           const float bn = args.bias ? __bfloat162float(args.bias[n]) : 0.f;
@@ -459,7 +590,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         }
       }
-      for (int g = g0; g < g1; g += GPS, ++it) {
+      for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
         const int ng = min(GPS, g1 - g);
         const int ss = it % Cfg::SSLOTS;
         const int tb = it % NTM;
@@ -467,54 +598,65 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tc_fence_after();
         const float* cs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::CS_OFF);
         const float* rs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::RS_OFF);
-        // Software pipeline over the stage's 16-column chunks: the TMEM load of
-        // chunk c+1 is in flight while chunk c is folded into the accumulators.
-        constexpr int NCH = CW / 16;  // chunks per group
-        uint32_t va[16], vb[Cfg::PIPE ? 16 : 1];
-        if (Cfg::PIPE) {
-          tmem_ld16(t_lane + static_cast<uint32_t>(tb * GPS * BN + h * CW), va);
-          tmem_ld_wait(va);
+        // The stage's partials are read from TMEM in batches of NB 16-column
+        // chunks.  tcgen05.wait::ld waits for every load the thread has issued,
+        // so the pipeline is one batch deep: the loads of batch i+1 are in
+        // flight while batch i is folded into the accumulators.
+        constexpr int NB = Cfg::DRAIN_BATCH;
+        constexpr int NCH = CW / 16;       // chunks per group
+        constexpr int BPG = NCH / NB;      // batches per group
+        const int nbt = ng * BPG;          // batches in this stage
+        uint32_t vbuf[Cfg::PIPE ? 2 : 1][NB][16];
+        auto issue = [&](int bi, uint32_t (&dst)[NB][16]) {
+          const int j = bi / BPG, c0 = (bi % BPG) * NB;
+#pragma unroll
+          for (int qq = 0; qq < NB; ++qq)
+            tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + (c0 + qq) * 16), dst[qq]);
+        };
+        auto wait_batch = [&](uint32_t (&dst)[NB][16]) {
+#pragma unroll
+          for (int qq = 0; qq < NB; ++qq) tmem_ld_wait(dst[qq]);
+        };
+        if constexpr (Cfg::PIPE) {
+          issue(0, vbuf[0]);
+          wait_batch(vbuf[0]);
         }
 #pragma unroll
-        for (int j = 0; j < GPS; ++j) {
-          if (j >= ng) break;  // warp-uniform
+        for (int bi = 0; bi < GPS * BPG; ++bi) {
+          if (bi >= nbt) break;  // warp-uniform
+          const int j = bi / BPG, c0 = (bi % BPG) * NB;
+          uint32_t(&cur)[NB][16] = vbuf[Cfg::PIPE ? (bi & 1) : 0];
+          if constexpr (Cfg::PIPE) {
+            if (bi + 1 < nbt) issue(bi + 1, vbuf[(bi + 1) & 1]);
+          } else {
+            issue(bi, cur);
+            wait_batch(cur);
+          }
           const float* cs = cs_stage + j * BN + h * CW;
-          // this row's scale of group g+j; 1/256 undoes the 16*q encoding of both operands
-          const float rs = rs_stage[j * BM + row_local] * (1.0f / 256.0f);
+          // this row's scale of group g+j, times the factor that undoes the operand
+          // encoding: 1/256 for 16*q (int8), 2^18 for q * 2^-9 (E4M3)
+          const float rs = rs_stage[j * BM + row_local] * (Cfg::F8 ? 262144.0f : (1.0f / 256.0f));
           const float2 rs2 = make_float2(rs, rs);
 #pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            const int k = j * NCH + c;  // running chunk index within the stage
-            uint32_t* cur = va;
-            if constexpr (Cfg::PIPE) {
-              cur = (k & 1) ? vb : va;
-              uint32_t(&nxt)[16] = *reinterpret_cast<uint32_t(*)[16]>((k & 1) ? va : vb);
-              const bool more = (c + 1 < NCH) || (j + 1 < ng);
-              if (more) {
-                const int jn = (c + 1 < NCH) ? j : j + 1;
-                const int cn = (c + 1 < NCH) ? c + 1 : 0;
-                tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + jn) * BN + h * CW + cn * 16), nxt);
-              }
-            } else {
-              tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + c * 16), va);
-              tmem_ld_wait(va);
-            }
+          for (int qq = 0; qq < NB; ++qq) {
+            const int c = c0 + qq;
 #pragma unroll
             for (int j4 = 0; j4 < 4; ++j4) {
               const float4 sc = *reinterpret_cast<const float4*>(cs + c * 16 + j4 * 4);
 #pragma unroll
               for (int e = 0; e < 4; e += 2) {
                 const int jj = c * 16 + j4 * 4 + e;
-                const float2 p = make_float2(__int2float_rn(static_cast<int>(cur[j4 * 4 + e])),
-                                             __int2float_rn(static_cast<int>(cur[j4 * 4 + e + 1])));
-                const float2 t = __fmul2_rn(p, e == 0 ? make_float2(sc.x, sc.y) : make_float2(sc.z, sc.w));
+                const uint32_t u0 = cur[qq][j4 * 4 + e], u1 = cur[qq][j4 * 4 + e + 1];
+                const float2 pp = Cfg::F8 ? make_float2(__uint_as_float(u0), __uint_as_float(u1))
+                                          : make_float2(__int2float_rn(static_cast<int>(u0)),
+                                                        __int2float_rn(static_cast<int>(u1)));
+                const float2 t = __fmul2_rn(pp, e == 0 ? make_float2(sc.x, sc.y) : make_float2(sc.z, sc.w));
                 acc2[jj >> 1] = __ffma2_rn(rs2, t, acc2[jj >> 1]);
               }
             }
-            if constexpr (Cfg::PIPE) {
-              const bool more = (c + 1 < NCH) || (j + 1 < ng);
-              if (more) tmem_ld_wait(*reinterpret_cast<uint32_t(*)[16]>((k & 1) ? va : vb));
-            }
+          }
+          if constexpr (Cfg::PIPE) {
+            if (bi + 1 < nbt) wait_batch(vbuf[(bi + 1) & 1]);
           }
         }
         tc_fence_before();

@@ -31,7 +31,32 @@ constexpr int kMaxRank = 32;
 #ifndef HSQ_LARGE_STAGES
 #define HSQ_LARGE_STAGES 6
 #endif
-using CfgLarge = hsq::GemmCfg<256, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, 1, 3, 2>;
+#ifndef HSQ_LARGE_F8
+#define HSQ_LARGE_F8 true
+#endif
+#ifndef HSQ_LARGE_BN
+#define HSQ_LARGE_BN 256
+#endif
+#ifndef HSQ_LARGE_GPS
+#define HSQ_LARGE_GPS 1
+#endif
+#ifndef HSQ_LARGE_NI8
+#define HSQ_LARGE_NI8 3
+#endif
+#ifndef HSQ_LARGE_NTM
+#define HSQ_LARGE_NTM 2
+#endif
+#ifndef HSQ_LR_MMA
+#define HSQ_LR_MMA 1  // U L2 + b as a tensor-core step where the kernel supports it
+#endif
+#ifndef HSQ_LARGE_BATCH
+#define HSQ_LARGE_BATCH 0
+#endif
+#ifndef HSQ_LARGE_PIPE
+#define HSQ_LARGE_PIPE -1
+#endif
+using CfgLarge = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, HSQ_LARGE_GPS, HSQ_LARGE_NI8,
+                              HSQ_LARGE_NTM, 6, HSQ_LARGE_STAGES + 4, HSQ_LARGE_F8, HSQ_LARGE_BATCH, HSQ_LARGE_PIPE>;
 #ifndef HSQ_DEC_UNPACK_WARPS
 #define HSQ_DEC_UNPACK_WARPS 10
 #endif
@@ -382,6 +407,8 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     a.ws_counters = static_cast<unsigned*>(workspace);
     a.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.counters_bytes);
   }
+  // U L2 + b as a bf16 MMA step when the kernel has one and the rank fits its K
+  a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge::LR_MMA && r <= CfgLarge::LR_MAX_RANK) ? 1 : 0;
   a.limit_ns = wait_limit_ns();
   if (t_debug_flags) {
     a.debug_flags = t_debug_flags;
