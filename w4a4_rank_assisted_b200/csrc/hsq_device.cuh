@@ -289,7 +289,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "memory");
 }
 
+// 16 lanes x 256 bits, twice along columns: with lane base L and column base C,
+// thread t gets v[4k + e] = (L + t/4, C + 8k + 2(t%4) + e) and
+// v[4k + 2 + e] = (L + t/4 + 8, C + 8k + 2(t%4) + e), for k, e in {0, 1}.
+__device__ __forceinline__ void tmem_ld_q8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Wait for this thread's TMEM loads, passing 8 destination registers through the asm.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7])
+               :
+               : "memory");
+}
 
 // Wait for this thread's TMEM loads; the 16 destination registers are passed
 // through the asm so that the compiler cannot read them before the wait.

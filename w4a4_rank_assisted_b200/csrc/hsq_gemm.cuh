@@ -76,7 +76,7 @@ struct GemmArgs {
 };
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
-          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int DRAIN_BATCH_ = 0, int PIPE_ = -1>
+          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -96,8 +96,6 @@ struct GemmCfg {
   static constexpr bool F8 = F8_;
   static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
-  // DRAIN_BATCH: 16-column chunks per TMEM load batch of the drain (larger
-  // batches hide more load latency; each costs 16 more registers, twice).
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
   // Register split (setmaxnreg): producer/MMA/unpack warpgroups give registers
   // to the drain warpgroups, which hold CW fp32 accumulators per thread.
@@ -106,16 +104,16 @@ struct GemmCfg {
   // ptxas allocates for kernels that reallocate), so the split is sized
   // against that total; the host checks the kernel's actual register count
   // against LAUNCH_REGS before the first launch.
-  static constexpr int DRAIN_BATCH = DRAIN_BATCH_ > 0 ? DRAIN_BATCH_ : (!SWAP && CW == 64 ? 2 : 1);
-  static constexpr bool REALLOC = CW >= 128 || THREADS >= 768 || DRAIN_BATCH >= 2;
+  static constexpr bool REALLOC = CW >= 128 || THREADS >= 768;
   static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8 * 8) > 255 ? 248 : (65536 / THREADS) / 8 * 8;
-  static constexpr int REGS_LOW = THREADS >= 768 ? 40 : 64;
+  static constexpr int LOW_THREADS = THREADS - 32 * NUM_DRAIN_WARPS;  // producer, MMA, unpack warpgroups
+  static constexpr int REGS_LOW = THREADS > 512 ? 40 : 64;
   static constexpr int REGS_HIGH_RAW =
-      ((THREADS * LAUNCH_REGS - 256 * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
+      ((THREADS * LAUNCH_REGS - LOW_THREADS * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
   static constexpr int REGS_HIGH = REGS_HIGH_RAW > 232 ? 232 : REGS_HIGH_RAW;
-  static_assert(!REALLOC || 256 * REGS_LOW + 32 * NUM_DRAIN_WARPS * REGS_HIGH <= THREADS * LAUNCH_REGS,
+  static_assert(!REALLOC || LOW_THREADS * REGS_LOW + 32 * NUM_DRAIN_WARPS * REGS_HIGH <= THREADS * LAUNCH_REGS,
                 "register split exceeds the block's launch allocation");
-  static_assert(!REALLOC || THREADS == 256 + 32 * NUM_DRAIN_WARPS, "two low warpgroups");
+  static_assert(LOW_THREADS % 128 == 0, "whole low warpgroups");
   static_assert((2 + NUM_UNPACK_WARPS) % 4 == 0, "drain warps start on a warpgroup boundary");
   static constexpr int A_PACK = BM * 32 * GPS;  // packed bytes per stage (row operand)
   static constexpr int B_PACK = BN * 32 * GPS;  // packed bytes per stage (col operand)
@@ -155,7 +153,6 @@ struct GemmCfg {
   static constexpr bool PIPE = PIPE_ >= 0 ? PIPE_ != 0 : NUM_DRAIN_WARPS <= 8;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(CW % 16 == 0, "drain chunks");
-  static_assert((CW / 16) % DRAIN_BATCH == 0, "drain batches");
   static_assert(TMEM_NEED <= 512, "TMEM");
   static_assert(32 * GPS <= 256, "TMA box width");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -521,8 +518,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const int dw = warp - (2 + Cfg::NUM_UNPACK_WARPS);
     const int q = warp & 3;            // TMEM lane quadrant
     const int h = dw >> 2;             // column slice
-    const int row_local = q * 32 + lane;
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const int qd = lane >> 2, qc = lane & 3;
+    // Thread <-> accumulator layout, that of tcgen05.ld.16x256b: the thread holds
+    // rows q*32 + qd + 8i (i = 0..3) of the tile and, in each 8-column block b of
+    // its slice, columns h*CW + 8b + 2qc + {0, 1}, as the pair acc2[i*NBLK + b].
+    // A column-scale pair then serves four rows, and the four threads of a quad
+    // read four different pairs, so the per-group scale loads stay few.
+    constexpr int NBLK = CW / 8;   // 8-column blocks of the slice
+    constexpr int NCC = CW / 16;   // 16-column chunks (one TMEM load per half quadrant)
+    const uint32_t t_q = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
     Unit un;
@@ -530,62 +534,59 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int tile = un.tile;
       const int tr = tile % args.tiles_r, tc = tile / args.tiles_r;
       const int g0 = un.g0, g1 = un.g1;
-      const int row = tr * BM + row_local;
-      const bool row_ok = row < args.rows_r;
+      const int rbase = tr * BM + q * 32 + qd;   // tile row of i = 0 (row i adds 8i)
+      const int col0 = tc * BN + h * CW + 2 * qc;  // column of block 0, first of the pair
       const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
-      // fp32 accumulators as pairs, for the packed f32x2 multiply-add
-      float2 acc2[CW / 2];
+      float2 acc2[4 * NBLK];
 #pragma unroll
-      for (int j = 0; j < CW / 2; ++j) acc2[j] = make_float2(0.f, 0.f);
-#define ACC(j) (((j) & 1) ? acc2[(j) >> 1].y : acc2[(j) >> 1].x)
-      const int col0 = tc * BN + h * CW;
+      for (int j = 0; j < 4 * NBLK; ++j) acc2[j] = make_float2(0.f, 0.f);
       // The unit that holds the tile's first stage starts its accumulators at
-      // U L2 + b, so these loads overlap the pipeline instead of lengthening
-      // the epilogue's chain of dependent global accesses.
-      if constexpr (!Cfg::SWAP) {
-        if (g0 == 0 && row_ok && !lr_unit) {
+      // U L2 + b (when no low-rank MMA step carries it).
+      if (g0 == 0 && !lr_unit) {
+        if constexpr (!Cfg::SWAP) {
           // rows are tokens m, columns are output features n
-          const float* urow = args.U + static_cast<size_t>(row) * args.r;
-          if (args.bias) {
 #pragma unroll
-            for (int j8 = 0; j8 < CW / 8; ++j8) {
-              const int n = col0 + j8 * 8;
-              if (n < args.N) {
-                float bb[8];
-                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), bb);
+          for (int i = 0; i < 4; ++i) {
+            const int m = rbase + 8 * i;
+            if (m >= args.rows_r) continue;
+            if (args.bias) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ACC(j8 * 8 + e) = bb[e];
+              for (int b = 0; b < NBLK; ++b) {
+                const int n = col0 + 8 * b;
+                if (n < args.N) acc2[i * NBLK + b] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(args.bias + n));
+              }
+            }
+            const float* urow = args.U + static_cast<size_t>(m) * args.r;
+            for (int kk = 0; kk < args.r; ++kk) {
+              const float um = __ldg(urow + kk);
+              const float2 um2 = make_float2(um, um);
+              const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(kk) * args.N;
+#pragma unroll
+              for (int b = 0; b < NBLK; ++b) {
+                const int n = col0 + 8 * b;
+                if (n < args.N)
+                  acc2[i * NBLK + b] = __ffma2_rn(um2, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(l2 + n)),
+                                                  acc2[i * NBLK + b]);
               }
             }
           }
-          for (int i = 0; i < args.r; ++i) {
-            const float um = __ldg(urow + i);
-            const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(i) * args.N;
-#pragma unroll
-            for (int j8 = 0; j8 < CW / 8; ++j8) {
-              const int n = col0 + j8 * 8;
-              if (n < args.N) {
-                float l[8];
-                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + n)), l);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ACC(j8 * 8 + e) = fmaf(um, l[e], ACC(j8 * 8 + e));
-              }
-            }
-          }
-        }
-      } else if (g0 == 0 && row_ok) {
-        {
+        } else {
           // rows are output features n, columns are tokens m
-          const int n = row;
-          const float bn = args.bias ? __bfloat162float(args.bias[n]) : 0.f;
 #pragma unroll
-          for (int j = 0; j < CW; ++j) ACC(j) = bn;
-          for (int i = 0; i < args.r; ++i) {
-            const float l2 = __bfloat162float(args.L2[static_cast<size_t>(i) * args.N + n]);
+          for (int i = 0; i < 4; ++i) {
+            const int n = rbase + 8 * i;
+            if (n >= args.rows_r) continue;
+            const float bn = args.bias ? __bfloat162float(args.bias[n]) : 0.f;
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
-              const int m = col0 + j;
-              if (m < args.M) ACC(j) = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + i), l2, ACC(j));
+            for (int b = 0; b < NBLK; ++b) acc2[i * NBLK + b] = make_float2(bn, bn);
+            for (int kk = 0; kk < args.r; ++kk) {
+              const float l2 = __bfloat162float(args.L2[static_cast<size_t>(kk) * args.N + n]);
+#pragma unroll
+              for (int b = 0; b < NBLK; ++b) {
+                const int m = col0 + 8 * b;
+                if (m < args.M) acc2[i * NBLK + b].x = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + kk), l2, acc2[i * NBLK + b].x);
+                if (m + 1 < args.M) acc2[i * NBLK + b].y = fmaf(__ldg(args.U + static_cast<size_t>(m + 1) * args.r + kk), l2, acc2[i * NBLK + b].y);
+              }
             }
           }
         }
@@ -598,65 +599,65 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tc_fence_after();
         const float* cs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::CS_OFF);
         const float* rs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::RS_OFF);
-        // The stage's partials are read from TMEM in batches of NB 16-column
-        // chunks.  tcgen05.wait::ld waits for every load the thread has issued,
-        // so the pipeline is one batch deep: the loads of batch i+1 are in
-        // flight while batch i is folded into the accumulators.
-        constexpr int NB = Cfg::DRAIN_BATCH;
-        constexpr int NCH = CW / 16;       // chunks per group
-        constexpr int BPG = NCH / NB;      // batches per group
-        const int nbt = ng * BPG;          // batches in this stage
-        uint32_t vbuf[Cfg::PIPE ? 2 : 1][NB][16];
-        auto issue = [&](int bi, uint32_t (&dst)[NB][16]) {
-          const int j = bi / BPG, c0 = (bi % BPG) * NB;
-#pragma unroll
-          for (int qq = 0; qq < NB; ++qq)
-            tmem_ld16(t_lane + static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + (c0 + qq) * 16), dst[qq]);
+        // The stage's partials are read from TMEM one 16-column chunk (both
+        // half quadrants) at a time.  tcgen05.wait::ld waits for every load the
+        // thread has issued, so the pipeline is one chunk deep: the loads of
+        // chunk i+1 are in flight while chunk i is folded into the accumulators.
+        const int nbt = ng * NCC;  // chunks in this stage
+        uint32_t vbuf[Cfg::PIPE ? 2 : 1][2][8];
+        auto issue = [&](int bi, uint32_t (&dst)[2][8]) {
+          const int j = bi / NCC, cc = bi % NCC;
+          const uint32_t col = static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + 16 * cc);
+          tmem_ld_q8(t_q + col, dst[0]);
+          tmem_ld_q8(t_q + (16u << 16) + col, dst[1]);
         };
-        auto wait_batch = [&](uint32_t (&dst)[NB][16]) {
-#pragma unroll
-          for (int qq = 0; qq < NB; ++qq) tmem_ld_wait(dst[qq]);
+        auto wait_chunk = [&](uint32_t (&dst)[2][8]) {
+          tmem_ld_wait(dst[0]);
+          tmem_ld_wait(dst[1]);
         };
         if constexpr (Cfg::PIPE) {
           issue(0, vbuf[0]);
-          wait_batch(vbuf[0]);
+          wait_chunk(vbuf[0]);
         }
+        float2 rs2[4];
+        int jrs = -1;
 #pragma unroll
-        for (int bi = 0; bi < GPS * BPG; ++bi) {
+        for (int bi = 0; bi < GPS * NCC; ++bi) {
           if (bi >= nbt) break;  // warp-uniform
-          const int j = bi / BPG, c0 = (bi % BPG) * NB;
-          uint32_t(&cur)[NB][16] = vbuf[Cfg::PIPE ? (bi & 1) : 0];
+          const int j = bi / NCC, cc = bi % NCC;
+          uint32_t(&cur)[2][8] = vbuf[Cfg::PIPE ? (bi & 1) : 0];
           if constexpr (Cfg::PIPE) {
             if (bi + 1 < nbt) issue(bi + 1, vbuf[(bi + 1) & 1]);
           } else {
             issue(bi, cur);
-            wait_batch(cur);
+            wait_chunk(cur);
           }
-          const float* cs = cs_stage + j * BN + h * CW;
-          // this row's scale of group g+j, times the factor that undoes the operand
-          // encoding: 1/256 for 16*q (int8), 2^18 for q * 2^-9 (E4M3)
-          const float rs = rs_stage[j * BM + row_local] * (Cfg::F8 ? 262144.0f : (1.0f / 256.0f));
-          const float2 rs2 = make_float2(rs, rs);
+          if (j != jrs) {
+            // the four rows' scales of group g+j, times the factor that undoes the
+            // operand encoding: 1/256 for 16*q (int8), 2^18 for q * 2^-9 (E4M3)
+            jrs = j;
 #pragma unroll
-          for (int qq = 0; qq < NB; ++qq) {
-            const int c = c0 + qq;
+            for (int i = 0; i < 4; ++i) {
+              const float rs = rs_stage[j * BM + q * 32 + qd + 8 * i] * (Cfg::F8 ? 262144.0f : (1.0f / 256.0f));
+              rs2[i] = make_float2(rs, rs);
+            }
+          }
+          const float* cs = cs_stage + j * BN + h * CW + 16 * cc + 2 * qc;
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const float4 sc = *reinterpret_cast<const float4*>(cs + c * 16 + j4 * 4);
+          for (int kb = 0; kb < 2; ++kb) {
+            const float2 c2 = *reinterpret_cast<const float2*>(cs + 8 * kb);
+            const int b = 2 * cc + kb;
 #pragma unroll
-              for (int e = 0; e < 4; e += 2) {
-                const int jj = c * 16 + j4 * 4 + e;
-                const uint32_t u0 = cur[qq][j4 * 4 + e], u1 = cur[qq][j4 * 4 + e + 1];
-                const float2 pp = Cfg::F8 ? make_float2(__uint_as_float(u0), __uint_as_float(u1))
-                                          : make_float2(__int2float_rn(static_cast<int>(u0)),
-                                                        __int2float_rn(static_cast<int>(u1)));
-                const float2 t = __fmul2_rn(pp, e == 0 ? make_float2(sc.x, sc.y) : make_float2(sc.z, sc.w));
-                acc2[jj >> 1] = __ffma2_rn(rs2, t, acc2[jj >> 1]);
-              }
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t u0 = cur[i >> 1][4 * kb + 2 * (i & 1)], u1 = cur[i >> 1][4 * kb + 2 * (i & 1) + 1];
+              const float2 pp = Cfg::F8 ? make_float2(__uint_as_float(u0), __uint_as_float(u1))
+                                        : make_float2(__int2float_rn(static_cast<int>(u0)),
+                                                      __int2float_rn(static_cast<int>(u1)));
+              acc2[i * NBLK + b] = __ffma2_rn(rs2[i], __fmul2_rn(pp, c2), acc2[i * NBLK + b]);
             }
           }
           if constexpr (Cfg::PIPE) {
-            if (bi + 1 < nbt) wait_batch(vbuf[(bi + 1) & 1]);
+            if (bi + 1 < nbt) wait_chunk(vbuf[(bi + 1) & 1]);
           }
         }
         tc_fence_before();
@@ -671,14 +672,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // ---------------------------------------------------------- epilogue
       if (un.nslots > 1) {
         // Stream-K: every drain warp owns a 32-row x CW-column sub-tile.  It
-        // writes its fp32 partial to this CTA's slot, and the warp that arrives
-        // last for that sub-tile sums the contributing CTAs' partials in CTA
-        // order (deterministic), runs the epilogue and re-zeroes the counter.
-        // No cross-warp or cross-CTA waiting.
-        float* part = args.ws_partials +
-                      ((static_cast<size_t>(blockIdx.x) * 2 + un.slot) * BN + h * CW) * BM + row_local;
+        // writes its fp32 partial to this CTA's slot (in the threads' own
+        // layout, so each store is 32 consecutive pairs), and the warp that
+        // arrives last for that sub-tile sums the contributing CTAs' partials
+        // in CTA order (deterministic), runs the epilogue and re-zeroes the
+        // counter.  No cross-warp or cross-CTA waiting.
+        constexpr int SLOT2 = BN * BM / 2;  // float2 per CTA slot
+        float2* part = reinterpret_cast<float2*>(args.ws_partials) +
+                       (static_cast<size_t>(blockIdx.x) * 2 + un.slot) * SLOT2 + dw * (4 * NBLK * 32) + lane;
 #pragma unroll
-        for (int j = 0; j < CW; ++j) part[static_cast<size_t>(j) * BM] = ACC(j);
+        for (int j = 0; j < 4 * NBLK; ++j) part[j * 32] = acc2[j];
         __threadfence();
         __syncwarp();
         unsigned* counter = args.ws_counters + static_cast<size_t>(tile) * Cfg::NUM_DRAIN_WARPS + dw;
@@ -688,58 +691,65 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (!last) continue;
         __threadfence();
 #pragma unroll
-        for (int j = 0; j < CW; ++j) ACC(j) = 0.f;
+        for (int j = 0; j < 4 * NBLK; ++j) acc2[j] = make_float2(0.f, 0.f);
         const unsigned S = static_cast<unsigned>(args.stages_per_tile);
         const unsigned L = static_cast<unsigned>(args.stream_len);
 #pragma unroll 2
         for (int c = un.first; c < un.first + un.nslots; ++c) {
           const int cslot = (static_cast<unsigned>(c) * L >= static_cast<unsigned>(tile) * S) ? 0 : 1;
-          const float* p = args.ws_partials + ((static_cast<size_t>(c) * 2 + cslot) * BN + h * CW) * BM + row_local;
+          const float2* p = reinterpret_cast<const float2*>(args.ws_partials) +
+                            (static_cast<size_t>(c) * 2 + cslot) * SLOT2 + dw * (4 * NBLK * 32) + lane;
 #pragma unroll
-          for (int j = 0; j < CW; ++j) ACC(j) += __ldcg(p + static_cast<size_t>(j) * BM);
+          for (int j = 0; j < 4 * NBLK; ++j) {
+            const float2 v = __ldcg(p + j * 32);
+            acc2[j].x += v.x;
+            acc2[j].y += v.y;
+          }
         }
         if (lane == 0) *counter = 0u;
       }
-      if (!row_ok) continue;
       // the accumulators already hold U L2 + b (added by the tile's first unit)
       if (!Cfg::SWAP) {
         // rows are tokens m, columns are output features n
-        const size_t rowoff = static_cast<size_t>(row) * args.N;
 #pragma unroll
-        for (int j8 = 0; j8 < CW / 8; ++j8) {
-          const int n = col0 + j8 * 8;
-          if (n < args.N) {
-            const size_t off = rowoff + n;
-            if (args.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + off);
-              dst[0] = make_float4(ACC(j8 * 8 + 0), ACC(j8 * 8 + 1), ACC(j8 * 8 + 2), ACC(j8 * 8 + 3));
-              dst[1] = make_float4(ACC(j8 * 8 + 4), ACC(j8 * 8 + 5), ACC(j8 * 8 + 6), ACC(j8 * 8 + 7));
-            } else {
-              uint4 o;
-              __nv_bfloat162* ob = reinterpret_cast<__nv_bfloat162*>(&o);
+        for (int i = 0; i < 4; ++i) {
+          const int m = rbase + 8 * i;
+          if (m >= args.rows_r) continue;
+          const size_t rowoff = static_cast<size_t>(m) * args.N;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) ob[e] = __floats2bfloat162_rn(ACC(j8 * 8 + 2 * e), ACC(j8 * 8 + 2 * e + 1));
-              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off) = o;
+          for (int b = 0; b < NBLK; ++b) {
+            const int n = col0 + 8 * b;
+            if (n < args.N) {
+              if (args.out_f32) *reinterpret_cast<float2*>(static_cast<float*>(args.Y) + rowoff + n) = acc2[i * NBLK + b];
+              else *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(args.Y) + rowoff + n) =
+                  __float22bfloat162_rn(acc2[i * NBLK + b]);
             }
           }
         }
       } else {
         // rows are output features n, columns are tokens m
-        const int n = row;
 #pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          const int m = col0 + j;
-          if (m < args.M) {
-            const size_t off = static_cast<size_t>(m) * args.N + n;
-            if (args.out_f32) static_cast<float*>(args.Y)[off] = ACC(j);
-            else static_cast<__nv_bfloat16*>(args.Y)[off] = __float2bfloat16_rn(ACC(j));
+        for (int i = 0; i < 4; ++i) {
+          const int n = rbase + 8 * i;
+          if (n >= args.rows_r) continue;
+#pragma unroll
+          for (int b = 0; b < NBLK; ++b) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int m = col0 + 8 * b + e;
+              if (m < args.M) {
+                const float v = e ? acc2[i * NBLK + b].y : acc2[i * NBLK + b].x;
+                const size_t off = static_cast<size_t>(m) * args.N + n;
+                if (args.out_f32) static_cast<float*>(args.Y)[off] = v;
+                else static_cast<__nv_bfloat16*>(args.Y)[off] = __float2bfloat16_rn(v);
+              }
+            }
           }
         }
       }
     }
   }
 
-#undef ACC
   // ------------------------------------------------------------ teardown
   __syncthreads();
   if (*abort_flag) {

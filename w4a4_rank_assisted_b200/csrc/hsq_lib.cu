@@ -46,17 +46,18 @@ constexpr int kMaxRank = 32;
 #ifndef HSQ_LARGE_NTM
 #define HSQ_LARGE_NTM 2
 #endif
+#ifndef HSQ_LARGE_UNPACK
+#define HSQ_LARGE_UNPACK 6
+#endif
 #ifndef HSQ_LR_MMA
 #define HSQ_LR_MMA 1  // U L2 + b as a tensor-core step where the kernel supports it
-#endif
-#ifndef HSQ_LARGE_BATCH
-#define HSQ_LARGE_BATCH 0
 #endif
 #ifndef HSQ_LARGE_PIPE
 #define HSQ_LARGE_PIPE -1
 #endif
 using CfgLarge = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, HSQ_LARGE_GPS, HSQ_LARGE_NI8,
-                              HSQ_LARGE_NTM, 6, HSQ_LARGE_STAGES + 4, HSQ_LARGE_F8, HSQ_LARGE_BATCH, HSQ_LARGE_PIPE>;
+                              HSQ_LARGE_NTM, HSQ_LARGE_UNPACK, HSQ_LARGE_STAGES + 4, HSQ_LARGE_F8,
+                              HSQ_LARGE_PIPE>;
 #ifndef HSQ_DEC_UNPACK_WARPS
 #define HSQ_DEC_UNPACK_WARPS 10
 #endif
