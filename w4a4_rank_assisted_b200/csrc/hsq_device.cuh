@@ -301,6 +301,15 @@ __device__ __forceinline__ void tmem_ld_q8(uint32_t taddr, uint32_t (&v)[8]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Wait for this thread's TMEM loads, passing 2 x 8 destination registers through the asm.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[8], uint32_t (&w)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(w[0]), "+r"(w[1]), "+r"(w[2]), "+r"(w[3]), "+r"(w[4]), "+r"(w[5]), "+r"(w[6]), "+r"(w[7])
+               :
+               : "memory");
+}
+
 // Wait for this thread's TMEM loads, passing 8 destination registers through the asm.
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[8]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"

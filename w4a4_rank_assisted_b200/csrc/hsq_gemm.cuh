@@ -501,9 +501,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < Cfg::TPT; ++i)  // all loads first (always inside the stage)
           pk[i] = *reinterpret_cast<const uint4*>(st + src_off[i]);
+        // with one group per stage and tasks filling every thread, no task test is needed
+        constexpr bool ALL_TASKS = GPS == 1 && Cfg::TASKS % NT == 0;
 #pragma unroll
         for (int i = 0; i < Cfg::TPT; ++i)
-          if (grp[i] < ng) unpack16<Cfg::F8>(pk[i], dst + dst_off[i]);
+          if (ALL_TASKS || grp[i] < ng) unpack16<Cfg::F8>(pk[i], dst + dst_off[i]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -592,7 +594,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
       }
       for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
-        const int ng = min(GPS, g1 - g);
+        const int ng = GPS == 1 ? 1 : min(GPS, g1 - g);
         const int ss = it % Cfg::SSLOTS;
         const int tb = it % NTM;
         if (!wait2_warp(&tfull[tb], (it / NTM) & 1, &sfull[ss], (it / Cfg::SSLOTS) & 1, wp)) { ok = false; break; }
@@ -611,16 +613,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           tmem_ld_q8(t_q + col, dst[0]);
           tmem_ld_q8(t_q + (16u << 16) + col, dst[1]);
         };
-        auto wait_chunk = [&](uint32_t (&dst)[2][8]) {
-          tmem_ld_wait(dst[0]);
-          tmem_ld_wait(dst[1]);
-        };
+        auto wait_chunk = [&](uint32_t (&dst)[2][8]) { tmem_ld_wait(dst[0], dst[1]); };
         if constexpr (Cfg::PIPE) {
           issue(0, vbuf[0]);
           wait_chunk(vbuf[0]);
         }
         float2 rs2[4];
-        int jrs = -1;
 #pragma unroll
         for (int bi = 0; bi < GPS * NCC; ++bi) {
           if (bi >= nbt) break;  // warp-uniform
@@ -632,10 +630,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             issue(bi, cur);
             wait_chunk(cur);
           }
-          if (j != jrs) {
+          if (cc == 0) {
             // the four rows' scales of group g+j, times the factor that undoes the
             // operand encoding: 1/256 for 16*q (int8), 2^18 for q * 2^-9 (E4M3)
-            jrs = j;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float rs = rs_stage[j * BM + q * 32 + qd + 8 * i] * (Cfg::F8 ? 262144.0f : (1.0f / 256.0f));
@@ -694,16 +691,23 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int j = 0; j < 4 * NBLK; ++j) acc2[j] = make_float2(0.f, 0.f);
         const unsigned S = static_cast<unsigned>(args.stages_per_tile);
         const unsigned L = static_cast<unsigned>(args.stream_len);
-#pragma unroll 2
+#pragma unroll 1
         for (int c = un.first; c < un.first + un.nslots; ++c) {
           const int cslot = (static_cast<unsigned>(c) * L >= static_cast<unsigned>(tile) * S) ? 0 : 1;
           const float2* p = reinterpret_cast<const float2*>(args.ws_partials) +
                             (static_cast<size_t>(c) * 2 + cslot) * SLOT2 + dw * (4 * NBLK * 32) + lane;
+          // 16 pairs in flight at a time (the accumulators already use most registers)
 #pragma unroll
-          for (int j = 0; j < 4 * NBLK; ++j) {
-            const float2 v = __ldcg(p + j * 32);
-            acc2[j].x += v.x;
-            acc2[j].y += v.y;
+          for (int j0 = 0; j0 < 4 * NBLK; j0 += 16) {
+            float2 v[16];
+#pragma unroll
+            for (int e = 0; e < 16 && j0 + e < 4 * NBLK; ++e) v[e] = __ldcg(p + (j0 + e) * 32);
+#pragma unroll
+            for (int e = 0; e < 16 && j0 + e < 4 * NBLK; ++e) {
+              acc2[j0 + e].x += v[e].x;
+              acc2[j0 + e].y += v[e].y;
+            }
+            asm volatile("" ::: "memory");
           }
         }
         if (lane == 0) *counter = 0u;
