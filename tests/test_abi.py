@@ -95,7 +95,9 @@ def test_pack_and_act_argument_validation():
 
 
 def test_workspace_needs_are_consistent():
-    # split-K is used only when the output tiles cannot fill the device
-    assert hsq.hsq_workspace_bytes(4608, 12288, 3072, 4) == 0
-    assert hsq.hsq_workspace_bytes(1, 4096, 12288, 4) > 0
+    # More than 64 tokens: both code matrices expanded to E4M3 bytes, rows padded
+    # to whole 128 x 256 tiles (no split-K: the 1728 tiles fill the device).
+    assert hsq.hsq_workspace_bytes(4608, 12288, 3072, 4) == (4608 + 12288) * 3072
+    # decode tiles: only split-K scratch (counters and partial tiles)
+    assert 0 < hsq.hsq_workspace_bytes(1, 4096, 12288, 4) < 16 << 20
     assert hsq.hsq_workspace_bytes(0, 4096, 12288, 4) == 0

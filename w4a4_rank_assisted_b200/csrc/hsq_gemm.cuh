@@ -73,10 +73,13 @@ struct GemmArgs {
   uint64_t limit_ns;      // wait limit
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
   int lr_mma;             // 1: a tile's first unit starts with the low-rank step (kernels with LR_MMA)
+  const uint8_t* xe;      // pre-expanded row operand (kernels with PRE): [G][rg_r][4][8][16] E4M3
+  const uint8_t* we;      // pre-expanded col operand: [G][rg_c][4][8][16]
+  int rg_r, rg_c;         // 8-row groups of each (rows padded to whole tiles)
 };
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
-          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1>
+          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -94,6 +97,15 @@ struct GemmCfg {
   // product and every partial sum (|P| <= 64 * 49) is exact in both, so both
   // give the same per-group partial P_g.
   static constexpr bool F8 = F8_;
+  // Pre-expanded operands (tokens x outputs tiles): both code matrices are
+  // expanded once per call (expand_e4m3_kernel) into E4M3 tiles laid out the
+  // way the MMA reads them, so a stage is two contiguous bulk copies and no
+  // warp unpacks in the main loop; the NUM_UNPACK_WARPS warps then only build
+  // the low-rank step's operands.
+  static constexpr bool PRE = PRE_;
+  static constexpr int E8_SBO = 512;  // pre-expanded tile: bytes per 8-row group (4 K-chunks of 8 rows x 16 B)
+  static constexpr int A_E8 = BM / 8 * E8_SBO;
+  static constexpr int B_E8 = BN / 8 * E8_SBO;
   static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
@@ -122,13 +134,14 @@ struct GemmCfg {
   // Packed stage: row tile then col tile (released by the unpack warps).  The
   // scales of the same stage go to a separate, deeper ring (released by the
   // drain), so a packed stage is free again as soon as it is unpacked.
-  static constexpr int STAGE_BYTES = ((A_PACK + B_PACK + 1023) / 1024) * 1024;
+  static constexpr int STAGE_BYTES = PRE ? ((A_E8 + B_E8 + 1023) / 1024) * 1024 : ((A_PACK + B_PACK + 1023) / 1024) * 1024;
   static constexpr int CS_OFF = 0;                        // scale slot: col scales,
   static constexpr int RS_OFF = GPS * CS_BYTES;           // then row scales
   static constexpr int SSLOT_BYTES = ((RS_OFF + GPS * RS_BYTES + 127) / 128) * 128;
   static constexpr int SA = i8_group_stride(BM);  // int8 bytes of one group, row operand
   static constexpr int SB = i8_group_stride(BN);  // int8 bytes of one group, col operand
   static constexpr int I8_BYTES = ((GPS * (SA + SB) + 1023) / 1024) * 1024;
+  static constexpr int NI8E = PRE ? 0 : NI8;   // int8 buffers actually laid out
   static constexpr int TMEM_NEED = NTM * GPS * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                  : TMEM_NEED <= 256 ? 256 : 512;
@@ -140,12 +153,15 @@ struct GemmCfg {
   static constexpr int LR_K = 32;
   static constexpr int LR_MAX_RANK = (LR_K - 2) / 2;
   static constexpr int LR_SBO = LR_K / 8 * 128;  // bytes per 8-row group (4 K-chunks of 16 B)
-  static_assert(!LR_MMA || (BM + BN) / 8 * LR_SBO <= I8_BYTES, "low-rank operands fit an int8 buffer");
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * SSLOTS + 2 * NI8 + 2 * NTM + 1;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8 * I8_BYTES +
+  static_assert(!LR_MMA || PRE || (BM + BN) / 8 * LR_SBO <= I8_BYTES, "low-rank operands fit an int8 buffer");
+  // with pre-expanded operands the low-rank operands get a buffer of their own
+  static constexpr int LR_BYTES = (PRE && LR_MMA) ? (BM + BN) / 8 * LR_SBO : 0;
+  static_assert(!PRE || (F8 && !SWAP && GPS == 1), "pre-expanded operands: E4M3, tokens x outputs, one group a stage");
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * SSLOTS + 2 * NI8E + 2 * NTM + 1 + 2;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8E * I8_BYTES + LR_BYTES +
                                     SSLOTS * SSLOT_BYTES + NUM_BARS * 8 + 64;
   // unpack tasks (16 packed bytes each) per stage, and per unpack thread
-  static constexpr int TASKS = 2 * GPS * (BM + BN);
+  static constexpr int TASKS = PRE ? 1 : 2 * GPS * (BM + BN);
   static constexpr int TPT = (TASKS + 32 * NUM_UNPACK_WARPS - 1) / (32 * NUM_UNPACK_WARPS);
   // Drain software pipeline (next chunk's TMEM load in flight during the current
   // chunk) when registers allow; with 4 drain warps per scheduler the warps
@@ -160,7 +176,7 @@ struct GemmCfg {
 
 // Unpack 16 packed bytes (32 codes) into two 16-byte int8 core-matrix rows
 // (even codes, odd codes).
-template <bool F8>
+template <bool F8, int HI_OFF = static_cast<int>(kLBO)>
 __device__ __forceinline__ void unpack16(const uint4& p, uint8_t* dst) {
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint4 lo, hi;
@@ -183,7 +199,32 @@ __device__ __forceinline__ void unpack16(const uint4& p, uint8_t* dst) {
     }
   }
   *reinterpret_cast<uint4*>(dst) = lo;
-  *reinterpret_cast<uint4*>(dst + kLBO) = hi;
+  *reinterpret_cast<uint4*>(dst + HI_OFF) = hi;
+}
+
+// Expands a packed INT4 code matrix [rows][Kp/2] into the layout in which the
+// pre-expanded large-tile kernel's MMA reads its operands: E4M3 bytes
+// [G][rows_pad/8][4 K-chunks][8 rows][16 B], chunk 2h+p of group g holding the
+// codes 32h + 2e + p (e = 0..15), the same even/odd order as the shared-memory
+// unpack (any order works if both operands share it).  Rows >= rows are zero,
+// so whole tiles can be copied.  One thread per (group, 8-row group, half,
+// row); the eight threads of a row group write 128 contiguous bytes.
+__global__ void __launch_bounds__(256) expand_e4m3_kernel(const uint8_t* __restrict__ codes, int rows, int Kp,
+                                                          int rows_pad, uint8_t* __restrict__ out) {
+  const size_t RG = static_cast<size_t>(rows_pad / 8);
+  const size_t total = static_cast<size_t>(Kp / 64) * RG * 16;
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int r8 = static_cast<int>(t & 7);
+    const int half = static_cast<int>((t >> 3) & 1);
+    const size_t gr = t >> 4;  // g * RG + rg
+    const int g = static_cast<int>(gr / RG);
+    const int row = static_cast<int>(gr % RG) * 8 + r8;
+    uint4 p = make_uint4(0u, 0u, 0u, 0u);
+    if (row < rows)
+      p = __ldg(reinterpret_cast<const uint4*>(codes + static_cast<size_t>(row) * (Kp / 2) + g * 32 + half * 16));
+    unpack16<true, 128>(p, out + (gr * 4 + 2 * half) * 128 + r8 * 16);
+  }
 }
 
 // Operands of the low-rank step for one tile (rows r0.. of tokens, columns c0..
@@ -284,12 +325,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_row, const __grid_constant__ CUtensorMap tm_col,
                      const GemmArgs args) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, CW = Cfg::CW, STAGES = Cfg::STAGES, GPS = Cfg::GPS;
-  constexpr int NI8 = Cfg::NI8, NTM = Cfg::NTM;
+  constexpr int NI8 = Cfg::NI8E, NTM = Cfg::NTM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* i8_base = smem + STAGES * Cfg::STAGE_BYTES;
-  uint8_t* sc_base = i8_base + NI8 * Cfg::I8_BYTES;
+  uint8_t* lr_buf = i8_base + NI8 * Cfg::I8_BYTES;  // low-rank operands (pre-expanded mode)
+  uint8_t* sc_base = lr_buf + Cfg::LR_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sc_base + Cfg::SSLOTS * Cfg::SSLOT_BYTES);
   uint64_t* full = bars;                   // [STAGES] packed stage landed
   uint64_t* empty = bars + STAGES;         // [STAGES] packed stage unpacked
@@ -300,6 +342,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* tfull = empty8 + NI8;          // [NTM] TMEM partials ready
   uint64_t* tempty = tfull + NTM;          // [NTM] TMEM partials drained
   uint64_t* final_bar = tempty + NTM;      // teardown: all MMAs done
+  uint64_t* lrfull = final_bar + 1;        // low-rank operands built (pre-expanded mode)
+  uint64_t* lrempty = lrfull + 1;          // low-rank operands consumed by the MMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* tail_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -311,7 +355,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], Cfg::NUM_UNPACK_WARPS);
+      mbar_init(&empty[s], Cfg::PRE ? 1 : Cfg::NUM_UNPACK_WARPS);  // PRE: released by the MMA's commit
     }
     for (int s = 0; s < Cfg::SSLOTS; ++s) {
       mbar_init(&sfull[s], 1);
@@ -326,6 +370,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(&tempty[b], Cfg::NUM_DRAIN_WARPS);
     }
     mbar_init(final_bar, 1);
+    mbar_init(lrfull, Cfg::NUM_UNPACK_WARPS);
+    mbar_init(lrempty, 1);
     *abort_flag = 0;
     *tail_flag = 0;
     fence_mbar_init();
@@ -381,9 +427,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
           uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
           uint8_t* sc = sc_base + ss * Cfg::SSLOT_BYTES;
-          mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
-          tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
-          tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * 32, c0);
+          if constexpr (Cfg::PRE) {
+            // MMA-ready E4M3 tiles: one contiguous block per operand
+            mbar_arrive_expect_tx(&full[s], Cfg::A_E8 + Cfg::B_E8);
+            bulk_load(st, args.xe + (static_cast<size_t>(g) * args.rg_r + tr * (BM / 8)) * Cfg::E8_SBO, Cfg::A_E8,
+                      &full[s]);
+            bulk_load(st + Cfg::A_E8, args.we + (static_cast<size_t>(g) * args.rg_c + tc * (BN / 8)) * Cfg::E8_SBO,
+                      Cfg::B_E8, &full[s]);
+          } else {
+            mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
+            tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
+            tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * 32, c0);
+          }
           mbar_arrive_expect_tx(&sfull[ss], ng * (cs_bytes + rs_bytes));
           for (int j = 0; j < ng; ++j) {
             bulk_load(sc + Cfg::CS_OFF + j * Cfg::CS_BYTES,
@@ -398,8 +453,47 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
-    if (lane == 0) {
+    if (Cfg::PRE && lane == 0) {
+      // pre-expanded operands: the MMAs read the stage itself and release it
+      constexpr uint32_t idesc = idesc_f8(BM, BN);
+      constexpr uint32_t idesc_lr = idesc_bf16(BM, BN);
+      uint32_t it = 0, nlr = 0;
+      bool ok = true;
+      Unit un;
+      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+        const int g0 = un.g0, g1 = un.g1;
+        const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
+        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+          const int s = it % STAGES;
+          const int tb = it % NTM;
+          if (!wait_one(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
+          if (!wait_one(&tempty[tb], ((it / NTM) & 1) ^ 1, wp)) { ok = false; break; }
+          const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
+          if (Cfg::LR_MMA && g < g0) {
+            // low-rank step: [U_hi U_lo 1] x [L2 L2 b] over K = LR_K, from the low-rank buffer
+            if (!wait_one(lrfull, nlr & 1, wp)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t abuf = smem_u32(lr_buf), bbuf = abuf + (BM / 8) * Cfg::LR_SBO;
+#pragma unroll
+            for (int q = 0; q < Cfg::LR_K / 16; ++q)
+              mma_bf16(d, smem_desc_kmajor(abuf + q * 256, 128, Cfg::LR_SBO),
+                       smem_desc_kmajor(bbuf + q * 256, 128, Cfg::LR_SBO), idesc_lr, q > 0 ? 1u : 0u);
+            mma_commit(lrempty);
+            ++nlr;
+          } else {
+            tc_fence_after();
+            const uint32_t abuf = smem_u32(stage_base + s * Cfg::STAGE_BYTES), bbuf = abuf + Cfg::A_E8;
+            mma_f8(d, smem_desc_kmajor(abuf, 128, Cfg::E8_SBO), smem_desc_kmajor(bbuf, 128, Cfg::E8_SBO), idesc, 0u);
+            mma_f8(d, smem_desc_kmajor(abuf + 256, 128, Cfg::E8_SBO), smem_desc_kmajor(bbuf + 256, 128, Cfg::E8_SBO),
+                   idesc, 1u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[tb]);
+        }
+      }
+    } else if (!Cfg::PRE && lane == 0) {
       constexpr uint32_t idesc = Cfg::F8 ? idesc_f8(BM, BN) : idesc_i8(BM, BN);
+      constexpr int NI8D = NI8 > 0 ? NI8 : 1;  // (unused when PRE)
       uint32_t it = 0;
       bool ok = true;
       Unit un;
@@ -408,9 +502,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
         for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
-          const int b = it % NI8;
+          const int b = it % NI8D;
           const int tb = it % NTM;
-          if (!wait_one(&full8[b], (it / NI8) & 1, wp)) { ok = false; break; }
+          if (!wait_one(&full8[b], (it / NI8D) & 1, wp)) { ok = false; break; }
           if (!wait_one(&tempty[tb], ((it / NTM) & 1) ^ 1, wp)) { ok = false; break; }
           tc_fence_after();
           const uint32_t buf = smem_u32(i8_base + b * Cfg::I8_BYTES);
@@ -449,68 +543,87 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else if (warp < 2 + Cfg::NUM_UNPACK_WARPS) {
     // ------------------------------------------------------------ unpack
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
-    constexpr int NT = 32 * Cfg::NUM_UNPACK_WARPS;
-    // This thread's tasks are the same at every stage: precompute their offsets.
-    // Task t -> operand (row tasks first), row, 16-byte chunk c of the row's
-    // 32*GPS packed bytes (c fastest, so 8 consecutive threads read 128
-    // contiguous bytes); group j = c/2, half = c%2.
-    uint32_t src_off[Cfg::TPT], dst_off[Cfg::TPT];
-    int grp[Cfg::TPT];
-    const int ut = (warp - 2) * 32 + lane;
-#pragma unroll
-    for (int i = 0; i < Cfg::TPT; ++i) {
-      int t = ut + i * NT;
-      grp[i] = GPS;  // GPS = no task
-      src_off[i] = dst_off[i] = 0;
-      if (t < Cfg::TASKS) {
-        const bool colop = t >= 2 * GPS * BM;
-        if (colop) t -= 2 * GPS * BM;
-        const int row = t / (2 * GPS), c = t % (2 * GPS);
-        const int j = c >> 1, half = c & 1;
-        grp[i] = j;
-        src_off[i] = (colop ? Cfg::A_PACK : 0) + row * 32 * GPS + c * 16;
-        dst_off[i] = (colop ? GPS * Cfg::SA + j * Cfg::SB : j * Cfg::SA) + (row >> 3) * kSBO + 2 * half * kLBO +
-                     (row & 7) * 16;
+    if constexpr (Cfg::PRE) {
+      // pre-expanded mode: these warps only build the low-rank step's operands,
+      // one tile ahead at most (single buffer)
+      const int ut = (warp - 2) * 32 + lane;
+      uint32_t nlr = 0;
+      bool ok = true;
+      Unit un;
+      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+        if (!(Cfg::LR_MMA && args.lr_mma && un.g0 == 0)) continue;
+        if (!wait_warp(lrempty, (nlr & 1) ^ 1, wp)) { ok = false; break; }
+        const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
+        build_lr_operands<Cfg>(args, tr * BM, tc * BN, lr_buf, ut, 32 * Cfg::NUM_UNPACK_WARPS);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(lrfull);
+        ++nlr;
       }
-    }
-    uint32_t it = 0;
-    bool ok = true;
-    Unit un;
-    for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
-      const int g0 = un.g0, g1 = un.g1;
-      const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
-      for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
-        const int ng = min(GPS, g1 - g);
-        const int s = it % STAGES;
-        const int b = it % NI8;
-        if (!wait2_warp(&full[s], (it / STAGES) & 1, &empty8[b], ((it / NI8) & 1) ^ 1, wp)) { ok = false; break; }
-        const uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
-        uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
-        if (Cfg::LR_MMA && g < g0) {
-          const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
-          build_lr_operands<Cfg>(args, tr * BM, tc * BN, dst, ut, NT);
+    } else {
+      constexpr int NT = 32 * Cfg::NUM_UNPACK_WARPS;
+      // This thread's tasks are the same at every stage: precompute their offsets.
+      // Task t -> operand (row tasks first), row, 16-byte chunk c of the row's
+      // 32*GPS packed bytes (c fastest, so 8 consecutive threads read 128
+      // contiguous bytes); group j = c/2, half = c%2.
+      uint32_t src_off[Cfg::TPT], dst_off[Cfg::TPT];
+      int grp[Cfg::TPT];
+      const int ut = (warp - 2) * 32 + lane;
+  #pragma unroll
+      for (int i = 0; i < Cfg::TPT; ++i) {
+        int t = ut + i * NT;
+        grp[i] = GPS;  // GPS = no task
+        src_off[i] = dst_off[i] = 0;
+        if (t < Cfg::TASKS) {
+          const bool colop = t >= 2 * GPS * BM;
+          if (colop) t -= 2 * GPS * BM;
+          const int row = t / (2 * GPS), c = t % (2 * GPS);
+          const int j = c >> 1, half = c & 1;
+          grp[i] = j;
+          src_off[i] = (colop ? Cfg::A_PACK : 0) + row * 32 * GPS + c * 16;
+          dst_off[i] = (colop ? GPS * Cfg::SA + j * Cfg::SB : j * Cfg::SA) + (row >> 3) * kSBO + 2 * half * kLBO +
+                       (row & 7) * 16;
+        }
+      }
+      uint32_t it = 0;
+      bool ok = true;
+      Unit un;
+      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+        const int g0 = un.g0, g1 = un.g1;
+        const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
+        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+          const int ng = min(GPS, g1 - g);
+          const int s = it % STAGES;
+          const int b = it % NI8;
+          if (!wait2_warp(&full[s], (it / STAGES) & 1, &empty8[b], ((it / NI8) & 1) ^ 1, wp)) { ok = false; break; }
+          const uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
+          uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
+          if (Cfg::LR_MMA && g < g0) {
+            const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
+            build_lr_operands<Cfg>(args, tr * BM, tc * BN, dst, ut, NT);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&full8[b]);
+              mbar_arrive(&empty[s]);
+            }
+            continue;
+          }
+          uint4 pk[Cfg::TPT];
+  #pragma unroll
+          for (int i = 0; i < Cfg::TPT; ++i)  // all loads first (always inside the stage)
+            pk[i] = *reinterpret_cast<const uint4*>(st + src_off[i]);
+          // with one group per stage and tasks filling every thread, no task test is needed
+          constexpr bool ALL_TASKS = GPS == 1 && Cfg::TASKS % NT == 0;
+  #pragma unroll
+          for (int i = 0; i < Cfg::TPT; ++i)
+            if (ALL_TASKS || grp[i] < ng) unpack16<Cfg::F8>(pk[i], dst + dst_off[i]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(&full8[b]);
             mbar_arrive(&empty[s]);
           }
-          continue;
-        }
-        uint4 pk[Cfg::TPT];
-#pragma unroll
-        for (int i = 0; i < Cfg::TPT; ++i)  // all loads first (always inside the stage)
-          pk[i] = *reinterpret_cast<const uint4*>(st + src_off[i]);
-        // with one group per stage and tasks filling every thread, no task test is needed
-        constexpr bool ALL_TASKS = GPS == 1 && Cfg::TASKS % NT == 0;
-#pragma unroll
-        for (int i = 0; i < Cfg::TPT; ++i)
-          if (ALL_TASKS || grp[i] < ng) unpack16<Cfg::F8>(pk[i], dst + dst_off[i]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&full8[b]);
-          mbar_arrive(&empty[s]);
         }
       }
     }

@@ -46,8 +46,11 @@ constexpr int kMaxRank = 32;
 #ifndef HSQ_LARGE_NTM
 #define HSQ_LARGE_NTM 2
 #endif
+#ifndef HSQ_LARGE_PRE
+#define HSQ_LARGE_PRE true  // operands expanded once per call; no unpack in the main loop
+#endif
 #ifndef HSQ_LARGE_UNPACK
-#define HSQ_LARGE_UNPACK 6
+#define HSQ_LARGE_UNPACK (HSQ_LARGE_PRE ? 2 : 6)
 #endif
 #ifndef HSQ_LR_MMA
 #define HSQ_LR_MMA 1  // U L2 + b as a tensor-core step where the kernel supports it
@@ -57,7 +60,7 @@ constexpr int kMaxRank = 32;
 #endif
 using CfgLarge = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, HSQ_LARGE_GPS, HSQ_LARGE_NI8,
                               HSQ_LARGE_NTM, HSQ_LARGE_UNPACK, HSQ_LARGE_STAGES + 4, HSQ_LARGE_F8,
-                              HSQ_LARGE_PIPE>;
+                              HSQ_LARGE_PIPE, HSQ_LARGE_PRE>;
 #ifndef HSQ_DEC_UNPACK_WARPS
 #define HSQ_DEC_UNPACK_WARPS 10
 #endif
@@ -137,7 +140,14 @@ struct Plan {
   int gps_stage;  // 64-groups per pipeline stage of the chosen kernel
   int tiles_r, tiles_c, stages_per_tile, stream_len, grid;
   size_t counters_bytes, partial_bytes;
-  size_t ws_bytes() const { return stream_len > 0 ? counters_bytes + partial_bytes : 0; }
+  // pre-expanded operands (large tiles with CfgLarge::PRE): 8-row groups and bytes
+  int rg_r, rg_c;
+  size_t pre_x_bytes, pre_w_bytes;
+  size_t split_bytes() const { return stream_len > 0 ? counters_bytes + partial_bytes : 0; }
+  // workspace: [stream-K counters][stream-K partials][expanded row operand][expanded col operand]
+  size_t pre_x_offset() const { return (split_bytes() + 255) / 256 * 256; }
+  size_t pre_w_offset() const { return pre_x_offset() + pre_x_bytes; }
+  size_t ws_bytes() const { return pre_x_bytes + pre_w_bytes > 0 ? pre_w_offset() + pre_w_bytes : split_bytes(); }
 };
 
 Plan make_plan(int M, int N, int K, int nsm) {
@@ -176,6 +186,12 @@ Plan make_plan(int M, int N, int K, int nsm) {
   }
   p.counters_bytes = ((static_cast<size_t>(tiles) * p.drain_warps * 4 + 255) / 256) * 256;
   p.partial_bytes = static_cast<size_t>(p.grid) * 2 * p.BN * 128 * 4;
+  if (p.kind == kLarge && CfgLarge::PRE) {
+    p.rg_r = p.tiles_r * (128 / 8);
+    p.rg_c = p.tiles_c * (CfgLarge::BN / 8);
+    p.pre_x_bytes = static_cast<size_t>(G) * p.rg_r * CfgLarge::E8_SBO;
+    p.pre_w_bytes = static_cast<size_t>(G) * p.rg_c * CfgLarge::E8_SBO;
+  }
   return p;
 }
 
@@ -407,6 +423,19 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   if (p.stream_len > 0) {
     a.ws_counters = static_cast<unsigned*>(workspace);
     a.ws_partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.counters_bytes);
+  }
+  if (p.pre_x_bytes > 0) {
+    // expand both code matrices into MMA-ready E4M3 tiles (rows padded to whole tiles)
+    uint8_t* xe = static_cast<uint8_t*>(workspace) + p.pre_x_offset();
+    uint8_t* we = static_cast<uint8_t*>(workspace) + p.pre_w_offset();
+    const int blocks = 4 * device_sm_count();
+    hsq::expand_e4m3_kernel<<<blocks, 256, 0, stream>>>(x_codes, M, Kp, p.rg_r * 8, xe);
+    hsq::expand_e4m3_kernel<<<blocks, 256, 0, stream>>>(w_codes, N, Kp, p.rg_c * 8, we);
+    if (cudaGetLastError() != cudaSuccess) return HSQ_ERR_CUDA;
+    a.xe = xe;
+    a.we = we;
+    a.rg_r = p.rg_r;
+    a.rg_c = p.rg_c;
   }
   // U L2 + b as a bf16 MMA step when the kernel has one and the rank fits its K
   a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge::LR_MMA && r <= CfgLarge::LR_MAX_RANK) ? 1 : 0;
