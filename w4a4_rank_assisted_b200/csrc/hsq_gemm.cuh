@@ -79,7 +79,7 @@ struct GemmArgs {
 };
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
-          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false>
+          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false, int CHB_ = 2>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -119,7 +119,7 @@ struct GemmCfg {
   static constexpr bool REALLOC = CW >= 128 || THREADS >= 768;
   static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8 * 8) > 255 ? 248 : (65536 / THREADS) / 8 * 8;
   static constexpr int LOW_THREADS = THREADS - 32 * NUM_DRAIN_WARPS;  // producer, MMA, unpack warpgroups
-  static constexpr int REGS_LOW = THREADS > 512 ? 40 : 64;
+  static constexpr int REGS_LOW = (THREADS <= 512 || LOW_THREADS <= 128) ? 64 : 40;
   static constexpr int REGS_HIGH_RAW =
       ((THREADS * LAUNCH_REGS - LOW_THREADS * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
   static constexpr int REGS_HIGH = REGS_HIGH_RAW > 232 ? 232 : REGS_HIGH_RAW;
@@ -157,9 +157,13 @@ struct GemmCfg {
   // with pre-expanded operands the low-rank operands get a buffer of their own
   static constexpr int LR_BYTES = (PRE && LR_MMA) ? (BM + BN) / 8 * LR_SBO : 0;
   static_assert(!PRE || (F8 && !SWAP && GPS == 1), "pre-expanded operands: E4M3, tokens x outputs, one group a stage");
+  // Tokens x outputs tiles write Y with TMA stores: each drain warp stages a
+  // 32-row x 128-byte box (128-byte swizzle) in its own 4 KB buffer.
+  static constexpr bool TMA_STORE = !SWAP;
+  static constexpr int YST_BYTES = TMA_STORE ? NUM_DRAIN_WARPS * 4096 : 0;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * SSLOTS + 2 * NI8E + 2 * NTM + 1 + 2;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NI8E * I8_BYTES + LR_BYTES +
-                                    SSLOTS * SSLOT_BYTES + NUM_BARS * 8 + 64;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + YST_BYTES + NI8E * I8_BYTES +
+                                    LR_BYTES + SSLOTS * SSLOT_BYTES + NUM_BARS * 8 + 64;
   // unpack tasks (16 packed bytes each) per stage, and per unpack thread
   static constexpr int TASKS = PRE ? 1 : 2 * GPS * (BM + BN);
   static constexpr int TPT = (TASKS + 32 * NUM_UNPACK_WARPS - 1) / (32 * NUM_UNPACK_WARPS);
@@ -167,8 +171,12 @@ struct GemmCfg {
   // chunk) when registers allow; with 4 drain warps per scheduler the warps
   // themselves hide the load latency.
   static constexpr bool PIPE = PIPE_ >= 0 ? PIPE_ != 0 : NUM_DRAIN_WARPS <= 8;
+  // 8-column blocks per TMEM load of the drain (2 or 4): one load and one wait
+  // cover 16 * CHB columns of both half quadrants
+  static constexpr int CHB = CHB_;
+  static_assert(CHB == 2 || CHB == 4, "drain chunk");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-  static_assert(CW % 16 == 0, "drain chunks");
+  static_assert(CW % (8 * CHB_) == 0, "drain chunks");
   static_assert(TMEM_NEED <= 512, "TMEM");
   static_assert(32 * GPS <= 256, "TMA box width");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -323,13 +331,14 @@ __device__ __forceinline__ bool next_unit(const GemmArgs& a, int k, Unit& u) {
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_row, const __grid_constant__ CUtensorMap tm_col,
-                     const GemmArgs args) {
+                     const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, CW = Cfg::CW, STAGES = Cfg::STAGES, GPS = Cfg::GPS;
   constexpr int NI8 = Cfg::NI8E, NTM = Cfg::NTM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint8_t* i8_base = smem + STAGES * Cfg::STAGE_BYTES;
+  uint8_t* ystage = smem + STAGES * Cfg::STAGE_BYTES;  // 1024-aligned (stage sizes are)
+  uint8_t* i8_base = ystage + Cfg::YST_BYTES;
   uint8_t* lr_buf = i8_base + NI8 * Cfg::I8_BYTES;  // low-rank operands (pre-expanded mode)
   uint8_t* sc_base = lr_buf + Cfg::LR_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sc_base + Cfg::SSLOTS * Cfg::SSLOT_BYTES);
@@ -640,7 +649,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // A column-scale pair then serves four rows, and the four threads of a quad
     // read four different pairs, so the per-group scale loads stay few.
     constexpr int NBLK = CW / 8;   // 8-column blocks of the slice
-    constexpr int NCC = CW / 16;   // 16-column chunks (one TMEM load per half quadrant)
+    constexpr int CHB = Cfg::CHB;  // blocks per chunk (one TMEM load per half quadrant)
+    constexpr int NCC = NBLK / CHB;  // chunks per group
     const uint32_t t_q = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
@@ -719,14 +729,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         // thread has issued, so the pipeline is one chunk deep: the loads of
         // chunk i+1 are in flight while chunk i is folded into the accumulators.
         const int nbt = ng * NCC;  // chunks in this stage
-        uint32_t vbuf[Cfg::PIPE ? 2 : 1][2][8];
-        auto issue = [&](int bi, uint32_t (&dst)[2][8]) {
+        uint32_t vbuf[Cfg::PIPE ? 2 : 1][2][4 * CHB];
+        auto issue = [&](int bi, uint32_t (&dst)[2][4 * CHB]) {
           const int j = bi / NCC, cc = bi % NCC;
-          const uint32_t col = static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + 16 * cc);
-          tmem_ld_q8(t_q + col, dst[0]);
-          tmem_ld_q8(t_q + (16u << 16) + col, dst[1]);
+          const uint32_t col = static_cast<uint32_t>((tb * GPS + j) * BN + h * CW + 8 * CHB * cc);
+          if constexpr (CHB == 2) {
+            tmem_ld_q8(t_q + col, dst[0]);
+            tmem_ld_q8(t_q + (16u << 16) + col, dst[1]);
+          } else {
+            tmem_ld_q16(t_q + col, dst[0]);
+            tmem_ld_q16(t_q + (16u << 16) + col, dst[1]);
+          }
         };
-        auto wait_chunk = [&](uint32_t (&dst)[2][8]) { tmem_ld_wait(dst[0], dst[1]); };
+        auto wait_chunk = [&](uint32_t (&dst)[2][4 * CHB]) { tmem_ld_wait(dst[0], dst[1]); };
         if constexpr (Cfg::PIPE) {
           issue(0, vbuf[0]);
           wait_chunk(vbuf[0]);
@@ -736,7 +751,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int bi = 0; bi < GPS * NCC; ++bi) {
           if (bi >= nbt) break;  // warp-uniform
           const int j = bi / NCC, cc = bi % NCC;
-          uint32_t(&cur)[2][8] = vbuf[Cfg::PIPE ? (bi & 1) : 0];
+          uint32_t(&cur)[2][4 * CHB] = vbuf[Cfg::PIPE ? (bi & 1) : 0];
           if constexpr (Cfg::PIPE) {
             if (bi + 1 < nbt) issue(bi + 1, vbuf[(bi + 1) & 1]);
           } else {
@@ -752,11 +767,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               rs2[i] = make_float2(rs, rs);
             }
           }
-          const float* cs = cs_stage + j * BN + h * CW + 16 * cc + 2 * qc;
+          const float* cs = cs_stage + j * BN + h * CW + 8 * CHB * cc + 2 * qc;
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
+          for (int kb = 0; kb < CHB; ++kb) {
             const float2 c2 = *reinterpret_cast<const float2*>(cs + 8 * kb);
-            const int b = 2 * cc + kb;
+            const int b = CHB * cc + kb;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const uint32_t u0 = cur[i >> 1][4 * kb + 2 * (i & 1)], u1 = cur[i >> 1][4 * kb + 2 * (i & 1) + 1];
@@ -826,7 +841,59 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (lane == 0) *counter = 0u;
       }
       // the accumulators already hold U L2 + b (added by the tile's first unit)
-      if (!Cfg::SWAP) {
+      if constexpr (Cfg::TMA_STORE) {
+        // Stage 32 rows x 128 bytes at a time in this warp's buffer, in the
+        // 128-byte swizzled layout (16-byte chunk c of row r at chunk c ^ (r % 8),
+        // so the quad-layout writes hit distinct banks), then one TMA store of
+        // that box; rows and columns outside Y are clipped by the TMA unit.
+        uint8_t* stg = ystage + dw * 4096;
+        const int y0 = tr * BM + q * 32;
+        const int x0 = tc * BN + h * CW;
+        if (!args.out_f32) {
+#pragma unroll
+          for (int pz = 0; pz < CW / 64; ++pz) {  // 8 blocks = 64 bf16 columns per box
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rl = qd + 8 * i;
+#pragma unroll
+              for (int kb = 0; kb < 8; ++kb) {
+                const __nv_bfloat162 v = __float22bfloat162_rn(acc2[i * NBLK + 8 * pz + kb]);
+                *reinterpret_cast<__nv_bfloat162*>(stg + rl * 128 + ((kb ^ (rl & 7)) << 4) + qc * 4) = v;
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && x0 + 64 * pz < args.N && y0 < args.M) {  // skip boxes wholly outside Y
+              tma_store_2d(&tm_y, stg, x0 + 64 * pz, y0);
+              bulk_commit_group();
+            }
+          }
+        } else {
+#pragma unroll
+          for (int pz = 0; pz < CW / 32; ++pz) {  // 4 blocks = 32 fp32 columns per box
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int rl = qd + 8 * i;
+#pragma unroll
+              for (int kb = 0; kb < 4; ++kb) {
+                const int c16 = 2 * kb + (qc >> 1);  // 16-byte chunk of the row
+                *reinterpret_cast<float2*>(stg + rl * 128 + ((c16 ^ (rl & 7)) << 4) + (qc & 1) * 8) =
+                    acc2[i * NBLK + 4 * pz + kb];
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && x0 + 32 * pz < args.N && y0 < args.M) {
+              tma_store_2d(&tm_y, stg, x0 + 32 * pz, y0);
+              bulk_commit_group();
+            }
+          }
+        }
+      } else if (!Cfg::SWAP) {
         // rows are tokens m, columns are output features n
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -865,6 +932,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
       }
     }
+    // the warp's TMA stores must be complete before the CTA's shared memory goes away
+    if (Cfg::TMA_STORE && lane == 0) bulk_wait_all();
   }
 
   // ------------------------------------------------------------ teardown

@@ -52,6 +52,9 @@ constexpr int kMaxRank = 32;
 #ifndef HSQ_LARGE_UNPACK
 #define HSQ_LARGE_UNPACK (HSQ_LARGE_PRE ? 2 : 6)
 #endif
+#ifndef HSQ_LARGE_CHB
+#define HSQ_LARGE_CHB 2  // 8-column blocks per TMEM load of the drain
+#endif
 #ifndef HSQ_LR_MMA
 #define HSQ_LR_MMA 1  // U L2 + b as a tensor-core step where the kernel supports it
 #endif
@@ -60,7 +63,7 @@ constexpr int kMaxRank = 32;
 #endif
 using CfgLarge = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, HSQ_LARGE_GPS, HSQ_LARGE_NI8,
                               HSQ_LARGE_NTM, HSQ_LARGE_UNPACK, HSQ_LARGE_STAGES + 4, HSQ_LARGE_F8,
-                              HSQ_LARGE_PIPE, HSQ_LARGE_PRE>;
+                              HSQ_LARGE_PIPE, HSQ_LARGE_PRE, HSQ_LARGE_CHB>;
 #ifndef HSQ_DEC_UNPACK_WARPS
 #define HSQ_DEC_UNPACK_WARPS 10
 #endif
@@ -225,9 +228,24 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Y [M][N] (bf16 or fp32) for the epilogue's TMA stores: boxes of 32 rows x
+// 128 bytes, 128-byte swizzle.
+bool make_y_map(CUtensorMap* map, void* Y, int M, int N, bool f32) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * es};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), 32u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class Cfg>
-hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& tc, const hsq::GemmArgs& a,
-                       cudaStream_t st) {
+hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& tc, const CUtensorMap& ty,
+                       const hsq::GemmArgs& a, cudaStream_t st) {
   static std::mutex mu;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -248,7 +266,7 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
   }
-  hsq::w4a4_gemm_kernel<Cfg><<<p.grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(tr, tc, a);
+  hsq::w4a4_gemm_kernel<Cfg><<<p.grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(tr, tc, ty, a);
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
@@ -411,6 +429,8 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     ok = make_codes_map(&tm_row, w_codes, N, Kp, 128, p.gps_stage) &&
          make_codes_map(&tm_col, x_codes, M, Kp, p.BN, p.gps_stage);
   }
+  CUtensorMap tm_y = tm_row;  // only the tokens x outputs kernel stores through a map
+  if (!p.swap) ok = make_y_map(&tm_y, Y, M, N, out == HSQ_OUT_F32);
   if (!ok) return HSQ_ERR_CUDA;
   a.U = U;
   a.L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
@@ -446,10 +466,10 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     t_debug_flags = 0;
   }
   switch (p.kind) {
-    case kLarge: return launch_gemm<CfgLarge>(p, tm_row, tm_col, a, stream);
-    case kDec16: return launch_gemm<CfgDec16>(p, tm_row, tm_col, a, stream);
-    case kDec32: return launch_gemm<CfgDec32>(p, tm_row, tm_col, a, stream);
-    case kDec64: return launch_gemm<CfgDec64>(p, tm_row, tm_col, a, stream);
+    case kLarge: return launch_gemm<CfgLarge>(p, tm_row, tm_col, tm_y, a, stream);
+    case kDec16: return launch_gemm<CfgDec16>(p, tm_row, tm_col, tm_y, a, stream);
+    case kDec32: return launch_gemm<CfgDec32>(p, tm_row, tm_col, tm_y, a, stream);
+    case kDec64: return launch_gemm<CfgDec64>(p, tm_row, tm_col, tm_y, a, stream);
   }
   return HSQ_ERR_INVALID_ARG;
 }
