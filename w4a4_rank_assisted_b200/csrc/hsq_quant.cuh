@@ -58,7 +58,14 @@ __device__ __forceinline__ int rint_small(float t) {
 }
 
 // Same result as quantize8, with the per-element divisions by the group scale
-// done as div_by_recip (one reciprocal per group).
+// done as one product and Markstein's correction against one reciprocal per
+// group.  With the scale in [2^-100, 2^100] no element needs the guarded
+// division: |v| <= 7 scale keeps the quotient and the remainder normal, and an
+// element below 2^-126 has a quotient below 2^-26, which rounds to code 0 either
+// way.  Nor does a code need clamping: scale = RN(absmax / 7) makes |v / scale|
+// at most 7 (1 + 2^-24), which rounds to 7.  The code's 4-bit two's complement
+// is read straight from the bits of t + 1.5 * 2^23 (its offset 0x4B400000 is a
+// multiple of 16).
 __device__ __forceinline__ uint32_t quantize8_fast(const float (&v)[8], float& scale) {
   float amax = 0.f;
 #pragma unroll
@@ -72,9 +79,9 @@ __device__ __forceinline__ uint32_t quantize8_fast(const float (&v)[8], float& s
     const float z = __frcp_rn(scale);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      int q = rint_small(div_by_recip(v[e], scale, z));
-      q = max(-7, min(7, q));
-      packed |= static_cast<uint32_t>(q & 0xF) << (4 * e);
+      const float q0 = __fmul_rn(v[e], z);
+      const float t = __fmaf_rn(__fmaf_rn(-q0, scale, v[e]), z, q0);
+      packed |= (static_cast<uint32_t>(__float_as_int(__fadd_rn(t, 12582912.0f))) & 0xFu) << (4 * e);
     }
   } else if (scale != 0.f) {
 #pragma unroll
@@ -228,8 +235,25 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
       if (m >= M) break;  // warp-uniform
       float x[8], xh[8];
       bf16x8_to_f32(xr[i], x);
+      // X_hat = x / s: product and correction (exact for normal operands and
+      // quotients, and for x = 0); the warp takes the guarded division only
+      // if some lane holds an element outside [2^-100, 2^100]
+      bool odd = false;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xh[e] = real ? div_by_recip(x[e], sv[e], sz[e]) : 0.f;
+      for (int e = 0; e < 8; ++e) {
+        const float ax = fabsf(x[e]);
+        odd |= (ax != 0.f) & ((ax < 0x1p-100f) | (ax > 0x1p100f));
+        const float q0 = __fmul_rn(x[e], sz[e]);
+        xh[e] = __fmaf_rn(__fmaf_rn(-q0, sv[e], x[e]), sz[e], q0);
+      }
+      if (__any_sync(0xffffffffu, odd)) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xh[e] = div_by_recip(x[e], sv[e], sz[e]);
+      }
+      if (!real) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xh[e] = 0.f;
+      }
       if constexpr (R > 0 && R <= 4) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
