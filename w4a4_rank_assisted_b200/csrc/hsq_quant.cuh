@@ -194,8 +194,26 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
 #pragma unroll
     for (int j = 0; j < RA; ++j) u[i][j] = 0.f;
 
+  // X rows of a chunk are loaded one chunk ahead, so their HBM latency overlaps
+  // the previous chunk's arithmetic
+  auto load_x = [&](int c, uint4 (&xr)[SUB]) {
+    const int k0 = c * 256 + lane * 8;
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      const int m = mb + i;
+      xr[i] = (c < nchunks && k0 < K && m < M)
+                  ? __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k0))
+                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 xnext[SUB];
+  load_x(warp / NSUB, xnext);
   for (int c = warp / NSUB; c < nchunks; c += NW / NSUB) {
     const int k0 = c * 256 + lane * 8;
+    uint4 xr[SUB];
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) xr[i] = xnext[i];
+    load_x(c + NW / NSUB, xnext);
     const bool real = k0 < K;  // K % 8 == 0: a lane's 8 channels are all real or all padding
     const bool in_k = k0 < Kp;
     float sv[8], sz[8];
@@ -221,13 +239,6 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
 #pragma unroll
         for (int t = 0; t < 8; ++t) l1s[(v * 8 + t) / R][(v * 8 + t) % R] = f[t];
       }
-    }
-    uint4 xr[SUB];
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) {
-      const int m = mb + i;
-      xr[i] = (real && m < M) ? __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k0))
-                              : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int i = 0; i < SUB; ++i) {
