@@ -193,6 +193,17 @@ __device__ __forceinline__ bool wait2_warp(uint64_t* a, uint32_t pa, uint64_t* b
   return true;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// The library's kernels are launched so that the next kernel in the stream may
+// start before this one ends.  grid_dep_wait() blocks the calling thread until
+// the preceding kernel has completed and its writes are visible (it returns at
+// once when there is none); every thread calls it before touching memory that
+// the preceding kernel may write.  grid_dep_launch() lets the next kernel launch;
+// a kernel calls it only after its own grid_dep_wait(), so that a kernel that
+// starts early always finds every kernel before its predecessor complete.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA / bulk copy
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(

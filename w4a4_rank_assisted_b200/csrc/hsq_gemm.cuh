@@ -219,6 +219,7 @@ __device__ __forceinline__ void unpack16(const uint4& p, uint8_t* dst) {
 // row); the eight threads of a row group write 128 contiguous bytes.
 __global__ void __launch_bounds__(256) expand_e4m3_kernel(const uint8_t* __restrict__ codes, int rows, int Kp,
                                                           int rows_pad, uint8_t* __restrict__ out) {
+  grid_dep_wait();  // the codes may come from the preceding kernel
   const size_t RG = static_cast<size_t>(rows_pad / 8);
   const size_t total = static_cast<size_t>(Kp / 64) * RG * 16;
   for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
@@ -233,6 +234,8 @@ __global__ void __launch_bounds__(256) expand_e4m3_kernel(const uint8_t* __restr
       p = __ldg(reinterpret_cast<const uint4*>(codes + static_cast<size_t>(row) * (Kp / 2) + g * 32 + half * 16));
     unpack16<true, 128>(p, out + (gr * 4 + 2 * half) * 128 + r8 * 16);
   }
+  // the next kernel (the GEMM, one CTA per SM) may launch once the blocks are done
+  if (threadIdx.x == 0) grid_dep_launch();
 }
 
 // Operands of the low-rank step for one tile (rows r0.. of tokens, columns c0..
@@ -397,6 +400,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // every warp but the producer reads or writes global memory only after the
+  // preceding kernel is complete (U, L2, bias, Y, the workspace)
+  if (warp != 0) grid_dep_wait();
 
   uint32_t issued = 0;  // producer: stages issued (for the teardown drain)
 
@@ -404,6 +410,24 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
     if (lane == 0 && !(args.debug_flags & 1)) {
+      // Weights x tokens tiles: the weight tiles of the first STAGES steps are
+      // requested before waiting for the preceding kernel (the packed weights
+      // are never written by the kernel just before this one: the packing
+      // kernel does not let its successor start early).  Their activation
+      // halves follow right after the wait, before anything that can give up.
+      uint32_t npre = 0;
+      if constexpr (Cfg::SWAP) {
+        Unit pu;
+        for (int k = 0; npre < static_cast<uint32_t>(STAGES) && next_unit<GPS>(args, k, pu); ++k) {
+          const int r0p = (pu.tile % args.tiles_r) * BM;
+          for (int g = pu.g0; g < pu.g1 && npre < static_cast<uint32_t>(STAGES); g += GPS, ++npre) {
+            mbar_arrive_expect_tx(&full[npre], Cfg::A_PACK + Cfg::B_PACK);
+            tma_load_2d(stage_base + npre * Cfg::STAGE_BYTES, &tm_row, &full[npre], g * 32, r0p);
+          }
+        }
+      }
+      grid_dep_wait();
+      grid_dep_launch();
       uint32_t it = 0;
       bool ok = true;
       Unit un;
@@ -444,8 +468,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             bulk_load(st + Cfg::A_E8, args.we + (static_cast<size_t>(g) * args.rg_c + tc * (BN / 8)) * Cfg::E8_SBO,
                       Cfg::B_E8, &full[s]);
           } else {
-            mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
-            tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
+            if (it >= npre) {
+              mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
+              tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
+            }
             tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * 32, c0);
           }
           mbar_arrive_expect_tx(&sfull[ss], ng * (cs_bytes + rs_bytes));

@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/hsq.h"
 #include "hsq_device.cuh"
@@ -101,6 +102,29 @@ hsq_status noalloc_scratch(void** out) {
   if (slot.err != cudaSuccess || !slot.ptr) return HSQ_ERR_CUDA;
   *out = slot.ptr;
   return HSQ_OK;
+}
+
+#ifndef HSQ_PDL
+#define HSQ_PDL 1  // launch with programmatic stream serialization (see grid_dep_wait)
+#endif
+
+// Launch `kernel` so that it may start while the preceding kernel in the stream
+// is still running; the kernel itself waits (grid_dep_wait) before touching
+// memory that kernel may write.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(bool allow, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (HSQ_PDL && allow) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 thread_local int t_debug_flags = 0;
@@ -266,7 +290,11 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
   }
-  hsq::w4a4_gemm_kernel<Cfg><<<p.grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(tr, tc, ty, a);
+  // decode tiles start early (their weight prefetch overlaps the activation
+  // step); the GPU-filling large tiles measured faster without an early start
+  if (launch_pdl(p.swap, hsq::w4a4_gemm_kernel<Cfg>, dim3(p.grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, tr, tc, ty, a) !=
+      cudaSuccess)
+    return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
@@ -368,10 +396,9 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   const int G = groups_of(K), Kp = G * kGroup, ld = scales_ld(M);
   const auto* X = static_cast<const __nv_bfloat16*>(X_bf16);
   const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
-#define HSQ_ACT_LAUNCH(RV, SM)                                                                     \
-  hsq::quantize_act_kernel<RV, SM><<<(M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB,      \
-                                     hsq::ActCfg<RV, SM>::NW * 32, 0, stream>>>(X, s, L1, M, K, r, Kp, ld, \
-                                                                                x_codes, x_scales, U)
+#define HSQ_ACT_LAUNCH(RV, SM)                                                                           \
+  lerr = launch_pdl(true, hsq::quantize_act_kernel<RV, SM>, dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB), \
+             dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U)
 #define HSQ_ACT_RANKS(SM)                   \
   switch (r) {                              \
     case 0: HSQ_ACT_LAUNCH(0, SM); break;   \
@@ -383,6 +410,7 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
     case 32: HSQ_ACT_LAUNCH(32, SM); break; \
     default: HSQ_ACT_LAUNCH(-1, SM); break; \
   }
+  cudaError_t lerr = cudaSuccess;
   // few rows: one block per sub-block with 32 warps spread over K; else 8 warps x 2 sub-blocks
   if (M <= 64) {
     HSQ_ACT_RANKS(true)
@@ -391,7 +419,7 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   }
 #undef HSQ_ACT_RANKS
 #undef HSQ_ACT_LAUNCH
-  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+  return (lerr == cudaSuccess && cudaGetLastError() == cudaSuccess) ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
 hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, const float* U, const uint8_t* w_codes,
@@ -449,9 +477,11 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     uint8_t* xe = static_cast<uint8_t*>(workspace) + p.pre_x_offset();
     uint8_t* we = static_cast<uint8_t*>(workspace) + p.pre_w_offset();
     const int blocks = 4 * device_sm_count();
-    hsq::expand_e4m3_kernel<<<blocks, 256, 0, stream>>>(x_codes, M, Kp, p.rg_r * 8, xe);
-    hsq::expand_e4m3_kernel<<<blocks, 256, 0, stream>>>(w_codes, N, Kp, p.rg_c * 8, we);
-    if (cudaGetLastError() != cudaSuccess) return HSQ_ERR_CUDA;
+    if (launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, x_codes, M, Kp, p.rg_r * 8,
+                   xe) != cudaSuccess ||
+        launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, w_codes, N, Kp, p.rg_c * 8,
+                   we) != cudaSuccess)
+      return HSQ_ERR_CUDA;
     a.xe = xe;
     a.we = we;
     a.rg_r = p.rg_r;

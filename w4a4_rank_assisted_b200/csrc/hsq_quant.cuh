@@ -180,6 +180,12 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
                         uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U) {
   using C = ActCfg<R, SMALL>;
   constexpr int SUB = C::SUB, NW = C::NW, RB = C::RB, NSUB = C::NSUB;
+  grid_dep_wait();  // X may come from the preceding kernel
+  // a grid of a few blocks lets the next kernel start right away (it runs on the
+  // idle SMs); a grid that fills the GPU lets it start only as blocks finish, so
+  // that early arrivals do not take SMs from this kernel's later blocks
+  const bool early = gridDim.x <= 64;
+  if (early && threadIdx.x == 0) grid_dep_launch();
   constexpr int RA = C::RMAX > 0 ? C::RMAX : 1;
   __shared__ float upart[R != 0 ? NW : 1][SUB][RA];
   const int warp = threadIdx.x >> 5;
@@ -307,6 +313,7 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
       }
     }
   }
+  if (!early && threadIdx.x == 0) grid_dep_launch();
   if constexpr (R != 0) {
 #pragma unroll
     for (int i = 0; i < SUB; ++i)
