@@ -9,15 +9,16 @@
  * Diffusion Transformers" (H-SVDQuant, arXiv 2610.11315):
  *   - Abstract: every weight is a low-bit residual plus a high-precision
  *     low-rank component; weights and activations are both 4-bit (W4A4).
- *   - Table 1 and Table 8 captions: quantization groups of 64 along K.
+ *   - Table 1 and Table 8 captions: quantization groups of 64 along K;
+ *     Table 3 and Table 4 captions: groups of 128 for the Qwen3-8B results.
  *   - rit.work blog, diagonal-scaling paragraph: the smoothing vector s moves
  *     range between activations and weights without changing the layer's
  *     full-precision map (X_hat R^T + X_hat L1 L2 = X W^T before quantizing).
  *
- * Quantizer (symmetric signed INT4, one fp32 scale per 64 values along K):
+ * Quantizer (symmetric signed INT4, one fp32 scale per group of `group` values along K):
  *   scale = fp32(absmax / 7); code = clamp(round_half_even(fp32(v / scale)), -7, 7);
  *   an all-zero group has scale 0 and codes 0.  K is zero-padded to
- *   Kp = 64 * ceil(K / 64).
+ *   Kp = group * ceil(K / group).
  *
  * Conventions shared by every call
  *   - Every data pointer is a DEVICE pointer owned by the caller; the library
@@ -26,7 +27,7 @@
  *   - Packed codes: row-major [rows][Kp/2] bytes; byte j of a row holds code
  *     2j in bits 0-3 and code 2j+1 in bits 4-7, 4-bit two's complement.
  *     Padded codes (k >= K) are 0.
- *   - Scales: group-major fp32 [G][ld] with G = ceil(K/64) and
+ *   - Scales: group-major fp32 [G][ld] with G = ceil(K/group) and
  *     ld = hsq_scales_ld(rows) = rows rounded up to a multiple of 4; entry
  *     [g][i] is the scale of group g of row i; entries i >= rows are written 0.
  *   - Calls are asynchronous on `stream`.  Arguments are validated on the host
@@ -34,7 +35,7 @@
  *   - Every wait inside a kernel is bounded; a kernel that gives up records
  *     HSQ_ERR_TIMEOUT in a device status word, which hsq_get_device_status()
  *     reports.
- *   - Supported: group == 64, 0 <= r <= 32, K % 8 == 0, N % 8 == 0,
+ *   - Supported: group == 64 or 128, 0 <= r <= 32, K % 8 == 0, N % 8 == 0,
  *     1 <= M, N, K <= 2^20.
  */
 #ifndef HSQ_H_
@@ -52,7 +53,7 @@ typedef enum {
   HSQ_OK = 0,
   HSQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, L1/L2 null with r > 0, ws too small */
   HSQ_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned */
-  HSQ_ERR_UNSUPPORTED = 3,   /* group != 64, r > 32, K or N not a multiple of 8 */
+  HSQ_ERR_UNSUPPORTED = 3,   /* group not 64 or 128, r > 32, K or N not a multiple of 8 */
   HSQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, tensor map) */
   HSQ_ERR_TIMEOUT = 5,       /* a kernel gave up waiting (reported by hsq_get_device_status) */
   HSQ_ERR_SCRATCH_LIMIT = 6  /* hsq_linear_forward_noalloc: shape needs more than HSQ_NOALLOC_SCRATCH_BYTES */
@@ -60,7 +61,7 @@ typedef enum {
 
 typedef enum { HSQ_OUT_BF16 = 0, HSQ_OUT_F32 = 1 } hsq_out_dtype;
 
-/* Number of 64-wide groups along K: ceil(K / group).  Returns 0 if group <= 0. */
+/* Number of groups along K: ceil(K / group).  Returns 0 if group <= 0. */
 int hsq_num_groups(int K, int group);
 
 /* Bytes of a packed code matrix with `rows` rows: rows * Kp / 2. */
@@ -73,10 +74,11 @@ int hsq_scales_ld(int rows);
 size_t hsq_scales_bytes(int rows, int K, int group);
 
 /*
- * Bytes of split-K scratch that hsq_linear_forward needs for this shape on the
- * current device (0 when the shape runs without split-K).  The caller zero-fills
- * the workspace once before its first use; every completed call leaves it
- * zero-filled again.
+ * Bytes of scratch that hsq_linear_forward needs for this shape on the current
+ * device, for either group size: split-K counters and partial tiles, and for
+ * M > 64 the two code matrices expanded to E4M3 bytes (0 when nothing is
+ * needed).  The caller zero-fills the workspace once before its first use;
+ * every completed call leaves the split-K counters zero again.
  */
 size_t hsq_workspace_bytes(int M, int N, int K, int r);
 
@@ -84,7 +86,7 @@ size_t hsq_workspace_bytes(int M, int N, int K, int r);
  * Offline weight packing (Abstract: low-bit residual + high-precision
  * low-rank part).  R[n,k] = fp32(W[n,k]*s[k] - sum_{j<r} L1[k,j]*L2[j,n]),
  * formed in fp64 with the sum taken for j = 0..r-1, each multiply and add
- * rounded separately; R is then quantized per 64-group of each row.
+ * rounded separately; R is then quantized per group of each row.
  *   W_bf16   [N][K] bf16        s   [K] fp32 (all > 0)
  *   L1_bf16  [K][r] bf16        L2_bf16 [r][N] bf16   (both NULL iff r == 0)
  *   w_codes  out [N][Kp/2] u8   w_scales out [G][hsq_scales_ld(N)] fp32
@@ -95,7 +97,7 @@ hsq_status hsq_pack_weights(const void* W_bf16, const float* s, const void* L1_b
 
 /*
  * Per-forward activation step (one fused kernel): X_hat = fp32(fp32(X)/s_k)
- * (rit.work blog: smoothing), its group-64 INT4 codes and scales, and the
+ * (rit.work blog: smoothing), its group-wise INT4 codes and scales, and the
  * low-rank down-projection U = X_hat L1 accumulated in fp32.
  *   X_bf16  [M][K] bf16          s [K] fp32        L1_bf16 [K][r] bf16 (NULL iff r == 0)
  *   x_codes out [M][Kp/2] u8     x_scales out [G][hsq_scales_ld(M)] fp32
@@ -146,15 +148,17 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
  * cudaFree synchronize the device and may fail under memory pressure).  For
  * them this call takes the same arguments as hsq_linear_forward minus
  * workspace/ws_bytes, and uses a file-scope device array of
- * HSQ_NOALLOC_SCRATCH_BYTES bytes for the split-K counters and partial tiles.
+ * HSQ_NOALLOC_SCRATCH_BYTES bytes for the scratch hsq_linear_forward would
+ * take from the workspace (split-K counters and partial tiles, expanded codes).
  * It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *
  *   - Inputs and outputs are still caller-owned device pointers, exactly as
  *     for hsq_linear_forward; the results are the same.
- *   - Shapes whose scratch need, hsq_workspace_bytes(M,N,K,r), exceeds
+ *   - Shapes whose scratch need for the given group exceeds
  *     HSQ_NOALLOC_SCRATCH_BYTES are rejected with HSQ_ERR_SCRATCH_LIMIT before
- *     anything is launched (split-K shapes with 128x256 tiles can need up to
- *     about 39 MB; the decode tiles, M <= 64, need at most about 10 MB).
+ *     anything is launched (M > 64 needs (M + N) * Kp bytes of expanded codes,
+ *     rows rounded up to whole tiles, plus any split-K scratch; the decode
+ *     tiles, M <= 64, need at most about 10 MB).
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any
  *     stream capture.

@@ -49,7 +49,7 @@ def check_y(Y_gpu: np.ndarray, Y_ref: np.ndarray, out_f32: bool, where: str = ""
     return (float(d.max()) / r if r > 0 else float(d.max())), r
 
 
-def oracle_layer(X, W, s, L1, L2, bias, rows=None):
+def oracle_layer(X, W, s, L1, L2, bias, rows=None, group=O.GROUP):
     """Oracle outputs for a layer given torch CPU tensors (bf16 / fp32).
     ``rows`` restricts the activation side to those token rows."""
     Xn = to_np(X)
@@ -59,9 +59,9 @@ def oracle_layer(X, W, s, L1, L2, bias, rows=None):
     L1n = None if L1 is None else to_np(L1)
     L2n = None if L2 is None else to_np(L2)
     bn = None if bias is None else to_np(bias)
-    wc, ws = O.pack_weights(Wn, sn, L1n, L2n)
-    xc, xs, U = O.quantize_act(Xn, sn, L1n)
-    Y = O.linear_forward(xc, xs, U, wc, ws, L2n, bn)
+    wc, ws = O.pack_weights(Wn, sn, L1n, L2n, group)
+    xc, xs, U = O.quantize_act(Xn, sn, L1n, group)
+    Y = O.linear_forward(xc, xs, U, wc, ws, L2n, bn, group)
     return dict(w_codes=wc, w_scales=ws, x_codes=xc, x_scales=xs, U=U, Y=Y)
 
 

@@ -19,15 +19,15 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _run_gpu(layer, out=hsq.HSQ_OUT_F32, X=None):
+def _run_gpu(layer, out=hsq.HSQ_OUT_F32, X=None, group=hsq.GROUP):
     X = layer.X if X is None else X
     M, K = X.shape
     N = layer.W.shape[0]
     r = layer.spec.r
     d = lambda t: None if t is None else t.to(DEV).contiguous()
     pl = hsq.PackedLinear(d(layer.W), d(layer.s), d(layer.L1) if r else None,
-                          d(layer.L2) if r else None, d(layer.bias))
-    act = hsq.ActBuffers(M, K, r, DEV)
+                          d(layer.L2) if r else None, d(layer.bias), group=group)
+    act = hsq.ActBuffers(M, K, r, DEV, group=group)
     Y = torch.empty((M, N), dtype=torch.float32 if out == hsq.HSQ_OUT_F32 else torch.bfloat16, device=DEV)
     ws = pl.workspace(M)
     hsq.forward(pl, d(X), act, Y, workspace=ws, out=out)
@@ -41,9 +41,9 @@ def _spec(M, K, N, r, seed=0, bias=True, act="outlier"):
                      seed=seed, bias=bias)
 
 
-def _check_all(layer, pl, act, Y, out_f32, where):
+def _check_all(layer, pl, act, Y, out_f32, where, group=hsq.GROUP):
     ref = oracle_layer(layer.X, layer.W, layer.s, layer.L1 if layer.spec.r else None,
-                       layer.L2 if layer.spec.r else None, layer.bias)
+                       layer.L2 if layer.spec.r else None, layer.bias, group=group)
     M, N = Y.shape
     # weights: bit-exact codes and scales (with the zero padding of the layout)
     assert np.array_equal(to_np(pl.w_codes), ref["w_codes"]), f"{where}: weight codes differ"
@@ -87,6 +87,31 @@ def test_layer_matches_oracle(M, K, N, r, out):
     layer = make_layer(_spec(M, K, N, r, seed=M + K + N + r))
     pl, act, Y, _ = _run_gpu(layer, out)
     _check_all(layer, pl, act, Y, out == hsq.HSQ_OUT_F32, f"{M}x{K}x{N} r{r}")
+
+
+# groups of 128 (the pages' Qwen3-8B setting): decode and large tiles, split-K,
+# K that pads the last group, the tensor-core and CUDA-core low-rank paths
+SHAPES_G128 = [
+    (1, 256, 128, 4),
+    (16, 4096, 1024, 4),     # stream-K decode tile
+    (17, 200, 264, 2),       # K = 200 pads to 256
+    (40, 640, 136, 32),
+    (64, 384, 520, 0),
+    (65, 1152, 256, 4),
+    (130, 320, 264, 15),
+    (200, 1024, 1160, 4),
+    (128, 2048, 1024, 4),    # large tile, split-K or whole tiles
+    (300, 640, 512, 32),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r", SHAPES_G128)
+@pytest.mark.parametrize("out", [hsq.HSQ_OUT_F32, hsq.HSQ_OUT_BF16])
+def test_layer_matches_oracle_groups_of_128(M, K, N, r, out):
+    layer = make_layer(_spec(M, K, N, r, seed=7 * M + K + N + r))
+    pl, act, Y, _ = _run_gpu(layer, out, group=128)
+    assert pl.w_scales.shape[0] == hsq.hsq_num_groups(K, 128)
+    _check_all(layer, pl, act, Y, out == hsq.HSQ_OUT_F32, f"g128 {M}x{K}x{N} r{r}", group=128)
 
 
 def test_strong_low_rank_branch_and_zero_bias():

@@ -318,3 +318,77 @@ def test_brute_force_tiny_layers():
                     y += U[m, j] * float(L2[j, n])
                 y += float(b[n])
                 assert Y[m, n] == pytest.approx(y, rel=1e-12, abs=1e-12)
+
+
+# ---------------------------------------------------------------- groups of 128
+# (Deflating the Hessian, Table 3 and Table 4 captions: the Qwen3-8B results use
+# groups of 128 along K.)
+def test_brute_force_quantizer_groups_of_128():
+    """Element-by-element restatement of the quantizer with 128-wide groups,
+    including a K that pads the last group."""
+    rng = np.random.default_rng(31)
+    for K in (128, 200, 256):
+        x = (rng.standard_normal((3, K)) * 3).astype(f32)
+        codes, sc = O.quantize_groups(x, 128)
+        assert codes.shape == (3, O.num_groups(K, 128) * 128)
+        for r in range(3):
+            for g in range(O.num_groups(K, 128)):
+                vals = [x[r, k] for k in range(g * 128, min(K, g * 128 + 128))]
+                amax = f32(0)
+                for v in vals:
+                    amax = max(amax, abs(v))
+                s = f32(amax / f32(7))
+                assert sc[r, g] == s
+                for i, v in enumerate(vals):
+                    t = f32(v / s)
+                    fl = np.floor(t)
+                    d = t - fl
+                    qq = fl + 1 if d > 0.5 else fl if d < 0.5 else (fl if fl % 2 == 0 else fl + 1)
+                    assert codes[r, g * 128 + i] == min(7, max(-7, int(qq)))
+            assert np.all(codes[r, K:] == 0)
+
+
+def test_groups_of_128_agree_with_64_when_halves_share_the_absmax():
+    """If both 64-halves of every 128-group have the same absmax, the two group
+    sizes give the same codes and the 128-group scale equals both 64-group
+    scales: a misplaced group boundary or a wrong group count breaks this."""
+    rng = np.random.default_rng(37)
+    x = (rng.standard_normal((4, 384)) * 2).astype(f32)
+    x = np.clip(x, -5, 5).astype(f32)
+    x[:, 0::64] = f32(6.5)  # the absmax of every 64-half, so also of every 128-group
+    c64, s64 = O.quantize_groups(x, 64)
+    c128, s128 = O.quantize_groups(x, 128)
+    assert np.array_equal(c64, c128)
+    assert np.array_equal(s128, s64[:, 0::2]) and np.array_equal(s128, s64[:, 1::2])
+    x[:, 64] = f32(6.6)  # now the second half of group 0 is larger: only that group changes
+    c64, s64 = O.quantize_groups(x, 64)
+    c128, s128 = O.quantize_groups(x, 128)
+    assert s128[0, 0] == f32(f32(6.6) / f32(7)) and s64[0, 0] == f32(f32(6.5) / f32(7))
+    assert np.array_equal(c128[:, 128:], c64[:, 128:])
+
+
+def test_brute_force_tiny_layers_groups_of_128():
+    """Tiny layers with 128-wide groups, every output by explicit loops."""
+    rng = np.random.default_rng(41)
+    for (M, N, K, r) in [(2, 3, 128, 0), (3, 2, 200, 2), (1, 4, 256, 4)]:
+        X = _bf16_round(rng.standard_normal((M, K)) * 2)
+        W = _bf16_round(rng.standard_normal((N, K)) * 0.02)
+        L1 = _bf16_round(rng.standard_normal((K, r)) * 0.1) if r else None
+        L2 = _bf16_round(rng.standard_normal((r, N)) * 0.1) if r else None
+        b = _bf16_round(rng.standard_normal(N))
+        s = np.exp(rng.uniform(-1, 1, K)).astype(f32)
+        wc, ws = O.pack_weights(W, s, L1, L2, 128)
+        xc, xs, U = O.quantize_act(X, s, L1, 128)
+        Y = O.linear_forward(xc, xs, U, wc, ws, L2, b, 128)
+        qx, qw = O.unpack_int4(xc), O.unpack_int4(wc)
+        assert xs.shape == (O.num_groups(K, 128), M) and ws.shape == (O.num_groups(K, 128), N)
+        for m in range(M):
+            for n in range(N):
+                y = 0.0
+                for k in range(qx.shape[1]):
+                    g = k // 128
+                    y += (float(xs[g, m]) * int(qx[m, k])) * (float(ws[g, n]) * int(qw[n, k]))
+                for j in range(r):
+                    y += U[m, j] * float(L2[j, n])
+                y += float(b[n])
+                assert Y[m, n] == pytest.approx(y, rel=1e-12, abs=1e-12)

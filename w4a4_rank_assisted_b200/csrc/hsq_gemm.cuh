@@ -79,7 +79,8 @@ struct GemmArgs {
 };
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
-          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false, int CHB_ = 2>
+          int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false, int CHB_ = 2,
+          int BPG_ = 1>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -87,7 +88,12 @@ struct GemmCfg {
   static constexpr int CW = BN / DH;           // columns per drain thread
   static constexpr int STAGES = STAGES_;
   static constexpr bool SWAP = SWAP_;
-  static constexpr int GPS = GPS_;             // 64-groups per pipeline stage
+  static constexpr int GPS = GPS_;             // scale groups per pipeline stage
+  // 64-wide K blocks per scale group: 1 for groups of 64, 2 for groups of 128.
+  // Codes move and multiply in 64-blocks (a block is two K = 32 MMAs); a group's
+  // blocks accumulate into one TMEM partial, which the drain rescales once.
+  static constexpr int BPG = BPG_;
+  static constexpr int BPS = GPS * BPG;        // 64-blocks per stage
   static constexpr int NI8 = NI8_;             // int8 operand buffers
   static constexpr int NTM = NTM_;             // TMEM partial buffers
   static constexpr int SSLOTS = SSLOTS_;       // scale ring slots (released by the drain)
@@ -104,8 +110,10 @@ struct GemmCfg {
   // the low-rank step's operands.
   static constexpr bool PRE = PRE_;
   static constexpr int E8_SBO = 512;  // pre-expanded tile: bytes per 8-row group (4 K-chunks of 8 rows x 16 B)
-  static constexpr int A_E8 = BM / 8 * E8_SBO;
-  static constexpr int B_E8 = BN / 8 * E8_SBO;
+  static constexpr int A_E8_BLK = BM / 8 * E8_SBO;  // one 64-block of a tile
+  static constexpr int B_E8_BLK = BN / 8 * E8_SBO;
+  static constexpr int A_E8 = BPG * A_E8_BLK;
+  static constexpr int B_E8 = BPG * B_E8_BLK;
   static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
   static constexpr int NUM_DRAIN_WARPS = 4 * DH;
   static constexpr int THREADS = 32 * (2 + NUM_UNPACK_WARPS + NUM_DRAIN_WARPS);
@@ -127,8 +135,8 @@ struct GemmCfg {
                 "register split exceeds the block's launch allocation");
   static_assert(LOW_THREADS % 128 == 0, "whole low warpgroups");
   static_assert((2 + NUM_UNPACK_WARPS) % 4 == 0, "drain warps start on a warpgroup boundary");
-  static constexpr int A_PACK = BM * 32 * GPS;  // packed bytes per stage (row operand)
-  static constexpr int B_PACK = BN * 32 * GPS;  // packed bytes per stage (col operand)
+  static constexpr int A_PACK = BM * 32 * BPS;  // packed bytes per stage (row operand)
+  static constexpr int B_PACK = BN * 32 * BPS;  // packed bytes per stage (col operand)
   static constexpr int CS_BYTES = BN * 4;       // col scales of one group
   static constexpr int RS_BYTES = BM * 4;       // row scales of one group
   // Packed stage: row tile then col tile (released by the unpack warps).  The
@@ -140,7 +148,7 @@ struct GemmCfg {
   static constexpr int SSLOT_BYTES = ((RS_OFF + GPS * RS_BYTES + 127) / 128) * 128;
   static constexpr int SA = i8_group_stride(BM);  // int8 bytes of one group, row operand
   static constexpr int SB = i8_group_stride(BN);  // int8 bytes of one group, col operand
-  static constexpr int I8_BYTES = ((GPS * (SA + SB) + 1023) / 1024) * 1024;
+  static constexpr int I8_BYTES = ((BPS * (SA + SB) + 1023) / 1024) * 1024;
   static constexpr int NI8E = PRE ? 0 : NI8;   // int8 buffers actually laid out
   static constexpr int TMEM_NEED = NTM * GPS * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
@@ -165,7 +173,7 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + YST_BYTES + NI8E * I8_BYTES +
                                     LR_BYTES + SSLOTS * SSLOT_BYTES + NUM_BARS * 8 + 64;
   // unpack tasks (16 packed bytes each) per stage, and per unpack thread
-  static constexpr int TASKS = PRE ? 1 : 2 * GPS * (BM + BN);
+  static constexpr int TASKS = PRE ? 1 : 2 * BPS * (BM + BN);
   static constexpr int TPT = (TASKS + 32 * NUM_UNPACK_WARPS - 1) / (32 * NUM_UNPACK_WARPS);
   // Drain software pipeline (next chunk's TMEM load in flight during the current
   // chunk) when registers allow; with 4 drain warps per scheduler the warps
@@ -178,7 +186,8 @@ struct GemmCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(CW % (8 * CHB_) == 0, "drain chunks");
   static_assert(TMEM_NEED <= 512, "TMEM");
-  static_assert(32 * GPS <= 256, "TMA box width");
+  static_assert(32 * BPS <= 256, "TMA box width");
+  static_assert(!PRE || GPS == 1, "pre-expanded operands: one group a stage");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -422,7 +431,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const int r0p = (pu.tile % args.tiles_r) * BM;
           for (int g = pu.g0; g < pu.g1 && npre < static_cast<uint32_t>(STAGES); g += GPS, ++npre) {
             mbar_arrive_expect_tx(&full[npre], Cfg::A_PACK + Cfg::B_PACK);
-            tma_load_2d(stage_base + npre * Cfg::STAGE_BYTES, &tm_row, &full[npre], g * 32, r0p);
+            tma_load_2d(stage_base + npre * Cfg::STAGE_BYTES, &tm_row, &full[npre], g * Cfg::BPG * 32, r0p);
           }
         }
       }
@@ -463,16 +472,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if constexpr (Cfg::PRE) {
             // MMA-ready E4M3 tiles: one contiguous block per operand
             mbar_arrive_expect_tx(&full[s], Cfg::A_E8 + Cfg::B_E8);
-            bulk_load(st, args.xe + (static_cast<size_t>(g) * args.rg_r + tr * (BM / 8)) * Cfg::E8_SBO, Cfg::A_E8,
-                      &full[s]);
-            bulk_load(st + Cfg::A_E8, args.we + (static_cast<size_t>(g) * args.rg_c + tc * (BN / 8)) * Cfg::E8_SBO,
-                      Cfg::B_E8, &full[s]);
+#pragma unroll
+            for (int b = 0; b < Cfg::BPG; ++b) {
+              const size_t blk = static_cast<size_t>(g) * Cfg::BPG + b;
+              bulk_load(st + b * Cfg::A_E8_BLK, args.xe + (blk * args.rg_r + tr * (BM / 8)) * Cfg::E8_SBO,
+                        Cfg::A_E8_BLK, &full[s]);
+              bulk_load(st + Cfg::A_E8 + b * Cfg::B_E8_BLK, args.we + (blk * args.rg_c + tc * (BN / 8)) * Cfg::E8_SBO,
+                        Cfg::B_E8_BLK, &full[s]);
+            }
           } else {
             if (it >= npre) {
               mbar_arrive_expect_tx(&full[s], Cfg::A_PACK + Cfg::B_PACK);
-              tma_load_2d(st, &tm_row, &full[s], g * 32, r0);
+              tma_load_2d(st, &tm_row, &full[s], g * Cfg::BPG * 32, r0);
             }
-            tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * 32, c0);
+            tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * Cfg::BPG * 32, c0);
           }
           mbar_arrive_expect_tx(&sfull[ss], ng * (cs_bytes + rs_bytes));
           for (int j = 0; j < ng; ++j) {
@@ -517,10 +530,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             ++nlr;
           } else {
             tc_fence_after();
-            const uint32_t abuf = smem_u32(stage_base + s * Cfg::STAGE_BYTES), bbuf = abuf + Cfg::A_E8;
-            mma_f8(d, smem_desc_kmajor(abuf, 128, Cfg::E8_SBO), smem_desc_kmajor(bbuf, 128, Cfg::E8_SBO), idesc, 0u);
-            mma_f8(d, smem_desc_kmajor(abuf + 256, 128, Cfg::E8_SBO), smem_desc_kmajor(bbuf + 256, 128, Cfg::E8_SBO),
-                   idesc, 1u);
+            const uint32_t stg = smem_u32(stage_base + s * Cfg::STAGE_BYTES);
+#pragma unroll
+            for (int b = 0; b < Cfg::BPG; ++b) {
+              const uint32_t abuf = stg + b * Cfg::A_E8_BLK, bbuf = stg + Cfg::A_E8 + b * Cfg::B_E8_BLK;
+              mma_f8(d, smem_desc_kmajor(abuf, 128, Cfg::E8_SBO), smem_desc_kmajor(bbuf, 128, Cfg::E8_SBO), idesc,
+                     b > 0 ? 1u : 0u);
+              mma_f8(d, smem_desc_kmajor(abuf + 256, 128, Cfg::E8_SBO),
+                     smem_desc_kmajor(bbuf + 256, 128, Cfg::E8_SBO), idesc, 1u);
+            }
           }
           mma_commit(&empty[s]);
           mma_commit(&tfull[tb]);
@@ -557,17 +575,22 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             continue;
           }
           for (int j = 0; j < ng; ++j) {
-            const uint32_t a_addr = buf + j * Cfg::SA;
-            const uint32_t b_addr = buf + GPS * Cfg::SA + j * Cfg::SB;
             const uint32_t d = tmem_base + static_cast<uint32_t>((tb * GPS + j) * BN);
-            if constexpr (Cfg::F8) {
-              mma_f8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
-              mma_f8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
-                     smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
-            } else {
-              mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, 0u);
-              mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
-                     smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+#pragma unroll
+            for (int bb = 0; bb < Cfg::BPG; ++bb) {
+              const int jb = j * Cfg::BPG + bb;  // 64-block within the stage
+              const uint32_t a_addr = buf + jb * Cfg::SA;
+              const uint32_t b_addr = buf + Cfg::BPS * Cfg::SA + jb * Cfg::SB;
+              const uint32_t acc0 = bb > 0 ? 1u : 0u;
+              if constexpr (Cfg::F8) {
+                mma_f8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, acc0);
+                mma_f8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
+                       smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+              } else {
+                mma_i8(d, smem_desc_kmajor(a_addr, kLBO, kSBO), smem_desc_kmajor(b_addr, kLBO, kSBO), idesc, acc0);
+                mma_i8(d, smem_desc_kmajor(a_addr + 2 * kLBO, kLBO, kSBO),
+                       smem_desc_kmajor(b_addr + 2 * kLBO, kLBO, kSBO), idesc, 1u);
+              }
             }
           }
           mma_commit(&empty8[b]);
@@ -599,8 +622,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       constexpr int NT = 32 * Cfg::NUM_UNPACK_WARPS;
       // This thread's tasks are the same at every stage: precompute their offsets.
       // Task t -> operand (row tasks first), row, 16-byte chunk c of the row's
-      // 32*GPS packed bytes (c fastest, so 8 consecutive threads read 128
-      // contiguous bytes); group j = c/2, half = c%2.
+      // 32*BPS packed bytes (c fastest, so 8 consecutive threads read 128
+      // contiguous bytes); 64-block jb = c/2, half = c%2, scale group jb/BPG.
       uint32_t src_off[Cfg::TPT], dst_off[Cfg::TPT];
       int grp[Cfg::TPT];
       const int ut = (warp - 2) * 32 + lane;
@@ -610,14 +633,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         grp[i] = GPS;  // GPS = no task
         src_off[i] = dst_off[i] = 0;
         if (t < Cfg::TASKS) {
-          const bool colop = t >= 2 * GPS * BM;
-          if (colop) t -= 2 * GPS * BM;
-          const int row = t / (2 * GPS), c = t % (2 * GPS);
-          const int j = c >> 1, half = c & 1;
-          grp[i] = j;
-          src_off[i] = (colop ? Cfg::A_PACK : 0) + row * 32 * GPS + c * 16;
-          dst_off[i] = (colop ? GPS * Cfg::SA + j * Cfg::SB : j * Cfg::SA) + (row >> 3) * kSBO + 2 * half * kLBO +
-                       (row & 7) * 16;
+          const bool colop = t >= 2 * Cfg::BPS * BM;
+          if (colop) t -= 2 * Cfg::BPS * BM;
+          const int row = t / (2 * Cfg::BPS), c = t % (2 * Cfg::BPS);
+          const int jb = c >> 1, half = c & 1;
+          grp[i] = jb / Cfg::BPG;
+          src_off[i] = (colop ? Cfg::A_PACK : 0) + row * 32 * Cfg::BPS + c * 16;
+          dst_off[i] = (colop ? Cfg::BPS * Cfg::SA + jb * Cfg::SB : jb * Cfg::SA) + (row >> 3) * kSBO +
+                       2 * half * kLBO + (row & 7) * 16;
         }
       }
       uint32_t it = 0;

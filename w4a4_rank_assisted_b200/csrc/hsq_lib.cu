@@ -19,63 +19,28 @@
 
 namespace {
 
-constexpr int kGroup = 64;
 constexpr int kMaxDim = 1 << 20;
 constexpr int kMaxRank = 32;
 
-// Kernel configurations (see hsq_gemm.cuh).
-//                           BN  DH STAGES SWAP  GPS NI8 NTM
-#ifndef HSQ_LARGE_DH
-#define HSQ_LARGE_DH 2
-#endif
-// M > 64: 128 tokens x 256 outputs per tile; HSQ_LARGE_DH column slices of drain warps
-#ifndef HSQ_LARGE_STAGES
-#define HSQ_LARGE_STAGES 6
-#endif
-#ifndef HSQ_LARGE_F8
-#define HSQ_LARGE_F8 true
-#endif
-#ifndef HSQ_LARGE_BN
-#define HSQ_LARGE_BN 256
-#endif
-#ifndef HSQ_LARGE_GPS
-#define HSQ_LARGE_GPS 1
-#endif
-#ifndef HSQ_LARGE_NI8
-#define HSQ_LARGE_NI8 3
-#endif
-#ifndef HSQ_LARGE_NTM
-#define HSQ_LARGE_NTM 2
-#endif
-#ifndef HSQ_LARGE_PRE
-#define HSQ_LARGE_PRE true  // operands expanded once per call; no unpack in the main loop
-#endif
-#ifndef HSQ_LARGE_UNPACK
-#define HSQ_LARGE_UNPACK (HSQ_LARGE_PRE ? 2 : 6)
-#endif
-#ifndef HSQ_LARGE_CHB
-#define HSQ_LARGE_CHB 2  // 8-column blocks per TMEM load of the drain
-#endif
+// Kernel configurations (hsq_gemm.cuh), for scale groups of 64 and of 128 along K.
+//   GemmCfg<BN, DH, STAGES, SWAP, GPS, NI8, NTM, UNPACK/helper warps, SSLOTS, E4M3, PIPE, PRE, CHB, BPG>
+// M > 64: 128 tokens x 256 outputs per tile, both operands pre-expanded to E4M3
+// tiles, 8 drain warps in two column slices, 2 warps building the low-rank step.
+using CfgLarge64 = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 2, 10, true, -1, true, 2, 1>;
+using CfgLarge128 = hsq::GemmCfg<256, 2, 3, false, 1, 3, 2, 2, 7, true, -1, true, 2, 2>;
+// M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; packed codes
+// unpacked in shared memory (the drain is light, so more warps unpack); four
+// 64-blocks per stage either way
+using CfgDec16_64 = hsq::GemmCfg<16, 1, 6, true, 4, 2, 4, 10>;
+using CfgDec32_64 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, 10>;
+using CfgDec64_64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
+using CfgDec16_128 = hsq::GemmCfg<16, 1, 6, true, 2, 2, 4, 10, 10, false, -1, false, 2, 2>;
+using CfgDec32_128 = hsq::GemmCfg<32, 1, 5, true, 2, 2, 2, 10, 9, false, -1, false, 2, 2>;
+using CfgDec64_128 = hsq::GemmCfg<64, 1, 8, true, 1, 2, 2, 6, 12, false, -1, false, 2, 2>;
+
 #ifndef HSQ_LR_MMA
 #define HSQ_LR_MMA 1  // U L2 + b as a tensor-core step where the kernel supports it
 #endif
-#ifndef HSQ_LARGE_PIPE
-#define HSQ_LARGE_PIPE -1
-#endif
-using CfgLarge = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_LARGE_STAGES, false, HSQ_LARGE_GPS, HSQ_LARGE_NI8,
-                              HSQ_LARGE_NTM, HSQ_LARGE_UNPACK, HSQ_LARGE_STAGES + 4, HSQ_LARGE_F8,
-                              HSQ_LARGE_PIPE, HSQ_LARGE_PRE, HSQ_LARGE_CHB>;
-#ifndef HSQ_DEC_UNPACK_WARPS
-#define HSQ_DEC_UNPACK_WARPS 10
-#endif
-// M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; the drain is light,
-// so more warps unpack
-#ifndef HSQ_DEC_STAGES
-#define HSQ_DEC_STAGES 6
-#endif
-using CfgDec16 = hsq::GemmCfg<16, 1, HSQ_DEC_STAGES, true, 4, 2, 4, HSQ_DEC_UNPACK_WARPS>;
-using CfgDec32 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, HSQ_DEC_UNPACK_WARPS>;
-using CfgDec64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
 
 // Scratch of hsq_linear_forward_noalloc (split-K counters, then partial tiles),
 // for callers that cannot provide a workspace.  In host code this name only
@@ -132,7 +97,7 @@ thread_local int t_debug_limit_ms = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int groups_of(int K) { return (K + kGroup - 1) / kGroup; }
+int groups_of(int K, int group) { return (K + group - 1) / group; }
 int scales_ld(int rows) { return (rows + 3) & ~3; }
 
 uint64_t wait_limit_ns() {
@@ -161,13 +126,15 @@ enum Kind { kLarge = 0, kDec16, kDec32, kDec64 };
 
 struct Plan {
   Kind kind;
+  int group;      // 64 or 128
   int BN;
   bool swap;
   int drain_warps;
-  int gps_stage;  // 64-groups per pipeline stage of the chosen kernel
+  int gps_stage;  // scale groups per pipeline stage of the chosen kernel
+  int bps_stage;  // 64-blocks per pipeline stage (the TMA box width / 32 bytes)
   int tiles_r, tiles_c, stages_per_tile, stream_len, grid;
   size_t counters_bytes, partial_bytes;
-  // pre-expanded operands (large tiles with CfgLarge::PRE): 8-row groups and bytes
+  // pre-expanded operands (large tiles): 8-row groups and bytes
   int rg_r, rg_c;
   size_t pre_x_bytes, pre_w_bytes;
   size_t split_bytes() const { return stream_len > 0 ? counters_bytes + partial_bytes : 0; }
@@ -177,25 +144,33 @@ struct Plan {
   size_t ws_bytes() const { return pre_x_bytes + pre_w_bytes > 0 ? pre_w_offset() + pre_w_bytes : split_bytes(); }
 };
 
-Plan make_plan(int M, int N, int K, int nsm) {
+template <class C>
+void plan_from(Plan& p) {
+  p.BN = C::BN;
+  p.gps_stage = C::GPS;
+  p.bps_stage = C::BPS;
+  p.drain_warps = C::NUM_DRAIN_WARPS;
+}
+
+Plan make_plan(int M, int N, int K, int group, int nsm) {
   Plan p{};
-  const int G = groups_of(K);
+  p.group = group;
+  const bool g128 = group == 128;
+  const int G = groups_of(K, group);
   if (M <= 64) {
     p.swap = true;
     p.kind = M <= 16 ? kDec16 : M <= 32 ? kDec32 : kDec64;
-    p.BN = M <= 16 ? CfgDec16::BN : M <= 32 ? CfgDec32::BN : CfgDec64::BN;
-    p.gps_stage = M <= 16 ? CfgDec16::GPS : M <= 32 ? CfgDec32::GPS : CfgDec64::GPS;
-    p.drain_warps = CfgDec16::NUM_DRAIN_WARPS;
+    if (p.kind == kDec16) g128 ? plan_from<CfgDec16_128>(p) : plan_from<CfgDec16_64>(p);
+    if (p.kind == kDec32) g128 ? plan_from<CfgDec32_128>(p) : plan_from<CfgDec32_64>(p);
+    if (p.kind == kDec64) g128 ? plan_from<CfgDec64_128>(p) : plan_from<CfgDec64_64>(p);
     p.tiles_r = (N + 127) / 128;
     p.tiles_c = (M + p.BN - 1) / p.BN;
   } else {
     p.swap = false;
     p.kind = kLarge;
-    p.BN = CfgLarge::BN;
-    p.gps_stage = CfgLarge::GPS;
-    p.drain_warps = CfgLarge::NUM_DRAIN_WARPS;
+    g128 ? plan_from<CfgLarge128>(p) : plan_from<CfgLarge64>(p);
     p.tiles_r = (M + 127) / 128;
-    p.tiles_c = (N + CfgLarge::BN - 1) / CfgLarge::BN;
+    p.tiles_c = (N + p.BN - 1) / p.BN;
   }
   const long tiles = static_cast<long>(p.tiles_r) * p.tiles_c;
   p.stages_per_tile = (G + p.gps_stage - 1) / p.gps_stage;
@@ -213,14 +188,16 @@ Plan make_plan(int M, int N, int K, int nsm) {
   }
   p.counters_bytes = ((static_cast<size_t>(tiles) * p.drain_warps * 4 + 255) / 256) * 256;
   p.partial_bytes = static_cast<size_t>(p.grid) * 2 * p.BN * 128 * 4;
-  if (p.kind == kLarge && CfgLarge::PRE) {
+  if (p.kind == kLarge) {  // both large configurations pre-expand their operands
+    const size_t blocks = static_cast<size_t>(G) * (group / 64);  // 64-wide K blocks
     p.rg_r = p.tiles_r * (128 / 8);
-    p.rg_c = p.tiles_c * (CfgLarge::BN / 8);
-    p.pre_x_bytes = static_cast<size_t>(G) * p.rg_r * CfgLarge::E8_SBO;
-    p.pre_w_bytes = static_cast<size_t>(G) * p.rg_c * CfgLarge::E8_SBO;
+    p.rg_c = p.tiles_c * (p.BN / 8);
+    p.pre_x_bytes = blocks * p.rg_r * CfgLarge64::E8_SBO;
+    p.pre_w_bytes = blocks * p.rg_c * CfgLarge64::E8_SBO;
   }
   return p;
 }
+static_assert(CfgLarge64::PRE && CfgLarge128::PRE && CfgLarge64::BN == CfgLarge128::BN, "large configurations");
 
 // ------------------------------------------------------------------ tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -321,7 +298,9 @@ size_t hsq_scales_bytes(int rows, int K, int group) {
 size_t hsq_workspace_bytes(int M, int N, int K, int r) {
   (void)r;
   if (M < 1 || N < 1 || K < 1) return 0;
-  return make_plan(M, N, K, device_sm_count()).ws_bytes();
+  // enough for either supported group size
+  const int nsm = device_sm_count();
+  return std::max(make_plan(M, N, K, 64, nsm).ws_bytes(), make_plan(M, N, K, 128, nsm).ws_bytes());
 }
 
 const char* hsq_status_string(hsq_status s) {
@@ -355,7 +334,7 @@ hsq_status hsq_get_device_status(cudaStream_t stream) {
 }
 
 static hsq_status check_common(int rows, int K, int r, int group) {
-  if (group != kGroup) return HSQ_ERR_UNSUPPORTED;
+  if (group != 64 && group != 128) return HSQ_ERR_UNSUPPORTED;
   if (rows < 1 || K < 1 || rows > kMaxDim || K > kMaxDim || r < 0) return HSQ_ERR_INVALID_ARG;
   if (r > kMaxRank || (K % 8) != 0) return HSQ_ERR_UNSUPPORTED;
   return HSQ_OK;
@@ -370,11 +349,16 @@ hsq_status hsq_pack_weights(const void* W_bf16, const float* s, const void* L1_b
   if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(w_codes) || !aligned16(w_scales) ||
       (L1_bf16 && !aligned16(L1_bf16)) || (L2_bf16 && !aligned16(L2_bf16)))
     return HSQ_ERR_ALIGNMENT;
-  const int G = groups_of(K), Kp = G * kGroup, ld = scales_ld(N);
+  const int G = groups_of(K, group), Kp = G * group, ld = scales_ld(N);
   const int blocks = (N + 7) / 8;
-  hsq::pack_weights_kernel<<<blocks, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(W_bf16), s, static_cast<const __nv_bfloat16*>(L1_bf16),
-      static_cast<const __nv_bfloat16*>(L2_bf16), N, K, r, Kp, ld, w_codes, w_scales);
+  if (group == 128)
+    hsq::pack_weights_kernel<16><<<blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(W_bf16), s, static_cast<const __nv_bfloat16*>(L1_bf16),
+        static_cast<const __nv_bfloat16*>(L2_bf16), N, K, r, Kp, ld, w_codes, w_scales);
+  else
+    hsq::pack_weights_kernel<8><<<blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(W_bf16), s, static_cast<const __nv_bfloat16*>(L1_bf16),
+        static_cast<const __nv_bfloat16*>(L2_bf16), N, K, r, Kp, ld, w_codes, w_scales);
   if (cudaGetLastError() != cudaSuccess) return HSQ_ERR_CUDA;
   if (ld > N) {
     const int n = (ld - N) * G;
@@ -393,12 +377,18 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(x_codes) || !aligned16(x_scales) ||
       (L1_bf16 && !aligned16(L1_bf16)) || (U && !aligned16(U)))
     return HSQ_ERR_ALIGNMENT;
-  const int G = groups_of(K), Kp = G * kGroup, ld = scales_ld(M);
+  const int G = groups_of(K, group), Kp = G * group, ld = scales_ld(M);
   const auto* X = static_cast<const __nv_bfloat16*>(X_bf16);
   const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
-#define HSQ_ACT_LAUNCH(RV, SM)                                                                           \
-  lerr = launch_pdl(true, hsq::quantize_act_kernel<RV, SM>, dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB), \
-             dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, x_codes, x_scales, U)
+#define HSQ_ACT_LAUNCH(RV, SM)                                                                              \
+  lerr = (group == 128 ? launch_pdl(true, hsq::quantize_act_kernel<RV, SM, 16>,                             \
+                                    dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),     \
+                                    dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, \
+                                    x_codes, x_scales, U)                                                  \
+                       : launch_pdl(true, hsq::quantize_act_kernel<RV, SM, 8>,                              \
+                                    dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),     \
+                                    dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, \
+                                    x_codes, x_scales, U))
 #define HSQ_ACT_RANKS(SM)                   \
   switch (r) {                              \
     case 0: HSQ_ACT_LAUNCH(0, SM); break;   \
@@ -438,8 +428,8 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
       (bias_bf16 && !aligned16(bias_bf16)) || (workspace && !aligned16(workspace)))
     return HSQ_ERR_ALIGNMENT;
 
-  const int G = groups_of(K), Kp = G * kGroup;
-  const Plan p = make_plan(M, N, K, device_sm_count());
+  const int G = groups_of(K, group), Kp = G * group;
+  const Plan p = make_plan(M, N, K, group, device_sm_count());
   if (p.ws_bytes() > 0 && (!workspace || ws_bytes < p.ws_bytes())) return HSQ_ERR_INVALID_ARG;
 
   hsq::GemmArgs a{};
@@ -449,13 +439,13 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   if (!p.swap) {
     a.scales_r = x_scales; a.ld_r = ldx; a.rows_r = M;
     a.scales_c = w_scales; a.ld_c = ldw; a.rows_c = N;
-    ok = make_codes_map(&tm_row, x_codes, M, Kp, 128, p.gps_stage) &&
-         make_codes_map(&tm_col, w_codes, N, Kp, p.BN, p.gps_stage);
+    ok = make_codes_map(&tm_row, x_codes, M, Kp, 128, p.bps_stage) &&
+         make_codes_map(&tm_col, w_codes, N, Kp, p.BN, p.bps_stage);
   } else {
     a.scales_r = w_scales; a.ld_r = ldw; a.rows_r = N;
     a.scales_c = x_scales; a.ld_c = ldx; a.rows_c = M;
-    ok = make_codes_map(&tm_row, w_codes, N, Kp, 128, p.gps_stage) &&
-         make_codes_map(&tm_col, x_codes, M, Kp, p.BN, p.gps_stage);
+    ok = make_codes_map(&tm_row, w_codes, N, Kp, 128, p.bps_stage) &&
+         make_codes_map(&tm_col, x_codes, M, Kp, p.BN, p.bps_stage);
   }
   CUtensorMap tm_y = tm_row;  // only the tokens x outputs kernel stores through a map
   if (!p.swap) ok = make_y_map(&tm_y, Y, M, N, out == HSQ_OUT_F32);
@@ -488,18 +478,28 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     a.rg_c = p.rg_c;
   }
   // U L2 + b as a bf16 MMA step when the kernel has one and the rank fits its K
-  a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge::LR_MMA && r <= CfgLarge::LR_MAX_RANK) ? 1 : 0;
+  a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge64::LR_MMA && CfgLarge128::LR_MMA &&
+              r <= CfgLarge64::LR_MAX_RANK) ? 1 : 0;
   a.limit_ns = wait_limit_ns();
   if (t_debug_flags) {
     a.debug_flags = t_debug_flags;
     a.limit_ns = static_cast<uint64_t>(t_debug_limit_ms > 0 ? t_debug_limit_ms : 50) * 1000000ull;
     t_debug_flags = 0;
   }
+  const bool g128 = group == 128;
   switch (p.kind) {
-    case kLarge: return launch_gemm<CfgLarge>(p, tm_row, tm_col, tm_y, a, stream);
-    case kDec16: return launch_gemm<CfgDec16>(p, tm_row, tm_col, tm_y, a, stream);
-    case kDec32: return launch_gemm<CfgDec32>(p, tm_row, tm_col, tm_y, a, stream);
-    case kDec64: return launch_gemm<CfgDec64>(p, tm_row, tm_col, tm_y, a, stream);
+    case kLarge:
+      return g128 ? launch_gemm<CfgLarge128>(p, tm_row, tm_col, tm_y, a, stream)
+                  : launch_gemm<CfgLarge64>(p, tm_row, tm_col, tm_y, a, stream);
+    case kDec16:
+      return g128 ? launch_gemm<CfgDec16_128>(p, tm_row, tm_col, tm_y, a, stream)
+                  : launch_gemm<CfgDec16_64>(p, tm_row, tm_col, tm_y, a, stream);
+    case kDec32:
+      return g128 ? launch_gemm<CfgDec32_128>(p, tm_row, tm_col, tm_y, a, stream)
+                  : launch_gemm<CfgDec32_64>(p, tm_row, tm_col, tm_y, a, stream);
+    case kDec64:
+      return g128 ? launch_gemm<CfgDec64_128>(p, tm_row, tm_col, tm_y, a, stream)
+                  : launch_gemm<CfgDec64_64>(p, tm_row, tm_col, tm_y, a, stream);
   }
   return HSQ_ERR_INVALID_ARG;
 }
@@ -521,7 +521,7 @@ hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_sca
       !aligned16(Y) || (U && !aligned16(U)) || (L2_bf16 && !aligned16(L2_bf16)) ||
       (bias_bf16 && !aligned16(bias_bf16)))
     return HSQ_ERR_ALIGNMENT;
-  const Plan p = make_plan(M, N, K, device_sm_count());
+  const Plan p = make_plan(M, N, K, group, device_sm_count());
   void* scratch = nullptr;
   if (p.ws_bytes() > 0) {
     if (p.ws_bytes() > kNoallocScratchBytes) return HSQ_ERR_SCRATCH_LIMIT;

@@ -2,27 +2,36 @@
 // fused per-forward activation step.
 //
 // Quantizer (Deflating the Hessian, Abstract: 4-bit weights and activations;
-// Table 1 caption: groups of 64 along K): symmetric signed INT4 with one fp32
-// scale per 64 values, scale = absmax / 7 (IEEE division), code =
-// round-half-even(v / scale) clamped to [-7, 7].  Both kernels give every lane
-// 8 consecutive K-elements, so one 64-group spans 8 adjacent lanes and its
-// absmax is a 3-step xor-shuffle reduction.
+// Table 1 caption: groups of 64 along K; Table 3 and Table 4 captions: groups of
+// 128 for the Qwen3-8B results): symmetric signed INT4 with one fp32 scale per
+// group, scale = absmax / 7 (IEEE division), code = round-half-even(v / scale)
+// clamped to [-7, 7].  Both kernels give every lane 8 consecutive K-elements, so
+// a group spans GL = group/8 adjacent lanes (8 or 16) and its absmax is a
+// log2(GL)-step xor-shuffle reduction.
 #pragma once
 
 #include "hsq_device.cuh"
 
 namespace hsq {
 
-// Quantize one lane's 8 values of a 64-group spread over 8 adjacent lanes.
-// Every lane of the warp must call this (it shuffles).  Returns the 8 codes
-// packed as 4 bytes (code e in bits 4e..4e+3) and the group's scale.
-__device__ __forceinline__ uint32_t quantize8(const float (&v)[8], float& scale) {
+// Absmax of a group spread over GL adjacent lanes (8 values each): GL = 8 for
+// groups of 64, 16 for groups of 128.  Every lane of the warp must call it.
+template <int GL>
+__device__ __forceinline__ float group_absmax(const float (&v)[8]) {
   float amax = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+#pragma unroll
+  for (int o = 1; o < GL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  return amax;
+}
+
+// Quantize one lane's 8 values of a group spread over GL adjacent lanes.
+// Every lane of the warp must call this (it shuffles).  Returns the 8 codes
+// packed as 4 bytes (code e in bits 4e..4e+3) and the group's scale.
+template <int GL>
+__device__ __forceinline__ uint32_t quantize8(const float (&v)[8], float& scale) {
+  const float amax = group_absmax<GL>(v);
   scale = __fdiv_rn(amax, 7.0f);
   uint32_t packed = 0;
   if (scale != 0.f) {
@@ -66,13 +75,9 @@ __device__ __forceinline__ int rint_small(float t) {
 // at most 7 (1 + 2^-24), which rounds to 7.  The code's 4-bit two's complement
 // is read straight from the bits of t + 1.5 * 2^23 (its offset 0x4B400000 is a
 // multiple of 16).
+template <int GL>
 __device__ __forceinline__ uint32_t quantize8_fast(const float (&v)[8], float& scale) {
-  float amax = 0.f;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  const float amax = group_absmax<GL>(v);
   scale = __fdiv_rn(amax, 7.0f);
   uint32_t packed = 0;
   if (scale >= 0x1p-100f && scale <= 0x1p100f) {
@@ -99,6 +104,7 @@ __device__ __forceinline__ uint32_t quantize8_fast(const float (&v)[8], float& s
 // the sum in fp64 for j = 0..r-1 with every multiply and add rounded on its own
 // (no fused multiply-add), then quantized.  One warp per output row n.
 // ---------------------------------------------------------------------------
+template <int GL>
 __global__ void __launch_bounds__(256) pack_weights_kernel(const __nv_bfloat16* __restrict__ W,
                                                            const float* __restrict__ s,
                                                            const __nv_bfloat16* __restrict__ L1,
@@ -133,10 +139,10 @@ __global__ void __launch_bounds__(256) pack_weights_kernel(const __nv_bfloat16* 
       for (int e = 0; e < 8; ++e) R[e] = 0.f;
     }
     float sc;
-    const uint32_t packed = quantize8(R, sc);
+    const uint32_t packed = quantize8<GL>(R, sc);
     if (k0 < Kp) {
       *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (Kp / 2) + k0 / 2) = packed;
-      if ((lane & 7) == 0) scales[static_cast<size_t>(k0 / 64) * ld + n] = sc;
+      if ((lane & (GL - 1)) == 0) scales[static_cast<size_t>(k0 / (8 * GL)) * ld + n] = sc;
     }
   }
 }
@@ -173,7 +179,7 @@ struct ActCfg {
   static constexpr int NSUB = RB / SUB;
 };
 
-template <int R, bool SMALL>
+template <int R, bool SMALL, int GL>
 __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
     quantize_act_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
                         const __nv_bfloat16* __restrict__ L1, int M, int K, int r, int Kp, int ld,
@@ -301,11 +307,11 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
         }
       }
       float sc;
-      const uint32_t packed = quantize8_fast(xh, sc);
+      const uint32_t packed = quantize8_fast<GL>(xh, sc);
       if (in_k) {
         *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
-        if ((lane & 7) == 0) {
-          float* srow = scales + static_cast<size_t>(k0 / 64) * ld;
+        if ((lane & (GL - 1)) == 0) {
+          float* srow = scales + static_cast<size_t>(k0 / (8 * GL)) * ld;
           srow[m] = sc;
           if (m == M - 1)
             for (int p = M; p < ld; ++p) srow[p] = 0.f;  // padding of the group-major layout

@@ -175,32 +175,32 @@ def hsq_debug_force_timeout(flags: int, limit_ms: int) -> None:
 
 
 # ---------------------------------------------------------------- buffers
-def alloc_codes(rows: int, K: int, device) -> torch.Tensor:
-    Kp = hsq_num_groups(K) * GROUP
+def alloc_codes(rows: int, K: int, device, group: int = GROUP) -> torch.Tensor:
+    Kp = hsq_num_groups(K, group) * group
     return torch.empty((rows, Kp // 2), dtype=torch.uint8, device=device)
 
 
-def alloc_scales(rows: int, K: int, device) -> torch.Tensor:
-    return torch.empty((hsq_num_groups(K), hsq_scales_ld(rows)), dtype=torch.float32, device=device)
+def alloc_scales(rows: int, K: int, device, group: int = GROUP) -> torch.Tensor:
+    return torch.empty((hsq_num_groups(K, group), hsq_scales_ld(rows)), dtype=torch.float32, device=device)
 
 
 class PackedLinear:
     """A packed layer: INT4 residual codes and scales plus the low-rank pair,
     the smoothing vector and the bias, all resident on one device."""
 
-    def __init__(self, W, s, L1, L2, bias=None, stream=None):
+    def __init__(self, W, s, L1, L2, bias=None, stream=None, group: int = GROUP):
         N, K = W.shape
         r = 0 if L1 is None else int(L1.shape[1])
         dev = W.device
-        self.N, self.K, self.r = N, K, r
+        self.N, self.K, self.r, self.group = N, K, r, group
         self.s = s.contiguous()
         self.L1 = None if r == 0 else L1.contiguous()
         self.L2 = None if r == 0 else L2.contiguous()
         self.bias = None if bias is None else bias.contiguous()
-        self.w_codes = alloc_codes(N, K, dev)
-        self.w_scales = alloc_scales(N, K, dev)
+        self.w_codes = alloc_codes(N, K, dev, group)
+        self.w_scales = alloc_scales(N, K, dev, group)
         hsq_pack_weights(W.contiguous(), self.s, self.L1, self.L2, N, K, r,
-                         self.w_codes, self.w_scales, stream=stream)
+                         self.w_codes, self.w_scales, group=group, stream=stream)
 
     def workspace(self, M: int) -> Optional[torch.Tensor]:
         n = hsq_workspace_bytes(M, self.N, self.K, self.r)
@@ -212,10 +212,10 @@ class PackedLinear:
 class ActBuffers:
     """Per-forward buffers of the activation step for M tokens."""
 
-    def __init__(self, M: int, K: int, r: int, device):
-        self.M, self.K, self.r = M, K, r
-        self.x_codes = alloc_codes(M, K, device)
-        self.x_scales = alloc_scales(M, K, device)
+    def __init__(self, M: int, K: int, r: int, device, group: int = GROUP):
+        self.M, self.K, self.r, self.group = M, K, r, group
+        self.x_codes = alloc_codes(M, K, device, group)
+        self.x_scales = alloc_scales(M, K, device, group)
         self.U = torch.empty((M, r), dtype=torch.float32, device=device) if r > 0 else None
 
 
@@ -223,10 +223,12 @@ def forward(layer: PackedLinear, X: torch.Tensor, act: ActBuffers, Y: torch.Tens
             workspace: Optional[torch.Tensor] = None, out: int = HSQ_OUT_BF16, stream=None) -> torch.Tensor:
     """One forward of the layer: the activation step, then the GEMM + epilogue."""
     M = X.shape[0]
+    if act.group != layer.group:
+        raise ValueError("activation buffers and packed layer use different group sizes")
     hsq_quantize_act(X, layer.s, layer.L1, M, layer.K, layer.r, act.x_codes, act.x_scales, act.U,
-                     stream=stream)
+                     group=layer.group, stream=stream)
     ws_bytes = 0 if workspace is None else workspace.numel()
     hsq_linear_forward(act.x_codes, act.x_scales, act.U, layer.w_codes, layer.w_scales, layer.L2,
                        layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace,
-                       ws_bytes=ws_bytes, stream=stream)
+                       ws_bytes=ws_bytes, group=layer.group, stream=stream)
     return Y
