@@ -62,7 +62,8 @@ def _fwd(lib, **kw):
 
 def test_forward_argument_validation():
     lib = hsq.load()
-    assert _fwd(lib, g=128) == hsq.HSQ_ERR_UNSUPPORTED
+    assert _fwd(lib, g=96) == hsq.HSQ_ERR_UNSUPPORTED
+    assert _fwd(lib, g=32) == hsq.HSQ_ERR_UNSUPPORTED
     assert _fwd(lib, r=33) == hsq.HSQ_ERR_UNSUPPORTED
     assert _fwd(lib, r=-1) == hsq.HSQ_ERR_INVALID_ARG
     assert _fwd(lib, K=100) == hsq.HSQ_ERR_UNSUPPORTED

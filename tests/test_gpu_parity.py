@@ -192,7 +192,7 @@ def test_invalid_arguments_launch_nothing():
     pl, act, Y, ws = _run_gpu(layer)
     with pytest.raises(hsq.HsqError) as e:
         hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, None,
-                               8, 64, 128, 4, Y, group=128)
+                               8, 64, 128, 4, Y, group=96)
     assert e.value.status == hsq.HSQ_ERR_UNSUPPORTED
     big = hsq.hsq_workspace_bytes(1, 4096, 12288, 4)
     with pytest.raises(hsq.HsqError) as e:
