@@ -60,18 +60,18 @@ def layer_ops(spec):
 
 def layer_gemm_bytes(spec):
     """Algorithmic HBM bytes of one hsq_linear_forward call (each operand once)."""
-    M, N, K, r = spec.M, spec.N, spec.K, spec.r
-    G = -(-K // 64)
-    Kp = 64 * G
+    M, N, K, r, gs = spec.M, spec.N, spec.K, spec.r, spec.group
+    G = -(-K // gs)
+    Kp = gs * G
     return (M * Kp // 2 + 4 * M * G + 4 * M * r      # x codes, scales, U
             + N * Kp // 2 + 4 * N * G + 2 * r * N    # w codes, scales, L2
             + 2 * M * N)                             # Y (bf16)
 
 
 def layer_act_bytes(spec):
-    M, K, r = spec.M, spec.K, spec.r
-    G = -(-K // 64)
-    return 2 * M * K + M * 64 * G // 2 + 4 * M * G + 4 * M * r + 4 * K + 2 * K * r
+    M, K, r, gs = spec.M, spec.K, spec.r, spec.group
+    G = -(-K // gs)
+    return 2 * M * K + M * gs * G // 2 + 4 * M * G + 4 * M * r + 4 * K + 2 * K * r
 
 
 class ClockSampler:
@@ -175,7 +175,7 @@ def oracle_timing(specs, budget_s: float = 12.0, seed_rows: int = 4):
         Wn, sn = lay.W.float().numpy(), lay.s.numpy()
         L1n = lay.L1.float().numpy() if spec.r else None
         L2n = lay.L2.float().numpy() if spec.r else None
-        wc, ws = O.pack_weights(Wn, sn, L1n, L2n)
+        wc, ws = O.pack_weights(Wn, sn, L1n, L2n, spec.group)
         packed.append((spec, lay.X.float().numpy(), sn, L1n, L2n, wc, ws))
 
     def run(rows):
@@ -183,8 +183,8 @@ def oracle_timing(specs, budget_s: float = 12.0, seed_rows: int = 4):
         ops = 0
         for spec, X, sn, L1n, L2n, wc, ws in packed:
             m = min(rows, spec.M)
-            xc, xs, U = O.quantize_act(X[:m], sn, L1n)
-            O.linear_forward(xc, xs, U, wc, ws, L2n, None)
+            xc, xs, U = O.quantize_act(X[:m], sn, L1n, spec.group)
+            O.linear_forward(xc, xs, U, wc, ws, L2n, None, spec.group)
             ops += layer_ops(spec) * m / spec.M
         return time.perf_counter() - t0, ops
 
@@ -234,9 +234,9 @@ def run_gpu(args, specs, wl_name, rank, world, local):
         lay = make_layer(spec)
         d = lambda t: None if t is None else t.to(dev).contiguous()
         pl = hsq.PackedLinear(d(lay.W), d(lay.s), d(lay.L1) if spec.r else None,
-                              d(lay.L2) if spec.r else None, None)
+                              d(lay.L2) if spec.r else None, None, group=spec.group)
         X = d(lay.X)
-        act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev)
+        act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
         Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
         ws = pl.workspace(spec.M)
         X_host = lay.X.pin_memory()
@@ -249,14 +249,14 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     def launch_act(L, st):
         s = L["spec"]
         hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
-                             L["act"].x_scales, L["act"].U, stream=st)
+                             L["act"].x_scales, L["act"].U, group=s.group, stream=st)
 
     def launch_gemm(L, st):
         s = L["spec"]
         hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
                                L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
                                workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
-                               stream=st)
+                               group=s.group, stream=st)
 
     def step(st):
         for L in layers:
@@ -426,7 +426,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes on i8/e4m3 tensor cores, f32 accumulate",
             "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",
             "config": {"workload": wl_name, "layers": [s.name for s in specs], "tokens_per_step": tokens_step,
-                       "r": specs[0].r, "group": 64, "parallelism": f"replicas x{world}",
+                       "r": specs[0].r, "group": specs[0].group, "parallelism": f"replicas x{world}",
                        "l2": (f"L2 flushed (256 MiB write) before every step and every timed kernel; flush "
                               f"time measured alone and subtracted; working set {ws_bytes / 2**20:.0f} MiB"
                               if flush else
