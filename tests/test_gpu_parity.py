@@ -75,8 +75,9 @@ SMALL_SHAPES = [
     (300, 640, 512, 32),
     (16, 4096, 2048, 4),     # stream-K, decode tile
     (128, 2048, 1024, 4),    # stream-K, large tile
-    (130, 320, 264, 15),     # largest rank of the tensor-core low-rank step
-    (97, 192, 136, 16),      # smallest rank past it (CUDA-core low-rank term)
+    (130, 320, 264, 15),     # largest rank of one tensor-core low-rank step
+    (97, 192, 136, 16),      # two low-rank steps
+    (96, 256, 200, 31),      # three low-rank steps, the last with one rank
     (129, 128, 256, 0),      # no low-rank pair: the step carries the bias alone
 ]
 

@@ -72,7 +72,7 @@ struct GemmArgs {
   unsigned* ws_counters;  // stream-K arrival counters per (tile, drain warp), zero between calls
   uint64_t limit_ns;      // wait limit
   int debug_flags;        // 1: producer issues nothing (forces the timeout path)
-  int lr_mma;             // 1: a tile's first unit starts with the low-rank step (kernels with LR_MMA)
+  int lr_mma;             // low-rank steps that start a tile's first unit (kernels with LR_MMA; 0: none)
   const uint8_t* xe;      // pre-expanded row operand (kernels with PRE): [G][rg_r][4][8][16] E4M3
   const uint8_t* we;      // pre-expanded col operand: [G][rg_c][4][8][16]
   int rg_r, rg_c;         // 8-row groups of each (rows padded to whole tiles)
@@ -153,10 +153,11 @@ struct GemmCfg {
   static constexpr int TMEM_NEED = NTM * GPS * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                  : TMEM_NEED <= 256 ? 256 : 512;
-  // Low-rank step (tokens x outputs tiles with E4M3 operands): U L2 + b enters
-  // a tile's accumulators as one extra pipeline step ahead of its groups, a
-  // bf16 MMA over an augmented K of LR_K = 32 (hi and lo bf16 parts of U
-  // against L2 twice, then ones against the bias), so that r <= LR_MAX_RANK.
+  // Low-rank steps (tokens x outputs tiles with E4M3 operands): U L2 + b enters
+  // a tile's accumulators as extra pipeline steps ahead of its groups, each a
+  // bf16 MMA over an augmented K of LR_K = 32 covering LR_MAX_RANK ranks (hi and
+  // lo bf16 parts of U against L2 twice) and, in the first step, ones against
+  // the bias.
   static constexpr bool LR_MMA = F8 && !SWAP && GPS == 1;
   static constexpr int LR_K = 32;
   static constexpr int LR_MAX_RANK = (LR_K - 2) / 2;
@@ -256,7 +257,8 @@ __global__ void __launch_bounds__(256) expand_e4m3_kernel(const uint8_t* __restr
 // outside the matrices and unused K are zero.  Threads t0, t0 + nt, ... each
 // build whole rows.
 template <class Cfg>
-__device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int c0, uint8_t* dst, int t0, int nt) {
+__device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int c0, int chunk, uint8_t* dst, int t0,
+                                                  int nt) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, K = Cfg::LR_K;
   for (int t = t0; t < BM + BN; t += nt) {
     const bool rowop = t < BM;
@@ -272,8 +274,8 @@ __device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int
       if (valid) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = 4 * c + e;
-          if (i < a.r && i < Cfg::LR_MAX_RANK) {
+          const int i = Cfg::LR_MAX_RANK * chunk + 4 * c + e;  // rank
+          if (4 * c + e < Cfg::LR_MAX_RANK && i < a.r) {
             if (rowop) {
               const float v = __ldg(a.U + static_cast<size_t>(idx) * a.r + i);
               f[2 * e] = __bfloat162float(__float2bfloat16_rn(v));
@@ -285,7 +287,7 @@ __device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int
             }
           }
         }
-        if (c == K / 8 - 1)  // element K-2: ones against the bias
+        if (c == K / 8 - 1 && chunk == 0)  // element K-2 of the first chunk: ones against the bias
           f[6] = rowop ? 1.f : (a.bias ? __bfloat162float(a.bias[idx]) : 0.f);
       }
       uint4 w;
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const uint32_t cs_bytes = static_cast<uint32_t>(min(BN, args.ld_c - c0)) * 4u;
         const uint32_t rs_bytes = static_cast<uint32_t>(min(BM, args.ld_r - r0)) * 4u;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
-        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+        for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
           const int s = it % STAGES;
           const int ss = it % Cfg::SSLOTS;
@@ -511,7 +513,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
-        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+        for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
           const int s = it % STAGES;
           const int tb = it % NTM;
           if (!wait_one(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
@@ -553,7 +555,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
-        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+        for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
           const int b = it % NI8D;
           const int tb = it % NTM;
@@ -610,13 +612,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       Unit un;
       for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
         if (!(Cfg::LR_MMA && args.lr_mma && un.g0 == 0)) continue;
-        if (!wait_warp(lrempty, (nlr & 1) ^ 1, wp)) { ok = false; break; }
         const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
-        build_lr_operands<Cfg>(args, tr * BM, tc * BN, lr_buf, ut, 32 * Cfg::NUM_UNPACK_WARPS);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(lrfull);
-        ++nlr;
+        for (int chunk = 0; chunk < args.lr_mma; ++chunk) {
+          if (!wait_warp(lrempty, (nlr & 1) ^ 1, wp)) { ok = false; break; }
+          // chunks as constants, so that each build unrolls over a fixed rank range
+          constexpr int LT = 32 * Cfg::NUM_UNPACK_WARPS;
+          if (chunk == 0) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 0, lr_buf, ut, LT);
+          else if (chunk == 1) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 1, lr_buf, ut, LT);
+          else build_lr_operands<Cfg>(args, tr * BM, tc * BN, 2, lr_buf, ut, LT);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(lrfull);
+          ++nlr;
+        }
       }
     } else {
       constexpr int NT = 32 * Cfg::NUM_UNPACK_WARPS;
@@ -649,7 +657,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
-        for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+        for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
           const int s = it % STAGES;
           const int b = it % NI8;
@@ -658,7 +666,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint8_t* dst = i8_base + b * Cfg::I8_BYTES;
           if (Cfg::LR_MMA && g < g0) {
             const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
-            build_lr_operands<Cfg>(args, tr * BM, tc * BN, dst, ut, NT);
+            const int chunk = (g - (g0 - GPS * args.lr_mma)) / GPS;
+            if (chunk == 0) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 0, dst, ut, NT);
+            else if (chunk == 1) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 1, dst, ut, NT);
+            else build_lr_operands<Cfg>(args, tr * BM, tc * BN, 2, dst, ut, NT);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -765,7 +776,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         }
       }
-      for (int g = lr_unit ? g0 - GPS : g0; g < g1; g += GPS, ++it) {
+      for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
         const int ng = GPS == 1 ? 1 : min(GPS, g1 - g);
         const int ss = it % Cfg::SSLOTS;
         const int tb = it % NTM;

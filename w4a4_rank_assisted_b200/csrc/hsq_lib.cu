@@ -478,8 +478,13 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     a.rg_c = p.rg_c;
   }
   // U L2 + b as a bf16 MMA step when the kernel has one and the rank fits its K
-  a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge64::LR_MMA && CfgLarge128::LR_MMA &&
-              r <= CfgLarge64::LR_MAX_RANK) ? 1 : 0;
+  // U L2 + b as tensor-core steps of LR_MAX_RANK ranks each (at least one: the bias)
+  static_assert(CfgLarge64::LR_MAX_RANK == CfgLarge128::LR_MAX_RANK, "low-rank chunk");
+  // (at most three steps: r <= 32 < 3 * LR_MAX_RANK; the kernel builds chunks 0..2)
+  static_assert(kMaxRank <= 3 * CfgLarge64::LR_MAX_RANK, "low-rank steps");
+  a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge64::LR_MMA && CfgLarge128::LR_MMA)
+                 ? std::max(1, (r + CfgLarge64::LR_MAX_RANK - 1) / CfgLarge64::LR_MAX_RANK)
+                 : 0;
   a.limit_ns = wait_limit_ns();
   if (t_debug_flags) {
     a.debug_flags = t_debug_flags;
