@@ -79,6 +79,10 @@ SMALL_SHAPES = [
     (97, 192, 136, 16),      # two low-rank steps
     (96, 256, 200, 31),      # three low-rank steps, the last with one rank
     (129, 128, 256, 0),      # no low-rank pair: the step carries the bias alone
+    (70, 200, 136, 8),       # rank 8: eight L1 rows per warp load, chunk of 200 channels
+    (40, 328, 264, 8),       # few rows, rank 8, ragged last chunk
+    (33, 328, 128, 7),       # generic odd rank, few rows
+    (150, 584, 136, 5),      # generic odd rank, ragged rows and last chunk
 ]
 
 

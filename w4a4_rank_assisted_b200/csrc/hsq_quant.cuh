@@ -161,22 +161,37 @@ __global__ void zero_scale_pad_kernel(float* scales, int rows, int ld, int G) {
 // A block of NW warps owns RB consecutive token rows, split into sub-blocks of
 // SUB rows.  Warp w works on sub-block w % (RB/SUB) and on the 256-wide K chunks
 // w / (RB/SUB), + NW/(RB/SUB), ...  Per chunk a lane loads the smoothing factors
-// and the L1 rows of its 8 channels once (16-byte loads) and reuses them for the
-// SUB rows, whose X loads are issued together.  U is reduced across lanes with
-// shuffles and across warps through shared memory in a fixed order, so the
-// result does not depend on scheduling.  Small M uses NW = 32 warps on one
-// sub-block so that K is spread over the whole block.
+// of its 8 channels once and reuses them for the SUB rows, whose X loads are
+// issued together (one chunk ahead).
+//
+// U = X_hat L1 takes one of two forms.  Ranks up to 4: a lane keeps the L1 rows
+// of its 8 channels in registers and accumulates all r columns.  Ranks of 8 and
+// more: the warp parks its SUB rows of X_hat in shared memory, and the lanes are
+// regrouped so that lane (kq, p) owns the rank pair (2p, 2p+1) of the channels
+// kq, kq + KP, kq + 2 KP, ... of the chunk; each L1 load of the warp is then one
+// contiguous run of KP rows of L1, applied to the SUB rows with packed fp32 FMAs.
+// U is reduced across lanes with shuffles and across warps through shared
+// memory in a fixed order, so the result does not depend on scheduling.  Small
+// M uses NW = 16 warps on one sub-block so that K is spread over the whole block.
 //
 // R is the rank as a compile-time constant (1, 2, 4, 8, 16, 32, or 0 for no
-// branch); R = -1 is the generic path for any other r <= 32 (scalar L1 loads).
+// branch); R = -1 is the generic path for any other r <= 32 (two 2-byte L1 loads
+// per rank pair).
 // ---------------------------------------------------------------------------
 template <int R, bool SMALL>
 struct ActCfg {
   static constexpr int RMAX = R < 0 ? 32 : R;  // accumulator width
-  static constexpr int SUB = (SMALL || R < 0 || R == 32) ? 2 : 4;
+  static constexpr int SUB = SMALL ? 2 : 4;
   static constexpr int NW = SMALL ? 16 : 8;
   static constexpr int RB = SMALL ? SUB : 2 * SUB;
   static constexpr int NSUB = RB / SUB;
+  // ranks of 8 and more: X_hat through shared memory, lanes over rank pairs
+  static constexpr bool PAIRS = R >= 8 || R < 0;
+  static constexpr int LPR = PAIRS ? RMAX / 2 : 1;  // lanes on one L1 row (one rank pair each)
+  static constexpr int KP = PAIRS ? 32 / LPR : 1;  // L1 rows per warp load
+  static constexpr int KS = 256 / KP;        // channels of one residue class in a chunk
+  static constexpr int KSP = KS + 4;         // padded: the KP classes start on different banks
+  static constexpr int XS_FLOATS = PAIRS ? NW * SUB * KP * KSP : 1;
 };
 
 template <int R, bool SMALL, int GL>
@@ -193,18 +208,26 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
   const bool early = gridDim.x <= 64;
   if (early && threadIdx.x == 0) grid_dep_launch();
   constexpr int RA = C::RMAX > 0 ? C::RMAX : 1;
+  constexpr bool PAIRS = C::PAIRS;
+  constexpr int KP = C::KP, KS = C::KS, KSP = C::KSP, LPR = C::LPR;
   __shared__ float upart[R != 0 ? NW : 1][SUB][RA];
+  __shared__ __align__(16) float xs_all[C::XS_FLOATS];
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
   const int sb = warp % NSUB;
   const int mb = blockIdx.x * RB + sb * SUB;  // first row of this warp's sub-block
   const int nchunks = (Kp + 255) / 256;
 
-  float u[SUB][RA];
+  float u[SUB][PAIRS ? 1 : RA];
+  float2 u2[PAIRS ? SUB : 1];
 #pragma unroll
-  for (int i = 0; i < SUB; ++i)
+  for (int i = 0; i < SUB; ++i) {
 #pragma unroll
-    for (int j = 0; j < RA; ++j) u[i][j] = 0.f;
+    for (int j = 0; j < (PAIRS ? 1 : RA); ++j) u[i][j] = 0.f;
+    if constexpr (PAIRS) u2[i] = make_float2(0.f, 0.f);
+  }
+  float* xw = xs_all + (PAIRS ? warp * SUB * KP * KSP : 0);  // this warp's X_hat rows
+  const int kq = lane / LPR, pr = lane % LPR;                // L1 row class, rank pair
 
   // X rows of a chunk are loaded one chunk ahead, so their HBM latency overlaps
   // the previous chunk's arithmetic
@@ -282,28 +305,20 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
         for (int e = 0; e < 8; ++e)
 #pragma unroll
           for (int j = 0; j < R; ++j) u[i][j] = fmaf(xh[e], l1s[e][j], u[i][j]);
-      } else if constexpr (R >= 8) {
-        // L1 row of channel k0+e, 8 ranks at a time (16-byte loads; L1-cache hits after the first row)
-        if (real) {
+      } else if constexpr (PAIRS) {
+        // park X_hat by residue class: channel lane*8+e goes to class (lane*8+e) % KP,
+        // slot (lane*8+e) / KP
+        float* xrow = xw + i * KP * KSP;
+        if constexpr (KP == 2) {
+          *reinterpret_cast<float4*>(xrow + lane * 4) = make_float4(xh[0], xh[2], xh[4], xh[6]);
+          *reinterpret_cast<float4*>(xrow + KSP + lane * 4) = make_float4(xh[1], xh[3], xh[5], xh[7]);
+        } else if constexpr (KP == 4) {
 #pragma unroll
-          for (int jc = 0; jc < R; jc += 8)
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<float2*>(xrow + e * KSP + lane * 2) = make_float2(xh[e], xh[e + 4]);
+        } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float f[8];
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(L1 + static_cast<size_t>(k0 + e) * R + jc)), f);
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) u[i][jc + jj] = fmaf(xh[e], f[jj], u[i][jc + jj]);
-            }
-        }
-      } else if constexpr (R < 0) {
-        if (real) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const __nv_bfloat16* row = L1 + static_cast<size_t>(k0 + e) * r;
-#pragma unroll
-            for (int j = 0; j < RA; ++j)
-              if (j < r) u[i][j] = fmaf(xh[e], __bfloat162float(__ldg(row + j)), u[i][j]);
-          }
+          for (int e = 0; e < 8; ++e) xrow[e * KSP + lane] = xh[e];
         }
       }
       float sc;
@@ -318,9 +333,60 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
         }
       }
     }
+    if constexpr (PAIRS) {
+      // U[i][2pr..2pr+1] += sum over this lane's channels k of X_hat[i][k] L1[k][2pr..2pr+1]
+      const int kv = min(256, K - c * 256);  // real channels of the chunk
+      const int nrows = min(SUB, M - mb);    // rows parked by this warp
+      __syncwarp();
+      if (nrows > 0) {
+        const __nv_bfloat16* l1c = L1 + static_cast<size_t>(c) * 256 * r;
+        const float* xq = xw + kq * KSP;
+        for (int t = 0; t < KS && kq + KP * t < kv; t += 4) {
+          float2 l[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int k = kq + KP * (t + q);
+            if constexpr (R > 0) {
+              uint32_t raw = 0u;
+              if (k < kv) raw = __ldg(reinterpret_cast<const unsigned int*>(l1c + static_cast<size_t>(k) * R) + pr);
+              l[q] = make_float2(__uint_as_float(raw << 16), __uint_as_float(raw & 0xffff0000u));
+            } else {
+              const __nv_bfloat16* row = l1c + static_cast<size_t>(k) * r + 2 * pr;
+              const bool k_ok = k < kv;
+              l[q].x = (k_ok && 2 * pr < r) ? __bfloat162float(__ldg(row)) : 0.f;
+              l[q].y = (k_ok && 2 * pr + 1 < r) ? __bfloat162float(__ldg(row + 1)) : 0.f;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < SUB; ++i) {
+            const float4 xv = *reinterpret_cast<const float4*>(xq + i * KP * KSP + t);
+            u2[i] = __ffma2_rn(make_float2(xv.x, xv.x), l[0], u2[i]);
+            u2[i] = __ffma2_rn(make_float2(xv.y, xv.y), l[1], u2[i]);
+            u2[i] = __ffma2_rn(make_float2(xv.z, xv.z), l[2], u2[i]);
+            u2[i] = __ffma2_rn(make_float2(xv.w, xv.w), l[3], u2[i]);
+          }
+        }
+      }
+      __syncwarp();  // the next chunk's rows overwrite the parked ones
+    }
   }
   if (!early && threadIdx.x == 0) grid_dep_launch();
-  if constexpr (R != 0) {
+  if constexpr (PAIRS) {
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      float2 v = u2[i];
+#pragma unroll
+      for (int o = LPR; o < 32; o <<= 1) {  // the KP lanes of one rank pair
+        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+      }
+      if (kq == 0) {
+        upart[warp][i][2 * pr] = v.x;
+        upart[warp][i][2 * pr + 1] = v.y;
+      }
+    }
+    __syncthreads();
+  } else if constexpr (R != 0) {
 #pragma unroll
     for (int i = 0; i < SUB; ++i)
 #pragma unroll
@@ -331,6 +397,8 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
         if (lane == 0) upart[warp][i][j] = v;
       }
     __syncthreads();
+  }
+  if constexpr (R != 0) {
     const int rows = min(RB, M - static_cast<int>(blockIdx.x) * RB);
     for (int t = threadIdx.x; t < rows * r; t += blockDim.x) {
       const int row = t / r, j = t - (t / r) * r;
