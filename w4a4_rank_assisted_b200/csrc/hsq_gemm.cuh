@@ -80,7 +80,7 @@ struct GemmArgs {
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
           int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false, int CHB_ = 2,
-          int BPG_ = 1>
+          int BPG_ = 1, bool PAIR_ = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -110,8 +110,18 @@ struct GemmCfg {
   // the low-rank step's operands.
   static constexpr bool PRE = PRE_;
   static constexpr int E8_SBO = 512;  // pre-expanded tile: bytes per 8-row group (4 K-chunks of 8 rows x 16 B)
+  // CTA pairs (pre-expanded tokens x outputs tiles only): the two CTAs of a
+  // cluster share one tile of 2 x 128 tokens x BN outputs; the even CTA issues
+  // cta_group::2 MMAs that read each CTA's 128 token rows and BN/2 output rows
+  // from that CTA's own shared memory and leave each CTA's 128 x BN partial in
+  // its own Tensor Memory.  Per CTA and step the operand bytes drop from
+  // (128 + BN) to (128 + BN/2) rows' worth, the drain work stays the same.
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int PM = PAIR ? 2 : 1;      // CTAs per tile
+  static constexpr int TILE_M = BM * PM;       // tokens per tile
+  static constexpr int B_ROWS = BN / PM;       // col-operand rows held by one CTA
   static constexpr int A_E8_BLK = BM / 8 * E8_SBO;  // one 64-block of a tile
-  static constexpr int B_E8_BLK = BN / 8 * E8_SBO;
+  static constexpr int B_E8_BLK = B_ROWS / 8 * E8_SBO;
   static constexpr int A_E8 = BPG * A_E8_BLK;
   static constexpr int B_E8 = BPG * B_E8_BLK;
   static constexpr int NUM_UNPACK_WARPS = UNPACK_WARPS_;
@@ -164,7 +174,9 @@ struct GemmCfg {
   static constexpr int LR_SBO = LR_K / 8 * 128;  // bytes per 8-row group (4 K-chunks of 16 B)
   static_assert(!LR_MMA || PRE || (BM + BN) / 8 * LR_SBO <= I8_BYTES, "low-rank operands fit an int8 buffer");
   // with pre-expanded operands the low-rank operands get a buffer of their own
-  static constexpr int LR_BYTES = (PRE && LR_MMA) ? (BM + BN) / 8 * LR_SBO : 0;
+  static constexpr int LR_BYTES = (PRE && LR_MMA) ? (BM + B_ROWS) / 8 * LR_SBO : 0;
+  static_assert(!PAIR || (PRE && LR_MMA), "CTA pairs: pre-expanded tokens x outputs tiles");
+  static_assert(!PAIR || A_E8_BLK == 8192 && B_E8_BLK == 8192, "CTA pairs: one 32 x 256-byte TMA box per block");
   static_assert(!PRE || (F8 && !SWAP && GPS == 1), "pre-expanded operands: E4M3, tokens x outputs, one group a stage");
   // Tokens x outputs tiles write Y with TMA stores: each drain warp stages a
   // 32-row x 128-byte box (128-byte swizzle) in its own 4 KB buffer.
@@ -248,8 +260,9 @@ __global__ void __launch_bounds__(256) expand_e4m3_kernel(const uint8_t* __restr
   if (threadIdx.x == 0) grid_dep_launch();
 }
 
-// Operands of the low-rank step for one tile (rows r0.. of tokens, columns c0..
-// of outputs), written as bf16 K-major core matrices (8 rows x 16 bytes,
+// Operands of the low-rank step for one tile (BM rows r0.. of tokens, B_ROWS
+// columns c0.. of outputs: this CTA's share of a pair tile), written as bf16
+// K-major core matrices (8 rows x 16 bytes,
 // K-chunks 128 bytes apart, 8-row groups LR_SBO apart) into an int8 buffer:
 //   A[m][2i] = bf16(U[m][i]),  A[m][2i+1] = bf16(U[m][i] - A[m][2i]),  A[m][LR_K-2] = 1
 //   B[n][2i] = B[n][2i+1] = L2[i][n],                               B[n][LR_K-2] = bias[n]
@@ -259,8 +272,8 @@ __global__ void __launch_bounds__(256) expand_e4m3_kernel(const uint8_t* __restr
 template <class Cfg>
 __device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int c0, int chunk, uint8_t* dst, int t0,
                                                   int nt) {
-  constexpr int BM = Cfg::BM, BN = Cfg::BN, K = Cfg::LR_K;
-  for (int t = t0; t < BM + BN; t += nt) {
+  constexpr int BM = Cfg::BM, BNR = Cfg::B_ROWS, K = Cfg::LR_K;
+  for (int t = t0; t < BM + BNR; t += nt) {
     const bool rowop = t < BM;
     const int row = rowop ? t : t - BM;
     const int idx = rowop ? r0 + row : c0 + row;  // token m or output n
@@ -315,17 +328,20 @@ struct Unit {
 // All stage arithmetic is 32-bit: the host uses stream-K only when the total
 // stage count is below 2^30 (64-bit division would expand into a long call-like
 // sequence inside warps running with a reduced register budget).
-template <int GPS>
+// With CTA pairs the workers are the pairs (both CTAs of a pair take the same units).
+template <int GPS, bool PAIR = false>
 __device__ __forceinline__ bool next_unit(const GemmArgs& a, int k, Unit& u) {
   const int tiles = a.tiles_r * a.tiles_c;
+  const unsigned wid = PAIR ? blockIdx.x >> 1 : blockIdx.x;
+  const int nwk = static_cast<int>(PAIR ? gridDim.x >> 1 : gridDim.x);
   if (a.stream_len == 0) {
-    const int t = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+    const int t = static_cast<int>(wid) + k * nwk;
     if (t >= tiles) return false;
-    u.tile = t; u.g0 = 0; u.g1 = a.G; u.nslots = 1; u.slot = 0; u.first = static_cast<int>(blockIdx.x);
+    u.tile = t; u.g0 = 0; u.g1 = a.G; u.nslots = 1; u.slot = 0; u.first = static_cast<int>(wid);
     return true;
   }
   const unsigned S = static_cast<unsigned>(a.stages_per_tile), L = static_cast<unsigned>(a.stream_len);
-  const unsigned begin = blockIdx.x * L;
+  const unsigned begin = wid * L;
   const unsigned end = min(begin + L, static_cast<unsigned>(tiles) * S);
   unsigned pos = begin;
   for (int i = 0; i < k && pos < end; ++i) pos = (pos / S + 1) * S;
@@ -348,6 +364,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                      const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
   constexpr int BM = Cfg::BM, BN = Cfg::BN, CW = Cfg::CW, STAGES = Cfg::STAGES, GPS = Cfg::GPS;
   constexpr int NI8 = Cfg::NI8E, NTM = Cfg::NTM;
+  constexpr bool PAIR = Cfg::PAIR;
+  constexpr int TILE_M = Cfg::TILE_M;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -374,6 +392,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
   const WaitPolicy wp{args.limit_ns, abort_flag};
+  // CTA pairs: rank 0 (the even CTA) issues the MMAs; each CTA owns tile rows
+  // crank*128 .. +127 and output rows crank*B_ROWS .. of the col operand
+  const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = crank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -390,10 +412,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     for (int b = 0; b < NTM; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], Cfg::NUM_DRAIN_WARPS);
+      mbar_init(&tempty[b], Cfg::NUM_DRAIN_WARPS * Cfg::PM);  // pairs: both CTAs' drain warps
     }
     mbar_init(final_bar, 1);
-    mbar_init(lrfull, Cfg::NUM_UNPACK_WARPS);
+    mbar_init(lrfull, Cfg::NUM_UNPACK_WARPS * Cfg::PM);
     mbar_init(lrempty, 1);
     *abort_flag = 0;
     *tail_flag = 0;
@@ -404,11 +426,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     prefetch_tensormap(&tm_col);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);  // the same warp of both CTAs
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote arrive
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // every warp but the producer reads or writes global memory only after the
@@ -429,7 +457,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t npre = 0;
       if constexpr (Cfg::SWAP) {
         Unit pu;
-        for (int k = 0; npre < static_cast<uint32_t>(STAGES) && next_unit<GPS>(args, k, pu); ++k) {
+        for (int k = 0; npre < static_cast<uint32_t>(STAGES) && next_unit<GPS, PAIR>(args, k, pu); ++k) {
           const int r0p = (pu.tile % args.tiles_r) * BM;
           for (int g = pu.g0; g < pu.g1 && npre < static_cast<uint32_t>(STAGES); g += GPS, ++npre) {
             mbar_arrive_expect_tx(&full[npre], Cfg::A_PACK + Cfg::B_PACK);
@@ -442,13 +470,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       Unit un;
-      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      for (int k = 0; ok && next_unit<GPS, PAIR>(args, k, un); ++k) {
         const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
         const int g0 = un.g0, g1 = un.g1;
         const int c0 = tc * BN;
-        const int r0 = tr * BM;
+        const int r0 = tr * TILE_M + static_cast<int>(crank) * BM;  // this CTA's first row
         const uint32_t cs_bytes = static_cast<uint32_t>(min(BN, args.ld_c - c0)) * 4u;
-        const uint32_t rs_bytes = static_cast<uint32_t>(min(BM, args.ld_r - r0)) * 4u;
+        // (the odd CTA of a pair tile past the last row has no row scales to load)
+        const uint32_t rs_bytes = static_cast<uint32_t>(max(0, min(BM, args.ld_r - r0))) * 4u;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
         for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
           const int ng = min(GPS, g1 - g);
@@ -465,13 +494,28 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             const float lo = 1.0f / 262144.0f;
             for (int i = 0; i < BM / 4; ++i) scw[(Cfg::RS_OFF / 16) + i] = make_float4(lo, lo, lo, lo);
             mbar_arrive(&sfull[ss]);
-            mbar_arrive(&full[s]);
+            if (leader) mbar_arrive(&full[s]);  // pairs: only the MMA issuer's barrier counts
             issued = it + 1;
             continue;
           }
           uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
           uint8_t* sc = sc_base + ss * Cfg::SSLOT_BYTES;
-          if constexpr (Cfg::PRE) {
+          if constexpr (PAIR) {
+            // MMA-ready E4M3 tiles, this CTA's share: 128 token rows and B_ROWS
+            // output rows per 64-block, one 32 x 256-byte box each.  Both CTAs'
+            // bytes are counted on the even CTA's barrier, which the even CTA
+            // arms with the pair's total (the odd CTA's bytes may land first:
+            // the phase cannot complete before that arrival).
+            if (leader) mbar_arrive_expect_tx(&full[s], Cfg::PM * (Cfg::A_E8 + Cfg::B_E8));
+            const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0u);
+#pragma unroll
+            for (int b = 0; b < Cfg::BPG; ++b) {
+              const int blk = g * Cfg::BPG + b;
+              tma_load_2d_pair(st + b * Cfg::A_E8_BLK, &tm_row, fb, 0, 2 * (blk * args.rg_r + r0 / 8));
+              tma_load_2d_pair(st + Cfg::A_E8 + b * Cfg::B_E8_BLK, &tm_col, fb, 0,
+                               2 * (blk * args.rg_c + (c0 + static_cast<int>(crank) * Cfg::B_ROWS) / 8));
+            }
+          } else if constexpr (Cfg::PRE) {
             // MMA-ready E4M3 tiles: one contiguous block per operand
             mbar_arrive_expect_tx(&full[s], Cfg::A_E8 + Cfg::B_E8);
 #pragma unroll
@@ -493,8 +537,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           for (int j = 0; j < ng; ++j) {
             bulk_load(sc + Cfg::CS_OFF + j * Cfg::CS_BYTES,
                       args.scales_c + static_cast<size_t>(g + j) * args.ld_c + c0, cs_bytes, &sfull[ss]);
-            bulk_load(sc + Cfg::RS_OFF + j * Cfg::RS_BYTES,
-                      args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, &sfull[ss]);
+            if (rs_bytes)
+              bulk_load(sc + Cfg::RS_OFF + j * Cfg::RS_BYTES,
+                        args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, &sfull[ss]);
           }
           issued = it + 1;
         }
@@ -503,32 +548,46 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
-    if (Cfg::PRE && lane == 0) {
-      // pre-expanded operands: the MMAs read the stage itself and release it
-      constexpr uint32_t idesc = idesc_f8(BM, BN);
-      constexpr uint32_t idesc_lr = idesc_bf16(BM, BN);
+    if (Cfg::PRE && lane == 0 && leader) {
+      // pre-expanded operands: the MMAs read the stage itself and release it.
+      // Pairs: one cta_group::2 MMA covers both CTAs' rows; its completion is
+      // signalled to the same barrier in both CTAs.
+      constexpr uint32_t idesc = idesc_f8(TILE_M, BN);
+      constexpr uint32_t idesc_lr = idesc_bf16(TILE_M, BN);
+      auto commit_both = [&](uint64_t* bar) {
+        if constexpr (PAIR) {
+          mma_commit_pair(mapa_shared(smem_u32(bar), 0u));
+          mma_commit_pair(mapa_shared(smem_u32(bar), 1u));
+        } else {
+          mma_commit(bar);
+        }
+      };
       uint32_t it = 0, nlr = 0;
       bool ok = true;
       Unit un;
-      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      for (int k = 0; ok && next_unit<GPS, PAIR>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
         for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
           const int s = it % STAGES;
           const int tb = it % NTM;
           if (!wait_one(&full[s], (it / STAGES) & 1, wp)) { ok = false; break; }
-          if (!wait_one(&tempty[tb], ((it / NTM) & 1) ^ 1, wp)) { ok = false; break; }
+          if (!(PAIR ? wait_one_cluster(&tempty[tb], ((it / NTM) & 1) ^ 1, wp)
+                     : wait_one(&tempty[tb], ((it / NTM) & 1) ^ 1, wp))) { ok = false; break; }
           const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
           if (Cfg::LR_MMA && g < g0) {
             // low-rank step: [U_hi U_lo 1] x [L2 L2 b] over K = LR_K, from the low-rank buffer
-            if (!wait_one(lrfull, nlr & 1, wp)) { ok = false; break; }
+            if (!(PAIR ? wait_one_cluster(lrfull, nlr & 1, wp) : wait_one(lrfull, nlr & 1, wp))) { ok = false; break; }
             tc_fence_after();
             const uint32_t abuf = smem_u32(lr_buf), bbuf = abuf + (BM / 8) * Cfg::LR_SBO;
 #pragma unroll
-            for (int q = 0; q < Cfg::LR_K / 16; ++q)
-              mma_bf16(d, smem_desc_kmajor(abuf + q * 256, 128, Cfg::LR_SBO),
-                       smem_desc_kmajor(bbuf + q * 256, 128, Cfg::LR_SBO), idesc_lr, q > 0 ? 1u : 0u);
-            mma_commit(lrempty);
+            for (int q = 0; q < Cfg::LR_K / 16; ++q) {
+              const uint64_t da = smem_desc_kmajor(abuf + q * 256, 128, Cfg::LR_SBO);
+              const uint64_t db = smem_desc_kmajor(bbuf + q * 256, 128, Cfg::LR_SBO);
+              if constexpr (PAIR) mma_bf16_pair(d, da, db, idesc_lr, q > 0 ? 1u : 0u);
+              else mma_bf16(d, da, db, idesc_lr, q > 0 ? 1u : 0u);
+            }
+            commit_both(lrempty);
             ++nlr;
           } else {
             tc_fence_after();
@@ -536,14 +595,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
             for (int b = 0; b < Cfg::BPG; ++b) {
               const uint32_t abuf = stg + b * Cfg::A_E8_BLK, bbuf = stg + Cfg::A_E8 + b * Cfg::B_E8_BLK;
-              mma_f8(d, smem_desc_kmajor(abuf, 128, Cfg::E8_SBO), smem_desc_kmajor(bbuf, 128, Cfg::E8_SBO), idesc,
-                     b > 0 ? 1u : 0u);
-              mma_f8(d, smem_desc_kmajor(abuf + 256, 128, Cfg::E8_SBO),
-                     smem_desc_kmajor(bbuf + 256, 128, Cfg::E8_SBO), idesc, 1u);
+#pragma unroll
+              for (int kh = 0; kh < 2; ++kh) {  // two K = 32 MMAs per 64-block
+                const uint64_t da = smem_desc_kmajor(abuf + 256 * kh, 128, Cfg::E8_SBO);
+                const uint64_t db = smem_desc_kmajor(bbuf + 256 * kh, 128, Cfg::E8_SBO);
+                const uint32_t acc = (b > 0 || kh > 0) ? 1u : 0u;
+                if constexpr (PAIR) mma_f8_pair(d, da, db, idesc, acc);
+                else mma_f8(d, da, db, idesc, acc);
+              }
             }
           }
-          mma_commit(&empty[s]);
-          mma_commit(&tfull[tb]);
+          commit_both(&empty[s]);
+          commit_both(&tfull[tb]);
         }
       }
     } else if (!Cfg::PRE && lane == 0) {
@@ -552,7 +615,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       Unit un;
-      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      for (int k = 0; ok && next_unit<GPS, PAIR>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
         for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
@@ -610,19 +673,24 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t nlr = 0;
       bool ok = true;
       Unit un;
-      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      for (int k = 0; ok && next_unit<GPS, PAIR>(args, k, un); ++k) {
         if (!(Cfg::LR_MMA && args.lr_mma && un.g0 == 0)) continue;
         const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
+        const int lr0 = tr * TILE_M + static_cast<int>(crank) * BM;        // this CTA's token rows
+        const int lc0 = tc * BN + static_cast<int>(crank) * Cfg::B_ROWS;  // and output rows
         for (int chunk = 0; chunk < args.lr_mma; ++chunk) {
           if (!wait_warp(lrempty, (nlr & 1) ^ 1, wp)) { ok = false; break; }
           // chunks as constants, so that each build unrolls over a fixed rank range
           constexpr int LT = 32 * Cfg::NUM_UNPACK_WARPS;
-          if (chunk == 0) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 0, lr_buf, ut, LT);
-          else if (chunk == 1) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 1, lr_buf, ut, LT);
-          else build_lr_operands<Cfg>(args, tr * BM, tc * BN, 2, lr_buf, ut, LT);
+          if (chunk == 0) build_lr_operands<Cfg>(args, lr0, lc0, 0, lr_buf, ut, LT);
+          else if (chunk == 1) build_lr_operands<Cfg>(args, lr0, lc0, 1, lr_buf, ut, LT);
+          else build_lr_operands<Cfg>(args, lr0, lc0, 2, lr_buf, ut, LT);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(lrfull);
+          if (lane == 0) {
+            if (leader) mbar_arrive(lrfull);
+            else mbar_arrive_cluster(mapa_shared(smem_u32(lrfull), 0u));  // the MMA issuer's barrier
+          }
           ++nlr;
         }
       }
@@ -654,7 +722,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t it = 0;
       bool ok = true;
       Unit un;
-      for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+      for (int k = 0; ok && next_unit<GPS, PAIR>(args, k, un); ++k) {
         const int g0 = un.g0, g1 = un.g1;
         const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
         for (int g = lr_unit ? g0 - GPS * args.lr_mma : g0; g < g1; g += GPS, ++it) {
@@ -715,11 +783,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     uint32_t it = 0;
     bool ok = true;
     Unit un;
-    for (int k = 0; ok && next_unit<GPS>(args, k, un); ++k) {
+    for (int k = 0; ok && next_unit<GPS, PAIR>(args, k, un); ++k) {
       const int tile = un.tile;
       const int tr = tile % args.tiles_r, tc = tile / args.tiles_r;
       const int g0 = un.g0, g1 = un.g1;
-      const int rbase = tr * BM + q * 32 + qd;   // tile row of i = 0 (row i adds 8i)
+      const int rbase = tr * TILE_M + static_cast<int>(crank) * BM + q * 32 + qd;  // row of i = 0 (row i adds 8i)
       const int col0 = tc * BN + h * CW + 2 * qc;  // column of block 0, first of the pair
       const bool lr_unit = Cfg::LR_MMA && args.lr_mma && g0 == 0;
       float2 acc2[4 * NBLK];
@@ -848,7 +916,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&tempty[tb]);
+          if (leader) mbar_arrive(&tempty[tb]);
+          else mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[tb]), 0u));  // the MMA issuer's barrier
           mbar_arrive(&sempty[ss]);
         }
       }
@@ -865,11 +934,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         constexpr int SLOT2 = BN * BM / 2;  // float2 per CTA slot
         float2* part = reinterpret_cast<float2*>(args.ws_partials) +
                        (static_cast<size_t>(blockIdx.x) * 2 + un.slot) * SLOT2 + dw * (4 * NBLK * 32) + lane;
+        // (pairs: a tile's sub-tiles are counted per CTA rank; worker c's CTA of this rank is 2c + crank)
 #pragma unroll
         for (int j = 0; j < 4 * NBLK; ++j) part[j * 32] = acc2[j];
         __threadfence();
         __syncwarp();
-        unsigned* counter = args.ws_counters + static_cast<size_t>(tile) * Cfg::NUM_DRAIN_WARPS + dw;
+        unsigned* counter =
+            args.ws_counters + (static_cast<size_t>(tile) * Cfg::PM + crank) * Cfg::NUM_DRAIN_WARPS + dw;
         int last = 0;
         if (lane == 0) last = (atomicAdd(counter, 1u) == static_cast<unsigned>(un.nslots - 1)) ? 1 : 0;
         last = __shfl_sync(0xffffffffu, last, 0);
@@ -882,8 +953,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll 1
         for (int c = un.first; c < un.first + un.nslots; ++c) {
           const int cslot = (static_cast<unsigned>(c) * L >= static_cast<unsigned>(tile) * S) ? 0 : 1;
+          const size_t cta = static_cast<size_t>(c) * Cfg::PM + crank;
           const float2* p = reinterpret_cast<const float2*>(args.ws_partials) +
-                            (static_cast<size_t>(c) * 2 + cslot) * SLOT2 + dw * (4 * NBLK * 32) + lane;
+                            (cta * 2 + cslot) * SLOT2 + dw * (4 * NBLK * 32) + lane;
           // 16 pairs in flight at a time (the accumulators already use most registers)
 #pragma unroll
           for (int j0 = 0; j0 < 4 * NBLK; j0 += 16) {
@@ -907,7 +979,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         // so the quad-layout writes hit distinct banks), then one TMA store of
         // that box; rows and columns outside Y are clipped by the TMA unit.
         uint8_t* stg = ystage + dw * 4096;
-        const int y0 = tr * BM + q * 32;
+        const int y0 = tr * TILE_M + static_cast<int>(crank) * BM + q * 32;
         const int x0 = tc * BN + h * CW;
         if (!args.out_f32) {
 #pragma unroll
@@ -1002,19 +1074,35 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const WaitPolicy tail{args.limit_ns, tail_flag};
     if (warp == 0 && lane == 0) {
       // let every load still in flight land before the CTA's shared memory goes away
+      // (pairs: operand bytes are counted on the even CTA's barriers only)
       const uint32_t first = issued > static_cast<uint32_t>(STAGES) ? issued - STAGES : 0u;
-      for (uint32_t i = first; i < issued; ++i) wait_one(&full[i % STAGES], (i / STAGES) & 1, tail);
+      if (leader)
+        for (uint32_t i = first; i < issued; ++i) wait_one(&full[i % STAGES], (i / STAGES) & 1, tail);
       const uint32_t sfirst = issued > static_cast<uint32_t>(Cfg::SSLOTS) ? issued - Cfg::SSLOTS : 0u;
       for (uint32_t i = sfirst; i < issued; ++i)
         wait_one(&sfull[i % Cfg::SSLOTS], (i / Cfg::SSLOTS) & 1, tail);
     }
-    if (warp == 1 && lane == 0) {
-      mma_commit(final_bar);  // arrives once every MMA issued above has completed
+    if (warp == 1 && lane == 0 && leader) {
+      // arrives once every MMA issued above has completed (pairs: the even CTA issues them)
+      if constexpr (PAIR) mma_commit_pair(mapa_shared(smem_u32(final_bar), 0u));
+      else mma_commit(final_bar);
       wait_one(final_bar, 0, tail);
     }
     __syncthreads();
   }
-  if (warp == 1) {
+  if constexpr (PAIR) {
+    // the pair's MMA completions are signalled to both CTAs' stage barriers:
+    // let the last of them land before this CTA's shared memory goes away
+    if (warp == 0 && lane == 0 && !*abort_flag) {
+      const WaitPolicy tail{args.limit_ns, tail_flag};
+      const uint32_t first = issued > static_cast<uint32_t>(STAGES) ? issued - STAGES : 0u;
+      for (uint32_t i = first; i < issued; ++i) wait_one(&empty[i % STAGES], (i / STAGES) & 1, tail);
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs are done with the pair's Tensor Memory and barriers
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  } else if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }

@@ -23,11 +23,21 @@ constexpr int kMaxDim = 1 << 20;
 constexpr int kMaxRank = 32;
 
 // Kernel configurations (hsq_gemm.cuh), for scale groups of 64 and of 128 along K.
-//   GemmCfg<BN, DH, STAGES, SWAP, GPS, NI8, NTM, UNPACK/helper warps, SSLOTS, E4M3, PIPE, PRE, CHB, BPG>
+//   GemmCfg<BN, DH, STAGES, SWAP, GPS, NI8, NTM, UNPACK/helper warps, SSLOTS, E4M3, PIPE, PRE, CHB, BPG, PAIR>
 // M > 64: 128 tokens x 256 outputs per tile, both operands pre-expanded to E4M3
 // tiles, 8 drain warps in two column slices, 2 warps building the low-rank step.
-using CfgLarge64 = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 2, 10, true, -1, true, 2, 1>;
-using CfgLarge128 = hsq::GemmCfg<256, 2, 3, false, 1, 3, 2, 2, 7, true, -1, true, 2, 2>;
+// HSQ_PAIR=1 builds CTA-pair tiles instead (clusters of 2 sharing 256 tokens x
+// 256 outputs, cta_group::2 MMAs, each CTA loading half of the outputs' operand
+// rows): a third less operand traffic per CTA, but measured slower on B200, since
+// every 64-group ends its accumulator chain and the pair adds a cross-CTA
+// hand-off to each of those chain ends.
+#ifndef HSQ_PAIR
+#define HSQ_PAIR 0
+#endif
+using CfgLarge64 = hsq::GemmCfg<256, 2, HSQ_PAIR ? 8 : 6, false, 1, 3, 2, 2, HSQ_PAIR ? 12 : 10, true, -1, true, 2,
+                                1, HSQ_PAIR != 0>;
+using CfgLarge128 = hsq::GemmCfg<256, 2, HSQ_PAIR ? 4 : 3, false, 1, 3, 2, 2, HSQ_PAIR ? 8 : 7, true, -1, true, 2,
+                                 2, HSQ_PAIR != 0>;
 // M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; packed codes
 // unpacked in shared memory (the drain is light, so more warps unpack); four
 // 64-blocks per stage either way
@@ -133,6 +143,7 @@ struct Plan {
   int gps_stage;  // scale groups per pipeline stage of the chosen kernel
   int bps_stage;  // 64-blocks per pipeline stage (the TMA box width / 32 bytes)
   int tiles_r, tiles_c, stages_per_tile, stream_len, grid;
+  int pm = 1;     // CTAs per tile (2: CTA pairs)
   size_t counters_bytes, partial_bytes;
   // pre-expanded operands (large tiles): 8-row groups and bytes
   int rg_r, rg_c;
@@ -152,6 +163,41 @@ void plan_from(Plan& p) {
   p.drain_warps = C::NUM_DRAIN_WARPS;
 }
 
+// Workers of the large-tile kernel: CTAs, or CTA pairs that the device can hold
+// at once (asked of the occupancy calculator once per device; half the SMs when
+// no device answers, as on a machine without a GPU).
+int large_workers(int nsm) {
+  if (!CfgLarge64::PAIR) return nsm;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nsm / 2;
+  }
+  static int cache[64] = {0};
+  if (cache[dev]) return cache[dev];
+  int n = nsm / 2;
+  auto* kern = hsq::w4a4_gemm_kernel<CfgLarge64>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CfgLarge64::SMEM_BYTES) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * n);
+    cfg.blockDim = dim3(CfgLarge64::THREADS);
+    cfg.dynamicSmemBytes = CfgLarge64::SMEM_BYTES;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, kern, &cfg) == cudaSuccess && c > 0) n = std::min(n, c);
+  }
+  cudaGetLastError();
+  cache[dev] = n;
+  return n;
+}
+
 Plan make_plan(int M, int N, int K, int group, int nsm) {
   Plan p{};
   p.group = group;
@@ -169,35 +215,40 @@ Plan make_plan(int M, int N, int K, int group, int nsm) {
     p.swap = false;
     p.kind = kLarge;
     g128 ? plan_from<CfgLarge128>(p) : plan_from<CfgLarge64>(p);
-    p.tiles_r = (M + 127) / 128;
+    p.pm = CfgLarge64::PM;
+    p.tiles_r = (M + CfgLarge64::TILE_M - 1) / CfgLarge64::TILE_M;
     p.tiles_c = (N + p.BN - 1) / p.BN;
   }
   const long tiles = static_cast<long>(p.tiles_r) * p.tiles_c;
   p.stages_per_tile = (G + p.gps_stage - 1) / p.gps_stage;
-  // Whole tiles per CTA when they fill the device in nearly full waves;
-  // otherwise stream-K: equal runs of stages per CTA across tile boundaries.
-  const long waves = (tiles + nsm - 1) / nsm;
-  const double fill = static_cast<double>(tiles) / static_cast<double>(waves * nsm);
+  // Whole tiles per worker (a CTA, or a CTA pair) when they fill the device in
+  // nearly full waves; otherwise stream-K: equal runs of stages per worker
+  // across tile boundaries.
+  const long nw = p.kind == kLarge ? large_workers(nsm) : nsm;
+  const long waves = (tiles + nw - 1) / nw;
+  const double fill = static_cast<double>(tiles) / static_cast<double>(waves * nw);
   const long total = tiles * p.stages_per_tile;
-  if ((tiles >= nsm && fill >= 0.9) || total <= nsm || total >= (1l << 30)) {
+  if ((tiles >= nw && fill >= 0.9) || total <= nw || total >= (1l << 30)) {
     p.stream_len = 0;
-    p.grid = static_cast<int>(std::min<long>(tiles, nsm));
+    p.grid = p.pm * static_cast<int>(std::min<long>(tiles, nw));
   } else {
-    p.stream_len = static_cast<int>((total + nsm - 1) / nsm);
-    p.grid = static_cast<int>((total + p.stream_len - 1) / p.stream_len);
+    p.stream_len = static_cast<int>((total + nw - 1) / nw);
+    p.grid = p.pm * static_cast<int>((total + p.stream_len - 1) / p.stream_len);
   }
-  p.counters_bytes = ((static_cast<size_t>(tiles) * p.drain_warps * 4 + 255) / 256) * 256;
+  p.counters_bytes = ((static_cast<size_t>(tiles) * p.pm * p.drain_warps * 4 + 255) / 256) * 256;
   p.partial_bytes = static_cast<size_t>(p.grid) * 2 * p.BN * 128 * 4;
   if (p.kind == kLarge) {  // both large configurations pre-expand their operands
     const size_t blocks = static_cast<size_t>(G) * (group / 64);  // 64-wide K blocks
-    p.rg_r = p.tiles_r * (128 / 8);
+    p.rg_r = p.tiles_r * (CfgLarge64::TILE_M / 8);
     p.rg_c = p.tiles_c * (p.BN / 8);
     p.pre_x_bytes = blocks * p.rg_r * CfgLarge64::E8_SBO;
     p.pre_w_bytes = blocks * p.rg_c * CfgLarge64::E8_SBO;
   }
   return p;
 }
-static_assert(CfgLarge64::PRE && CfgLarge128::PRE && CfgLarge64::BN == CfgLarge128::BN, "large configurations");
+static_assert(CfgLarge64::PRE && CfgLarge128::PRE && CfgLarge64::BN == CfgLarge128::BN &&
+                  CfgLarge64::PAIR == CfgLarge128::PAIR,
+              "large configurations");
 
 // ------------------------------------------------------------------ tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -225,6 +276,20 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, in
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(32 * groups), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Pre-expanded E4M3 tiles (large tiles with CTA pairs) viewed as rows of 256
+// bytes; one box of 32 rows is one 8 KB block of 128 rows x 64 codes.
+bool make_e8_map(CUtensorMap* map, const uint8_t* base, size_t bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || bytes % 256 != 0) return false;
+  const cuuint64_t dims[2] = {256u, static_cast<cuuint64_t>(bytes / 256)};
+  const cuuint64_t strides[1] = {256u};
+  const cuuint32_t box[2] = {256u, 32u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -267,11 +332,30 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
   }
-  // decode tiles start early (their weight prefetch overlaps the activation
-  // step); the GPU-filling large tiles measured faster without an early start
-  if (launch_pdl(p.swap, hsq::w4a4_gemm_kernel<Cfg>, dim3(p.grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, tr, tc, ty, a) !=
-      cudaSuccess)
-    return HSQ_ERR_CUDA;
+  cudaError_t e;
+  if constexpr (Cfg::PAIR) {
+    // CTA pairs: clusters of two, no early start
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (p.grid % 2 != 0) return HSQ_ERR_INVALID_ARG;
+    e = cudaLaunchKernelEx(&cfg, hsq::w4a4_gemm_kernel<Cfg>, tr, tc, ty, a);
+  } else {
+    // decode tiles start early (their weight prefetch overlaps the activation
+    // step); the GPU-filling large tiles measured faster without an early start
+    e = launch_pdl(p.swap, hsq::w4a4_gemm_kernel<Cfg>, dim3(p.grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, tr,
+                   tc, ty, a);
+  }
+  if (e != cudaSuccess) return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
@@ -476,6 +560,10 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     a.we = we;
     a.rg_r = p.rg_r;
     a.rg_c = p.rg_c;
+    // CTA pairs read the expanded tiles with tiled loads (the row and col maps
+    // of the pre-expanded kernel)
+    if (CfgLarge64::PAIR && !(make_e8_map(&tm_row, xe, p.pre_x_bytes) && make_e8_map(&tm_col, we, p.pre_w_bytes)))
+      return HSQ_ERR_CUDA;
   }
   // U L2 + b as a bf16 MMA step when the kernel has one and the rank fits its K
   // U L2 + b as tensor-core steps of LR_MAX_RANK ranks each (at least one: the bias)
