@@ -100,5 +100,8 @@ def test_workspace_needs_are_consistent():
     # to whole 128 x 256 tiles (no split-K: the 1728 tiles fill the device).
     assert hsq.hsq_workspace_bytes(4608, 12288, 3072, 4) == (4608 + 12288) * 3072
     # decode tiles: only split-K scratch (counters and partial tiles)
-    assert 0 < hsq.hsq_workspace_bytes(1, 4096, 12288, 4) < 16 << 20
+    assert 0 < hsq.hsq_workspace_bytes(16, 4096, 12288, 4) < 16 << 20
+    # up to 8 tokens: the weight stream needs no workspace
+    assert hsq.hsq_workspace_bytes(1, 4096, 12288, 4) == 0
+    assert hsq.hsq_workspace_bytes(8, 12288, 4096, 4) == 0
     assert hsq.hsq_workspace_bytes(0, 4096, 12288, 4) == 0

@@ -83,6 +83,13 @@ SMALL_SHAPES = [
     (40, 328, 264, 8),       # few rows, rank 8, ragged last chunk
     (33, 328, 128, 7),       # generic odd rank, few rows
     (150, 584, 136, 5),      # generic odd rank, ragged rows and last chunk
+    # M <= 8: the CUDA-core weight stream
+    (2, 640, 264, 32),
+    (3, 1152, 1160, 0),
+    (4, 200, 136, 7),        # K = 200 pads to 256
+    (8, 4096, 520, 4),
+    (7, 12288, 256, 4),      # long rows: several load batches per row
+    (8, 32768, 128, 4),      # activations too large for one block's shared memory: decode tiles
 ]
 
 
@@ -107,6 +114,8 @@ SHAPES_G128 = [
     (200, 1024, 1160, 4),
     (128, 2048, 1024, 4),    # large tile, split-K or whole tiles
     (300, 640, 512, 32),
+    (6, 640, 264, 16),       # the CUDA-core weight stream, four lanes per group
+    (8, 1024, 1160, 4),
 ]
 
 
@@ -166,13 +175,24 @@ def test_unit_smoothing_lossless_grid_matches_dense_product():
 
 
 def test_repeated_calls_are_deterministic_and_reuse_workspace():
-    layer = make_layer(_spec(3, 4096, 2048, 4, seed=2))
+    layer = make_layer(_spec(16, 4096, 2048, 4, seed=2))
     pl, act, Y, ws = _run_gpu(layer)
     assert ws is not None  # stream-K path (tiles cut between CTAs)
     assert int(ws[:16].view(torch.int32).abs().sum()) == 0  # counters back at zero
     Y0 = Y.clone()
     for _ in range(3):
         hsq.forward(pl, layer.X.to(DEV), act, Y, workspace=ws, out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y0)
+
+
+def test_few_token_stream_is_deterministic_without_workspace():
+    layer = make_layer(_spec(3, 4096, 2048, 4, seed=2))
+    pl, act, Y, ws = _run_gpu(layer)
+    assert ws is None  # up to 8 tokens: the CUDA-core weight stream, no scratch
+    Y0 = Y.clone()
+    for _ in range(3):
+        hsq.forward(pl, layer.X.to(DEV), act, Y, workspace=None, out=hsq.HSQ_OUT_F32)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y0)
 
@@ -199,8 +219,10 @@ def test_invalid_arguments_launch_nothing():
         hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, None,
                                8, 64, 128, 4, Y, group=96)
     assert e.value.status == hsq.HSQ_ERR_UNSUPPORTED
-    big = hsq.hsq_workspace_bytes(1, 4096, 12288, 4)
+    # a shape that needs split-K scratch, called without it: rejected before any
+    # launch (the buffers above are far too small for it, so nothing may run)
+    big = hsq.hsq_workspace_bytes(16, 4096, 12288, 4)
     with pytest.raises(hsq.HsqError) as e:
         hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, None,
-                               1, 4096, 12288, 4, Y, workspace=None)
+                               16, 4096, 12288, 4, Y, workspace=None)
     assert big > 0 and e.value.status == hsq.HSQ_ERR_INVALID_ARG

@@ -1,0 +1,170 @@
+// hsq_gemv.cuh -- the forward for a few tokens (M <= 8) as a weight stream on
+// the CUDA cores.
+//
+// Computes the same layer as hsq_gemm.cuh (Deflating the Hessian, Abstract:
+// 4-bit residual product plus the high-precision low-rank branch)
+//     Y[m,n] = sum_g sx[g][m] sw[g][n] P_g[m,n] + sum_j U[m,j] L2[j,n] + b[n],
+//     P_g[m,n] = sum_{k in group g} qx[m,k] qw[n,k]   (exact, int32)
+// for M <= 8 tokens.  There the product is a matrix-vector stream: every weight
+// byte is used for at most 16 multiply-adds, so the work is bound by reading the
+// packed weights once, and a tensor-core tile (128 rows, its TMA/unpack/MMA/drain
+// hand-offs per stage) only adds latency.  Here every warp streams whole weight
+// rows with 16-byte loads (a warp reads 512 contiguous bytes per instruction);
+// codes are widened in registers to int8 16*q (one AND or shift+AND per four
+// codes, the same trick as the tensor-core unpack), and __dp4a forms the exact
+// group partial 256*P_g in int32 (|256 P_g| <= 256 * 128 * 49 < 2^24, so its fp32
+// conversion is exact).  The block's activation codes are widened the same way
+// once into shared memory.  Each group partial is scaled by sx*sw in fp32, the
+// low-rank branch and the bias are added, and the warp's sum is written.
+#pragma once
+
+#include "hsq_device.cuh"
+
+namespace hsq {
+
+struct GemvArgs {
+  const uint8_t* x_codes;  // [M][Kp/2]
+  const float* x_scales;   // [G][ldx]
+  const float* U;          // [M][r]
+  const uint8_t* w_codes;  // [N][Kp/2]
+  const float* w_scales;   // [G][ldw]
+  const __nv_bfloat16* L2;    // [r][N]
+  const __nv_bfloat16* bias;  // [N] or nullptr
+  void* Y;                    // [M][N]
+  int ldx, ldw, r, out_f32;
+  int M, N, Kp, G;
+  int rows_per_block;
+};
+
+constexpr int kGemvThreads = 512;
+constexpr int kGemvBatch = 4;  // 16-byte weight chunks per lane per batch (two batches in flight)
+
+// Shared memory of one block: widened activation codes (even and odd codes of
+// every packed word, MT*Kp bytes) and the activation scales [G][MT].
+__host__ __device__ constexpr size_t gemv_smem_bytes(int MT, int Kp, int G) {
+  return static_cast<size_t>(MT) * Kp + static_cast<size_t>(G) * MT * 4;
+}
+
+// MT: tokens the kernel is built for (M <= MT); LPG: lanes per scale group (a
+// lane holds 32 codes, so 2 for groups of 64 and 4 for groups of 128).
+template <int MT, int LPG>
+__global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvArgs a) {
+  extern __shared__ __align__(16) uint8_t gemv_smem[];
+  const int W4 = a.Kp / 8;  // packed 32-bit words per row
+  uint32_t* xlo = reinterpret_cast<uint32_t*>(gemv_smem);  // [MT][W4] even codes, int8 16*q
+  uint32_t* xhi = xlo + MT * W4;                           // [MT][W4] odd codes
+  float* sxs = reinterpret_cast<float*>(xhi + MT * W4);     // [G][MT]
+  grid_dep_wait();  // the activation codes come from the preceding kernel
+  for (int i = threadIdx.x; i < MT * W4; i += blockDim.x) {
+    const int m = i / W4, j = i - m * W4;
+    uint32_t w = 0u;
+    if (m < a.M) w = __ldg(reinterpret_cast<const unsigned int*>(a.x_codes + static_cast<size_t>(m) * (a.Kp / 2)) + j);
+    xlo[i] = (w << 4) & 0xF0F0F0F0u;
+    xhi[i] = w & 0xF0F0F0F0u;
+  }
+  for (int i = threadIdx.x; i < a.G * MT; i += blockDim.x) {
+    const int g = i / MT, m = i - g * MT;
+    sxs[i] = m < a.M ? __ldg(a.x_scales + static_cast<size_t>(g) * a.ldx + m) : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) grid_dep_launch();
+
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int nwarps = blockDim.x >> 5;
+  const int nch = a.Kp / 32;  // 16-byte chunks per row (a multiple of LPG)
+  const int n0 = blockIdx.x * a.rows_per_block;
+  const int n1 = min(a.N, n0 + a.rows_per_block);
+  // The warp's rows n0 + warp, + nwarps, ... are streamed as one sequence of
+  // batches (kGemvBatch chunks per lane); the next batch's loads are issued
+  // before the current one is used, across row ends too, so that a lane always
+  // has one to two batches of loads in flight.
+  const int nrows = n1 > n0 + warp ? (n1 - n0 - warp + nwarps - 1) / nwarps : 0;
+  const int bpr = (nch + 32 * kGemvBatch - 1) / (32 * kGemvBatch);  // batches per row
+  const int total = nrows * bpr;
+  // (a batch's weight scales are loaded with its codes: they are as far away)
+  auto load = [&](int t, uint4 (&dst)[kGemvBatch], float (&dsw)[kGemvBatch]) {
+    const int n = n0 + warp + (t / bpr) * nwarps;
+    const int c0 = (t % bpr) * 32 * kGemvBatch;
+    const uint4* wrow = reinterpret_cast<const uint4*>(a.w_codes + static_cast<size_t>(n) * (a.Kp / 2));
+#pragma unroll
+    for (int b = 0; b < kGemvBatch; ++b) {
+      const int c = c0 + 32 * b + lane;
+      dst[b] = c < nch ? __ldg(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+      dsw[b] = c < nch ? __ldg(a.w_scales + static_cast<size_t>(c / LPG) * a.ldw + n) : 0.f;
+    }
+  };
+  float acc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) acc[m] = 0.f;
+  uint4 wv[kGemvBatch], wn[kGemvBatch];
+  float swv[kGemvBatch], swn[kGemvBatch];
+  if (total > 0) load(0, wv, swv);
+  for (int t = 0; t < total; ++t) {
+    if (t + 1 < total) load(t + 1, wn, swn);
+    const int n = n0 + warp + (t / bpr) * nwarps;
+    const int c0 = (t % bpr) * 32 * kGemvBatch;
+#pragma unroll
+    for (int b = 0; b < kGemvBatch; ++b) {
+      if (c0 + 32 * b >= nch) break;  // warp-uniform
+      const int c = c0 + 32 * b + lane;
+      const bool valid = c < nch;  // the LPG lanes of a group agree
+      const int g = c / LPG;
+      const float sw = swv[b];
+      const uint32_t w[4] = {wv[b].x, wv[b].y, wv[b].z, wv[b].w};
+      int wl[4], wh[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wl[j] = static_cast<int>((w[j] << 4) & 0xF0F0F0F0u);  // even codes, 16*q
+        wh[j] = static_cast<int>(w[j] & 0xF0F0F0F0u);         // odd codes, 16*q
+      }
+      const int cc = valid ? c : 0;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint4 l = *reinterpret_cast<const uint4*>(xlo + m * W4 + 4 * cc);
+        const uint4 h = *reinterpret_cast<const uint4*>(xhi + m * W4 + 4 * cc);
+        int p = __dp4a(wl[0], static_cast<int>(l.x), 0);
+        p = __dp4a(wl[1], static_cast<int>(l.y), p);
+        p = __dp4a(wl[2], static_cast<int>(l.z), p);
+        p = __dp4a(wl[3], static_cast<int>(l.w), p);
+        p = __dp4a(wh[0], static_cast<int>(h.x), p);
+        p = __dp4a(wh[1], static_cast<int>(h.y), p);
+        p = __dp4a(wh[2], static_cast<int>(h.z), p);
+        p = __dp4a(wh[3], static_cast<int>(h.w), p);
+#pragma unroll
+        for (int o = 1; o < LPG; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);  // 256 * P_g
+        if (valid && (lane & (LPG - 1)) == 0)
+          acc[m] = fmaf(static_cast<float>(p) * (1.0f / 256.0f), sxs[g * MT + m] * sw, acc[m]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kGemvBatch; ++b) {
+      wv[b] = wn[b];
+      swv[b] = swn[b];
+    }
+    if ((t + 1) % bpr != 0) continue;
+    // end of row n: low-rank branch (lane j adds U[m][j] L2[j][n]), the warp's sum, the bias
+    if (lane < a.r) {
+      const float l2 = __bfloat162float(a.L2[static_cast<size_t>(lane) * a.N + n]);
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (m < a.M) acc[m] = fmaf(__ldg(a.U + static_cast<size_t>(m) * a.r + lane), l2, acc[m]);
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
+    const float bn = a.bias ? __bfloat162float(a.bias[n]) : 0.f;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (lane == m && m < a.M) {
+        const float y = acc[m] + bn;
+        const size_t off = static_cast<size_t>(m) * a.N + n;
+        if (a.out_f32) static_cast<float*>(a.Y)[off] = y;
+        else static_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(y);
+      }
+      acc[m] = 0.f;
+    }
+  }
+}
+
+}  // namespace hsq

@@ -15,6 +15,7 @@
 #include "../../include/hsq.h"
 #include "hsq_device.cuh"
 #include "hsq_gemm.cuh"
+#include "hsq_gemv.cuh"
 #include "hsq_quant.cuh"
 
 namespace {
@@ -132,7 +133,13 @@ int device_sm_count() {
 }
 
 // ------------------------------------------------------------------ planning
-enum Kind { kLarge = 0, kDec16, kDec32, kDec64 };
+enum Kind { kLarge = 0, kDec16, kDec32, kDec64, kGemv };
+
+// M <= 8: the weight stream on the CUDA cores (hsq_gemv.cuh) when the block's
+// widened activation codes fit in shared memory; otherwise the decode tiles.
+constexpr int kGemvMaxM = 8;
+constexpr size_t kGemvSmemMax = 200 * 1024;
+int gemv_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
 struct Plan {
   Kind kind;
@@ -203,6 +210,16 @@ Plan make_plan(int M, int N, int K, int group, int nsm) {
   p.group = group;
   const bool g128 = group == 128;
   const int G = groups_of(K, group);
+  if (M <= kGemvMaxM && hsq::gemv_smem_bytes(gemv_mt(M), G * group, G) <= kGemvSmemMax) {
+    // one block of 16 warps per SM at most, whole weight rows per warp; no workspace
+    p.kind = kGemv;
+    p.swap = true;
+    p.grid = static_cast<int>(std::min<long>(nsm, (N + 15) / 16));
+    p.tiles_r = (N + p.grid - 1) / p.grid;  // rows per block
+    p.tiles_c = 1;
+    p.stream_len = 0;
+    return p;
+  }
   if (M <= 64) {
     p.swap = true;
     p.kind = M <= 16 ? kDec16 : M <= 32 ? kDec32 : kDec64;
@@ -356,6 +373,29 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
                    tc, ty, a);
   }
   if (e != cudaSuccess) return HSQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
+template <int MT, int LPG>
+hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
+  static std::mutex mu;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      if (cudaFuncSetAttribute(hsq::w4a4_gemv_kernel<MT, LPG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kGemvSmemMax)) != cudaSuccess)
+        return HSQ_ERR_CUDA;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
+  const size_t smem = hsq::gemv_smem_bytes(MT, a.Kp, a.G);
+  // starts early: it waits for the activation step before reading its codes
+  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG>, dim3(p.grid), dim3(hsq::kGemvThreads), smem, st, a) !=
+      cudaSuccess)
+    return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
@@ -515,6 +555,24 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   const int G = groups_of(K, group), Kp = G * group;
   const Plan p = make_plan(M, N, K, group, device_sm_count());
   if (p.ws_bytes() > 0 && (!workspace || ws_bytes < p.ws_bytes())) return HSQ_ERR_INVALID_ARG;
+  if (p.kind == kGemv) {
+    hsq::GemvArgs ga{};
+    ga.x_codes = x_codes; ga.x_scales = x_scales; ga.ldx = scales_ld(M);
+    ga.w_codes = w_codes; ga.w_scales = w_scales; ga.ldw = scales_ld(N);
+    ga.U = U; ga.r = r;
+    ga.L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
+    ga.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+    ga.Y = Y;
+    ga.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
+    ga.M = M; ga.N = N; ga.Kp = Kp; ga.G = G;
+    ga.rows_per_block = p.tiles_r;
+    const int mt = gemv_mt(M);
+    const bool g128 = group == 128;
+    if (mt == 1) return g128 ? launch_gemv<1, 4>(p, ga, stream) : launch_gemv<1, 2>(p, ga, stream);
+    if (mt == 2) return g128 ? launch_gemv<2, 4>(p, ga, stream) : launch_gemv<2, 2>(p, ga, stream);
+    if (mt == 4) return g128 ? launch_gemv<4, 4>(p, ga, stream) : launch_gemv<4, 2>(p, ga, stream);
+    return g128 ? launch_gemv<8, 4>(p, ga, stream) : launch_gemv<8, 2>(p, ga, stream);
+  }
 
   hsq::GemmArgs a{};
   const int ldx = scales_ld(M), ldw = scales_ld(N);
