@@ -37,7 +37,9 @@ struct GemvArgs {
 };
 
 constexpr int kGemvThreads = 512;
-constexpr int kGemvBatch = 4;  // 16-byte weight chunks per lane per batch (two batches in flight)
+// 16-byte weight chunks per lane per batch (two batches in flight; 4 measured
+// better than 8, which half-fills a batch when a row has 4 chunks per lane)
+constexpr int kGemvBatch = 4;
 
 // Shared memory of one block: widened activation codes (even and odd codes of
 // every packed word, MT*Kp bytes) and the activation scales [G][MT].
@@ -54,21 +56,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
   uint32_t* xlo = reinterpret_cast<uint32_t*>(gemv_smem);  // [MT][W4] even codes, int8 16*q
   uint32_t* xhi = xlo + MT * W4;                           // [MT][W4] odd codes
   float* sxs = reinterpret_cast<float*>(xhi + MT * W4);     // [G][MT]
-  grid_dep_wait();  // the activation codes come from the preceding kernel
-  for (int i = threadIdx.x; i < MT * W4; i += blockDim.x) {
-    const int m = i / W4, j = i - m * W4;
-    uint32_t w = 0u;
-    if (m < a.M) w = __ldg(reinterpret_cast<const unsigned int*>(a.x_codes + static_cast<size_t>(m) * (a.Kp / 2)) + j);
-    xlo[i] = (w << 4) & 0xF0F0F0F0u;
-    xhi[i] = w & 0xF0F0F0F0u;
-  }
-  for (int i = threadIdx.x; i < a.G * MT; i += blockDim.x) {
-    const int g = i / MT, m = i - g * MT;
-    sxs[i] = m < a.M ? __ldg(a.x_scales + static_cast<size_t>(g) * a.ldx + m) : 0.f;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) grid_dep_launch();
-
   const int warp = threadIdx.x >> 5, lane = lane_id();
   const int nwarps = blockDim.x >> 5;
   const int nch = a.Kp / 32;  // 16-byte chunks per row (a multiple of LPG)
@@ -98,7 +85,24 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
   for (int m = 0; m < MT; ++m) acc[m] = 0.f;
   uint4 wv[kGemvBatch], wn[kGemvBatch];
   float swv[kGemvBatch], swn[kGemvBatch];
+  // the packed weights are never written by the kernel just before this one (the
+  // activation step), so the first batch is requested before waiting for it
   if (total > 0) load(0, wv, swv);
+  grid_dep_wait();  // the activation codes come from the preceding kernel
+  for (int i = threadIdx.x; i < MT * W4; i += blockDim.x) {
+    const int m = i / W4, j = i - m * W4;
+    uint32_t w = 0u;
+    if (m < a.M) w = __ldg(reinterpret_cast<const unsigned int*>(a.x_codes + static_cast<size_t>(m) * (a.Kp / 2)) + j);
+    xlo[i] = (w << 4) & 0xF0F0F0F0u;
+    xhi[i] = w & 0xF0F0F0F0u;
+  }
+  for (int i = threadIdx.x; i < a.G * MT; i += blockDim.x) {
+    const int g = i / MT, m = i - g * MT;
+    sxs[i] = m < a.M ? __ldg(a.x_scales + static_cast<size_t>(g) * a.ldx + m) : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) grid_dep_launch();
+
   for (int t = 0; t < total; ++t) {
     if (t + 1 < total) load(t + 1, wn, swn);
     const int n = n0 + warp + (t / bpr) * nwarps;
