@@ -37,9 +37,11 @@ struct GemvArgs {
 };
 
 constexpr int kGemvThreads = 512;
-// 16-byte weight chunks per lane per batch (two batches in flight; 4 measured
-// better than 8, which half-fills a batch when a row has 4 chunks per lane)
+// 16-byte weight chunks per lane per batch (4 measured better than 8, which
+// half-fills a batch when a row has 4 chunks per lane), and batches in flight
+// (3 measured no better than 2)
 constexpr int kGemvBatch = 4;
+constexpr int kGemvDepth = 2;
 
 // Shared memory of one block: widened activation codes (even and odd codes of
 // every packed word, MT*Kp bytes) and the activation scales [G][MT].
@@ -62,9 +64,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
   const int n0 = blockIdx.x * a.rows_per_block;
   const int n1 = min(a.N, n0 + a.rows_per_block);
   // The warp's rows n0 + warp, + nwarps, ... are streamed as one sequence of
-  // batches (kGemvBatch chunks per lane); the next batch's loads are issued
-  // before the current one is used, across row ends too, so that a lane always
-  // has one to two batches of loads in flight.
+  // batches (kGemvBatch chunks per lane), kGemvDepth - 1 batches ahead of the
+  // one in use, across row ends too.
   const int nrows = n1 > n0 + warp ? (n1 - n0 - warp + nwarps - 1) / nwarps : 0;
   const int bpr = (nch + 32 * kGemvBatch - 1) / (32 * kGemvBatch);  // batches per row
   const int total = nrows * bpr;
@@ -83,11 +84,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
   float acc[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-  uint4 wv[kGemvBatch], wn[kGemvBatch];
-  float swv[kGemvBatch], swn[kGemvBatch];
+  uint4 wb[kGemvDepth][kGemvBatch];
+  float sb[kGemvDepth][kGemvBatch];
   // the packed weights are never written by the kernel just before this one (the
-  // activation step), so the first batch is requested before waiting for it
-  if (total > 0) load(0, wv, swv);
+  // activation step), so the first batches are requested before waiting for it
+#pragma unroll
+  for (int d = 0; d + 1 < kGemvDepth; ++d)
+    if (d < total) load(d, wb[d], sb[d]);
   grid_dep_wait();  // the activation codes come from the preceding kernel
   for (int i = threadIdx.x; i < MT * W4; i += blockDim.x) {
     const int m = i / W4, j = i - m * W4;
@@ -103,8 +106,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
   __syncthreads();
   if (threadIdx.x == 0) grid_dep_launch();
 
-  for (int t = 0; t < total; ++t) {
-    if (t + 1 < total) load(t + 1, wn, swn);
+  // one batch: its chunks' group partials, scaled, into acc; at a row's end the
+  // low-rank branch (lane j adds U[m][j] L2[j][n]), the warp's sum, the bias, Y
+  auto consume = [&](int t, const uint4 (&wv)[kGemvBatch], const float (&swv)[kGemvBatch]) {
     const int n = n0 + warp + (t / bpr) * nwarps;
     const int c0 = (t % bpr) * 32 * kGemvBatch;
 #pragma unroll
@@ -113,7 +117,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
       const int c = c0 + 32 * b + lane;
       const bool valid = c < nch;  // the LPG lanes of a group agree
       const int g = c / LPG;
-      const float sw = swv[b];
       const uint32_t w[4] = {wv[b].x, wv[b].y, wv[b].z, wv[b].w};
       int wl[4], wh[4];
 #pragma unroll
@@ -137,16 +140,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
 #pragma unroll
         for (int o = 1; o < LPG; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);  // 256 * P_g
         if (valid && (lane & (LPG - 1)) == 0)
-          acc[m] = fmaf(static_cast<float>(p) * (1.0f / 256.0f), sxs[g * MT + m] * sw, acc[m]);
+          acc[m] = fmaf(static_cast<float>(p) * (1.0f / 256.0f), sxs[g * MT + m] * swv[b], acc[m]);
       }
     }
-#pragma unroll
-    for (int b = 0; b < kGemvBatch; ++b) {
-      wv[b] = wn[b];
-      swv[b] = swn[b];
-    }
-    if ((t + 1) % bpr != 0) continue;
-    // end of row n: low-rank branch (lane j adds U[m][j] L2[j][n]), the warp's sum, the bias
+    if ((t + 1) % bpr != 0) return;
     if (lane < a.r) {
       const float l2 = __bfloat162float(a.L2[static_cast<size_t>(lane) * a.N + n]);
 #pragma unroll
@@ -167,6 +164,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
         else static_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(y);
       }
       acc[m] = 0.f;
+    }
+  };
+  // a ring of kGemvDepth batches: batch t + kGemvDepth - 1 is requested before batch t is used
+  constexpr int kAhead = kGemvDepth - 1;
+  for (int t0 = 0; t0 < total; t0 += kGemvDepth) {
+#pragma unroll
+    for (int d = 0; d < kGemvDepth; ++d) {
+      const int t = t0 + d;
+      if (t >= total) break;
+      if (t + kAhead < total) load(t + kAhead, wb[(d + kAhead) % kGemvDepth], sb[(d + kAhead) % kGemvDepth]);
+      consume(t, wb[d], sb[d]);
     }
   }
 }
