@@ -68,6 +68,16 @@ def layer_gemm_bytes(spec):
             + 2 * M * N)                             # Y (bf16)
 
 
+def layer_fused_bytes(spec):
+    """Algorithmic HBM bytes of one hsq_linear_forward_fused call: X, s, L1, the
+    packed weights and their scales, L2 and Y (the activation codes, scales and U
+    stay on chip)."""
+    M, N, K, r, gs = spec.M, spec.N, spec.K, spec.r, spec.group
+    G = -(-K // gs)
+    Kp = gs * G
+    return 2 * M * K + 4 * K + 2 * K * r + N * Kp // 2 + 4 * N * G + 2 * r * N + 2 * M * N
+
+
 def layer_act_bytes(spec):
     M, K, r, gs = spec.M, spec.K, spec.r, spec.group
     G = -(-K // gs)
@@ -272,15 +282,30 @@ def run_gpu(args, specs, wl_name, rank, world, local):
                                workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
                                group=s.group, stream=st)
 
+    # decode sizes the single-launch forward takes (up to 4 tokens, r in {0,1,2,4}):
+    # the activation step runs inside the weight-stream kernel
+    fused = all(hsq.fused_supported(s.M, s.K, s.r, s.group) for s in specs)
+
+    def launch_fused(L, st):
+        s = L["spec"]
+        hsq.hsq_linear_forward_fused(L["X"], L["pl"].s, L["pl"].L1, L["pl"].w_codes, L["pl"].w_scales,
+                                     L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"], group=s.group, stream=st)
+
     def step(st, rep=0):
         for L in replicas[rep]:
-            launch_act(L, st)
-            launch_gemm(L, st)
+            if fused:
+                launch_fused(L, st)
+            else:
+                launch_act(L, st)
+                launch_gemm(L, st)
 
     def step_e2e():
         for L in layers:
             L["X"].copy_(L["X_host"], non_blocking=True)
-            hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
+            if fused:
+                hsq.forward_fused(L["pl"], L["X"], L["Y"], stream=stream)
+            else:
+                hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
             L["Y_host"].copy_(L["Y"], non_blocking=True)
 
     # A step (one replica's layers) is captured once into a CUDA graph and
@@ -347,8 +372,12 @@ def run_gpu(args, specs, wl_name, rank, world, local):
         torch.cuda.synchronize()
         return replay_ms(g, 3) * 1e3 / (3 * reps)
 
-    gemm_us = [kernel_us(launch_gemm, li) for li in range(len(layers))]
-    act_us = [kernel_us(launch_act, li) for li in range(len(layers))]
+    if fused:  # one kernel per layer: its time is reported as the GEMM's, the activation step's as 0
+        gemm_us = [kernel_us(launch_fused, li) for li in range(len(layers))]
+        act_us = [0.0 for _ in layers]
+    else:
+        gemm_us = [kernel_us(launch_gemm, li) for li in range(len(layers))]
+        act_us = [kernel_us(launch_act, li) for li in range(len(layers))]
 
     # ---- end to end through the public API with host buffers (no graph)
     for _ in range(max(1, args.warmup // 2)):
@@ -376,7 +405,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     int8_peak = peaks["bf16_sustained"] * INT8_OVER_BF16_NOMINAL
     gemm_ops = sum(2 * L["spec"].M * L["spec"].N * L["spec"].K + 2 * L["spec"].M * L["spec"].N * L["spec"].r
                    for L in layers)
-    gemm_bytes = sum(layer_gemm_bytes(L["spec"]) for L in layers)
+    gemm_bytes = sum((layer_fused_bytes if fused else layer_gemm_bytes)(L["spec"]) for L in layers)
     gemm_time = sum(gemm_us) * 1e-6
     # hsq_linear_forward launches, for more than 64 tokens, two operand
     # expansions ahead of the GEMM: its time (and so the roofline) includes them
@@ -384,6 +413,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     # up to 8 tokens the forward is the CUDA-core weight stream (its shared-memory
     # limit is far above these shapes' K)
     gemm_label = ("w4a4_gemm_kernel (+ 2 expand_e4m3_kernel: one hsq_linear_forward)" if any(large)
+                  else "w4a4_gemv_kernel, activation step fused in (one hsq_linear_forward_fused)" if fused
                   else "w4a4_gemv_kernel" if all(L["spec"].M <= 8 for L in layers) else "w4a4_gemm_kernel")
     t_tensor = gemm_ops / (int8_peak * 1e12)
     t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
@@ -407,8 +437,8 @@ def run_gpu(args, specs, wl_name, rank, world, local):
         layer_detail.append({"layer": s.name, "M": s.M, "K": s.K, "N": s.N, "r": s.r,
                              "gemm_us": g, "act_us": a,
                              "gemm_tops": gops / (g * 1e-6) / 1e12,
-                             "gemm_gbs": layer_gemm_bytes(s) / (g * 1e-6) / 1e9,
-                             "act_gbs": layer_act_bytes(s) / (a * 1e-6) / 1e9})
+                             "gemm_gbs": (layer_fused_bytes if fused else layer_gemm_bytes)(s) / (g * 1e-6) / 1e9,
+                             "act_gbs": layer_act_bytes(s) / (a * 1e-6) / 1e9 if a > 0 else None})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -423,6 +453,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",
             "config": {"workload": wl_name, "layers": [s.name for s in specs], "tokens_per_step": tokens_step,
                        "r": specs[0].r, "group": specs[0].group, "parallelism": f"replicas x{world}",
+                       "fused_activation_step": fused,
                        "l2": (f"inputs larger than L2: {nrep} replicas of the step's layers (distinct weights, "
                               f"activations, outputs), steps and per-kernel launches cycle through them; "
                               f"{nrep * ws_bytes / 2**20:.0f} MiB in all, {ws_bytes / 2**20:.1f} MiB per step"
@@ -431,7 +462,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             "tokens_per_s": tokens_step * world / (ms_step * 1e-3),
             "e2e": {"value": tops_e2e, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": ms_e2e},
-            "gpu_launches": sum(4 if big else 2 for big in large) * args.steps,
+            "gpu_launches": sum(1 if fused else 4 if big else 2 for big in large) * args.steps,
             "graph": "one step captured in a CUDA graph, replayed K times",
             "roofline": roofline,
             "layers": layer_detail,

@@ -111,11 +111,13 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
  * The layer's forward (Abstract: 4-bit residual product plus the 16-bit
  * low-rank branch):
  *   Y[m,n] = sum_g sx[g][m] * sw[g][n] * P_g[m,n] + sum_j U[m,j] * L2[j,n] + b[n],
- * with P_g the exact integer dot product of group g's codes.  The INT4 codes are
- * multiplied on the tensor cores (tcgen05, kind::i8) one group at a time into
- * Tensor Memory and each group's int32 partial is rescaled into an fp32
+ * with P_g the exact integer dot product of group g's codes.  For M > 8 the
+ * INT4 codes are multiplied on the tensor cores (tcgen05) one group at a time
+ * into Tensor Memory and each group's exact partial is rescaled into an fp32
  * accumulator, which also receives the low-rank branch and the bias before
- * the single rounding to the output type.
+ * the single rounding to the output type.  For M <= 8 the same sums run as a
+ * weight stream on the CUDA cores (integer dot products of the codes), which
+ * needs no workspace.
  *   x_codes/x_scales/U   as written by hsq_quantize_act (U NULL iff r == 0)
  *   w_codes/w_scales     as written by hsq_pack_weights
  *   L2_bf16 [r][N] (NULL iff r == 0), bias_bf16 [N] or NULL for no bias
@@ -173,6 +175,26 @@ hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_sca
                                       const void* L2_bf16, const void* bias_bf16,
                                       int M, int N, int K, int r, int group,
                                       void* Y, hsq_out_dtype out, cudaStream_t stream);
+
+/*
+ * Activation step and forward in one launch, for decode-sized inputs: the
+ * same results as hsq_quantize_act followed by hsq_linear_forward (the same
+ * codes, scales and U, which are kept on chip and not written out), for
+ *   M <= 4 tokens, rank r in {0, 1, 2, 4}, and K small enough that one block
+ *   holds the rows' codes: T * (Kp + 4 * G + 272) bytes <= 200 KiB, T being M
+ *   rounded up to 1, 2 or 4 (so any K <= 47872 for M <= 4).
+ * Other shapes return HSQ_ERR_UNSUPPORTED before anything is launched (use the
+ * two calls).  The pages do not name this fusion; it is the step before the
+ * path (activations quantized online) moved into the path's first kernel.
+ *   X_bf16 [M][K] bf16, s [K] fp32, L1_bf16 [K][r] bf16 (NULL iff r == 0)
+ *   w_codes/w_scales as written by hsq_pack_weights; L2_bf16, bias_bf16, Y, out
+ *   as for hsq_linear_forward.  No workspace.
+ */
+hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const void* L1_bf16,
+                                    const uint8_t* w_codes, const float* w_scales,
+                                    const void* L2_bf16, const void* bias_bf16,
+                                    int M, int N, int K, int r, int group,
+                                    void* Y, hsq_out_dtype out, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* hsq_status_string(hsq_status status);

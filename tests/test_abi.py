@@ -80,6 +80,30 @@ def test_forward_argument_validation():
     assert _fwd(lib, b=MIS) == hsq.HSQ_ERR_ALIGNMENT
 
 
+def test_fused_forward_argument_validation():
+    lib = hsq.load()
+    f = lib.hsq_linear_forward_fused
+
+    def call(**kw):
+        a = dict(X=A, s=A, L1=A, wc=A, ws=A, L2=A, b=None, M=1, N=64, K=64, r=4, g=64, Y=A, out=0)
+        a.update(kw)
+        return f(a["X"], a["s"], a["L1"], a["wc"], a["ws"], a["L2"], a["b"], a["M"], a["N"], a["K"], a["r"],
+                 a["g"], a["Y"], a["out"], None)
+
+    assert call(M=5) == hsq.HSQ_ERR_UNSUPPORTED          # more than 4 tokens: the two-call path
+    assert call(r=3) == hsq.HSQ_ERR_UNSUPPORTED
+    assert call(r=8) == hsq.HSQ_ERR_UNSUPPORTED
+    assert call(M=4, K=65536) == hsq.HSQ_ERR_UNSUPPORTED  # the rows' codes do not fit one block
+    assert call(g=96) == hsq.HSQ_ERR_UNSUPPORTED
+    assert call(M=0) == hsq.HSQ_ERR_INVALID_ARG
+    assert call(X=None) == hsq.HSQ_ERR_INVALID_ARG
+    assert call(L1=None) == hsq.HSQ_ERR_INVALID_ARG      # r > 0 needs L1 and L2
+    assert call(r=0) == hsq.HSQ_ERR_INVALID_ARG          # r == 0 wants L1 == L2 == NULL
+    assert call(X=MIS) == hsq.HSQ_ERR_ALIGNMENT
+    assert hsq.fused_supported(1, 4096, 4) and not hsq.fused_supported(5, 4096, 4)
+    assert hsq.fused_supported(4, 47872, 4) and not hsq.fused_supported(4, 47936, 4)
+
+
 def test_pack_and_act_argument_validation():
     lib = hsq.load()
     pk = lib.hsq_pack_weights

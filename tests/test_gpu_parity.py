@@ -128,6 +128,36 @@ def test_layer_matches_oracle_groups_of_128(M, K, N, r, out):
     _check_all(layer, pl, act, Y, out == hsq.HSQ_OUT_F32, f"g128 {M}x{K}x{N} r{r}", group=128)
 
 
+FUSED_SHAPES = [
+    # (M, K, N, r, group)  -- the single-launch decode forward
+    (1, 4096, 1160, 4, 64),
+    (2, 640, 264, 2, 64),
+    (3, 200, 136, 1, 64),     # K = 200 pads to 256
+    (4, 1152, 520, 0, 64),
+    (1, 1024, 264, 4, 128),
+    (4, 384, 136, 2, 128),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,group", FUSED_SHAPES)
+@pytest.mark.parametrize("out", [hsq.HSQ_OUT_F32, hsq.HSQ_OUT_BF16])
+def test_fused_forward_matches_oracle_and_two_calls(M, K, N, r, group, out):
+    layer = make_layer(_spec(M, K, N, r, seed=11 * M + K + N + r + group))
+    pl, act, Y2, _ = _run_gpu(layer, out, group=group)  # the two calls
+    Yf = torch.empty_like(Y2)
+    hsq.forward_fused(pl, layer.X.to(DEV), Yf, out=out)
+    torch.cuda.synchronize()
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    ref = oracle_layer(layer.X, layer.W, layer.s, layer.L1 if r else None, layer.L2 if r else None, layer.bias,
+                       group=group)
+    check_y(to_np(Yf), ref["Y"], out == hsq.HSQ_OUT_F32, f"fused {M}x{K}x{N} r{r} g{group}")
+    # the same codes and scales, and U up to its fp32 summation order
+    a, b = to_np(Yf).astype(np.float64), to_np(Y2).astype(np.float64)
+    rms = np.sqrt(np.mean(ref["Y"] ** 2))
+    tol = 1e-5 * rms if out == hsq.HSQ_OUT_F32 else 1e-5 * rms + np.abs(b) * 2.0 ** -8
+    assert np.all(np.abs(a - b) <= tol), "fused forward differs from the two calls"
+
+
 def test_strong_low_rank_branch_and_zero_bias():
     """Scale up L1, L2 so that the branch carries a large share of Y: a dropped
     or transposed branch would fail the tolerance by a wide margin."""

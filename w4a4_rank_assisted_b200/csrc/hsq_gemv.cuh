@@ -16,9 +16,17 @@
 // conversion is exact).  The block's activation codes are widened the same way
 // once into shared memory.  Each group partial is scaled by sx*sw in fp32, the
 // low-rank branch and the bias are added, and the warp's sum is written.
+//
+// Fused form (RF >= 0, up to 4 tokens and rank 0, 1, 2 or 4): the block runs the
+// activation step itself in its prologue -- X_hat = X/s, the group codes and
+// scales, U = X_hat L1, with the same arithmetic as quantize_act_kernel, so the
+// codes are the same bits -- straight into shared memory, so that a layer is one
+// launch and nothing of the activation step goes through HBM.  Every block
+// repeats that small step (M*K elements and K*r L1 values, from L2).
 #pragma once
 
 #include "hsq_device.cuh"
+#include "hsq_quant.cuh"
 
 namespace hsq {
 
@@ -34,6 +42,11 @@ struct GemvArgs {
   int ldx, ldw, r, out_f32;
   int M, N, Kp, G;
   int rows_per_block;
+  // fused form: the layer's input instead of x_codes / x_scales / U
+  const __nv_bfloat16* X;   // [M][K]
+  const float* s;           // [K]
+  const __nv_bfloat16* L1;  // [K][r]
+  int K, group;
 };
 
 constexpr int kGemvThreads = 512;
@@ -44,20 +57,24 @@ constexpr int kGemvBatch = 4;
 constexpr int kGemvDepth = 2;
 
 // Shared memory of one block: widened activation codes (even and odd codes of
-// every packed word, MT*Kp bytes) and the activation scales [G][MT].
+// every packed word, MT*Kp bytes), the activation scales [G][MT] and, fused, U
+// [MT][4] with its per-warp partials [16][MT][4].
 __host__ __device__ constexpr size_t gemv_smem_bytes(int MT, int Kp, int G) {
-  return static_cast<size_t>(MT) * Kp + static_cast<size_t>(G) * MT * 4;
+  return static_cast<size_t>(MT) * Kp + static_cast<size_t>(G) * MT * 4 + (kGemvThreads / 32 + 1) * MT * 4 * 4;
 }
 
 // MT: tokens the kernel is built for (M <= MT); LPG: lanes per scale group (a
-// lane holds 32 codes, so 2 for groups of 64 and 4 for groups of 128).
-template <int MT, int LPG>
+// lane holds 32 codes, so 2 for groups of 64 and 4 for groups of 128); RF: -1
+// reads the activation step's outputs, 0/1/2/4 is the fused form of that rank.
+template <int MT, int LPG, int RF = -1>
 __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvArgs a) {
   extern __shared__ __align__(16) uint8_t gemv_smem[];
   const int W4 = a.Kp / 8;  // packed 32-bit words per row
   uint32_t* xlo = reinterpret_cast<uint32_t*>(gemv_smem);  // [MT][W4] even codes, int8 16*q
   uint32_t* xhi = xlo + MT * W4;                           // [MT][W4] odd codes
   float* sxs = reinterpret_cast<float*>(xhi + MT * W4);     // [G][MT]
+  float* Us = sxs + a.G * MT;                               // fused: U [MT][4]
+  float* upart = Us + MT * 4;                               // fused: [warp][MT][4]
   const int warp = threadIdx.x >> 5, lane = lane_id();
   const int nwarps = blockDim.x >> 5;
   const int nch = a.Kp / 32;  // 16-byte chunks per row (a multiple of LPG)
@@ -91,17 +108,98 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
 #pragma unroll
   for (int d = 0; d + 1 < kGemvDepth; ++d)
     if (d < total) load(d, wb[d], sb[d]);
-  grid_dep_wait();  // the activation codes come from the preceding kernel
-  for (int i = threadIdx.x; i < MT * W4; i += blockDim.x) {
-    const int m = i / W4, j = i - m * W4;
-    uint32_t w = 0u;
-    if (m < a.M) w = __ldg(reinterpret_cast<const unsigned int*>(a.x_codes + static_cast<size_t>(m) * (a.Kp / 2)) + j);
-    xlo[i] = (w << 4) & 0xF0F0F0F0u;
-    xhi[i] = w & 0xF0F0F0F0u;
-  }
-  for (int i = threadIdx.x; i < a.G * MT; i += blockDim.x) {
-    const int g = i / MT, m = i - g * MT;
-    sxs[i] = m < a.M ? __ldg(a.x_scales + static_cast<size_t>(g) * a.ldx + m) : 0.f;
+  grid_dep_wait();  // the activation codes (or X) come from the preceding kernel
+  const float* Uv = a.U;  // U [M][r]: the activation step's, or this block's own (fused)
+  if constexpr (RF < 0) {
+    for (int i = threadIdx.x; i < MT * W4; i += blockDim.x) {
+      const int m = i / W4, j = i - m * W4;
+      uint32_t w = 0u;
+      if (m < a.M) w = __ldg(reinterpret_cast<const unsigned int*>(a.x_codes + static_cast<size_t>(m) * (a.Kp / 2)) + j);
+      xlo[i] = (w << 4) & 0xF0F0F0F0u;
+      xhi[i] = w & 0xF0F0F0F0u;
+    }
+    for (int i = threadIdx.x; i < a.G * MT; i += blockDim.x) {
+      const int g = i / MT, m = i - g * MT;
+      sxs[i] = m < a.M ? __ldg(a.x_scales + static_cast<size_t>(g) * a.ldx + m) : 0.f;
+    }
+  } else {
+    // the activation step: warp w takes (token, 256-channel chunk) pairs w, w + 16, ...;
+    // a lane handles 8 channels, as in quantize_act_kernel
+    constexpr int RA = RF > 0 ? RF : 1;
+    const int nchk = (a.Kp + 255) / 256;
+    float u[MT][RA];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int j = 0; j < RA; ++j) u[m][j] = 0.f;
+    for (int pc = warp; pc < MT * nchk; pc += nwarps) {
+      const int m = pc / nchk, c = pc - (pc / nchk) * nchk;  // warp-uniform
+      const int k0 = c * 256 + lane * 8;
+      const bool real = m < a.M && k0 < a.K;  // K % 8 == 0: all 8 channels real or all padding
+      const bool in_k = k0 < a.Kp;
+      float sv[8], sz[8];
+      if (real) {
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(a.s + k0));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(a.s + k0 + 4));
+        sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+        sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sv[e] = 1.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sz[e] = __frcp_rn(sv[e]);
+      const uint4 raw = real ? __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(m) * a.K + k0))
+                             : make_uint4(0u, 0u, 0u, 0u);
+      float xh[8];
+      smooth8(raw, sv, sz, real, xh);
+      float sc;
+      const uint32_t packed = LPG == 2 ? quantize8_fast<8>(xh, sc) : quantize8_fast<16>(xh, sc);
+      if (in_k) {
+        const int j = k0 / 8;  // the lane's packed word
+        xlo[m * W4 + j] = (packed << 4) & 0xF0F0F0F0u;
+        xhi[m * W4 + j] = packed & 0xF0F0F0F0u;
+        if ((lane & (4 * LPG - 1)) == 0) sxs[(k0 / a.group) * MT + m] = sc;  // (0 for padding rows)
+      }
+      if constexpr (RF > 0) {
+        // the 8 channels' L1 rows (8*RF bf16, contiguous)
+        if (real) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.L1 + static_cast<size_t>(k0) * RF);
+#pragma unroll
+          for (int v = 0; v < RF; ++v) {
+            float f[8];
+            bf16x8_to_f32(__ldg(src + v), f);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              const int e = (v * 8 + t) / RF, jr = (v * 8 + t) % RF;
+#pragma unroll
+              for (int mm = 0; mm < MT; ++mm)
+                if (mm == m) u[mm][jr] = fmaf(xh[e], f[t], u[mm][jr]);
+            }
+          }
+        }
+      }
+    }
+    if constexpr (RF > 0) {
+      // U: lanes, then warps in a fixed order
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < RF; ++j) {
+          float v = u[m][j];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) upart[(warp * MT + m) * 4 + j] = v;
+        }
+      __syncthreads();
+      if (threadIdx.x < MT * RF) {
+        const int m = threadIdx.x / RF, j = threadIdx.x - (threadIdx.x / RF) * RF;
+        float v = 0.f;
+        for (int w = 0; w < nwarps; ++w) v += upart[(w * MT + m) * 4 + j];
+        Us[m * RF + j] = v;
+      }
+    }
+    Uv = Us;
   }
   __syncthreads();
   if (threadIdx.x == 0) grid_dep_launch();
@@ -148,7 +246,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
       const float l2 = __bfloat162float(a.L2[static_cast<size_t>(lane) * a.N + n]);
 #pragma unroll
       for (int m = 0; m < MT; ++m)
-        if (m < a.M) acc[m] = fmaf(__ldg(a.U + static_cast<size_t>(m) * a.r + lane), l2, acc[m]);
+        if (m < a.M) acc[m] = fmaf(Uv[m * a.r + lane], l2, acc[m]);
     }
 #pragma unroll
     for (int m = 0; m < MT; ++m)

@@ -376,7 +376,7 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
-template <int MT, int LPG>
+template <int MT, int LPG, int RF = -1>
 hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
   static std::mutex mu;
   static bool attr_set[64] = {false};
@@ -385,7 +385,7 @@ hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-      if (cudaFuncSetAttribute(hsq::w4a4_gemv_kernel<MT, LPG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(hsq::w4a4_gemv_kernel<MT, LPG, RF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kGemvSmemMax)) != cudaSuccess)
         return HSQ_ERR_CUDA;
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
@@ -393,7 +393,7 @@ hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
   }
   const size_t smem = hsq::gemv_smem_bytes(MT, a.Kp, a.G);
   // starts early: it waits for the activation step before reading its codes
-  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG>, dim3(p.grid), dim3(hsq::kGemvThreads), smem, st, a) !=
+  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG, RF>, dim3(p.grid), dim3(hsq::kGemvThreads), smem, st, a) !=
       cudaSuccess)
     return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
@@ -683,6 +683,57 @@ hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_sca
   }
   return hsq_linear_forward(x_codes, x_scales, U, w_codes, w_scales, L2_bf16, bias_bf16, M, N, K, r, group, Y, out,
                             scratch, scratch ? kNoallocScratchBytes : 0, stream);
+}
+
+hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const void* L1_bf16, const uint8_t* w_codes,
+                                    const float* w_scales, const void* L2_bf16, const void* bias_bf16, int M, int N,
+                                    int K, int r, int group, void* Y, hsq_out_dtype out, cudaStream_t stream) {
+  hsq_status st = check_common(M, K, r, group);
+  if (st != HSQ_OK) return st;
+  if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return HSQ_ERR_UNSUPPORTED;
+  if (out != HSQ_OUT_BF16 && out != HSQ_OUT_F32) return HSQ_ERR_INVALID_ARG;
+  if (!X_bf16 || !s || !w_codes || !w_scales || !Y) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1_bf16 != nullptr) || (r > 0) != (L2_bf16 != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(Y) ||
+      (L1_bf16 && !aligned16(L1_bf16)) || (L2_bf16 && !aligned16(L2_bf16)) || (bias_bf16 && !aligned16(bias_bf16)))
+    return HSQ_ERR_ALIGNMENT;
+  const int G = groups_of(K, group), Kp = G * group;
+  const int mt = gemv_mt(M);
+  if (M > 4 || !(r == 0 || r == 1 || r == 2 || r == 4) || hsq::gemv_smem_bytes(mt, Kp, G) > kGemvSmemMax)
+    return HSQ_ERR_UNSUPPORTED;
+  const int nsm = device_sm_count();
+  Plan p{};
+  p.kind = kGemv;
+  p.grid = std::min(nsm, (N + 15) / 16);
+  hsq::GemvArgs ga{};
+  ga.w_codes = w_codes; ga.w_scales = w_scales; ga.ldw = scales_ld(N);
+  ga.r = r;
+  ga.L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
+  ga.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+  ga.Y = Y;
+  ga.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
+  ga.M = M; ga.N = N; ga.Kp = Kp; ga.G = G;
+  ga.rows_per_block = (N + p.grid - 1) / p.grid;
+  ga.X = static_cast<const __nv_bfloat16*>(X_bf16);
+  ga.s = s;
+  ga.L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
+  ga.K = K; ga.group = group;
+  const bool g128 = group == 128;
+#define HSQ_FUSED(MTV, RV) \
+  return g128 ? launch_gemv<MTV, 4, RV>(p, ga, stream) : launch_gemv<MTV, 2, RV>(p, ga, stream)
+#define HSQ_FUSED_R(MTV)          \
+  switch (r) {                    \
+    case 0: HSQ_FUSED(MTV, 0);    \
+    case 1: HSQ_FUSED(MTV, 1);    \
+    case 2: HSQ_FUSED(MTV, 2);    \
+    default: HSQ_FUSED(MTV, 4);   \
+  }
+  if (mt == 1) HSQ_FUSED_R(1);
+  if (mt == 2) HSQ_FUSED_R(2);
+  HSQ_FUSED_R(4);
+#undef HSQ_FUSED_R
+#undef HSQ_FUSED
 }
 
 }  // extern "C"

@@ -60,6 +60,33 @@ __device__ __forceinline__ float div_by_recip(float x, float y, float z) {
   return __fmaf_rn(r, z, q);
 }
 
+// X_hat = x / s for a lane's 8 channels (bf16 x, fp32 s and its reciprocal z):
+// product and correction, exact for normal operands and quotients and for
+// x = 0; the warp takes the guarded division only if some lane holds an element
+// outside [2^-100, 2^100].  Padding channels (real = false) give 0.  Every lane
+// of the warp must call it (it votes).
+__device__ __forceinline__ void smooth8(const uint4& raw, const float (&sv)[8], const float (&sz)[8], bool real,
+                                        float (&xh)[8]) {
+  float x[8];
+  bf16x8_to_f32(raw, x);
+  bool odd = false;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float ax = fabsf(x[e]);
+    odd |= (ax != 0.f) & ((ax < 0x1p-100f) | (ax > 0x1p100f));
+    const float q0 = __fmul_rn(x[e], sz[e]);
+    xh[e] = __fmaf_rn(__fmaf_rn(-q0, sv[e], x[e]), sz[e], q0);
+  }
+  if (__any_sync(0xffffffffu, odd)) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xh[e] = div_by_recip(x[e], sv[e], sz[e]);
+  }
+  if (!real) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xh[e] = 0.f;
+  }
+}
+
 // Round-half-even of |t| < 2^22 to an integer: add 1.5*2^23 (the sum's last
 // mantissa bit is then the units place) and read the integer from the bits.
 __device__ __forceinline__ int rint_small(float t) {
@@ -279,27 +306,8 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
     for (int i = 0; i < SUB; ++i) {
       const int m = mb + i;
       if (m >= M) break;  // warp-uniform
-      float x[8], xh[8];
-      bf16x8_to_f32(xr[i], x);
-      // X_hat = x / s: product and correction (exact for normal operands and
-      // quotients, and for x = 0); the warp takes the guarded division only
-      // if some lane holds an element outside [2^-100, 2^100]
-      bool odd = false;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float ax = fabsf(x[e]);
-        odd |= (ax != 0.f) & ((ax < 0x1p-100f) | (ax > 0x1p100f));
-        const float q0 = __fmul_rn(x[e], sz[e]);
-        xh[e] = __fmaf_rn(__fmaf_rn(-q0, sv[e], x[e]), sz[e], q0);
-      }
-      if (__any_sync(0xffffffffu, odd)) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xh[e] = div_by_recip(x[e], sv[e], sz[e]);
-      }
-      if (!real) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xh[e] = 0.f;
-      }
+      float xh[8];
+      smooth8(xr[i], sv, sz, real, xh);
       if constexpr (R > 0 && R <= 4) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)

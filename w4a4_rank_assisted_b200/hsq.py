@@ -35,7 +35,7 @@ EXPORTED = (
     "hsq_num_groups", "hsq_codes_bytes", "hsq_scales_ld", "hsq_scales_bytes",
     "hsq_workspace_bytes", "hsq_pack_weights", "hsq_quantize_act",
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
-    "hsq_debug_force_timeout", "hsq_linear_forward_noalloc",
+    "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused",
 )
 
 
@@ -77,6 +77,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_linear_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, sz, vp]
     lib.hsq_linear_forward.restype = i
     lib.hsq_linear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
+    lib.hsq_linear_forward_fused.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
+    lib.hsq_linear_forward_fused.restype = i
     lib.hsq_linear_forward_noalloc.restype = i
     lib.hsq_status_string.argtypes = [i]; lib.hsq_status_string.restype = c.c_char_p
     lib.hsq_get_device_status.argtypes = [vp]; lib.hsq_get_device_status.restype = i
@@ -166,6 +168,25 @@ def hsq_linear_forward_noalloc(x_codes, x_scales, U, w_codes, w_scales, L2, bias
            "hsq_linear_forward_noalloc")
 
 
+def hsq_linear_forward_fused(X, s, L1, w_codes, w_scales, L2, bias, M, N, K, r, Y,
+                             out: int = HSQ_OUT_BF16, group=GROUP, stream=None) -> None:
+    """The activation step and the forward in one launch (M <= 4, r in
+    {0, 1, 2, 4}); HSQ_ERR_UNSUPPORTED otherwise."""
+    _check(load().hsq_linear_forward_fused(_ptr(X), _ptr(s), _ptr(L1), _ptr(w_codes), _ptr(w_scales),
+                                           _ptr(L2), _ptr(bias), M, N, K, r, group, _ptr(Y), int(out),
+                                           _stream(stream)),
+           "hsq_linear_forward_fused")
+
+
+def fused_supported(M: int, K: int, r: int, group: int = GROUP) -> bool:
+    """Whether hsq_linear_forward_fused takes this shape (mirrors its checks)."""
+    if M < 1 or M > 4 or r not in (0, 1, 2, 4):
+        return False
+    G = hsq_num_groups(K, group)
+    mt = 1 if M <= 1 else 2 if M <= 2 else 4
+    return mt * (G * group + 4 * G + 272) <= 200 * 1024
+
+
 def hsq_get_device_status(stream=None) -> int:
     return load().hsq_get_device_status(_stream(stream))
 
@@ -217,6 +238,16 @@ class ActBuffers:
         self.x_codes = alloc_codes(M, K, device, group)
         self.x_scales = alloc_scales(M, K, device, group)
         self.U = torch.empty((M, r), dtype=torch.float32, device=device) if r > 0 else None
+
+
+def forward_fused(layer: PackedLinear, X: torch.Tensor, Y: torch.Tensor, out: int = HSQ_OUT_BF16,
+                  stream=None) -> torch.Tensor:
+    """One forward of the layer in a single launch (decode sizes, see
+    hsq_linear_forward_fused)."""
+    hsq_linear_forward_fused(X, layer.s, layer.L1, layer.w_codes, layer.w_scales, layer.L2, layer.bias,
+                             X.shape[0], layer.N, layer.K, layer.r, Y, out=out, group=layer.group,
+                             stream=stream)
+    return Y
 
 
 def forward(layer: PackedLinear, X: torch.Tensor, act: ActBuffers, Y: torch.Tensor,
