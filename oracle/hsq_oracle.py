@@ -239,6 +239,29 @@ def dense_forward(X, W, bias):
     return Y
 
 
+def lowrank_init(W, s, r):
+    """Plain truncated-SVD initialisation of the low-rank pair.
+
+    The pages name it as the "Plain SVD" row of the L1-initialisation ablation
+    (Table 6 of the paper, shd-paper.top): the protected subspace L1 is taken
+    from the singular vectors of the smoothed weight.  Reading: L1 [K, r] holds
+    the top-r right singular vectors of W_hat = W diag(s) (orthonormal columns,
+    the protected subspace of Figure 1's caption) and L2 [r, N] = L1^T W_hat^T,
+    its least-squares partner, so that (L1 L2)^T is the best rank-r
+    approximation of W_hat (Eckart-Young).  Sign convention: each column of L1
+    has its entry of largest magnitude positive (lowest index on ties).  All in
+    fp64; returns (L1, L2, singular values of W_hat)."""
+    What = np.asarray(W, dtype=f64) * np.asarray(s, dtype=f64)[None, :]
+    _, sv, Vt = np.linalg.svd(What, full_matrices=False)
+    L1 = Vt[:r].T.copy()
+    for j in range(r):
+        i = int(np.argmax(np.abs(L1[:, j])))
+        if L1[i, j] < 0:
+            L1[:, j] = -L1[:, j]
+    L2 = L1.T @ What.T
+    return L1, L2, sv
+
+
 def bf16_ulp(y):
     """Spacing of bf16 numbers at |y| (fp64), used by the bf16-output tolerance."""
     y = np.abs(np.asarray(y, dtype=f64))

@@ -392,3 +392,61 @@ def test_brute_force_tiny_layers_groups_of_128():
                     y += U[m, j] * float(L2[j, n])
                 y += float(b[n])
                 assert Y[m, n] == pytest.approx(y, rel=1e-12, abs=1e-12)
+
+
+# ---------------------------------------------------------------- truncated-SVD initialisation
+def _orthonormal(rng, n, k):
+    q, _ = np.linalg.qr(rng.standard_normal((n, k)))
+    return q
+
+
+def test_lowrank_init_recovers_a_planted_decomposition():
+    """W_hat = U diag(sigma) V^T built from known orthonormal factors and known
+    singular values: L1 spans V's first r columns, (L1 L2)^T leaves exactly the
+    tail energy sqrt(sum_{i>r} sigma_i^2), and L1 is orthonormal."""
+    rng = np.random.default_rng(5)
+    N, K, r = 40, 24, 4
+    U, V = _orthonormal(rng, N, K), _orthonormal(rng, K, K)
+    sigma = np.array([50.0, 30.0, 20.0, 12.0] + list(np.linspace(3.0, 0.5, K - 4)))
+    What = U @ np.diag(sigma) @ V.T
+    s = rng.uniform(0.5, 2.0, K)
+    W = What / s[None, :]  # so that W diag(s) is the planted matrix
+    L1, L2, _ = O.lowrank_init(W, s, r)
+    assert np.allclose(L1.T @ L1, np.eye(r), atol=1e-12)
+    P1, Pv = L1 @ L1.T, V[:, :r] @ V[:, :r].T
+    assert np.max(np.abs(P1 - Pv)) < 1e-10
+    err = np.linalg.norm(What.T - L1 @ L2)
+    assert abs(err - np.sqrt(np.sum(sigma[r:] ** 2))) < 1e-9 * err
+    # sign convention: the largest-magnitude entry of each column is positive
+    for j in range(r):
+        assert L1[np.argmax(np.abs(L1[:, j])), j] > 0
+
+
+def test_lowrank_init_exact_for_rank_r_weights():
+    rng = np.random.default_rng(6)
+    N, K, r = 30, 20, 3
+    What = rng.standard_normal((N, r)) @ rng.standard_normal((r, K))
+    L1, L2, _ = O.lowrank_init(What, np.ones(K), r)
+    assert np.max(np.abs(L1 @ L2 - What.T)) < 1e-11 * np.max(np.abs(What))
+
+
+def test_lowrank_init_picks_the_largest_axes_of_a_scaled_selection():
+    """W with one nonzero per row in distinct columns: its singular vectors are
+    coordinate axes, so L1's columns are the unit vectors of the r largest |W|
+    entries (in that order, positive) and L2 holds those entries."""
+    N, K, r = 6, 8, 3
+    W = np.zeros((N, K))
+    cols, vals = [5, 1, 7, 2, 0, 4], [2.0, -9.0, 4.0, -1.0, 6.5, 3.0]
+    for n, (c, v) in enumerate(zip(cols, vals)):
+        W[n, c] = v
+    s = np.full(K, 0.5)  # smoothing scales every singular value by 0.5
+    L1, L2, sv = O.lowrank_init(W, s, r)
+    order = [1, 4, 2]  # rows with |v| = 9, 6.5, 4
+    for j, n in enumerate(order):
+        e = np.zeros(K)
+        e[cols[n]] = 1.0
+        assert np.allclose(L1[:, j], e, atol=1e-12)
+        expect = np.zeros(N)
+        expect[n] = 0.5 * vals[n]
+        assert np.allclose(L2[j], expect, atol=1e-12)
+    assert np.allclose(sv[:r], [4.5, 3.25, 2.0])
