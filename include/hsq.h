@@ -196,6 +196,28 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
                                     int M, int N, int K, int r, int group,
                                     void* Y, hsq_out_dtype out, cudaStream_t stream);
 
+/*
+ * Pack-time helper: plain truncated-SVD initialisation of the low-rank pair
+ * (Table 6 of the paper, "Plain SVD" row of the L1-initialisation ablation), so
+ * that weights without a calibrated pair can be packed.  Not on the forward path.
+ *   L1 out [K][r] bf16: the top-r right singular vectors of W_hat = W diag(s)
+ *     (orthonormal columns; each column's entry of largest magnitude positive)
+ *   L2 out [r][N] bf16: L1^T W_hat^T, so that (L1 L2)^T approximates the best
+ *     rank-r approximation of W_hat
+ * by subspace iteration with r + 8 columns from a random start drawn from
+ * `seed` (the same seed gives the same result), `iters` iterations (0..64;
+ * more sharpen the subspace when W_hat's singular values r and r+1 are close),
+ * then Rayleigh-Ritz.  W_bf16 [N][K], s [K] as for hsq_pack_weights; 1 <= r <=
+ * min(32, N, K) (else HSQ_ERR_UNSUPPORTED).  workspace: at least
+ * hsq_lowrank_workspace_bytes(N, K, r) bytes (about 4 N K).  The large products
+ * are fp32 cuBLAS GEMMs; the library keeps one cuBLAS handle per device (which
+ * holds device memory of its own) and serialises these calls.
+ */
+size_t hsq_lowrank_workspace_bytes(int N, int K, int r);
+hsq_status hsq_lowrank_init(const void* W_bf16, const float* s, int N, int K, int r, int iters,
+                            unsigned long long seed, void* L1_bf16, void* L2_bf16,
+                            void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* hsq_status_string(hsq_status status);
 

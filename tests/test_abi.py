@@ -104,6 +104,29 @@ def test_fused_forward_argument_validation():
     assert hsq.fused_supported(4, 47872, 4) and not hsq.fused_supported(4, 47936, 4)
 
 
+def test_lowrank_helper_argument_validation():
+    lib = hsq.load()
+    f = lib.hsq_lowrank_init
+    ws = hsq.hsq_lowrank_workspace_bytes(64, 32, 4)
+    assert ws >= 4 * 64 * 32
+    assert hsq.hsq_lowrank_workspace_bytes(64, 32, 0) == 0
+    assert hsq.hsq_lowrank_workspace_bytes(64, 32, 33) == 0
+
+    def call(**kw):
+        a = dict(W=A, s=A, N=64, K=32, r=4, it=8, seed=0, L1=A, L2=A, ws=A, wsb=ws)
+        a.update(kw)
+        return f(a["W"], a["s"], a["N"], a["K"], a["r"], a["it"], a["seed"], a["L1"], a["L2"], a["ws"], a["wsb"],
+                 None)
+
+    assert call(r=0) == hsq.HSQ_ERR_UNSUPPORTED
+    assert call(r=33) == hsq.HSQ_ERR_UNSUPPORTED
+    assert call(N=16, K=8, r=9) == hsq.HSQ_ERR_UNSUPPORTED   # rank above min(N, K)
+    assert call(it=65) == hsq.HSQ_ERR_INVALID_ARG
+    assert call(ws=None) == hsq.HSQ_ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == hsq.HSQ_ERR_INVALID_ARG
+    assert call(W=MIS) == hsq.HSQ_ERR_ALIGNMENT
+
+
 def test_pack_and_act_argument_validation():
     lib = hsq.load()
     pk = lib.hsq_pack_weights

@@ -4,6 +4,7 @@
 // Everything numeric happens in the kernels of hsq_quant.cuh and hsq_gemm.cuh;
 // this file only checks arguments (synchronously, before any launch) and
 // launches them.  It allocates no device memory.
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -16,6 +17,7 @@
 #include "hsq_device.cuh"
 #include "hsq_gemm.cuh"
 #include "hsq_gemv.cuh"
+#include "hsq_lowrank.cuh"
 #include "hsq_quant.cuh"
 
 namespace {
@@ -399,9 +401,134 @@ hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ truncated-SVD helper
+// Workspace carve-up of hsq_lowrank_init (each part 256-byte aligned).
+struct LrLayout {
+  int p;
+  size_t A, Q, Y, Z, Z64, Q64, Y64, G, Rinv, V, L1c, C, end;
+};
+
+LrLayout lr_layout(int N, int K, int r) {
+  LrLayout L{};
+  L.p = std::min(r + hsq::kLrOversample, std::min(N, K));
+  const size_t p = static_cast<size_t>(L.p);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return at;
+  };
+  L.A = take(4ull * N * K);
+  L.Q = take(4 * K * p);
+  L.Y = take(4 * N * p);
+  L.Z = take(4 * K * p);
+  L.Z64 = take(8 * K * p);
+  L.Q64 = take(8 * K * p);
+  L.Y64 = take(8 * N * p);
+  L.G = take(8 * p * p);
+  L.Rinv = take(8 * p * p);
+  L.V = take(4 * p * p);
+  L.L1c = take(4ull * K * r);
+  L.C = take(4ull * N * r);
+  L.end = off;
+  return L;
+}
+
+// One cuBLAS handle per device, created on first use (creating one costs
+// milliseconds); calls on it are serialised.
+struct BlasSlot {
+  std::mutex mu;
+  cublasHandle_t h = nullptr;
+};
+BlasSlot g_blas[kMaxDevices];
+
 }  // namespace
 
 extern "C" {
+
+size_t hsq_lowrank_workspace_bytes(int N, int K, int r) {
+  if (N < 1 || K < 1 || r < 1 || r > kMaxRank || r > std::min(N, K)) return 0;
+  return lr_layout(N, K, r).end;
+}
+
+hsq_status hsq_lowrank_init(const void* W_bf16, const float* s, int N, int K, int r, int iters,
+                            unsigned long long seed, void* L1_bf16, void* L2_bf16, void* workspace,
+                            size_t ws_bytes, cudaStream_t stream) {
+  if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return HSQ_ERR_INVALID_ARG;
+  if (r < 1 || r > kMaxRank || r > std::min(N, K)) return HSQ_ERR_UNSUPPORTED;
+  if (iters < 0 || iters > 64) return HSQ_ERR_INVALID_ARG;
+  if (!W_bf16 || !s || !L1_bf16 || !L2_bf16 || !workspace) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(L1_bf16) || !aligned16(L2_bf16) || !aligned16(workspace))
+    return HSQ_ERR_ALIGNMENT;
+  const LrLayout L = lr_layout(N, K, r);
+  if (ws_bytes < L.end) return HSQ_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSQ_ERR_CUDA;
+  BlasSlot& slot = g_blas[dev];
+  std::lock_guard<std::mutex> lk(slot.mu);
+  if (!slot.h && cublasCreate(&slot.h) != CUBLAS_STATUS_SUCCESS) {
+    slot.h = nullptr;
+    return HSQ_ERR_CUDA;
+  }
+  cublasHandle_t h = slot.h;
+  if (cublasSetStream(h, stream) != CUBLAS_STATUS_SUCCESS ||
+      cublasSetMathMode(h, CUBLAS_DEFAULT_MATH) != CUBLAS_STATUS_SUCCESS)  // plain fp32, no TF32
+    return HSQ_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* A = reinterpret_cast<float*>(ws + L.A);
+  float* Q = reinterpret_cast<float*>(ws + L.Q);
+  float* Y = reinterpret_cast<float*>(ws + L.Y);
+  float* Z = reinterpret_cast<float*>(ws + L.Z);
+  double* Z64 = reinterpret_cast<double*>(ws + L.Z64);
+  double* Q64 = reinterpret_cast<double*>(ws + L.Q64);
+  double* Y64 = reinterpret_cast<double*>(ws + L.Y64);
+  double* G = reinterpret_cast<double*>(ws + L.G);
+  double* Rinv = reinterpret_cast<double*>(ws + L.Rinv);
+  float* V = reinterpret_cast<float*>(ws + L.V);
+  float* L1c = reinterpret_cast<float*>(ws + L.L1c);
+  float* C = reinterpret_cast<float*>(ws + L.C);
+  const int p = L.p;
+  const int blocks = 4 * device_sm_count();
+  const float one = 1.f, zero = 0.f;
+  const double done = 1.0, dzero = 0.0;
+  bool ok = true;
+  auto blas = [&](cublasStatus_t st) { ok = ok && st == CUBLAS_STATUS_SUCCESS; };
+  // orthonormalise the K x p matrix Z (fp32) into Q (fp32): CholeskyQR twice, in fp64
+  auto orth = [&]() {
+    hsq::lr_to_f64_kernel<<<blocks, 256, 0, stream>>>(Z, Z64, static_cast<size_t>(K) * p);
+    double* src = Z64;
+    double* dst = Q64;
+    for (int pass = 0; pass < 2; ++pass) {
+      blas(cublasDgemm(h, CUBLAS_OP_T, CUBLAS_OP_N, p, p, K, &done, src, K, src, K, &dzero, G, p));
+      hsq::lr_chol_inv_kernel<<<1, hsq::kLrMaxP, 0, stream>>>(G, p, Rinv);
+      blas(cublasDgemm(h, CUBLAS_OP_N, CUBLAS_OP_N, K, p, p, &done, src, K, Rinv, p, &dzero, dst, K));
+      std::swap(src, dst);
+    }
+    hsq::lr_to_f32_kernel<<<blocks, 256, 0, stream>>>(src, Q, static_cast<size_t>(K) * p);
+  };
+  hsq::lr_smooth_kernel<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(W_bf16), s, N, K, A);
+  hsq::lr_random_kernel<<<blocks, 256, 0, stream>>>(Z, static_cast<size_t>(K) * p, seed);
+  orth();
+  for (int it = 0; it < iters && ok; ++it) {
+    // Z = W_hat^T (W_hat Q): Y = A^T Q (N x p), Z = A Y (K x p)
+    blas(cublasSgemm(h, CUBLAS_OP_T, CUBLAS_OP_N, N, p, K, &one, A, K, Q, K, &zero, Y, N));
+    blas(cublasSgemm(h, CUBLAS_OP_N, CUBLAS_OP_N, K, p, N, &one, A, K, Y, N, &zero, Z, K));
+    orth();
+  }
+  // Rayleigh-Ritz: T = (W_hat Q)^T (W_hat Q) in fp64, its eigenvectors V
+  blas(cublasSgemm(h, CUBLAS_OP_T, CUBLAS_OP_N, N, p, K, &one, A, K, Q, K, &zero, Y, N));
+  hsq::lr_to_f64_kernel<<<blocks, 256, 0, stream>>>(Y, Y64, static_cast<size_t>(N) * p);
+  blas(cublasDgemm(h, CUBLAS_OP_T, CUBLAS_OP_N, p, p, N, &done, Y64, N, Y64, N, &dzero, G, p));
+  hsq::lr_jacobi_kernel<<<1, hsq::kLrMaxP, 0, stream>>>(G, p, V);
+  // L1 = Q V[:, :r] (K x r), C = W_hat L1 (N x r) = L2^T
+  blas(cublasSgemm(h, CUBLAS_OP_N, CUBLAS_OP_N, K, r, p, &one, Q, K, V, p, &zero, L1c, K));
+  blas(cublasSgemm(h, CUBLAS_OP_T, CUBLAS_OP_N, N, r, K, &one, A, K, L1c, K, &zero, C, N));
+  hsq::lr_sign_out_kernel<<<r, 256, 0, stream>>>(L1c, C, K, N, r, static_cast<__nv_bfloat16*>(L1_bf16),
+                                                   static_cast<__nv_bfloat16*>(L2_bf16));
+  if (!ok) return HSQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
 
 int hsq_num_groups(int K, int group) {
   if (group <= 0 || K < 0) return 0;

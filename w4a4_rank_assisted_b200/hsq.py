@@ -36,6 +36,7 @@ EXPORTED = (
     "hsq_workspace_bytes", "hsq_pack_weights", "hsq_quantize_act",
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
     "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused",
+    "hsq_lowrank_workspace_bytes", "hsq_lowrank_init",
 )
 
 
@@ -79,6 +80,9 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_linear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
     lib.hsq_linear_forward_fused.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
     lib.hsq_linear_forward_fused.restype = i
+    lib.hsq_lowrank_workspace_bytes.argtypes = [i, i, i]; lib.hsq_lowrank_workspace_bytes.restype = sz
+    lib.hsq_lowrank_init.argtypes = [vp, vp, i, i, i, i, c.c_ulonglong, vp, vp, vp, sz, vp]
+    lib.hsq_lowrank_init.restype = i
     lib.hsq_linear_forward_noalloc.restype = i
     lib.hsq_status_string.argtypes = [i]; lib.hsq_status_string.restype = c.c_char_p
     lib.hsq_get_device_status.argtypes = [vp]; lib.hsq_get_device_status.restype = i
@@ -185,6 +189,23 @@ def fused_supported(M: int, K: int, r: int, group: int = GROUP) -> bool:
     G = hsq_num_groups(K, group)
     mt = 1 if M <= 1 else 2 if M <= 2 else 4
     return mt * (G * group + 4 * G + 272) <= 200 * 1024
+
+
+def hsq_lowrank_workspace_bytes(N: int, K: int, r: int) -> int:
+    return int(load().hsq_lowrank_workspace_bytes(N, K, r))
+
+
+def lowrank_init(W: torch.Tensor, s: torch.Tensor, r: int, iters: int = 8, seed: int = 0, stream=None):
+    """Plain truncated-SVD L1 [K, r], L2 [r, N] (bf16) of W diag(s) on the GPU
+    (pack-time helper; see hsq_lowrank_init)."""
+    N, K = W.shape
+    ws = torch.empty(max(1, hsq_lowrank_workspace_bytes(N, K, r)), dtype=torch.uint8, device=W.device)
+    L1 = torch.empty((K, r), dtype=torch.bfloat16, device=W.device)
+    L2 = torch.empty((r, N), dtype=torch.bfloat16, device=W.device)
+    _check(load().hsq_lowrank_init(_ptr(W), _ptr(s), N, K, r, iters, int(seed) & ((1 << 64) - 1), _ptr(L1),
+                                   _ptr(L2), _ptr(ws), ws.numel(), _stream(stream)),
+           "hsq_lowrank_init")
+    return L1, L2
 
 
 def hsq_get_device_status(stream=None) -> int:
