@@ -132,25 +132,40 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
     for (int m = 0; m < MT; ++m)
 #pragma unroll
       for (int j = 0; j < RA; ++j) u[m][j] = 0.f;
+    // a chunk's X row, smoothing factors and L1 rows are requested one chunk ahead
+    constexpr int RL = RF > 0 ? RF : 1;
+    auto ld = [&](int pc, uint4& raw, float4& s0, float4& s1, uint4 (&l1)[RL]) {
+      const bool live = pc < MT * nchk;
+      const int m = live ? pc / nchk : 0;
+      const int k0 = (live ? pc - m * nchk : 0) * 256 + lane * 8;
+      const bool real = live && m < a.M && k0 < a.K;
+      s0 = real ? __ldg(reinterpret_cast<const float4*>(a.s + k0)) : make_float4(1.f, 1.f, 1.f, 1.f);
+      s1 = real ? __ldg(reinterpret_cast<const float4*>(a.s + k0 + 4)) : make_float4(1.f, 1.f, 1.f, 1.f);
+      raw = real ? __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(m) * a.K + k0))
+                 : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int v = 0; v < RF; ++v)
+        l1[v] = real ? __ldg(reinterpret_cast<const uint4*>(a.L1 + static_cast<size_t>(k0) * RF) + v)
+                     : make_uint4(0u, 0u, 0u, 0u);
+    };
+    uint4 rawn, l1n[RL];
+    float4 s0n, s1n;
+    ld(warp, rawn, s0n, s1n, l1n);
     for (int pc = warp; pc < MT * nchk; pc += nwarps) {
+      const uint4 raw = rawn;
+      const float4 s0 = s0n, s1 = s1n;
+      uint4 l1c[RL];
+#pragma unroll
+      for (int v = 0; v < RL; ++v) l1c[v] = l1n[v];
+      ld(pc + nwarps, rawn, s0n, s1n, l1n);
       const int m = pc / nchk, c = pc - (pc / nchk) * nchk;  // warp-uniform
       const int k0 = c * 256 + lane * 8;
       const bool real = m < a.M && k0 < a.K;  // K % 8 == 0: all 8 channels real or all padding
       const bool in_k = k0 < a.Kp;
-      float sv[8], sz[8];
-      if (real) {
-        const float4 s0 = __ldg(reinterpret_cast<const float4*>(a.s + k0));
-        const float4 s1 = __ldg(reinterpret_cast<const float4*>(a.s + k0 + 4));
-        sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-        sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sv[e] = 1.f;
-      }
+      const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      float sz[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) sz[e] = __frcp_rn(sv[e]);
-      const uint4 raw = real ? __ldg(reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(m) * a.K + k0))
-                             : make_uint4(0u, 0u, 0u, 0u);
       float xh[8];
       smooth8(raw, sv, sz, real, xh);
       float sc;
@@ -162,20 +177,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
         if ((lane & (4 * LPG - 1)) == 0) sxs[(k0 / a.group) * MT + m] = sc;  // (0 for padding rows)
       }
       if constexpr (RF > 0) {
-        // the 8 channels' L1 rows (8*RF bf16, contiguous)
-        if (real) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.L1 + static_cast<size_t>(k0) * RF);
+        // the 8 channels' L1 rows (8*RF bf16, contiguous; zero for padding)
 #pragma unroll
-          for (int v = 0; v < RF; ++v) {
-            float f[8];
-            bf16x8_to_f32(__ldg(src + v), f);
+        for (int v = 0; v < RF; ++v) {
+          float f[8];
+          bf16x8_to_f32(l1c[v], f);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const int e = (v * 8 + t) / RF, jr = (v * 8 + t) % RF;
+          for (int t = 0; t < 8; ++t) {
+            const int e = (v * 8 + t) / RF, jr = (v * 8 + t) % RF;
 #pragma unroll
-              for (int mm = 0; mm < MT; ++mm)
-                if (mm == m) u[mm][jr] = fmaf(xh[e], f[t], u[mm][jr]);
-            }
+            for (int mm = 0; mm < MT; ++mm)
+              if (mm == m) u[mm][jr] = fmaf(xh[e], f[t], u[mm][jr]);
           }
         }
       }
