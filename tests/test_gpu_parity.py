@@ -74,6 +74,7 @@ SMALL_SHAPES = [
     (256, 1152, 1152, 4),
     (300, 640, 512, 32),
     (16, 4096, 2048, 4),     # stream-K, decode tile
+    (24, 4096, 2048, 4),     # stream-K, decode tile of 32 tokens
     (128, 2048, 1024, 4),    # stream-K, large tile
     (130, 320, 264, 15),     # largest rank of one tensor-core low-rank step
     (97, 192, 136, 16),      # two low-rank steps
@@ -205,7 +206,7 @@ def test_unit_smoothing_lossless_grid_matches_dense_product():
 
 
 def test_repeated_calls_are_deterministic_and_reuse_workspace():
-    layer = make_layer(_spec(16, 4096, 2048, 4, seed=2))
+    layer = make_layer(_spec(24, 4096, 2048, 4, seed=2))
     pl, act, Y, ws = _run_gpu(layer)
     assert ws is not None  # stream-K path (tiles cut between CTAs)
     assert int(ws[:16].view(torch.int32).abs().sum()) == 0  # counters back at zero
@@ -228,7 +229,7 @@ def test_few_token_stream_is_deterministic_without_workspace():
 
 
 def test_forced_timeout_reports_status_and_library_recovers():
-    layer = make_layer(_spec(16, 256, 256, 4, seed=3))
+    layer = make_layer(_spec(24, 256, 256, 4, seed=3))  # a decode tile (the weight stream has no waits)
     pl, act, Y, ws = _run_gpu(layer)
     Y_ok = Y.clone()
     hsq.hsq_debug_force_timeout(1, 30)
@@ -251,8 +252,8 @@ def test_invalid_arguments_launch_nothing():
     assert e.value.status == hsq.HSQ_ERR_UNSUPPORTED
     # a shape that needs split-K scratch, called without it: rejected before any
     # launch (the buffers above are far too small for it, so nothing may run)
-    big = hsq.hsq_workspace_bytes(16, 4096, 12288, 4)
+    big = hsq.hsq_workspace_bytes(24, 4096, 12288, 4)
     with pytest.raises(hsq.HsqError) as e:
         hsq.hsq_linear_forward(act.x_codes, act.x_scales, act.U, pl.w_codes, pl.w_scales, pl.L2, None,
-                               16, 4096, 12288, 4, Y, workspace=None)
+                               24, 4096, 12288, 4, Y, workspace=None)
     assert big > 0 and e.value.status == hsq.HSQ_ERR_INVALID_ARG
