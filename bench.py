@@ -299,14 +299,34 @@ def run_gpu(args, specs, wl_name, rank, world, local):
                 launch_act(L, st)
                 launch_gemm(L, st)
 
+    # End to end: every step copies each layer's X from pinned host memory and its
+    # Y back.  The copies run on their own streams (host-to-device and device-to-
+    # host use the two directions of the link at once) and overlap the other
+    # layers' kernels; the step ends on the compute stream once its outputs landed.
+    copy_in = torch.cuda.Stream(device=dev)
+    copy_out = torch.cuda.Stream(device=dev)
+
     def step_e2e():
-        for L in layers:
-            L["X"].copy_(L["X_host"], non_blocking=True)
+        copy_in.wait_stream(stream)  # the previous step is done with the input buffers
+        arrived = []
+        with torch.cuda.stream(copy_in):
+            for L in layers:
+                L["X"].copy_(L["X_host"], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_in)
+                arrived.append(ev)
+        for L, ev in zip(layers, arrived):
+            stream.wait_event(ev)
             if fused:
                 hsq.forward_fused(L["pl"], L["X"], L["Y"], stream=stream)
             else:
                 hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
-            L["Y_host"].copy_(L["Y"], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(stream)
+            copy_out.wait_event(done)
+            with torch.cuda.stream(copy_out):
+                L["Y_host"].copy_(L["Y"], non_blocking=True)
+        stream.wait_stream(copy_out)  # outputs on the host before the step counts as done
 
     # A step (one replica's layers) is captured once into a CUDA graph and
     # replayed: at decode sizes a kernel runs for a few microseconds, less than
