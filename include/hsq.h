@@ -77,7 +77,7 @@ size_t hsq_scales_bytes(int rows, int K, int group);
  * Bytes of scratch that hsq_linear_forward needs for this shape on the current
  * device, for either group size: split-K counters and partial tiles, and for
  * M > 64 the two code matrices expanded to E4M3 bytes (0 when nothing is
- * needed).  The caller zero-fills the workspace once before its first use;
+ * needed, as for M <= 8 whenever the weight stream takes the shape).  The caller zero-fills the workspace once before its first use;
  * every completed call leaves the split-K counters zero again.
  */
 size_t hsq_workspace_bytes(int M, int N, int K, int r);

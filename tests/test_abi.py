@@ -148,7 +148,9 @@ def test_workspace_needs_are_consistent():
     assert hsq.hsq_workspace_bytes(4608, 12288, 3072, 4) == (4608 + 12288) * 3072
     # decode tiles: only split-K scratch (counters and partial tiles)
     assert 0 < hsq.hsq_workspace_bytes(16, 4096, 12288, 4) < 16 << 20
-    # up to 8 tokens: the weight stream needs no workspace
+    # up to 8 tokens: the weight stream needs no workspace, unless K is too long
+    # for one block's shared memory (then the decode tiles and their scratch)
     assert hsq.hsq_workspace_bytes(1, 4096, 12288, 4) == 0
     assert hsq.hsq_workspace_bytes(8, 12288, 4096, 4) == 0
+    assert hsq.hsq_workspace_bytes(8, 4096, 32768, 4) > 0  # K = 32768
     assert hsq.hsq_workspace_bytes(0, 4096, 12288, 4) == 0
