@@ -39,6 +39,14 @@ L2_BYTES = 126 * 2 ** 20
 METRIC = "W4A4 rank-4 linear TOPS & tokens/s at FLUX/SANA/Qwen3 shapes; % of roofline"
 INT8_OVER_BF16_NOMINAL = 2.0  # dense INT8 (4.5 POPS) over dense BF16 (2.25 PFLOP/s), nominal
 
+# DRAM bytes (read + write) per GEMM launch, averaged over the step's layers,
+# from one ncu capture of the current kernel (profiles/w4a4_gemm_kernel_flux_mlp_up.md
+# gives the command and the per-layer counters).  A workload without a capture,
+# or whose GEMM changed after its capture, reports null.
+NCU_TRAFFIC_PER_LAUNCH = {
+    "flux_block_r4": (45407488 + 40368896 + 55537408 + 66134528 + 215083776 + 19456512) / 3,
+}
+
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -440,14 +448,16 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     if t_tensor >= t_hbm:
         achieved = gemm_ops / gemm_time / 1e12
         roofline = {"bound": "tensor", "kernel": gemm_label, "achieved": achieved, "peak": int8_peak,
-                    "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": None,
+                    "unit": "TFLOP/s", "frac": achieved / int8_peak,
+                    "traffic": NCU_TRAFFIC_PER_LAUNCH.get(wl_name),
                     "peak_source": f"{peaks['source']}: bf16 sustained {peaks['bf16_sustained']} TFLOP/s x nominal "
                                    f"INT8/BF16 ratio {INT8_OVER_BF16_NOMINAL}",
                     "frac_of_spec_4500": achieved / 4500.0}
     else:
         achieved = gemm_bytes / gemm_time / 1e9
         roofline = {"bound": "hbm", "kernel": gemm_label, "achieved": achieved, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": NCU_TRAFFIC_PER_LAUNCH.get(wl_name),
                     "peak_source": f"{peaks['source']} copy bandwidth", "frac_of_spec_8000": achieved / 8000.0}
     roofline["algorithmic_per_launch"] = {"ops": gemm_ops / len(layers), "bytes": gemm_bytes / len(layers)}
     layer_detail = []
