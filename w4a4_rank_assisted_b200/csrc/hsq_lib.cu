@@ -41,6 +41,14 @@ using CfgLarge64 = hsq::GemmCfg<256, 2, HSQ_PAIR ? 8 : 6, false, 1, 3, 2, 2, HSQ
                                 1, HSQ_PAIR != 0>;
 using CfgLarge128 = hsq::GemmCfg<256, 2, HSQ_PAIR ? 4 : 3, false, 1, 3, 2, 2, HSQ_PAIR ? 8 : 7, true, -1, true, 2,
                                  2, HSQ_PAIR != 0>;
+// 64 < M <= 256, groups of 64 ("mid"): tokens x outputs tiles of 128 x 256 that
+// unpack both packed operands in shared memory (6 warps) instead of expanding
+// them in HBM first -- with one or two token tiles each weight tile is read about
+// once, so the per-call expansion of the whole weight matrix would only add traffic.
+#ifndef HSQ_MID_MAX_M
+#define HSQ_MID_MAX_M 256
+#endif
+using CfgMid64 = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 6, 10, true, -1, false, 2, 1>;
 // M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; packed codes
 // unpacked in shared memory (the drain is light, so more warps unpack); four
 // 64-blocks per stage either way
@@ -135,7 +143,7 @@ int device_sm_count() {
 }
 
 // ------------------------------------------------------------------ planning
-enum Kind { kLarge = 0, kDec16, kDec32, kDec64, kGemv };
+enum Kind { kLarge = 0, kDec16, kDec32, kDec64, kGemv, kMid };
 
 // M <= 8: the weight stream on the CUDA cores (hsq_gemv.cuh) when the block's
 // widened activation codes fit in shared memory; otherwise the decode tiles.
@@ -230,6 +238,12 @@ Plan make_plan(int M, int N, int K, int group, int nsm) {
     if (p.kind == kDec64) g128 ? plan_from<CfgDec64_128>(p) : plan_from<CfgDec64_64>(p);
     p.tiles_r = (N + 127) / 128;
     p.tiles_c = (M + p.BN - 1) / p.BN;
+  } else if (M <= HSQ_MID_MAX_M && !g128) {
+    p.swap = false;
+    p.kind = kMid;
+    plan_from<CfgMid64>(p);
+    p.tiles_r = (M + 127) / 128;
+    p.tiles_c = (N + p.BN - 1) / p.BN;
   } else {
     p.swap = false;
     p.kind = kLarge;
@@ -755,7 +769,8 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   static_assert(CfgLarge64::LR_MAX_RANK == CfgLarge128::LR_MAX_RANK, "low-rank chunk");
   // (at most three steps: r <= 32 < 3 * LR_MAX_RANK; the kernel builds chunks 0..2)
   static_assert(kMaxRank <= 3 * CfgLarge64::LR_MAX_RANK, "low-rank steps");
-  a.lr_mma = (HSQ_LR_MMA && p.kind == kLarge && CfgLarge64::LR_MMA && CfgLarge128::LR_MMA)
+  static_assert(CfgMid64::LR_MMA && CfgMid64::LR_MAX_RANK == CfgLarge64::LR_MAX_RANK, "mid tiles: low-rank steps");
+  a.lr_mma = (HSQ_LR_MMA && (p.kind == kLarge || p.kind == kMid) && CfgLarge64::LR_MMA && CfgLarge128::LR_MMA)
                  ? std::max(1, (r + CfgLarge64::LR_MAX_RANK - 1) / CfgLarge64::LR_MAX_RANK)
                  : 0;
   a.limit_ns = wait_limit_ns();
@@ -769,6 +784,8 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
     case kLarge:
       return g128 ? launch_gemm<CfgLarge128>(p, tm_row, tm_col, tm_y, a, stream)
                   : launch_gemm<CfgLarge64>(p, tm_row, tm_col, tm_y, a, stream);
+    case kMid:
+      return launch_gemm<CfgMid64>(p, tm_row, tm_col, tm_y, a, stream);
     case kDec16:
       return g128 ? launch_gemm<CfgDec16_128>(p, tm_row, tm_col, tm_y, a, stream)
                   : launch_gemm<CfgDec16_64>(p, tm_row, tm_col, tm_y, a, stream);
