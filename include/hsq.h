@@ -76,8 +76,9 @@ size_t hsq_scales_bytes(int rows, int K, int group);
 /*
  * Bytes of scratch that hsq_linear_forward needs for this shape on the current
  * device, for either group size: split-K counters and partial tiles, and for
- * M > 64 the two code matrices expanded to E4M3 bytes (0 when nothing is
- * needed, as for M <= 8 whenever the weight stream takes the shape).  The caller zero-fills the workspace once before its first use;
+ * M > 64 (groups of 128; M > 256 for groups of 64) the two code matrices
+ * expanded to E4M3 bytes (0 when nothing is needed, as for M <= 8 whenever the
+ * weight stream takes the shape).  The caller zero-fills the workspace once before its first use;
  * every completed call leaves the split-K counters zero again.
  */
 size_t hsq_workspace_bytes(int M, int N, int K, int r);
@@ -158,9 +159,10 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
  *     for hsq_linear_forward; the results are the same.
  *   - Shapes whose scratch need for the given group exceeds
  *     HSQ_NOALLOC_SCRATCH_BYTES are rejected with HSQ_ERR_SCRATCH_LIMIT before
- *     anything is launched (M > 64 needs (M + N) * Kp bytes of expanded codes,
- *     rows rounded up to whole tiles, plus any split-K scratch; the decode
- *     tiles, M <= 64, need at most about 10 MB).
+ *     anything is launched (M > 256, or M > 64 with groups of 128, needs
+ *     (M + N) * Kp bytes of expanded codes, rows rounded up to whole tiles, plus
+ *     any split-K scratch; smaller M needs only split-K scratch, at most about
+ *     40 MB, and none up to 8 tokens).
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any
  *     stream capture.
