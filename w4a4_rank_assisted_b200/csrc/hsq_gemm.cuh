@@ -1,15 +1,22 @@
-// hsq_gemm.cuh -- packed INT4 x INT4 GEMM on tcgen05 (kind::i8) with a per-group
-// fp32 rescale and a fused low-rank + bias epilogue.
+// hsq_gemm.cuh -- packed INT4 x INT4 GEMM on tcgen05 with a per-group fp32
+// rescale and a fused low-rank + bias epilogue.
 //
 // Computes (Deflating the Hessian, Abstract: 4-bit residual product plus the
 // high-precision low-rank branch)
 //     Y[m,n] = sum_g sx[g][m] sw[g][n] P_g[m,n] + sum_j U[m,j] L2[j,n] + b[n],
-//     P_g[m,n] = sum_{k in group g} qx[m,k] qw[n,k]   (exact, int32)
+//     P_g[m,n] = sum_{k in group g} qx[m,k] qw[n,k]   (exact integers)
 //
-// Blackwell has no INT4 tensor-core mode, so each 64-wide group is unpacked in
-// shared memory to INT8 and multiplied with two tcgen05.mma.kind::i8 (K = 32
-// each) into its own Tensor Memory region; drain warps read the int32 partial
-// with tcgen05.ld and fold it into fp32 register accumulators with its scales.
+// Blackwell has no INT4 tensor-core mode.  Each 64-wide block of codes is fed
+// to the tensor cores in an 8-bit form whose products and 64-term sums are
+// exact, two K = 32 MMAs per block into a group's own Tensor Memory partial;
+// drain warps read that partial with tcgen05.ld and fold it into fp32 register
+// accumulators with the group's two scales.  The 8-bit forms:
+//   kind::i8      int8 16*q (decode tiles): the MMA sums 256*q_x*q_w in int32,
+//                 the drain folds 1/256 into the row scale (a power of two);
+//   kind::f8f6f4  E4M3 subnormals q*2^-9 (tokens x outputs tiles): every product
+//                 and partial is exact in fp32, so the drain needs no int->fp32
+//                 conversion and folds 2^18 into the row scale instead.
+// Either way the group partial is the same number.
 //
 // Operands are named by their role in the MMA:
 //   "row" operand  -> MMA A, 128 rows per tile, one TMEM lane per row;
@@ -18,22 +25,32 @@
 // outputs); for decode-sized M the roles swap (128 weight rows x BN tokens), so
 // the MMA's M=128 side is always filled.
 //
-// Unpack: a packed byte holds two 4-bit two's-complement codes.  Masking a code
-// into the HIGH nibble of a byte gives the int8 value 16*q, so one AND (odd
-// codes) or one shift+AND (even codes) unpacks four codes; the MMA then sums
-// 256*q_x*q_w, and the drain folds 1/256 into the per-row scale (a power of two,
-// so the fp32 result is unchanged).  The even/odd split permutes K inside a
-// group identically for both operands, which leaves every P_g unchanged.
+// Where the 8-bit operands come from (GemmCfg):
+//   packed codes staged by TMA and widened in shared memory by unpack warps
+//     (decode tiles; tokens x outputs tiles for up to 256 tokens): a packed
+//     byte holds two 4-bit two's-complement codes; masking a code into the
+//     HIGH nibble of a byte gives 16*q (one AND or shift+AND per four codes),
+//     or the E4M3 byte sign<<7 | |q|.  The even/odd split permutes K inside a
+//     block identically for both operands, which leaves every P_g unchanged;
+//   pre-expanded (PRE; more tokens): expand_e4m3_kernel writes both code
+//     matrices once per call as MMA-ready E4M3 tiles, and a stage is two bulk
+//     copies.
+// The low-rank branch U L2 + b enters the same accumulators as bf16 MMA steps
+// ahead of a tile's first group (tokens x outputs tiles) or is added by the
+// drain at the tile's start (decode tiles).
 //
 // Pipeline (one CTA per SM, persistent over work units).  One pipeline step
-// ("stage") carries GPS consecutive 64-groups, so that the fixed cost of each
+// ("stage") carries GPS consecutive scale groups, so that the fixed cost of each
 // hand-off is shared by GPS groups:
-//   warp 0      TMA producer: packed row/col tiles (GPS groups wide) + the row
-//               and col scales of each group, into a STAGES-deep ring
+//   warp 0      TMA producer: row/col tiles + the row and col scales of each
+//               group, into a STAGES-deep ring (scales in a deeper ring of their own)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2-7   unpack packed -> int8 canonical K-major layout, NI8 buffers
-//   warps 8..   drain / epilogue; warp w reads TMEM lanes 32*(w%4)..+31; NTM
+//   warps 2..   unpack (packed -> 8-bit K-major layout, NI8 buffers) or, with
+//               PRE, the builders of the low-rank step's operands
+//   last warps  drain / epilogue; warp w reads TMEM lanes 32*(w%4)..+31; NTM
 //               TMEM buffers of GPS x BN columns
+// Work is whole tiles per CTA, or stream-K runs of stages with a deterministic
+// last-arriver reduction when the tiles do not fill the SMs.
 #pragma once
 
 #include "hsq_device.cuh"

@@ -1,9 +1,11 @@
 // hsq_lib.cu -- the C ABI of libhsq (declared in include/hsq.h): argument
 // validation, launch planning, tensor-map construction and kernel launches.
 //
-// Everything numeric happens in the kernels of hsq_quant.cuh and hsq_gemm.cuh;
-// this file only checks arguments (synchronously, before any launch) and
-// launches them.  It allocates no device memory.
+// Everything numeric happens in the kernels of hsq_quant.cuh, hsq_gemm.cuh,
+// hsq_gemv.cuh and hsq_lowrank.cuh (and, for the pack-time truncated-SVD
+// helper only, plain fp32/fp64 cuBLAS GEMMs); this file checks arguments
+// (synchronously, before any launch), plans and launches.  It allocates no
+// device memory, except the helper's one cuBLAS handle per device.
 #include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
