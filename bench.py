@@ -435,9 +435,10 @@ def run_gpu(args, specs, wl_name, rank, world, local):
                    for L in layers)
     gemm_bytes = sum((layer_fused_bytes if fused else layer_gemm_bytes)(L["spec"]) for L in layers)
     gemm_time = sum(gemm_us) * 1e-6
-    # hsq_linear_forward launches, for more than 64 tokens, two operand
-    # expansions ahead of the GEMM: its time (and so the roofline) includes them
-    large = [L["spec"].M > 64 for L in layers]
+    # hsq_linear_forward launches two operand expansions ahead of the GEMM when
+    # the codes are pre-expanded (more than 256 tokens, or more than 64 at groups
+    # of 128): its time (and so the roofline) includes them
+    large = [L["spec"].M > 256 or (L["spec"].M > 64 and L["spec"].group == 128) for L in layers]
     # up to 8 tokens the forward is the CUDA-core weight stream (its shared-memory
     # limit is far above these shapes' K)
     gemm_label = ("w4a4_gemm_kernel (+ 2 expand_e4m3_kernel: one hsq_linear_forward)" if any(large)
