@@ -20,7 +20,7 @@ shd-paper.top, thelatestinai.com and rit.work.
 Together:  Y = Q4(X_hat) Q4(R)^T + (X_hat L1) L2 + b, with
 X_hat = X diag(s)^-1 and R = W diag(s) - (L1 L2)^T  (W stored [N, K]).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * symmetric signed INT4, codes in [-7, 7], scale = absmax / 7 in fp32 with
     IEEE division, code = round-half-even(fp32(x / scale)), clamp to [-7, 7];
   * an all-zero group has scale 0 and codes 0;

@@ -15,7 +15,7 @@ layer is otherwise the one of oracle.hsq_oracle (smoothed activations X_hat,
 residual R = W diag(s) - (L1 L2)^T, high-precision low-rank branch), with both
 4-bit operands in NVFP4 instead of group-64 INT4.
 
-Readings where the page is silent (listed in the design doc):
+Readings where the page is silent:
   * element format E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit):
     magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}; a 4-bit code is sign << 3 | index
     (index = exponent << 1 | mantissa, i.e. the position in that list); values
