@@ -39,15 +39,6 @@ L2_BYTES = 126 * 2 ** 20
 METRIC = "W4A4 rank-4 linear TOPS & tokens/s at FLUX/SANA/Qwen3 shapes; % of roofline"
 INT8_OVER_BF16_NOMINAL = 2.0  # dense INT8 (4.5 POPS) over dense BF16 (2.25 PFLOP/s), nominal
 
-# DRAM bytes (read + write) per GEMM launch, averaged over the step's layers,
-# from one ncu capture of the current kernel (profiles/w4a4_gemm_kernel_flux_mlp_up.md
-# gives the command and the per-layer counters).  A workload without a capture,
-# or whose GEMM changed after its capture, reports null.
-NCU_TRAFFIC_PER_LAUNCH = {
-    "flux_block_r4": (45407488 + 40368896 + 55537408 + 66134528 + 215083776 + 19456512) / 3,
-}
-
-
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -90,6 +81,81 @@ def layer_act_bytes(spec):
     M, K, r, gs = spec.M, spec.K, spec.r, spec.group
     G = -(-K // gs)
     return 2 * M * K + M * gs * G // 2 + 4 * M * G + 4 * M * r + 4 * K + 2 * K * r
+
+
+def _cu(res):
+    """Unpack a cuda-python driver call's result, raising on an error code."""
+    err, *rest = res if isinstance(res, tuple) else (res,)
+    if int(err) != 0:
+        raise RuntimeError(f"CUDA driver call failed: {err}")
+    return rest[0] if len(rest) == 1 else rest
+
+
+def time_kernel_nodes(launch, stream, name_part: str, calls: int, repeats: int = 3):
+    """Device time of one kind of kernel inside a multi-kernel library call.
+
+    ``launch(i, stream)`` issues call i (all of its kernels) on ``stream``.  The
+    ``calls`` calls are captured into one CUDA graph; every kernel node whose
+    name does not contain ``name_part`` is removed and the remaining nodes are
+    chained in launch order, so they run one after another exactly as launched
+    (same grid, arguments and inputs: the removed kernels' outputs are already
+    in memory from earlier calls).  The graph is replayed ``repeats`` times
+    between CUDA events on ``stream``; returns (microseconds per kept node,
+    kept nodes per call)."""
+    from cuda.bindings import driver as cu
+    hs = cu.CUstream(stream.cuda_stream)
+    _cu(cu.cuStreamBeginCapture(hs, cu.CUstreamCaptureMode.CU_STREAM_CAPTURE_MODE_RELAXED))
+    try:
+        for i in range(calls):
+            launch(i, stream)
+    finally:
+        graph = _cu(cu.cuStreamEndCapture(hs))
+    try:
+        n = _cu(cu.cuGraphGetNodes(graph, 0))[1]
+        nodes = _cu(cu.cuGraphGetNodes(graph, n))[0]
+        key = lambda nd: int(nd)
+        deps = {key(nd): {key(d) for d in _cu(cu.cuGraphNodeGetDependencies(
+            nd, _cu(cu.cuGraphNodeGetDependencies(nd, 0))[1]))[0]} for nd in nodes}
+        order, placed = [], set()
+        while len(order) < len(nodes):  # launch order (the capture is a chain)
+            for nd in nodes:
+                k = key(nd)
+                if k not in placed and deps[k] <= placed:
+                    order.append(nd)
+                    placed.add(k)
+        kept = []
+        for nd in order:
+            name = ""
+            if _cu(cu.cuGraphNodeGetType(nd)) == cu.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
+                prm = _cu(cu.cuGraphKernelNodeGetParams(nd))
+                if int(prm.func):
+                    name = _cu(cu.cuFuncGetName(prm.func))
+                elif int(prm.kern):
+                    name = _cu(cu.cuKernelGetName(prm.kern))
+                name = name.decode() if isinstance(name, bytes) else str(name)
+            if name_part in name:
+                kept.append(nd)
+            else:
+                _cu(cu.cuGraphDestroyNode(nd))
+        for a, b in zip(kept[:-1], kept[1:]):
+            _cu(cu.cuGraphAddDependencies(graph, [a], [b], 1))
+        exe = _cu(cu.cuGraphInstantiate(graph, 0))
+        try:
+            _cu(cu.cuGraphLaunch(exe, hs))
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(repeats):
+                _cu(cu.cuGraphLaunch(exe, hs))
+            e1.record(stream)
+            torch.cuda.synchronize()
+        finally:
+            _cu(cu.cuGraphExecDestroy(exe))
+    finally:
+        _cu(cu.cuGraphDestroy(graph))
+    if not kept:
+        raise RuntimeError(f"no kernel named like {name_part!r} in the call")
+    return e0.elapsed_time(e1) * 1e3 / (repeats * len(kept)), len(kept) / calls
 
 
 class ClockSampler:
@@ -241,76 +307,269 @@ def run_reference(args, specs, wl_name, rank, world):
 
 
 # ------------------------------------------------------------------ GPU leg
+def _sources_sha() -> str:
+    """Hash of the CUDA sources: an ncu traffic figure is reported only for the
+    build it was captured from."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "w4a4_rank_assisted_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+# DRAM read + write bytes per launch of the dominant kernel (mean over the
+# step's layers) from one ncu capture, keyed by workload, with the hash of the
+# CUDA sources it was captured from; any other build reports null.
+NCU_TRAFFIC = {}
+
+
+class Workload:
+    """One workload on one GPU: packed layers, their replicas (decode sizes),
+    one CUDA graph per replica step, and the launch helpers of the public API."""
+
+    def __init__(self, hsq, specs, dev, host_buffers=False):
+        self.hsq, self.specs, self.dev = hsq, specs, dev
+        d = lambda t: None if t is None else t.to(dev).contiguous()
+        host_layers = [make_layer(spec) for spec in specs]
+
+        def build_layers():
+            out = []
+            for spec, lay in zip(specs, host_layers):
+                pl = hsq.PackedLinear(d(lay.W), d(lay.s), d(lay.L1) if spec.r else None,
+                                      d(lay.L2) if spec.r else None, None, group=spec.group)
+                act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
+                Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
+                out.append(dict(spec=spec, pl=pl, X=d(lay.X), act=act, Y=Y, ws=pl.workspace(spec.M)))
+            return out
+
+        self.layers = build_layers()
+        if host_buffers:
+            for L, lay in zip(self.layers, host_layers):
+                L["X_host"] = lay.X.pin_memory()
+                L["Y_host"] = torch.empty((L["spec"].M, L["spec"].N), dtype=torch.bfloat16).pin_memory()
+        # Working sets smaller than 2 x L2 (decode sizes): the layers are replicated
+        # (distinct packed weights, activations, outputs and workspaces) and the timed
+        # steps and kernels cycle through the replicas, so that every launch reads
+        # inputs that are not in L2 (inputs larger than L2, as a model's many layers
+        # are).  Enough replicas that even one layer's launches span 2 x L2.
+        self.ws_bytes = sum(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in self.layers)
+        min_layer = min(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in self.layers)
+        self.nrep = 1 if self.ws_bytes >= 2 * L2_BYTES else min(128, -(-2 * L2_BYTES // min_layer))
+        self.replicas = [self.layers] + [build_layers() for _ in range(self.nrep - 1)]
+        # decode sizes the single-launch forward takes: the activation step runs
+        # inside the forward's kernel
+        self.fused = all(hsq.fused_supported(s.M, s.K, s.r, s.group) for s in specs)
+        torch.cuda.synchronize()
+        if hsq.hsq_get_device_status() != hsq.HSQ_OK:
+            raise RuntimeError("device status not clean after packing")
+        self.gstream = torch.cuda.Stream(device=dev)
+
+    # the public API's calls, one layer at a time
+    def launch_act(self, L, st):
+        s = L["spec"]
+        self.hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
+                                  L["act"].x_scales, L["act"].U, group=s.group, stream=st)
+
+    def launch_gemm(self, L, st):
+        s = L["spec"]
+        self.hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
+                                    L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
+                                    workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
+                                    group=s.group, stream=st)
+
+    def launch_fused(self, L, st):
+        s = L["spec"]
+        self.hsq.hsq_linear_forward_fused(L["X"], L["pl"].s, L["pl"].L1, L["pl"].w_codes, L["pl"].w_scales,
+                                          L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"], group=s.group, stream=st)
+
+    def step(self, st, rep=0):
+        for L in self.replicas[rep]:
+            if self.fused:
+                self.launch_fused(L, st)
+            else:
+                self.launch_act(L, st)
+                self.launch_gemm(L, st)
+
+    def capture(self, fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.gstream):
+            fn(self.gstream)
+        return g
+
+    def replay_ms(self, g, n):
+        # CUDAGraph.replay() launches on the current stream: make it gstream
+        with torch.cuda.stream(self.gstream):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(self.gstream)
+            for _ in range(n):
+                g.replay()
+            b.record(self.gstream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    def prepare_steps(self, warmup):
+        """One CUDA graph per replica step (at decode sizes a kernel runs for a few
+        microseconds, less than its host-side launch), warmed up."""
+        self.gstream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.gstream):
+            for i in range(self.nrep):
+                self.step(self.gstream, i)
+        torch.cuda.synchronize()
+        self.g_steps = [self.capture(lambda st, i=i: self.step(st, i)) for i in range(self.nrep)]
+        with torch.cuda.stream(self.gstream):
+            for k in range(max(warmup, self.nrep)):
+                self.g_steps[k % self.nrep].replay()
+        torch.cuda.synchronize()
+
+    def timed_steps_ms(self, steps):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.gstream):
+            t0.record(self.gstream)
+            for k in range(steps):
+                self.g_steps[k % self.nrep].replay()
+            t1.record(self.gstream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
+    def launches_per_step(self):
+        """Kernels of this library launched by one step."""
+        n = 0
+        for L in self.layers:
+            if self.fused:
+                n += 1
+            else:
+                n += 1 + (3 if self.expands(L["spec"]) else 1)
+        return n
+
+    @staticmethod
+    def expands(s):
+        """hsq_linear_forward expands both code matrices to E4M3 tiles ahead of
+        the GEMM (two more launches) for more than 256 tokens, or more than 64 at
+        groups of 128."""
+        return s.M > 256 or (s.M > 64 and s.group == 128)
+
+    def kernel_times(self):
+        """Per layer: device microseconds of each kernel, each timed alone over
+        >= 20 launches in a CUDA graph (cycling through the replicas), CUDA events
+        on the replaying stream.  For calls of several kernels the GEMM kernel and
+        the expansions are also timed apart (time_kernel_nodes)."""
+        reps = max(20, self.nrep)
+        out = []
+        for li, L in enumerate(self.layers):
+            def per_call(fn):
+                g = self.capture(lambda st: [fn(self.replicas[j % self.nrep][li], st) for j in range(reps)])
+                with torch.cuda.stream(self.gstream):
+                    g.replay()
+                torch.cuda.synchronize()
+                return self.replay_ms(g, 3) * 1e3 / (3 * reps)
+            d = {}
+            if self.fused:
+                d["call_us"] = per_call(self.launch_fused)
+                d["gemm_kernel_us"] = d["call_us"]
+                d["act_us"] = 0.0
+            else:
+                d["call_us"] = per_call(self.launch_gemm)
+                d["act_us"] = per_call(self.launch_act)
+                if self.expands(L["spec"]):
+                    call = lambda i, st: self.launch_gemm(self.replicas[i % self.nrep][li], st)
+                    d["gemm_kernel_us"], _ = time_kernel_nodes(call, self.gstream, "w4a4_gemm_kernel", reps)
+                    e_us, e_n = time_kernel_nodes(call, self.gstream, "expand_e4m3_kernel", reps)
+                    d["expand_us"] = e_us * e_n  # both launches of one call
+                else:
+                    d["gemm_kernel_us"] = d["call_us"]
+            out.append(d)
+        return out
+
+    def roofline(self, kt, peaks, wl_name):
+        """Roofline of the dominant kernel (the forward's GEMM, or the weight
+        stream at decode sizes) over the step's layers, against the measured
+        peaks: tensor-bound when its INT8 time floor exceeds its HBM floor."""
+        specs = [L["spec"] for L in self.layers]
+        # each kernel is timed alone in a short graph: the burst peaks apply
+        int8_peak = peaks["bf16"] * INT8_OVER_BF16_NOMINAL
+        gemm_ops = sum(2 * s.M * s.N * s.K + 2 * s.M * s.N * s.r for s in specs)
+        gemm_bytes = sum((layer_fused_bytes if self.fused else layer_gemm_bytes)(s) for s in specs)
+        gemm_time = sum(d["gemm_kernel_us"] for d in kt) * 1e-6
+        label = ("w4a4_gemv_kernel, activation step fused in (one hsq_linear_forward_fused)" if self.fused
+                 else "w4a4_gemv_kernel" if all(s.M <= 8 for s in specs) else "w4a4_gemm_kernel")
+        t_tensor = gemm_ops / (int8_peak * 1e12)
+        t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
+        tr = NCU_TRAFFIC.get(wl_name)
+        traffic = tr[1] if tr and tr[0] == _sources_sha() else None
+        if t_tensor >= t_hbm:
+            achieved = gemm_ops / gemm_time / 1e12
+            r = {"bound": "tensor", "kernel": label, "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
+                 "frac": achieved / int8_peak, "traffic": traffic,
+                 "peak_source": (f"{peaks['source']}: bf16 burst {peaks['bf16']} TFLOP/s x nominal INT8/BF16 "
+                                 f"ratio {INT8_OVER_BF16_NOMINAL} (each kernel timed alone)"),
+                 "frac_of_spec_4500": achieved / 4500.0}
+        else:
+            achieved = gemm_bytes / gemm_time / 1e9
+            r = {"bound": "hbm", "kernel": label, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                 "peak_source": f"{peaks['source']} copy bandwidth", "frac_of_spec_8000": achieved / 8000.0}
+        r["algorithmic_per_launch"] = {"ops": gemm_ops / len(specs), "bytes": gemm_bytes / len(specs)}
+        r["time_per_launch_us"] = gemm_time * 1e6 / len(specs)
+        return r
+
+    def layer_detail(self, kt):
+        out = []
+        for L, d in zip(self.layers, kt):
+            s = L["spec"]
+            gops = 2 * s.M * s.N * s.K + 2 * s.M * s.N * s.r
+            g = d["gemm_kernel_us"]
+            row = {"layer": s.name, "M": s.M, "K": s.K, "N": s.N, "r": s.r, "group": s.group,
+                   "call_us": d["call_us"], "gemm_kernel_us": g, "act_us": d["act_us"],
+                   "gemm_tops": gops / (g * 1e-6) / 1e12,
+                   "gemm_gbs": (layer_fused_bytes if self.fused else layer_gemm_bytes)(s) / (g * 1e-6) / 1e9,
+                   "act_gbs": layer_act_bytes(s) / (d["act_us"] * 1e-6) / 1e9 if d["act_us"] > 0 else None}
+            if "expand_us" in d:
+                row["expand_us"] = d["expand_us"]
+            out.append(row)
+        return out
+
+    def l2_note(self):
+        if self.nrep > 1:
+            return (f"inputs larger than L2: {self.nrep} replicas of the step's layers (distinct weights, "
+                    f"activations, outputs), steps and per-kernel launches cycle through them; "
+                    f"{self.nrep * self.ws_bytes / 2**20:.0f} MiB in all, {self.ws_bytes / 2**20:.1f} MiB per step")
+        return f"no flush; per-step working set {self.ws_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2"
+
+
 def run_gpu(args, specs, wl_name, rank, world, local):
     from w4a4_rank_assisted_b200 import hsq
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    d = lambda t: None if t is None else t.to(dev).contiguous()
-    host_layers = [make_layer(spec) for spec in specs]
+    W = Workload(hsq, specs, dev, host_buffers=True)
+    layers = W.layers
+    W.prepare_steps(args.warmup)
 
-    def build_layers():
-        out = []
-        for spec, lay in zip(specs, host_layers):
-            pl = hsq.PackedLinear(d(lay.W), d(lay.s), d(lay.L1) if spec.r else None,
-                                  d(lay.L2) if spec.r else None, None, group=spec.group)
-            X = d(lay.X)
-            act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
-            Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
-            out.append(dict(spec=spec, pl=pl, X=X, act=act, Y=Y, ws=pl.workspace(spec.M)))
-        return out
-
-    layers = build_layers()
-    for L, lay in zip(layers, host_layers):
-        L["X_host"] = lay.X.pin_memory()
-        L["Y_host"] = torch.empty((L["spec"].M, L["spec"].N), dtype=torch.bfloat16).pin_memory()
-    # Working sets smaller than 2 x L2 (decode sizes): the layers are replicated
-    # (distinct packed weights, activations, outputs and workspaces) and the timed
-    # steps and kernels cycle through the replicas, so that every launch reads
-    # inputs that are not in L2 (inputs larger than L2, as a model's many layers
-    # are).  Enough replicas that even one layer's launches span 2 x L2.
-    ws_bytes = sum(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in layers)
-    min_layer = min(layer_act_bytes(L["spec"]) + layer_gemm_bytes(L["spec"]) for L in layers)
-    nrep = 1 if ws_bytes >= 2 * L2_BYTES else min(128, -(-2 * L2_BYTES // min_layer))
-    replicas = [layers] + [build_layers() for _ in range(nrep - 1)]
+    # ---- timed region: exactly K steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    _barrier(world)
     torch.cuda.synchronize()
+    ms_total = W.timed_steps_ms(args.steps)
+    _barrier(world)
+    clk = clocks.stop()
+    ms_total = _max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
     if hsq.hsq_get_device_status() != hsq.HSQ_OK:
-        raise RuntimeError("device status not clean after packing")
+        raise RuntimeError("a kernel reported a timeout during the timed region")
 
-    def launch_act(L, st):
-        s = L["spec"]
-        hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
-                             L["act"].x_scales, L["act"].U, group=s.group, stream=st)
+    kt = W.kernel_times()
 
-    def launch_gemm(L, st):
-        s = L["spec"]
-        hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
-                               L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
-                               workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
-                               group=s.group, stream=st)
-
-    # decode sizes the single-launch forward takes (up to 4 tokens, r in {0,1,2,4}):
-    # the activation step runs inside the weight-stream kernel
-    fused = all(hsq.fused_supported(s.M, s.K, s.r, s.group) for s in specs)
-
-    def launch_fused(L, st):
-        s = L["spec"]
-        hsq.hsq_linear_forward_fused(L["X"], L["pl"].s, L["pl"].L1, L["pl"].w_codes, L["pl"].w_scales,
-                                     L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"], group=s.group, stream=st)
-
-    def step(st, rep=0):
-        for L in replicas[rep]:
-            if fused:
-                launch_fused(L, st)
-            else:
-                launch_act(L, st)
-                launch_gemm(L, st)
-
-    # End to end: every step copies each layer's X from pinned host memory and its
-    # Y back.  The copies run on their own streams (host-to-device and device-to-
-    # host use the two directions of the link at once) and overlap the other
-    # layers' kernels; the step ends on the compute stream once its outputs landed.
+    # ---- end to end through the public API with host buffers (no graph): every
+    # step copies each layer's X from pinned host memory and its Y back.  The
+    # copies run on their own streams (host-to-device and device-to-host use the
+    # two directions of the link at once) and overlap the other layers' kernels;
+    # the step ends on the compute stream once its outputs landed.
     copy_in = torch.cuda.Stream(device=dev)
     copy_out = torch.cuda.Stream(device=dev)
 
@@ -325,7 +584,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
                 arrived.append(ev)
         for L, ev in zip(layers, arrived):
             stream.wait_event(ev)
-            if fused:
+            if W.fused:
                 hsq.forward_fused(L["pl"], L["X"], L["Y"], stream=stream)
             else:
                 hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
@@ -336,78 +595,6 @@ def run_gpu(args, specs, wl_name, rank, world, local):
                 L["Y_host"].copy_(L["Y"], non_blocking=True)
         stream.wait_stream(copy_out)  # outputs on the host before the step counts as done
 
-    # A step (one replica's layers) is captured once into a CUDA graph and
-    # replayed: at decode sizes a kernel runs for a few microseconds, less than
-    # its host-side launch.
-    gstream = torch.cuda.Stream(device=dev)
-    gstream.wait_stream(stream)
-    with torch.cuda.stream(gstream):
-        for i in range(nrep):
-            step(gstream, i)
-    torch.cuda.synchronize()
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=gstream):
-            fn(gstream)
-        return g
-
-    g_steps = [capture(lambda st, i=i: step(st, i)) for i in range(nrep)]
-    with torch.cuda.stream(gstream):
-        for k in range(max(args.warmup, nrep)):
-            g_steps[k % nrep].replay()
-    torch.cuda.synchronize()
-
-    def replay_ms(g, n):
-        # CUDAGraph.replay() launches on the current stream: make it gstream
-        with torch.cuda.stream(gstream):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(gstream)
-            for _ in range(n):
-                g.replay()
-            b.record(gstream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b)
-
-    # ---- timed region: exactly K steps
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    _barrier(world)
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(gstream):
-        t0.record(gstream)
-        for k in range(args.steps):
-            g_steps[k % nrep].replay()
-        t1.record(gstream)
-    torch.cuda.synchronize()
-    _barrier(world)
-    clk = clocks.stop()
-    ms_total = t0.elapsed_time(t1)
-    ms_total = _max_over_ranks(ms_total, world)
-    ms_step = ms_total / args.steps
-    if hsq.hsq_get_device_status() != hsq.HSQ_OK:
-        raise RuntimeError("a kernel reported a timeout during the timed region")
-
-    # ---- per-kernel device time: each kernel alone, REPS launches per graph
-    # (cycling through the replicas), CUDA events on the replaying stream
-    def kernel_us(fn, li):
-        reps = max(20, nrep)
-        g = capture(lambda st: [fn(replicas[j % nrep][li], st) for j in range(reps)])
-        with torch.cuda.stream(gstream):
-            g.replay()
-        torch.cuda.synchronize()
-        return replay_ms(g, 3) * 1e3 / (3 * reps)
-
-    if fused:  # one kernel per layer: its time is reported as the GEMM's, the activation step's as 0
-        gemm_us = [kernel_us(launch_fused, li) for li in range(len(layers))]
-        act_us = [0.0 for _ in layers]
-    else:
-        gemm_us = [kernel_us(launch_gemm, li) for li in range(len(layers))]
-        act_us = [kernel_us(launch_act, li) for li in range(len(layers))]
-
-    # ---- end to end through the public API with host buffers (no graph)
     for _ in range(max(1, args.warmup // 2)):
         step_e2e()
     torch.cuda.synchronize()
@@ -426,50 +613,30 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     tops_e2e = ops_step * world / (ms_e2e * 1e-3) / 1e12
     h2d = sum(L["X_host"].numel() * 2 for L in layers)
     d2h = sum(L["Y_host"].numel() * 2 for L in layers)
-
-    # ---- roofline of the dominant kernel (the GEMM, all layers of the step):
-    # tensor-bound when its INT8 time floor exceeds its HBM floor, else HBM-bound
     peaks = _peaks()
-    int8_peak = peaks["bf16_sustained"] * INT8_OVER_BF16_NOMINAL
-    gemm_ops = sum(2 * L["spec"].M * L["spec"].N * L["spec"].K + 2 * L["spec"].M * L["spec"].N * L["spec"].r
-                   for L in layers)
-    gemm_bytes = sum((layer_fused_bytes if fused else layer_gemm_bytes)(L["spec"]) for L in layers)
-    gemm_time = sum(gemm_us) * 1e-6
-    # hsq_linear_forward launches two operand expansions ahead of the GEMM when
-    # the codes are pre-expanded (more than 256 tokens, or more than 64 at groups
-    # of 128): its time (and so the roofline) includes them
-    large = [L["spec"].M > 256 or (L["spec"].M > 64 and L["spec"].group == 128) for L in layers]
-    # up to 8 tokens the forward is the CUDA-core weight stream (its shared-memory
-    # limit is far above these shapes' K)
-    gemm_label = ("w4a4_gemm_kernel (+ 2 expand_e4m3_kernel: one hsq_linear_forward)" if any(large)
-                  else "w4a4_gemv_kernel, activation step fused in (one hsq_linear_forward_fused)" if fused
-                  else "w4a4_gemv_kernel" if all(L["spec"].M <= 8 for L in layers) else "w4a4_gemm_kernel")
-    t_tensor = gemm_ops / (int8_peak * 1e12)
-    t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
-    if t_tensor >= t_hbm:
-        achieved = gemm_ops / gemm_time / 1e12
-        roofline = {"bound": "tensor", "kernel": gemm_label, "achieved": achieved, "peak": int8_peak,
-                    "unit": "TFLOP/s", "frac": achieved / int8_peak,
-                    "traffic": NCU_TRAFFIC_PER_LAUNCH.get(wl_name),
-                    "peak_source": f"{peaks['source']}: bf16 sustained {peaks['bf16_sustained']} TFLOP/s x nominal "
-                                   f"INT8/BF16 ratio {INT8_OVER_BF16_NOMINAL}",
-                    "frac_of_spec_4500": achieved / 4500.0}
-    else:
-        achieved = gemm_bytes / gemm_time / 1e9
-        roofline = {"bound": "hbm", "kernel": gemm_label, "achieved": achieved, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": NCU_TRAFFIC_PER_LAUNCH.get(wl_name),
-                    "peak_source": f"{peaks['source']} copy bandwidth", "frac_of_spec_8000": achieved / 8000.0}
-    roofline["algorithmic_per_launch"] = {"ops": gemm_ops / len(layers), "bytes": gemm_bytes / len(layers)}
-    layer_detail = []
-    for L, g, a in zip(layers, gemm_us, act_us):
-        s = L["spec"]
-        gops = 2 * s.M * s.N * s.K + 2 * s.M * s.N * s.r
-        layer_detail.append({"layer": s.name, "M": s.M, "K": s.K, "N": s.N, "r": s.r,
-                             "gemm_us": g, "act_us": a,
-                             "gemm_tops": gops / (g * 1e-6) / 1e12,
-                             "gemm_gbs": (layer_fused_bytes if fused else layer_gemm_bytes)(s) / (g * 1e-6) / 1e9,
-                             "act_gbs": layer_act_bytes(s) / (a * 1e-6) / 1e9 if a > 0 else None})
+    roofline = W.roofline(kt, peaks, wl_name)
+
+    # ---- decode-sized layers (Qwen3-8B, 1 and 16 tokens), timed the same way:
+    # their own step graphs cycling through replicas, per-kernel times, roofline
+    decode = None
+    if not args.no_decode:
+        decode = {}
+        for dname in ("qwen3_8b_m1", "qwen3_8b_m16"):
+            D = Workload(hsq, WORKLOADS[dname], dev)
+            D.prepare_steps(args.warmup)
+            dsteps = max(50, args.steps)
+            d_ms = _max_over_ranks(D.timed_steps_ms(dsteps), world) / dsteps
+            dkt = D.kernel_times()
+            dops = sum(layer_ops(L["spec"]) for L in D.layers)
+            decode[dname] = {"ms_per_step": d_ms, "tops": dops * world / (d_ms * 1e-3) / 1e12,
+                             "tokens_per_s": D.specs[0].M * world / (d_ms * 1e-3),
+                             "fused_activation_step": D.fused, "gpu_launches_per_step": D.launches_per_step(),
+                             "l2": D.l2_note(), "roofline": D.roofline(dkt, peaks, dname),
+                             "layers": D.layer_detail(dkt)}
+            del D
+            torch.cuda.empty_cache()
+        if hsq.hsq_get_device_status() != hsq.HSQ_OK:
+            raise RuntimeError("a kernel reported a timeout in the decode measurements")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -480,23 +647,20 @@ def run_gpu(args, specs, wl_name, rank, world, local):
         line = {
             "metric": METRIC, "value": tops, "unit": "TOPS",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes on i8/e4m3 tensor cores, f32 accumulate",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int4 codes on i8/e4m3 tensor cores, f32 accumulate",
             "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",
             "config": {"workload": wl_name, "layers": [s.name for s in specs], "tokens_per_step": tokens_step,
                        "r": specs[0].r, "group": specs[0].group, "parallelism": f"replicas x{world}",
-                       "fused_activation_step": fused,
-                       "l2": (f"inputs larger than L2: {nrep} replicas of the step's layers (distinct weights, "
-                              f"activations, outputs), steps and per-kernel launches cycle through them; "
-                              f"{nrep * ws_bytes / 2**20:.0f} MiB in all, {ws_bytes / 2**20:.1f} MiB per step"
-                              if nrep > 1 else
-                              f"no flush; per-step working set {ws_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2")},
+                       "fused_activation_step": W.fused, "l2": W.l2_note()},
             "tokens_per_s": tokens_step * world / (ms_step * 1e-3),
             "e2e": {"value": tops_e2e, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": ms_e2e},
-            "gpu_launches": sum(1 if fused else 4 if big else 2 for big in large) * args.steps,
+            "gpu_launches": W.launches_per_step() * args.steps,
             "graph": "one step captured in a CUDA graph, replayed K times",
             "roofline": roofline,
-            "layers": layer_detail,
+            "layers": W.layer_detail(kt),
+            "decode": decode,
             "cpu_baseline": cpu,
             "clocks": clk,
         }
@@ -511,6 +675,7 @@ def main():
     ap.add_argument("--impl", default="hsq", choices=["hsq", "reference"])
     ap.add_argument("--workload", default="flux_block_r4", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-size sub-measurements")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3

@@ -263,7 +263,14 @@ def lowrank_init(W, s, r):
 
 
 def bf16_ulp(y):
-    """Spacing of bf16 numbers at |y| (fp64), used by the bf16-output tolerance."""
+    """Spacing of bf16 numbers at |y| (fp64), used by the bf16-output tolerance.
+
+    bf16 keeps 8 significant bits (7 stored) and the fp32 exponent range, so in
+    the binade [2^E, 2^(E+1)) its spacing is 2^(E-7); below the smallest normal
+    2^-126 the spacing stays 2^-133.  E is read exactly from the fp64 exponent
+    (frexp), not from a rounded logarithm.
+    """
     y = np.abs(np.asarray(y, dtype=f64))
-    e = np.floor(np.log2(np.maximum(y, 2.0 ** -126)))
-    return 2.0 ** (e - 7)
+    _, e = np.frexp(y)                    # y = m 2^e with m in [0.5, 1)
+    E = np.maximum(np.where(y > 0, e - 1, -126), -126)
+    return np.ldexp(np.ones_like(y), E - 7)

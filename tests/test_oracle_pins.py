@@ -11,6 +11,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import hsq_oracle as O
 
@@ -450,3 +451,40 @@ def test_lowrank_init_picks_the_largest_axes_of_a_scaled_selection():
         expect[n] = 0.5 * vals[n]
         assert np.allclose(L2[j], expect, atol=1e-12)
     assert np.allclose(sv[:r], [4.5, 3.25, 2.0])
+
+
+# --------------------------------------------------------------------------
+# bf16_ulp: the spacing the bf16-output tolerance adds, fixed by the bf16 format
+# --------------------------------------------------------------------------
+def _bf16_values_from_bits(bits):
+    """bf16 bit patterns (uint16) -> their values, decoded by torch's bfloat16."""
+    t = torch.tensor(np.asarray(bits, dtype=np.int32).astype(np.int16), dtype=torch.int16)
+    return t.view(torch.bfloat16).double().numpy()
+
+
+def test_bf16_ulp_hand_values():
+    # 8 significant bits: spacing 2^-7 in [1, 2), 2^-6 in [2, 4)
+    assert O.bf16_ulp(np.array([1.0]))[0] == 2.0 ** -7
+    assert O.bf16_ulp(np.array([1.5]))[0] == 2.0 ** -7
+    assert O.bf16_ulp(np.array([2.0]))[0] == 2.0 ** -6
+    assert O.bf16_ulp(np.array([-3.0]))[0] == 2.0 ** -6
+    assert O.bf16_ulp(np.array([0.75]))[0] == 2.0 ** -8
+    # just below a power of two stays in the lower binade (no rounding of a logarithm)
+    assert O.bf16_ulp(np.array([2.0 - 2.0 ** -40]))[0] == 2.0 ** -7
+    assert O.bf16_ulp(np.array([np.nextafter(1.0, 0.0)]))[0] == 2.0 ** -8
+    # subnormal range: the spacing stays that of the smallest binade, 2^-133
+    assert O.bf16_ulp(np.array([3 * 2.0 ** -130]))[0] == 2.0 ** -133
+    assert O.bf16_ulp(np.array([0.0]))[0] == 2.0 ** -133
+    assert O.bf16_ulp(np.array([2.0 ** -126]))[0] == 2.0 ** -133
+
+
+def test_bf16_ulp_equals_gap_to_next_bf16_pattern():
+    """For every positive finite bf16 value x except the largest, the gap to the
+    next bit pattern is the spacing at x."""
+    bits = np.arange(1, 0x7F7F, dtype=np.int64)  # 0x7F7F is the largest finite bf16
+    lo = _bf16_values_from_bits(bits)
+    hi = _bf16_values_from_bits(bits + 1)
+    assert np.all(hi > lo)
+    assert np.array_equal(O.bf16_ulp(lo), hi - lo)
+    # and at a point inside each gap
+    assert np.array_equal(O.bf16_ulp((lo + hi) / 2), hi - lo)

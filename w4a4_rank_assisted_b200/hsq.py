@@ -183,10 +183,12 @@ def hsq_linear_forward_fused(X, s, L1, w_codes, w_scales, L2, bias, M, N, K, r, 
 
 
 def fused_supported(M: int, K: int, r: int, group: int = GROUP) -> bool:
-    """Whether hsq_linear_forward_fused takes this shape (mirrors its checks)."""
-    if M < 1 or M > 4 or r not in (0, 1, 2, 4):
+    """Whether hsq_linear_forward_fused takes this shape: the limits stated in
+    include/hsq.h, restated in integer arithmetic (no library call, so that it
+    can be asked without a GPU)."""
+    if M < 1 or M > 4 or r not in (0, 1, 2, 4) or group not in (64, 128):
         return False
-    G = hsq_num_groups(K, group)
+    G = -(-K // group)
     mt = 1 if M <= 1 else 2 if M <= 2 else 4
     return mt * (G * group + 4 * G + 272) <= 200 * 1024
 
