@@ -137,8 +137,10 @@ def time_kernel_nodes(launch, stream, name_part: str, calls: int, repeats: int =
                 kept.append(nd)
             else:
                 _cu(cu.cuGraphDestroyNode(nd))
-        for a, b in zip(kept[:-1], kept[1:]):
-            _cu(cu.cuGraphAddDependencies(graph, [a], [b], 1))
+        for a, b in zip(kept[:-1], kept[1:]):  # chain the kept nodes (edges not already there)
+            have = _cu(cu.cuGraphNodeGetDependencies(b, _cu(cu.cuGraphNodeGetDependencies(b, 0))[1]))[0]
+            if int(a) not in {int(x) for x in have}:
+                _cu(cu.cuGraphAddDependencies(graph, [a], [b], 1))
         exe = _cu(cu.cuGraphInstantiate(graph, 0))
         try:
             _cu(cu.cuGraphLaunch(exe, hs))

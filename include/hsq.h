@@ -220,6 +220,60 @@ hsq_status hsq_lowrank_init(const void* W_bf16, const float* s, int N, int K, in
                             unsigned long long seed, void* L1_bf16, void* L2_bf16,
                             void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * NVFP4 variant.  The DiRotQ page (papernotes.org, quantization settings)
+ * names, next to INT4 W4A4 with groups of 64, the 4-bit floating-point W4A4
+ * setting of Blackwell: the standard NVFP4 format, E2M1 values sharing one FP8
+ * scale per 16 values.  The same layer (smoothed X_hat, residual R, the 16-bit
+ * low-rank branch and the bias as above) with both 4-bit operands in NVFP4:
+ *
+ *   g  = fp32(amax(|V|) / 2688) per tensor (2688 = 6 * 448)
+ *   b  = E4M3(fp32(blockmax / fp32(6 g))) per 16 values along K: round to
+ *        nearest, ties to even, saturating at 448
+ *   code = E2M1(fp32(v / fp32(b g))): nearest of {0, .5, 1, 1.5, 2, 3, 4, 6},
+ *        ties to the even mantissa, saturating at 6; sign in bit 3; a value
+ *        that rounds to 0 has code 0
+ *   g = 0 gives scales 0 and codes 0; a block whose scale is 0 has codes 0.
+ *   Y = gx gw sum_k (ex bx)(ew bw) + U L2 + b   (the tensor-core MMA applies
+ *       the block scales; fp32 accumulation)
+ *
+ * Layouts (K rounded up to Kq = 64 * ceil(K/64); padding codes and scales 0):
+ *   codes   [rows][Kq/2] bytes, code 2j in bits 0-3 and 2j+1 in bits 4-7
+ *   scales  E4M3 bytes in atoms of 128 rows x 64 K, [ceil(rows/128)][Kq/64][512]:
+ *           in atom (t, c) the byte at 16 (i % 32) + 4 (i / 32) + j is the
+ *           scale of row 128 t + i, values 64 c + 16 j .. + 15 (rows past
+ *           `rows` are written 0)
+ *   gs      device float[2]: gs[0] receives g; gs[1] is the call's scratch
+ * Supported: K % 8 == 0, N % 8 == 0, 0 <= r <= 32, 1 <= M, N, K <= 2^20;
+ * pointers 16-byte aligned; calls asynchronous on `stream`.
+ */
+size_t hsq_fp4_codes_bytes(int rows, int K);   /* rows * Kq / 2 */
+size_t hsq_fp4_scales_bytes(int rows, int K);  /* ceil(rows/128) * Kq/64 * 512 */
+
+/* Offline: R as in hsq_pack_weights (fp64, fixed order, one fp32 rounding),
+ * then NVFP4 codes, block scales and the tensor scale (two passes over W). */
+hsq_status hsq_fp4_pack_weights(const void* W_bf16, const float* s, const void* L1_bf16,
+                                const void* L2_bf16, int N, int K, int r, uint8_t* w_codes,
+                                uint8_t* w_sf, float* w_gs, cudaStream_t stream);
+
+/* Per forward: X_hat = fp32(fp32(X)/s), its NVFP4 codes, block scales and
+ * tensor scale (a first kernel takes the tensor's absmax), and U = X_hat L1 in
+ * fp32 exactly as hsq_quantize_act computes it. */
+hsq_status hsq_fp4_quantize_act(const void* X_bf16, const float* s, const void* L1_bf16, int M, int K,
+                                int r, uint8_t* x_codes, uint8_t* x_sf, float* x_gs, float* U,
+                                cudaStream_t stream);
+
+/* The forward on tcgen05 block-scaled MMAs (kind::mxf4nvf4, E4M3 scales per
+ * 16 values applied inside the instruction, one accumulator chain per tile),
+ * then Y = acc * fp32(gx gw) + U L2 + b rounded once to the output type.  No
+ * workspace.  Arguments as written by the two calls above; L2, bias, Y, out as
+ * for hsq_linear_forward. */
+hsq_status hsq_fp4_linear_forward(const uint8_t* x_codes, const uint8_t* x_sf, const float* x_gs,
+                                  const float* U, const uint8_t* w_codes, const uint8_t* w_sf,
+                                  const float* w_gs, const void* L2_bf16, const void* bias_bf16,
+                                  int M, int N, int K, int r, void* Y, hsq_out_dtype out,
+                                  cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* hsq_status_string(hsq_status status);
 

@@ -108,7 +108,10 @@ def quantize_nvfp4(V):
     denom = (scales.astype(f32) * g).astype(f32)        # fp32(b * g)
     with np.errstate(divide="ignore", invalid="ignore"):
         t = np.where(denom[..., None] > 0, blocks / denom[..., None], f32(0)).astype(f32)
-    codes = e2m1_encode(t.astype(f64)).reshape(rows, Kp)
+    t = t.reshape(rows, Kp)
+    codes = np.zeros((rows, Kp), dtype=np.uint8)
+    for i in range(0, rows, 256):  # in row slices, to bound the encoder's temporaries
+        codes[i:i + 256] = e2m1_encode(t[i:i + 256].astype(f64))
     return codes, scales, g
 
 
@@ -125,21 +128,45 @@ def pack_fp4(codes):
 
 
 # ---------------------------------------------------------------- the layer
-def nvfp4_layer_forward(X, W, s, L1, L2, bias):
-    """Y = deq(NVFP4(X_hat)) deq(NVFP4(R))^T + (X_hat L1) L2 + b, with X_hat and
-    R formed exactly as in oracle.hsq_oracle (fp32 X_hat, fp32 residual) and the
-    products and sums in fp64."""
-    from . import hsq_oracle as H  # the INT4 oracle's smoothing and residual steps
+def nvfp4_quantize_act(X, s, L1):
+    """The per-forward step: X_hat = fp32(X)/s exactly as oracle.hsq_oracle forms
+    it, its NVFP4 codes, block scales and tensor scale, and U = X_hat L1 in fp64."""
+    from . import hsq_oracle as H  # the INT4 oracle's smoothing step
     Xh = H.smooth_activation(X, s)
-    R = H.residual_weight(W, s, L1, L2)
-    xc, xs, xg = quantize_nvfp4(Xh)
-    wc, ws, wg = quantize_nvfp4(R)
-    K = np.asarray(X).shape[1]
+    c, sc, g = quantize_nvfp4(Xh)
+    if L1 is None or np.asarray(L1).shape[1] == 0:
+        U = np.zeros((Xh.shape[0], 0), dtype=f64)
+    else:
+        U = Xh.astype(f64) @ np.asarray(L1, dtype=f64)
+    return c, sc, g, U
+
+
+def nvfp4_pack_weights(W, s, L1, L2):
+    """Offline: the residual R = W diag(s) - (L1 L2)^T as oracle.hsq_oracle forms
+    it (fp64, fixed order, one fp32 rounding), then its NVFP4 codes, block scales
+    and tensor scale."""
+    from . import hsq_oracle as H  # the INT4 oracle's residual step
+    return quantize_nvfp4(H.residual_weight(W, s, L1, L2))
+
+
+def nvfp4_linear_forward(xc, xs, xg, U, wc, ws, wg, L2, bias, K):
+    """Y = deq(x) deq(w)^T + U L2 + b in fp64, from the codes [rows, Kp] (one code
+    per byte), block scales [rows, Kp/16] and tensor scales of both operands;
+    K is the layer's true width (the padding is dropped)."""
     Xq = dequantize_nvfp4(xc, xs, xg)[:, :K]
     Rq = dequantize_nvfp4(wc, ws, wg)[:, :K]
     Y = Xq @ Rq.T
-    if L1 is not None and np.asarray(L1).shape[1] > 0:
-        Y += (Xh.astype(f64) @ np.asarray(L1, dtype=f64)) @ np.asarray(L2, dtype=f64)
+    if U is not None and np.asarray(U).shape[1] > 0:
+        Y += np.asarray(U, dtype=f64) @ np.asarray(L2, dtype=f64)
     if bias is not None:
         Y += np.asarray(bias, dtype=f64)[None, :]
     return Y
+
+
+def nvfp4_layer_forward(X, W, s, L1, L2, bias):
+    """Y = deq(NVFP4(X_hat)) deq(NVFP4(R))^T + (X_hat L1) L2 + b, with X_hat and
+    R formed exactly as in oracle.hsq_oracle (fp32 X_hat, fp32 residual) and the
+    products and sums in fp64: the three steps above in order."""
+    wc, ws, wg = nvfp4_pack_weights(W, s, L1, L2)
+    xc, xs, xg, U = nvfp4_quantize_act(X, s, L1)
+    return nvfp4_linear_forward(xc, xs, xg, U, wc, ws, wg, L2, bias, np.asarray(X).shape[1])

@@ -21,7 +21,7 @@ MIS = (1 << 20) + 4  # misaligned
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(hsq_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(hsq_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -154,3 +154,33 @@ def test_workspace_needs_are_consistent():
     assert hsq.hsq_workspace_bytes(8, 12288, 4096, 4) == 0
     assert hsq.hsq_workspace_bytes(8, 4096, 32768, 4) > 0  # K = 32768
     assert hsq.hsq_workspace_bytes(0, 4096, 12288, 4) == 0
+
+
+def test_fp4_size_helpers():
+    # K rounded up to 64; scale atoms of 128 rows x 64 K (512 bytes)
+    assert hsq.hsq_fp4_codes_bytes(3, 96) == 3 * 64
+    assert hsq.hsq_fp4_codes_bytes(4608, 3072) == 4608 * 1536
+    assert hsq.hsq_fp4_scales_bytes(1, 64) == 512
+    assert hsq.hsq_fp4_scales_bytes(129, 200) == 2 * 4 * 512
+    assert hsq.hsq_fp4_scales_bytes(12288, 3072) == 96 * 48 * 512
+
+
+def test_fp4_argument_validation():
+    lib = hsq.load()
+    # weights: K % 8, rank, L1/L2 presence, alignment
+    assert lib.hsq_fp4_pack_weights(A, A, A, A, 64, 60, 4, A, A, A, None) == hsq.HSQ_ERR_UNSUPPORTED
+    assert lib.hsq_fp4_pack_weights(A, A, A, A, 64, 64, 33, A, A, A, None) == hsq.HSQ_ERR_UNSUPPORTED
+    assert lib.hsq_fp4_pack_weights(A, A, None, A, 64, 64, 4, A, A, A, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert lib.hsq_fp4_pack_weights(A, A, A, A, 64, 64, 4, A, A, None, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert lib.hsq_fp4_pack_weights(A, A, A, A, 64, 64, 4, A, MIS, A, None) == hsq.HSQ_ERR_ALIGNMENT
+    # activations
+    assert lib.hsq_fp4_quantize_act(A, A, A, 0, 64, 4, A, A, A, A, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert lib.hsq_fp4_quantize_act(A, A, A, 8, 64, 4, A, A, A, None, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert lib.hsq_fp4_quantize_act(A, A, A, 8, 64, 4, A, A, MIS, A, None) == hsq.HSQ_ERR_ALIGNMENT
+    # forward: N % 8, output type, scales present
+    f = lib.hsq_fp4_linear_forward
+    assert f(A, A, A, A, A, A, A, A, None, 16, 60, 64, 4, A, 0, None) == hsq.HSQ_ERR_UNSUPPORTED
+    assert f(A, A, A, A, A, A, A, A, None, 16, 64, 64, 4, A, 7, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert f(A, None, A, A, A, A, A, A, None, 16, 64, 64, 4, A, 0, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert f(A, A, A, None, A, A, A, A, None, 16, 64, 64, 4, A, 0, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert f(A, A, A, A, A, A, A, A, MIS, 16, 64, 64, 4, A, 0, None) == hsq.HSQ_ERR_ALIGNMENT

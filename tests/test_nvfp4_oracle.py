@@ -4,6 +4,7 @@ E2M1 grid and its ties (derived by hand), a scalar re-derivation of the block
 quantizer, on-grid round trips, and a lossless layer."""
 import numpy as np
 import pytest
+import torch
 
 from oracle import nvfp4_oracle as F
 
@@ -140,3 +141,34 @@ def test_lossless_layer_equals_the_dense_product():
     bias = rng.standard_normal(5)
     Y = F.nvfp4_layer_forward(X.astype(f32), W.astype(f32), np.ones(48, dtype=f32), None, None, bias)
     assert np.array_equal(Y, X @ W.T + bias[None, :])
+
+
+def test_lossless_layer_with_low_rank_branch_equals_the_dense_product():
+    """s = 1, r = 2: the residual R = W - (L1 L2)^T and X are on the NVFP4 grid
+    with values that are multiples of 2^-8, so W = R + (L1 L2)^T is exact in bf16
+    and the quantization is lossless.  Then X R^T + (X L1) L2 = X W^T exactly:
+    a dropped, transposed or sign-flipped branch fails."""
+    rng = np.random.default_rng(5)
+    K, M, N, r = 64, 3, 5, 2
+    g = 2.0 ** -12
+    # block scales that are multiples of 32, so every k b g is a multiple of 2^-8
+    bvals = np.array([32.0, 64.0, 96.0, 128.0, 192.0, 256.0, 320.0, 384.0, 448.0])
+
+    def grid(rows):
+        b = rng.choice(bvals, (rows, K // 16))
+        b[0, 0] = 448.0
+        k = rng.choice(np.concatenate([F.E2M1_GRID, -F.E2M1_GRID]), (rows, K // 16, 16))
+        k[..., 0] = 6.0
+        return (k * b[..., None] * g).reshape(rows, K)
+
+    X, R = grid(M), grid(N)
+    L1 = rng.integers(-2, 3, (K, r)) * 2.0 ** -4
+    L2 = rng.integers(-2, 3, (r, N)) * 2.0 ** -4
+    W = R + (L1 @ L2).T
+    Wb = torch.tensor(W, dtype=torch.float64).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(Wb, W), "W must be exact in bf16"
+    bias = rng.standard_normal(N)
+    Y = F.nvfp4_layer_forward(X.astype(f32), W.astype(f32), np.ones(K, dtype=f32), L1.astype(f32),
+                              L2.astype(f32), bias)
+    assert np.array_equal(Y, X @ W.T + bias[None, :])
+    assert np.max(np.abs((X @ L1) @ L2)) > 0  # the branch is not trivially zero

@@ -54,7 +54,7 @@ def _noalloc(pl, act, M, K, N, r, group):
     (16, 4096, 2048, 4, 64),    # split-K decode tiles: uses the scratch array
     (128, 2048, 1024, 4, 64),   # split-K 128x256 tiles: uses the scratch array
     (200, 224, 1160, 32, 64),   # whole tiles: no scratch
-    (320, 1024, 1024, 4, 64),   # more than 256 tokens: expanded codes in the scratch array
+    (320, 640, 1024, 4, 64),    # more than 256 tokens: expanded codes in the scratch array (whole tiles)
     (128, 2048, 1024, 4, 128),  # groups of 128 above 64 tokens: expanded codes in the scratch array
 ])
 def test_noalloc_matches_regular_entry_point_twice(M, K, N, r, group):

@@ -548,6 +548,89 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// ---------------------------------------------------------------- block-scaled MMA (NVFP4)
+// D[tmem] (+)= (A * SFA) x (B * SFB)^T with E2M1 A and B (packed two per byte,
+// K-major, K = 64 per instruction) and one E4M3 scale per 16 K-values of every
+// row of A and of B, read from Tensor Memory at tsfa / tsfb (block16 =
+// scale_vec::4X: one 32-bit column word holds a row's 4 scales of the
+// instruction's K = 64).  fp32 accumulator.
+__device__ __forceinline__ void mma_fp4_block16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with block scales: A, B E2M1, E4M3
+// scale factors (scale format bit 0), both K-major, dense K = 64, scale-factor
+// ids 0 (the scales of an instruction fill whole 32-bit TMEM words).
+__host__ __device__ constexpr uint32_t idesc_fp4_block16(int M, int N) {
+  return (1u << 7)                                   // A: E2M1
+         | (1u << 10)                                // B: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (0u << 23)                                // scale factors: E4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Copy 32 rows x 16 bytes of shared memory (one scale-factor atom: row i of the
+// atom holds the 4-byte words of matrix rows i, i+32, i+64, i+96) into Tensor
+// Memory at column `taddr`, replicated into the four 32-lane quadrants: lane
+// 32q + i, column c + j receives bytes 4j..4j+3 of atom row i, so matrix row m
+// finds its word at lane m, column c + m / 32.
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor for a K-major operand laid out by a TMA load with
+// 128-byte swizzle: 8-row x 128-byte atoms, `sbo` bytes between 8-row groups
+// (the atom base must be 1024-byte aligned; the start may advance along K by a
+// multiple of 16 bytes inside the 128-byte row).
+__device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;  // leading byte offset (unused by swizzled K-major)
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+  d |= static_cast<uint64_t>(2) << 61;  // layout: 128-byte swizzle
+  return d;
+}
+
+// fp32 -> E4M3 byte, round to nearest even, saturating at +-448 (finite).
+__device__ __forceinline__ uint32_t f32_to_e4m3_rn_sat(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return static_cast<uint32_t>(r) & 0xFFu;  // the second source lands in the low byte
+}
+
+// E4M3 byte (finite, sign 0) -> fp32, exactly.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+  // subnormal m * 2^-9, normal (1 + m/8) 2^(e-7)
+  return e == 0 ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Eight fp32 -> eight E2M1 codes (code e in bits 4e..4e+3), each rounded to the
+// nearest of {0, 0.5, 1, 1.5, 2, 3, 4, 6} with ties to the even mantissa bit and
+// saturating at 6; a value that rounds to zero gets code 0 (never the -0 pattern).
+__device__ __forceinline__ uint32_t f32x8_to_e2m1(const float (&v)[8]) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  const uint32_t mag = w & 0x77777777u;
+  const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;  // bit 3 of a nibble: magnitude > 0
+  return mag | (w & nonzero);
+}
+
 // Warpgroup register reallocation.
 template <int N>
 __device__ __forceinline__ void regs_dealloc() {

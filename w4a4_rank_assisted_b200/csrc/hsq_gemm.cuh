@@ -55,6 +55,12 @@
 
 #include "hsq_device.cuh"
 
+// Registers per thread left to the producer / MMA / helper warpgroups of
+// blocks of up to 512 threads (the rest go to the drain warpgroups).
+#ifndef HSQ_REGS_LOW_SMALL
+#define HSQ_REGS_LOW_SMALL 64
+#endif
+
 namespace hsq {
 
 // Canonical no-swizzle K-major layout of one operand and one 64-wide group:
@@ -154,7 +160,7 @@ struct GemmCfg {
   static constexpr bool REALLOC = CW >= 128 || THREADS >= 768;
   static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8 * 8) > 255 ? 248 : (65536 / THREADS) / 8 * 8;
   static constexpr int LOW_THREADS = THREADS - 32 * NUM_DRAIN_WARPS;  // producer, MMA, unpack warpgroups
-  static constexpr int REGS_LOW = (THREADS <= 512 || LOW_THREADS <= 128) ? 64 : 40;
+  static constexpr int REGS_LOW = (THREADS <= 512 || LOW_THREADS <= 128) ? HSQ_REGS_LOW_SMALL : 40;
   static constexpr int REGS_HIGH_RAW =
       ((THREADS * LAUNCH_REGS - LOW_THREADS * REGS_LOW) / (32 * NUM_DRAIN_WARPS)) / 8 * 8;
   static constexpr int REGS_HIGH = REGS_HIGH_RAW > 232 ? 232 : REGS_HIGH_RAW;

@@ -17,6 +17,7 @@
 
 #include "../../include/hsq.h"
 #include "hsq_device.cuh"
+#include "hsq_fp4.cuh"
 #include "hsq_gemm.cuh"
 #include "hsq_gemv.cuh"
 #include "hsq_lowrank.cuh"
@@ -39,10 +40,30 @@ constexpr int kMaxRank = 32;
 #ifndef HSQ_PAIR
 #define HSQ_PAIR 0
 #endif
-using CfgLarge64 = hsq::GemmCfg<256, 2, HSQ_PAIR ? 8 : 6, false, 1, 3, 2, 2, HSQ_PAIR ? 12 : 10, true, -1, true, 2,
+// Drain layout of the large tiles: HSQ_LARGE_DH column slices of 4 warps each,
+// HSQ_LARGE_CHB 8-column blocks per Tensor Memory load, HSQ_LARGE_PIPE (-1: by
+// register budget) for the next load in flight during the current chunk's math.
+#ifndef HSQ_LARGE_DH
+#define HSQ_LARGE_DH 2
+#endif
+#ifndef HSQ_LARGE_STAGES
+#define HSQ_LARGE_STAGES 6
+#endif
+#ifndef HSQ_LARGE128_STAGES
+#define HSQ_LARGE128_STAGES 3
+#endif
+#ifndef HSQ_LARGE_CHB
+#define HSQ_LARGE_CHB 2
+#endif
+#ifndef HSQ_LARGE_PIPE
+#define HSQ_LARGE_PIPE -1
+#endif
+using CfgLarge64 = hsq::GemmCfg<256, HSQ_LARGE_DH, HSQ_PAIR ? 8 : HSQ_LARGE_STAGES, false, 1, 3, 2, 2,
+                                HSQ_PAIR ? 12 : HSQ_LARGE_STAGES + 4, true, HSQ_LARGE_PIPE, true, HSQ_LARGE_CHB,
                                 1, HSQ_PAIR != 0>;
-using CfgLarge128 = hsq::GemmCfg<256, 2, HSQ_PAIR ? 4 : 3, false, 1, 3, 2, 2, HSQ_PAIR ? 8 : 7, true, -1, true, 2,
-                                 2, HSQ_PAIR != 0>;
+using CfgLarge128 = hsq::GemmCfg<256, HSQ_LARGE_DH, HSQ_PAIR ? 4 : HSQ_LARGE128_STAGES, false, 1, 3, 2, 2,
+                                 HSQ_PAIR ? 8 : HSQ_LARGE128_STAGES + 4, true,
+                                 HSQ_LARGE_PIPE, true, HSQ_LARGE_CHB, 2, HSQ_PAIR != 0>;
 // 64 < M <= 256, groups of 64 ("mid"): tokens x outputs tiles of 128 x 256 that
 // unpack both packed operands in shared memory (6 warps) instead of expanding
 // them in HBM first -- with one or two token tiles each weight tile is read about
@@ -312,6 +333,21 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, in
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over NVFP4 codes [rows][Kq/2] bytes for the block-scaled kernel: box =
+// 128 bytes (a stage's K = 256) x 128 rows, 128-byte swizzle (the layout its
+// MMA descriptors read).
+bool make_fp4_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kq) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Kq / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Kq / 2)};
+  const cuuint32_t box[2] = {128u, 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -651,11 +687,11 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   lerr = (group == 128 ? launch_pdl(true, hsq::quantize_act_kernel<RV, SM, 16>,                             \
                                     dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),     \
                                     dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, \
-                                    x_codes, x_scales, U)                                                  \
+                                    x_codes, x_scales, U, static_cast<float*>(nullptr))                    \
                        : launch_pdl(true, hsq::quantize_act_kernel<RV, SM, 8>,                              \
                                     dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),     \
                                     dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, \
-                                    x_codes, x_scales, U))
+                                    x_codes, x_scales, U, static_cast<float*>(nullptr)))
 #define HSQ_ACT_RANKS(SM)                   \
   switch (r) {                              \
     case 0: HSQ_ACT_LAUNCH(0, SM); break;   \
@@ -880,6 +916,150 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
   HSQ_FUSED_R(4);
 #undef HSQ_FUSED_R
 #undef HSQ_FUSED
+}
+
+// ------------------------------------------------------------------ NVFP4 variant
+static int fp4_kq(int K) { return (K + 63) / 64 * 64; }
+
+size_t hsq_fp4_codes_bytes(int rows, int K) {
+  if (rows < 0 || K < 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(fp4_kq(K)) / 2;
+}
+
+size_t hsq_fp4_scales_bytes(int rows, int K) {
+  if (rows < 0 || K < 0) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>(fp4_kq(K) / 64) * 512;
+}
+
+static hsq_status fp4_check(int rows, int K, int r) {
+  if (rows < 1 || K < 1 || rows > kMaxDim || K > kMaxDim || r < 0) return HSQ_ERR_INVALID_ARG;
+  if (r > kMaxRank || (K % 8) != 0) return HSQ_ERR_UNSUPPORTED;
+  return HSQ_OK;
+}
+
+hsq_status hsq_fp4_pack_weights(const void* W_bf16, const float* s, const void* L1_bf16, const void* L2_bf16, int N,
+                                int K, int r, uint8_t* w_codes, uint8_t* w_sf, float* w_gs, cudaStream_t stream) {
+  hsq_status st = fp4_check(N, K, r);
+  if (st != HSQ_OK) return st;
+  if (!W_bf16 || !s || !w_codes || !w_sf || !w_gs) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1_bf16 != nullptr) || (r > 0) != (L2_bf16 != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(W_bf16) || !aligned16(s) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(w_gs) ||
+      (L1_bf16 && !aligned16(L1_bf16)) || (L2_bf16 && !aligned16(L2_bf16)))
+    return HSQ_ERR_ALIGNMENT;
+  const int Kq = fp4_kq(K), KC = Kq / 64;
+  const auto* W = static_cast<const __nv_bfloat16*>(W_bf16);
+  const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
+  const auto* L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
+  const int blocks = (N + 7) / 8;
+  if (cudaMemsetAsync(w_gs, 0, 2 * sizeof(float), stream) != cudaSuccess) return HSQ_ERR_CUDA;
+  // first pass: absmax of the residual; second pass: codes and block scales
+  hsq::pack_weights_kernel<2, 1><<<blocks, 256, 0, stream>>>(W, s, L1, L2, N, K, r, Kq, 0, w_codes, nullptr, w_gs);
+  hsq::pack_weights_kernel<2, 2><<<blocks, 256, 0, stream>>>(W, s, L1, L2, N, K, r, Kq, 0, w_codes,
+                                                             reinterpret_cast<float*>(w_sf), w_gs);
+  const int pad = (N + 127) / 128 * 128 - N;
+  if (pad > 0) hsq::nvfp4_zero_sf_pad_kernel<<<(pad * KC + 255) / 256, 256, 0, stream>>>(w_sf, N, KC);
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
+hsq_status hsq_fp4_quantize_act(const void* X_bf16, const float* s, const void* L1_bf16, int M, int K, int r,
+                                uint8_t* x_codes, uint8_t* x_sf, float* x_gs, float* U, cudaStream_t stream) {
+  hsq_status st = fp4_check(M, K, r);
+  if (st != HSQ_OK) return st;
+  if (!X_bf16 || !s || !x_codes || !x_sf || !x_gs) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1_bf16 != nullptr) || (r > 0 && !U)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(x_codes) || !aligned16(x_sf) || !aligned16(x_gs) ||
+      (L1_bf16 && !aligned16(L1_bf16)) || (U && !aligned16(U)))
+    return HSQ_ERR_ALIGNMENT;
+  const int Kq = fp4_kq(K), KC = Kq / 64;
+  const auto* X = static_cast<const __nv_bfloat16*>(X_bf16);
+  const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
+  float* sf = reinterpret_cast<float*>(x_sf);
+  if (cudaMemsetAsync(x_gs, 0, 2 * sizeof(float), stream) != cudaSuccess) return HSQ_ERR_CUDA;
+  const long groups = static_cast<long>(M) * (K / 8);
+  const int ablocks = static_cast<int>(std::min<long>(4l * device_sm_count(), (groups + 255) / 256));
+  if (launch_pdl(false, hsq::nvfp4_act_amax_kernel, dim3(ablocks), dim3(256), 0, stream, X, s, M, K, x_gs) !=
+      cudaSuccess)
+    return HSQ_ERR_CUDA;
+  cudaError_t lerr = cudaSuccess;
+#define HSQ_FP4_ACT(RV, SM)                                                                                \
+  lerr = launch_pdl(false, hsq::quantize_act_kernel<RV, SM, 2, true>,                                      \
+                    dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),                     \
+                    dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kq, 0, x_codes, sf, U, \
+                    x_gs)
+#define HSQ_FP4_RANKS(SM)                  \
+  switch (r) {                             \
+    case 0: HSQ_FP4_ACT(0, SM); break;     \
+    case 1: HSQ_FP4_ACT(1, SM); break;     \
+    case 2: HSQ_FP4_ACT(2, SM); break;     \
+    case 4: HSQ_FP4_ACT(4, SM); break;     \
+    case 8: HSQ_FP4_ACT(8, SM); break;     \
+    case 16: HSQ_FP4_ACT(16, SM); break;   \
+    case 32: HSQ_FP4_ACT(32, SM); break;   \
+    default: HSQ_FP4_ACT(-1, SM); break;   \
+  }
+  if (M <= 64) {
+    HSQ_FP4_RANKS(true)
+  } else {
+    HSQ_FP4_RANKS(false)
+  }
+#undef HSQ_FP4_RANKS
+#undef HSQ_FP4_ACT
+  if (lerr != cudaSuccess) return HSQ_ERR_CUDA;
+  const int pad = (M + 127) / 128 * 128 - M;
+  if (pad > 0) hsq::nvfp4_zero_sf_pad_kernel<<<(pad * KC + 255) / 256, 256, 0, stream>>>(x_sf, M, KC);
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
+hsq_status hsq_fp4_linear_forward(const uint8_t* x_codes, const uint8_t* x_sf, const float* x_gs, const float* U,
+                                  const uint8_t* w_codes, const uint8_t* w_sf, const float* w_gs,
+                                  const void* L2_bf16, const void* bias_bf16, int M, int N, int K, int r, void* Y,
+                                  hsq_out_dtype out, cudaStream_t stream) {
+  hsq_status st = fp4_check(M, K, r);
+  if (st != HSQ_OK) return st;
+  if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return HSQ_ERR_UNSUPPORTED;
+  if (out != HSQ_OUT_BF16 && out != HSQ_OUT_F32) return HSQ_ERR_INVALID_ARG;
+  if (!x_codes || !x_sf || !x_gs || !w_codes || !w_sf || !w_gs || !Y) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L2_bf16 != nullptr) || (r > 0) != (U != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(x_codes) || !aligned16(x_sf) || !aligned16(x_gs) || !aligned16(w_codes) || !aligned16(w_sf) ||
+      !aligned16(w_gs) || !aligned16(Y) || (U && !aligned16(U)) || (L2_bf16 && !aligned16(L2_bf16)) ||
+      (bias_bf16 && !aligned16(bias_bf16)))
+    return HSQ_ERR_ALIGNMENT;
+  using Cfg = hsq::Fp4Cfg;
+  const int Kq = fp4_kq(K);
+  CUtensorMap tm_a, tm_b, tm_y;
+  if (!make_fp4_codes_map(&tm_a, x_codes, M, Kq) || !make_fp4_codes_map(&tm_b, w_codes, N, Kq) ||
+      !make_y_map(&tm_y, Y, M, N, out == HSQ_OUT_F32))
+    return HSQ_ERR_CUDA;
+  hsq::Fp4Args a{};
+  a.x_sf = x_sf; a.w_sf = w_sf; a.x_gs = x_gs; a.w_gs = w_gs;
+  a.U = U;
+  a.L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
+  a.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+  a.M = M; a.N = N; a.KC = Kq / 64; a.r = r;
+  a.tiles_m = (M + Cfg::BM - 1) / Cfg::BM;
+  a.tiles_n = (N + Cfg::BN - 1) / Cfg::BN;
+  a.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
+  a.limit_ns = wait_limit_ns();
+  static std::mutex mu;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      if (cudaFuncSetAttribute(hsq::fp4_gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::SMEM_BYTES) != cudaSuccess)
+        return HSQ_ERR_CUDA;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
+  const int tiles = a.tiles_m * a.tiles_n;
+  const int grid = std::min(tiles, device_sm_count());
+  if (launch_pdl(false, hsq::fp4_gemm_kernel<Cfg>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, stream, tm_a,
+                 tm_b, tm_y, a) != cudaSuccess)
+    return HSQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -126,22 +126,134 @@ __device__ __forceinline__ uint32_t quantize8_fast(const float (&v)[8], float& s
   return packed;
 }
 
+// NVFP4 (the DiRotQ page's FP4 setting: E2M1 values, one E4M3 scale per 16
+// values, and one fp32 scale g per tensor).  One lane's 8 values of a 16-value
+// block that spans two adjacent lanes: the block scale is the E4M3 byte
+// b = RN_sat(fp32(blockmax / sixg)), sixg = fp32(6 g); each code is the E2M1
+// rounding of fp32(v / fp32(b g)).  A zero g or a zero block scale gives codes
+// 0.  Returns the 8 codes (code e in bits 4e..4e+3) and sets `sf` to b.  Every
+// lane of the warp must call it (it shuffles).
+__device__ __forceinline__ uint32_t quantize8_nvfp4(const float (&v)[8], float g, float sixg, uint32_t& sf) {
+  float bmax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) bmax = fmaxf(bmax, fabsf(v[e]));
+  bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+  sf = 0u;
+  if (g == 0.f) return 0u;
+  sf = f32_to_e4m3_rn_sat(__fdiv_rn(bmax, sixg));
+  const float denom = __fmul_rn(e4m3_to_f32(sf), g);
+  if (denom == 0.f) return 0u;
+  float t[8];
+  if (denom >= 0x1p-100f && denom <= 0x1p100f) {
+    const float z = __frcp_rn(denom);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = div_by_recip(v[e], denom, z);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = __fdiv_rn(v[e], denom);
+  }
+  return f32x8_to_e2m1(t);
+}
+
+// The per-tensor NVFP4 scale from the tensor's absmax: g = fp32(amax / 2688)
+// (2688 = 6 * 448: the largest E2M1 magnitude times the largest E4M3 scale).
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax) { return __fdiv_rn(amax, 2688.0f); }
+
+// Byte offset of the scale word of matrix row `row` and 64-wide K chunk `kc` in
+// the NVFP4 scale layout: atoms of 128 rows x 64 K (512 bytes) ordered
+// [row tile][K chunk]; inside an atom, row i's four block scales form the
+// 32-bit word at 16 (i % 32) + 4 (i / 32).
+__device__ __forceinline__ size_t nvfp4_sf_word_offset(int row, int kc, int kchunks) {
+  return (static_cast<size_t>(row >> 7) * kchunks + kc) * 512 + 16 * (row & 31) + 4 * ((row & 127) >> 5);
+}
+
+// Gather the block-scale bytes of lanes 8p, 8p+2, 8p+4, 8p+6 (the four 16-value
+// blocks of a 64-wide K chunk) into one word on lane 8p.  Every lane calls it.
+__device__ __forceinline__ uint32_t gather_sf_word(uint32_t sf) {
+  const uint32_t b1 = __shfl_down_sync(0xffffffffu, sf, 2);
+  const uint32_t b2 = __shfl_down_sync(0xffffffffu, sf, 4);
+  const uint32_t b3 = __shfl_down_sync(0xffffffffu, sf, 6);
+  return sf | (b1 << 8) | (b2 << 16) | (b3 << 24);
+}
+
+// Zero the scale words of rows [rows, rows_pad) (rows_pad: rows rounded up to
+// 128) in every K chunk of an NVFP4 scale matrix.
+__global__ void nvfp4_zero_sf_pad_kernel(uint8_t* sf, int rows, int kchunks) {
+  const int pad = ((rows + 127) & ~127) - rows;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < pad * kchunks) {
+    const int row = rows + i / kchunks, kc = i % kchunks;
+    *reinterpret_cast<uint32_t*>(sf + nvfp4_sf_word_offset(row, kc, kchunks)) = 0u;
+  }
+}
+
+// Absmax of the smoothed activations X_hat = fp32(X)/s over the whole tensor
+// (the NVFP4 tensor scale's input), as the same quotients the quantizer forms;
+// folded into gs[1] (zeroed before the launch) with an integer atomicMax on the
+// float's bits (valid for values >= 0).  Warps stride over 8-element groups.
+__global__ void __launch_bounds__(256) nvfp4_act_amax_kernel(const __nv_bfloat16* __restrict__ X,
+                                                             const float* __restrict__ s, int M, int K,
+                                                             float* gs) {
+  grid_dep_wait();  // X may come from the preceding kernel
+  const int lane = lane_id();
+  const size_t groups = static_cast<size_t>(M) * (K / 8);
+  const size_t nwarps = static_cast<size_t>(gridDim.x) * (blockDim.x / 32);
+  float amax = 0.f;
+  for (size_t base = (static_cast<size_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5)) * 32;
+       base < groups; base += nwarps * 32) {
+    const size_t i = base + lane;
+    const bool valid = i < groups;
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    float sv[8], sz[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sv[e] = 1.f;
+    if (valid) {
+      const int m = static_cast<int>(i / (K / 8)), k0 = static_cast<int>(i % (K / 8)) * 8;
+      raw = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k0));
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + k0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + k0 + 4));
+      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+      sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sz[e] = __frcp_rn(sv[e]);
+    float xh[8];
+    smooth8(raw, sv, sz, valid, xh);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(xh[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0 && amax > 0.f) atomicMax(reinterpret_cast<unsigned int*>(gs + 1), __float_as_uint(amax));
+}
+
 // ---------------------------------------------------------------------------
 // Weight packing (offline): R[n,k] = fp32(W[n,k]*s[k] - sum_j L1[k,j]*L2[j,n]),
 // the sum in fp64 for j = 0..r-1 with every multiply and add rounded on its own
 // (no fused multiply-add), then quantized.  One warp per output row n.
 // ---------------------------------------------------------------------------
-template <int GL>
+// MODE 0: INT4 codes and fp32 group scales (GL lanes per group).
+// MODE 1 (NVFP4, first pass): only the absmax of R, folded into gs[1].
+// MODE 2 (NVFP4, second pass): E2M1 codes and E4M3 block scales (scale layout of
+//   nvfp4_sf_word_offset, `scales` taken as its bytes) with g from gs[1]; the
+//   first warp writes g to gs[0].
+template <int GL, int MODE = 0>
 __global__ void __launch_bounds__(256) pack_weights_kernel(const __nv_bfloat16* __restrict__ W,
                                                            const float* __restrict__ s,
                                                            const __nv_bfloat16* __restrict__ L1,
                                                            const __nv_bfloat16* __restrict__ L2, int N,
                                                            int K, int r, int Kp, int ld,
                                                            uint8_t* __restrict__ codes,
-                                                           float* __restrict__ scales) {
+                                                           float* __restrict__ scales, float* gs = nullptr) {
   const int n = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = lane_id();
   if (n >= N) return;  // warp-uniform
+  float g = 0.f, sixg = 0.f, amax = 0.f;
+  if constexpr (MODE == 2) {
+    g = nvfp4_tensor_scale(gs[1]);
+    sixg = __fmul_rn(6.0f, g);
+    if (n == 0 && lane == 0) gs[0] = g;
+  }
   for (int c0 = 0; c0 < Kp; c0 += 256) {
     const int k0 = c0 + lane * 8;
     float R[8];
@@ -165,12 +277,32 @@ __global__ void __launch_bounds__(256) pack_weights_kernel(const __nv_bfloat16* 
 #pragma unroll
       for (int e = 0; e < 8; ++e) R[e] = 0.f;
     }
-    float sc;
-    const uint32_t packed = quantize8<GL>(R, sc);
-    if (k0 < Kp) {
-      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (Kp / 2) + k0 / 2) = packed;
-      if ((lane & (GL - 1)) == 0) scales[static_cast<size_t>(k0 / (8 * GL)) * ld + n] = sc;
+    if constexpr (MODE == 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(R[e]));
+    } else if constexpr (MODE == 2) {
+      uint32_t sf;
+      const uint32_t packed = quantize8_nvfp4(R, g, sixg, sf);
+      const uint32_t word = gather_sf_word(sf);
+      if (k0 < Kp) {
+        *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (Kp / 2) + k0 / 2) = packed;
+        if ((lane & 7) == 0)
+          *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(scales) +
+                                       nvfp4_sf_word_offset(n, k0 / 64, Kp / 64)) = word;
+      }
+    } else {
+      float sc;
+      const uint32_t packed = quantize8<GL>(R, sc);
+      if (k0 < Kp) {
+        *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (Kp / 2) + k0 / 2) = packed;
+        if ((lane & (GL - 1)) == 0) scales[static_cast<size_t>(k0 / (8 * GL)) * ld + n] = sc;
+      }
     }
+  }
+  if constexpr (MODE == 1) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0 && amax > 0.f) atomicMax(reinterpret_cast<unsigned int*>(gs + 1), __float_as_uint(amax));
   }
 }
 
@@ -221,14 +353,24 @@ struct ActCfg {
   static constexpr int XS_FLOATS = PAIRS ? NW * SUB * KP * KSP : 1;
 };
 
-template <int R, bool SMALL, int GL>
+// FP4 = true: the NVFP4 form (quantize8_nvfp4; `scales` is taken as the bytes of
+// the NVFP4 scale layout, `ld` is unused, g comes from the absmax in gs[1] and
+// the first block writes it to gs[0]).
+template <int R, bool SMALL, int GL, bool FP4 = false>
 __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
     quantize_act_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
                         const __nv_bfloat16* __restrict__ L1, int M, int K, int r, int Kp, int ld,
-                        uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U) {
+                        uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U,
+                        float* gs = nullptr) {
   using C = ActCfg<R, SMALL>;
   constexpr int SUB = C::SUB, NW = C::NW, RB = C::RB, NSUB = C::NSUB;
-  grid_dep_wait();  // X may come from the preceding kernel
+  grid_dep_wait();  // X (and for FP4 the absmax) may come from the preceding kernel
+  float g = 0.f, sixg = 0.f;
+  if constexpr (FP4) {
+    g = nvfp4_tensor_scale(gs[1]);
+    sixg = __fmul_rn(6.0f, g);
+    if (blockIdx.x == 0 && threadIdx.x == 0) gs[0] = g;
+  }
   // a grid of a few blocks lets the next kernel start right away (it runs on the
   // idle SMs); a grid that fills the GPU lets it start only as blocks finish, so
   // that early arrivals do not take SMs from this kernel's later blocks
@@ -329,15 +471,27 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
           for (int e = 0; e < 8; ++e) xrow[e * KSP + lane] = xh[e];
         }
       }
-      float sc;
-      const uint32_t packed = quantize8_fast<GL>(xh, sc);
-      if (in_k) {
-        *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
-        if ((lane & (GL - 1)) == 0) {
-          float* srow = scales + static_cast<size_t>(k0 / (8 * GL)) * ld;
-          srow[m] = sc;
-          if (m == M - 1)
-            for (int p = M; p < ld; ++p) srow[p] = 0.f;  // padding of the group-major layout
+      if constexpr (FP4) {
+        uint32_t sf;
+        const uint32_t packed = quantize8_nvfp4(xh, g, sixg, sf);
+        const uint32_t word = gather_sf_word(sf);
+        if (in_k) {
+          *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
+          if ((lane & 7) == 0)
+            *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(scales) +
+                                         nvfp4_sf_word_offset(m, k0 / 64, Kp / 64)) = word;
+        }
+      } else {
+        float sc;
+        const uint32_t packed = quantize8_fast<GL>(xh, sc);
+        if (in_k) {
+          *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
+          if ((lane & (GL - 1)) == 0) {
+            float* srow = scales + static_cast<size_t>(k0 / (8 * GL)) * ld;
+            srow[m] = sc;
+            if (m == M - 1)
+              for (int p = M; p < ld; ++p) srow[p] = 0.f;  // padding of the group-major layout
+          }
         }
       }
     }

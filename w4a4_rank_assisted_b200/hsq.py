@@ -37,6 +37,8 @@ EXPORTED = (
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
     "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused",
     "hsq_lowrank_workspace_bytes", "hsq_lowrank_init",
+    "hsq_fp4_codes_bytes", "hsq_fp4_scales_bytes", "hsq_fp4_pack_weights", "hsq_fp4_quantize_act",
+    "hsq_fp4_linear_forward",
 )
 
 
@@ -87,6 +89,14 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_status_string.argtypes = [i]; lib.hsq_status_string.restype = c.c_char_p
     lib.hsq_get_device_status.argtypes = [vp]; lib.hsq_get_device_status.restype = i
     lib.hsq_debug_force_timeout.argtypes = [i, i]; lib.hsq_debug_force_timeout.restype = None
+    lib.hsq_fp4_codes_bytes.argtypes = [i, i]; lib.hsq_fp4_codes_bytes.restype = sz
+    lib.hsq_fp4_scales_bytes.argtypes = [i, i]; lib.hsq_fp4_scales_bytes.restype = sz
+    lib.hsq_fp4_pack_weights.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp, vp, vp]
+    lib.hsq_fp4_pack_weights.restype = i
+    lib.hsq_fp4_quantize_act.argtypes = [vp, vp, vp, i, i, i, vp, vp, vp, vp, vp]
+    lib.hsq_fp4_quantize_act.restype = i
+    lib.hsq_fp4_linear_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, i, vp]
+    lib.hsq_fp4_linear_forward.restype = i
     _lib = lib
     return lib
 
@@ -285,4 +295,76 @@ def forward(layer: PackedLinear, X: torch.Tensor, act: ActBuffers, Y: torch.Tens
     hsq_linear_forward(act.x_codes, act.x_scales, act.U, layer.w_codes, layer.w_scales, layer.L2,
                        layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace,
                        ws_bytes=ws_bytes, group=layer.group, stream=stream)
+    return Y
+
+
+# ---------------------------------------------------------------- NVFP4 variant
+def hsq_fp4_codes_bytes(rows: int, K: int) -> int:
+    return int(load().hsq_fp4_codes_bytes(rows, K))
+
+
+def hsq_fp4_scales_bytes(rows: int, K: int) -> int:
+    return int(load().hsq_fp4_scales_bytes(rows, K))
+
+
+def hsq_fp4_pack_weights(W, s, L1, L2, N, K, r, w_codes, w_sf, w_gs, stream=None) -> None:
+    _check(load().hsq_fp4_pack_weights(_ptr(W), _ptr(s), _ptr(L1), _ptr(L2), N, K, r, _ptr(w_codes),
+                                       _ptr(w_sf), _ptr(w_gs), _stream(stream)), "hsq_fp4_pack_weights")
+
+
+def hsq_fp4_quantize_act(X, s, L1, M, K, r, x_codes, x_sf, x_gs, U, stream=None) -> None:
+    _check(load().hsq_fp4_quantize_act(_ptr(X), _ptr(s), _ptr(L1), M, K, r, _ptr(x_codes), _ptr(x_sf),
+                                       _ptr(x_gs), _ptr(U), _stream(stream)), "hsq_fp4_quantize_act")
+
+
+def hsq_fp4_linear_forward(x_codes, x_sf, x_gs, U, w_codes, w_sf, w_gs, L2, bias, M, N, K, r, Y,
+                           out: int = HSQ_OUT_BF16, stream=None) -> None:
+    _check(load().hsq_fp4_linear_forward(_ptr(x_codes), _ptr(x_sf), _ptr(x_gs), _ptr(U), _ptr(w_codes),
+                                         _ptr(w_sf), _ptr(w_gs), _ptr(L2), _ptr(bias), M, N, K, r, _ptr(Y),
+                                         int(out), _stream(stream)), "hsq_fp4_linear_forward")
+
+
+def _fp4_kq(K: int) -> int:
+    return -(-K // 64) * 64
+
+
+class Fp4Linear:
+    """A layer packed in the NVFP4 variant: E2M1 residual codes, E4M3 block
+    scales and the tensor scale, plus the low-rank pair, smoothing and bias."""
+
+    def __init__(self, W, s, L1, L2, bias=None, stream=None):
+        N, K = W.shape
+        r = 0 if L1 is None else int(L1.shape[1])
+        dev = W.device
+        self.N, self.K, self.r = N, K, r
+        self.s = s.contiguous()
+        self.L1 = None if r == 0 else L1.contiguous()
+        self.L2 = None if r == 0 else L2.contiguous()
+        self.bias = None if bias is None else bias.contiguous()
+        self.w_codes = torch.empty((N, _fp4_kq(K) // 2), dtype=torch.uint8, device=dev)
+        self.w_sf = torch.empty(hsq_fp4_scales_bytes(N, K), dtype=torch.uint8, device=dev)
+        self.w_gs = torch.empty(4, dtype=torch.float32, device=dev)
+        hsq_fp4_pack_weights(W.contiguous(), self.s, self.L1, self.L2, N, K, r, self.w_codes, self.w_sf,
+                             self.w_gs, stream=stream)
+
+
+class Fp4ActBuffers:
+    """Per-forward buffers of the NVFP4 activation step for M tokens."""
+
+    def __init__(self, M: int, K: int, r: int, device):
+        self.M, self.K, self.r = M, K, r
+        self.x_codes = torch.empty((M, _fp4_kq(K) // 2), dtype=torch.uint8, device=device)
+        self.x_sf = torch.empty(hsq_fp4_scales_bytes(M, K), dtype=torch.uint8, device=device)
+        self.x_gs = torch.empty(4, dtype=torch.float32, device=device)
+        self.U = torch.empty((M, r), dtype=torch.float32, device=device) if r > 0 else None
+
+
+def fp4_forward(layer: Fp4Linear, X: torch.Tensor, act: Fp4ActBuffers, Y: torch.Tensor,
+                out: int = HSQ_OUT_BF16, stream=None) -> torch.Tensor:
+    """One NVFP4 forward: the activation step, then the block-scaled GEMM + epilogue."""
+    M = X.shape[0]
+    hsq_fp4_quantize_act(X, layer.s, layer.L1, M, layer.K, layer.r, act.x_codes, act.x_sf, act.x_gs, act.U,
+                         stream=stream)
+    hsq_fp4_linear_forward(act.x_codes, act.x_sf, act.x_gs, act.U, layer.w_codes, layer.w_sf, layer.w_gs,
+                           layer.L2, layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, stream=stream)
     return Y
