@@ -363,7 +363,7 @@ class Workload:
         self.replicas = [self.layers] + [build_layers() for _ in range(self.nrep - 1)]
         # decode sizes the single-launch forward takes: the activation step runs
         # inside the forward's kernel
-        self.fused = all(hsq.fused_supported(s.M, s.K, s.r, s.group) for s in specs)
+        self.fused = all(hsq.fused_supported(s.M, s.K, s.r, s.group, N=s.N) for s in specs)
         torch.cuda.synchronize()
         if hsq.hsq_get_device_status() != hsq.HSQ_OK:
             raise RuntimeError("device status not clean after packing")

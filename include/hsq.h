@@ -182,9 +182,13 @@ hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_sca
  * Activation step and forward in one launch, for decode-sized inputs: the
  * same results as hsq_quantize_act followed by hsq_linear_forward (the same
  * codes, scales and U, which are kept on chip and not written out), for
- *   M <= 4 tokens, rank r in {0, 1, 2, 4}, and K small enough that one block
- *   holds the rows' codes: T * (Kp + 4 * G + 272) bytes <= 200 KiB, T being M
- *   rounded up to 1, 2 or 4 (so any K <= 47872 for M <= 4).
+ *   M <= 4 tokens, rank r in {0, 1, 2, 4}, and K small enough that one block's
+ *   shared memory holds the rows' widened codes, the block's weight scales and a
+ *   ring of weight rows: T (Kp + 4 G + 272) + 4 G RB + S rs Kp/2 + 1024 bytes
+ *   <= 227 KiB, T = M rounded up to 1, 2 or 4, RB = ceil(N / SMs) rounded up
+ *   to 4 (the rows of one block), rs = min(RB, max(1, 32768 / Kp)) rows per
+ *   ring stage and S = 2 stages (1 when one stage holds all RB rows); e.g.
+ *   K <= 21888 for M = 4 and N = 12288 on 148 SMs.
  * Other shapes return HSQ_ERR_UNSUPPORTED before anything is launched (use the
  * two calls).  The pages do not name this fusion; it is the step before the
  * path (activations quantized online) moved into the path's first kernel.

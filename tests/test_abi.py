@@ -100,8 +100,16 @@ def test_fused_forward_argument_validation():
     assert call(L1=None) == hsq.HSQ_ERR_INVALID_ARG      # r > 0 needs L1 and L2
     assert call(r=0) == hsq.HSQ_ERR_INVALID_ARG          # r == 0 wants L1 == L2 == NULL
     assert call(X=MIS) == hsq.HSQ_ERR_ALIGNMENT
-    assert hsq.fused_supported(1, 4096, 4) and not hsq.fused_supported(5, 4096, 4)
-    assert hsq.fused_supported(4, 47872, 4) and not hsq.fused_supported(4, 47936, 4)
+    assert hsq.fused_supported(1, 4096, 4, N=12288) and not hsq.fused_supported(5, 4096, 4, N=12288)
+    # the Python restatement of the shared-memory limit agrees with the library at its edge
+    for N, M in ((4096, 4), (12288, 1), (12288, 4)):
+        lo, hi = 64, 1 << 17
+        while hi - lo > 64:  # the largest K (a multiple of 64) the restatement accepts
+            mid = (lo + hi) // 2 // 64 * 64
+            lo, hi = (mid, hi) if hsq.fused_supported(M, mid, 4, N=N, nsm=148) else (lo, mid)
+        # (only the rejected side is called: fake pointers must never reach a launch)
+        if hsq._sm_count() == 148:
+            assert call(M=M, N=N, K=lo + 64) == hsq.HSQ_ERR_UNSUPPORTED
 
 
 def test_lowrank_helper_argument_validation():

@@ -26,7 +26,7 @@ DEV = "cuda:0"
 LAYERS = [(w, i) for w, specs in WORKLOADS.items() for i in range(len(specs))]
 FUSED_LAYERS = [(w, i) for w, i in LAYERS
                 if hsq.fused_supported(WORKLOADS[w][i].M, WORKLOADS[w][i].K, WORKLOADS[w][i].r,
-                                            WORKLOADS[w][i].group)]
+                                       WORKLOADS[w][i].group, N=WORKLOADS[w][i].N)]
 
 
 def _sample_rows(M, n=40, seed=0):

@@ -168,11 +168,18 @@ int device_sm_count() {
 // ------------------------------------------------------------------ planning
 enum Kind { kLarge = 0, kDec16, kDec32, kDec64, kGemv, kMid };
 
-// M <= 8: the weight stream on the CUDA cores (hsq_gemv.cuh) when the block's
-// widened activation codes fit in shared memory; otherwise the decode tiles.
+// M <= 8: the weight stream on the CUDA cores (hsq_gemv.cuh) when its shared
+// memory (the block's widened activation codes and weight scales, and a ring of
+// at least two stages of weight rows) fits; otherwise the decode tiles.
 constexpr int kGemvMaxM = 8;
-constexpr size_t kGemvSmemMax = 200 * 1024;
+constexpr size_t kGemvSmemMax = 227 * 1024;
 int gemv_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+// Rows per block of the weight stream: N spread evenly over the SMs, rounded up
+// to a multiple of 4 (so that each group's run of block scales is 16-byte aligned).
+int gemv_rows_per_block(int N, int nsm) { return ((N + nsm - 1) / nsm + 3) / 4 * 4; }
+hsq::GemvLayout gemv_plan_layout(int M, int N, int Kp, int G, int nsm) {
+  return hsq::gemv_layout(gemv_mt(M), Kp, G, gemv_rows_per_block(N, nsm), kGemvSmemMax);
+}
 
 struct Plan {
   Kind kind;
@@ -243,12 +250,12 @@ Plan make_plan(int M, int N, int K, int group, int nsm) {
   p.group = group;
   const bool g128 = group == 128;
   const int G = groups_of(K, group);
-  if (M <= kGemvMaxM && hsq::gemv_smem_bytes(gemv_mt(M), G * group, G) <= kGemvSmemMax) {
-    // one block of 16 warps per SM at most, whole weight rows per warp; no workspace
+  if (M <= kGemvMaxM && gemv_plan_layout(M, N, G * group, G, nsm).stages > 0) {
+    // one block per SM at most, a contiguous run of weight rows per block; no workspace
     p.kind = kGemv;
     p.swap = true;
-    p.grid = static_cast<int>(std::min<long>(nsm, (N + 15) / 16));
-    p.tiles_r = (N + p.grid - 1) / p.grid;  // rows per block
+    p.tiles_r = gemv_rows_per_block(N, nsm);  // rows per block
+    p.grid = (N + p.tiles_r - 1) / p.tiles_r;
     p.tiles_c = 1;
     p.stream_len = 0;
     return p;
@@ -430,8 +437,10 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
+// `a` has the shape, rows_per_block and pointers set; the ring layout and the
+// wait limit are filled in here.
 template <int MT, int LPG, int RF = -1>
-hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
+hsq_status launch_gemv(const Plan& p, hsq::GemvArgs a, cudaStream_t st) {
   static std::mutex mu;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -445,9 +454,14 @@ hsq_status launch_gemv(const Plan& p, const hsq::GemvArgs& a, cudaStream_t st) {
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
   }
-  const size_t smem = hsq::gemv_smem_bytes(MT, a.Kp, a.G);
-  // starts early: it waits for the activation step before reading its codes
-  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG, RF>, dim3(p.grid), dim3(hsq::kGemvThreads), smem, st, a) !=
+  const hsq::GemvLayout L = hsq::gemv_layout(MT, a.Kp, a.G, a.rows_per_block, kGemvSmemMax);
+  if (L.stages < 1 || L.bytes > kGemvSmemMax) return HSQ_ERR_UNSUPPORTED;
+  a.rs = L.rs; a.stages = L.stages;
+  a.off_sws = L.off_sws; a.off_x = L.off_x; a.off_sxs = L.off_sxs; a.off_us = L.off_us; a.off_bars = L.off_bars;
+  a.limit_ns = wait_limit_ns();
+  // starts early: its weight copies do not depend on the preceding kernel, and
+  // it waits for the activation step before reading its codes
+  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG, RF>, dim3(p.grid), dim3(hsq::kGemvThreads), L.bytes, st, a) !=
       cudaSuccess)
     return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
@@ -882,12 +896,13 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
     return HSQ_ERR_ALIGNMENT;
   const int G = groups_of(K, group), Kp = G * group;
   const int mt = gemv_mt(M);
-  if (M > 4 || !(r == 0 || r == 1 || r == 2 || r == 4) || hsq::gemv_smem_bytes(mt, Kp, G) > kGemvSmemMax)
-    return HSQ_ERR_UNSUPPORTED;
   const int nsm = device_sm_count();
+  if (M > 4 || !(r == 0 || r == 1 || r == 2 || r == 4) || gemv_plan_layout(M, N, Kp, G, nsm).stages < 1)
+    return HSQ_ERR_UNSUPPORTED;
   Plan p{};
   p.kind = kGemv;
-  p.grid = std::min(nsm, (N + 15) / 16);
+  p.tiles_r = gemv_rows_per_block(N, nsm);
+  p.grid = (N + p.tiles_r - 1) / p.tiles_r;
   hsq::GemvArgs ga{};
   ga.w_codes = w_codes; ga.w_scales = w_scales; ga.ldw = scales_ld(N);
   ga.r = r;
@@ -896,7 +911,7 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
   ga.Y = Y;
   ga.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
   ga.M = M; ga.N = N; ga.Kp = Kp; ga.G = G;
-  ga.rows_per_block = (N + p.grid - 1) / p.grid;
+  ga.rows_per_block = p.tiles_r;
   ga.X = static_cast<const __nv_bfloat16*>(X_bf16);
   ga.s = s;
   ga.L1 = static_cast<const __nv_bfloat16*>(L1_bf16);

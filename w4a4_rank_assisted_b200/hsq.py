@@ -192,15 +192,41 @@ def hsq_linear_forward_fused(X, s, L1, w_codes, w_scales, L2, bias, M, N, K, r, 
            "hsq_linear_forward_fused")
 
 
-def fused_supported(M: int, K: int, r: int, group: int = GROUP) -> bool:
-    """Whether hsq_linear_forward_fused takes this shape: the limits stated in
-    include/hsq.h, restated in integer arithmetic (no library call, so that it
-    can be asked without a GPU)."""
+def _sm_count() -> int:
+    if torch.cuda.is_available():
+        return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return 148
+
+
+def _a16(v: int) -> int:
+    return (v + 15) // 16 * 16
+
+
+def stream_smem_fits(M: int, N: int, K: int, group: int = GROUP, nsm: Optional[int] = None) -> bool:
+    """Whether the weight stream's shared memory fits one block for this shape:
+    the restatement, in integer arithmetic, of the limit include/hsq.h gives for
+    hsq_linear_forward_fused (no library call, so it can be asked without a GPU).
+    T = M rounded up to 1, 2, 4 or 8; RB = rows per block = ceil(N / SMs) rounded
+    up to 4; a ring of at least two stages (one if one stage holds all RB rows)
+    of min(RB, max(1, 16384 // (Kp/2))) rows."""
+    nsm = nsm or _sm_count()
+    G = -(-K // group)
+    Kp = G * group
+    T = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8
+    RB = (-(-N // nsm) + 3) // 4 * 4
+    rowbytes = Kp // 2
+    rs = min(RB, 1 if rowbytes >= 16384 else 16384 // rowbytes)
+    fixed = _a16(G * RB * 4) + _a16(T * Kp) + _a16(G * T * 4) + _a16(T * 16) + _a16(16 * T * 16)
+    min_stages = 1 if -(-RB // rs) == 1 else 2
+    return fixed + 1024 + min_stages * rs * rowbytes <= 227 * 1024
+
+
+def fused_supported(M: int, K: int, r: int, group: int = GROUP, N: int = 8, nsm: Optional[int] = None) -> bool:
+    """Whether hsq_linear_forward_fused takes this shape (the limits stated in
+    include/hsq.h: M <= 4, r in {0, 1, 2, 4}, and the stream's shared memory)."""
     if M < 1 or M > 4 or r not in (0, 1, 2, 4) or group not in (64, 128):
         return False
-    G = -(-K // group)
-    mt = 1 if M <= 1 else 2 if M <= 2 else 4
-    return mt * (G * group + 4 * G + 272) <= 200 * 1024
+    return stream_smem_fits(M, N, K, group, nsm)
 
 
 def hsq_lowrank_workspace_bytes(N: int, K: int, r: int) -> int:
