@@ -38,6 +38,7 @@ from w4a4_rank_assisted_b200.synth import WORKLOADS, make_layer  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 METRIC = "W4A4 rank-4 linear TOPS & tokens/s at FLUX/SANA/Qwen3 shapes; % of roofline"
 INT8_OVER_BF16_NOMINAL = 2.0  # dense INT8 (4.5 POPS) over dense BF16 (2.25 PFLOP/s), nominal
+FP4_OVER_BF16_NOMINAL = 4.0   # dense FP4 (9 PFLOP/s) over dense BF16, nominal
 
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -250,6 +251,7 @@ def oracle_timing(specs, budget_s: float = 12.0, seed_rows: int = 4):
     """Time the CPU oracle (as it stands) on a bounded row sample of every layer
     with pre-packed weights; returns (ops/s, cores, sample description)."""
     from oracle import hsq_oracle as O
+    from oracle import nvfp4_oracle as F
     try:
         from threadpoolctl import threadpool_info
         cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
@@ -261,16 +263,23 @@ def oracle_timing(specs, budget_s: float = 12.0, seed_rows: int = 4):
         Wn, sn = lay.W.float().numpy(), lay.s.numpy()
         L1n = lay.L1.float().numpy() if spec.r else None
         L2n = lay.L2.float().numpy() if spec.r else None
-        wc, ws = O.pack_weights(Wn, sn, L1n, L2n, spec.group)
-        packed.append((spec, lay.X.float().numpy(), sn, L1n, L2n, wc, ws))
+        if spec.fmt == "nvfp4":
+            wq = F.nvfp4_pack_weights(Wn, sn, L1n, L2n)
+        else:
+            wq = O.pack_weights(Wn, sn, L1n, L2n, spec.group)
+        packed.append((spec, lay.X.float().numpy(), sn, L1n, L2n, wq))
 
     def run(rows):
         t0 = time.perf_counter()
         ops = 0
-        for spec, X, sn, L1n, L2n, wc, ws in packed:
+        for spec, X, sn, L1n, L2n, wq in packed:
             m = min(rows, spec.M)
-            xc, xs, U = O.quantize_act(X[:m], sn, L1n, spec.group)
-            O.linear_forward(xc, xs, U, wc, ws, L2n, None, spec.group)
+            if spec.fmt == "nvfp4":
+                xc, xs, xg, U = F.nvfp4_quantize_act(X[:m], sn, L1n)
+                F.nvfp4_linear_forward(xc, xs, xg, U, *wq, L2n, None, spec.K)
+            else:
+                xc, xs, U = O.quantize_act(X[:m], sn, L1n, spec.group)
+                O.linear_forward(xc, xs, U, *wq, L2n, None, spec.group)
             ops += layer_ops(spec) * m / spec.M
         return time.perf_counter() - t0, ops
 
@@ -340,9 +349,14 @@ class Workload:
         def build_layers():
             out = []
             for spec, lay in zip(specs, host_layers):
-                pl = hsq.PackedLinear(d(lay.W), d(lay.s), d(lay.L1) if spec.r else None,
-                                      d(lay.L2) if spec.r else None, None, group=spec.group)
-                act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
+                L1 = d(lay.L1) if spec.r else None
+                L2 = d(lay.L2) if spec.r else None
+                if spec.fmt == "nvfp4":
+                    pl = hsq.Fp4Linear(d(lay.W), d(lay.s), L1, L2, None)
+                    act = hsq.Fp4ActBuffers(spec.M, spec.K, spec.r, dev)
+                else:
+                    pl = hsq.PackedLinear(d(lay.W), d(lay.s), L1, L2, None, group=spec.group)
+                    act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
                 Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
                 out.append(dict(spec=spec, pl=pl, X=d(lay.X), act=act, Y=Y, ws=pl.workspace(spec.M)))
             return out
@@ -363,7 +377,8 @@ class Workload:
         self.replicas = [self.layers] + [build_layers() for _ in range(self.nrep - 1)]
         # decode sizes the single-launch forward takes: the activation step runs
         # inside the forward's kernel
-        self.fused = all(hsq.fused_supported(s.M, s.K, s.r, s.group, N=s.N) for s in specs)
+        self.fp4 = all(s.fmt == "nvfp4" for s in specs)
+        self.fused = not self.fp4 and all(hsq.fused_supported(s.M, s.K, s.r, s.group, N=s.N) for s in specs)
         torch.cuda.synchronize()
         if hsq.hsq_get_device_status() != hsq.HSQ_OK:
             raise RuntimeError("device status not clean after packing")
@@ -372,11 +387,21 @@ class Workload:
     # the public API's calls, one layer at a time
     def launch_act(self, L, st):
         s = L["spec"]
+        if s.fmt == "nvfp4":
+            a = L["act"]
+            self.hsq.hsq_fp4_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, a.x_codes, a.x_sf, a.x_gs,
+                                          a.U, stream=st)
+            return
         self.hsq.hsq_quantize_act(L["X"], L["pl"].s, L["pl"].L1, s.M, s.K, s.r, L["act"].x_codes,
                                   L["act"].x_scales, L["act"].U, group=s.group, stream=st)
 
     def launch_gemm(self, L, st):
         s = L["spec"]
+        if s.fmt == "nvfp4":
+            a, pl = L["act"], L["pl"]
+            self.hsq.hsq_fp4_linear_forward(a.x_codes, a.x_sf, a.x_gs, a.U, pl.w_codes, pl.w_sf, pl.w_gs, pl.L2, None,
+                                            s.M, s.N, s.K, s.r, L["Y"], stream=st)
+            return
         self.hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
                                     L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
                                     workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
@@ -437,13 +462,17 @@ class Workload:
         return t0.elapsed_time(t1)
 
     def launches_per_step(self):
-        """Kernels of this library launched by one step."""
+        """Kernels of this library launched by one step (an NVFP4 activation step
+        is two kernels and a tiny pad-zeroing kernel when M is not a multiple of 128)."""
         n = 0
         for L in self.layers:
+            s = L["spec"]
             if self.fused:
                 n += 1
+            elif s.fmt == "nvfp4":
+                n += 2 + (1 if s.M % 128 else 0) + 1
             else:
-                n += 1 + (3 if self.expands(L["spec"]) else 1)
+                n += 1 + (3 if self.expands(s) else 1)
         return n
 
     @staticmethod
@@ -451,7 +480,7 @@ class Workload:
         """hsq_linear_forward expands both code matrices to E4M3 tiles ahead of
         the GEMM (two more launches) for more than 256 tokens, or more than 64 at
         groups of 128."""
-        return s.M > 256 or (s.M > 64 and s.group == 128)
+        return s.fmt == "int4" and (s.M > 256 or (s.M > 64 and s.group == 128))
 
     def kernel_times(self):
         """Per layer: device microseconds of each kernel, each timed alone over
@@ -490,12 +519,15 @@ class Workload:
         stream at decode sizes) over the step's layers, against the measured
         peaks: tensor-bound when its INT8 time floor exceeds its HBM floor."""
         specs = [L["spec"] for L in self.layers]
-        # each kernel is timed alone in a short graph: the burst peaks apply
-        int8_peak = peaks["bf16"] * INT8_OVER_BF16_NOMINAL
+        # each kernel is timed alone in a short graph: the burst peaks apply; the
+        # INT4 codes run on the 8-bit tensor pipe, the NVFP4 variant on the FP4 one
+        ratio = FP4_OVER_BF16_NOMINAL if self.fp4 else INT8_OVER_BF16_NOMINAL
+        int8_peak = peaks["bf16"] * ratio
         gemm_ops = sum(2 * s.M * s.N * s.K + 2 * s.M * s.N * s.r for s in specs)
         gemm_bytes = sum((layer_fused_bytes if self.fused else layer_gemm_bytes)(s) for s in specs)
         gemm_time = sum(d["gemm_kernel_us"] for d in kt) * 1e-6
-        label = ("w4a4_gemv_kernel, activation step fused in (one hsq_linear_forward_fused)" if self.fused
+        label = ("fp4_gemm_kernel (kind::mxf4nvf4 block-scaled)" if self.fp4
+                 else "w4a4_gemv_kernel, activation step fused in (one hsq_linear_forward_fused)" if self.fused
                  else "w4a4_gemv_kernel" if all(s.M <= 8 for s in specs) else "w4a4_gemm_kernel")
         t_tensor = gemm_ops / (int8_peak * 1e12)
         t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
@@ -505,9 +537,9 @@ class Workload:
             achieved = gemm_ops / gemm_time / 1e12
             r = {"bound": "tensor", "kernel": label, "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
                  "frac": achieved / int8_peak, "traffic": traffic,
-                 "peak_source": (f"{peaks['source']}: bf16 burst {peaks['bf16']} TFLOP/s x nominal INT8/BF16 "
-                                 f"ratio {INT8_OVER_BF16_NOMINAL} (each kernel timed alone)"),
-                 "frac_of_spec_4500": achieved / 4500.0}
+                 "peak_source": (f"{peaks['source']}: bf16 burst {peaks['bf16']} TFLOP/s x nominal "
+                                 f"{'FP4' if self.fp4 else 'INT8'}/BF16 ratio {ratio} (each kernel timed alone)"),
+                 f"frac_of_spec_{int(2250 * ratio)}": achieved / (2250.0 * ratio)}
         else:
             achieved = gemm_bytes / gemm_time / 1e9
             r = {"bound": "hbm", "kernel": label, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -618,27 +650,31 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     peaks = _peaks()
     roofline = W.roofline(kt, peaks, wl_name)
 
-    # ---- decode-sized layers (Qwen3-8B, 1 and 16 tokens), timed the same way:
-    # their own step graphs cycling through replicas, per-kernel times, roofline
-    decode = None
-    if not args.no_decode:
-        decode = {}
-        for dname in ("qwen3_8b_m1", "qwen3_8b_m16"):
-            D = Workload(hsq, WORKLOADS[dname], dev)
-            D.prepare_steps(args.warmup)
-            dsteps = max(50, args.steps)
-            d_ms = _max_over_ranks(D.timed_steps_ms(dsteps), world) / dsteps
-            dkt = D.kernel_times()
-            dops = sum(layer_ops(L["spec"]) for L in D.layers)
-            decode[dname] = {"ms_per_step": d_ms, "tops": dops * world / (d_ms * 1e-3) / 1e12,
-                             "tokens_per_s": D.specs[0].M * world / (d_ms * 1e-3),
-                             "fused_activation_step": D.fused, "gpu_launches_per_step": D.launches_per_step(),
-                             "l2": D.l2_note(), "roofline": D.roofline(dkt, peaks, dname),
-                             "layers": D.layer_detail(dkt)}
-            del D
-            torch.cuda.empty_cache()
+    # ---- other workloads timed the same way (their own step graphs, cycling
+    # through replicas where the step is smaller than 2 x L2; per-kernel times;
+    # roofline): the decode-sized Qwen3-8B layers (1 and 16 tokens) and the FLUX.1
+    # block in the NVFP4 variant
+    def sub_measure(name):
+        D = Workload(hsq, WORKLOADS[name], dev)
+        D.prepare_steps(args.warmup)
+        dsteps = max(50, args.steps)
+        d_ms = _max_over_ranks(D.timed_steps_ms(dsteps), world) / dsteps
+        dkt = D.kernel_times()
+        dops = sum(layer_ops(L["spec"]) for L in D.layers)
+        out = {"ms_per_step": d_ms, "tops": dops * world / (d_ms * 1e-3) / 1e12,
+               "tokens_per_s": D.specs[0].M * world / (d_ms * 1e-3),
+               "fused_activation_step": D.fused, "gpu_launches_per_step": D.launches_per_step(),
+               "l2": D.l2_note(), "roofline": D.roofline(dkt, peaks, name), "layers": D.layer_detail(dkt)}
+        del D
+        torch.cuda.empty_cache()
         if hsq.hsq_get_device_status() != hsq.HSQ_OK:
-            raise RuntimeError("a kernel reported a timeout in the decode measurements")
+            raise RuntimeError(f"a kernel reported a timeout in the {name} measurements")
+        return out
+
+    decode = None if args.no_decode else {d: sub_measure(d) for d in ("qwen3_8b_m1", "qwen3_8b_m16")}
+    nvfp4 = None
+    if not args.no_decode and wl_name == "flux_block_r4":
+        nvfp4 = {"workload": "flux_block_r4_nvfp4", **sub_measure("flux_block_r4_nvfp4")}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -650,7 +686,8 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             "metric": METRIC, "value": tops, "unit": "TOPS",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int4 codes on i8/e4m3 tensor cores, f32 accumulate",
+            "dtype": ("e2m1 codes, e4m3 block scales on fp4 tensor cores, f32 accumulate" if W.fp4
+                      else "int4 codes on i8/e4m3 tensor cores, f32 accumulate"),
             "data": "synthetic (seeded; layer shapes of the pages' backbones, random weights)",
             "config": {"workload": wl_name, "layers": [s.name for s in specs], "tokens_per_step": tokens_step,
                        "r": specs[0].r, "group": specs[0].group, "parallelism": f"replicas x{world}",
@@ -663,6 +700,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             "roofline": roofline,
             "layers": W.layer_detail(kt),
             "decode": decode,
+            "nvfp4": nvfp4,
             "cpu_baseline": cpu,
             "clocks": clk,
         }

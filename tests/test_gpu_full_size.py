@@ -23,7 +23,8 @@ from _helpers import check_y, pad_scales, to_np
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
-LAYERS = [(w, i) for w, specs in WORKLOADS.items() for i in range(len(specs))]
+# the INT4 layers (the NVFP4 variant's full-size case is in test_gpu_nvfp4.py)
+LAYERS = [(w, i) for w, specs in WORKLOADS.items() for i in range(len(specs)) if specs[i].fmt == "int4"]
 FUSED_LAYERS = [(w, i) for w, i in LAYERS
                 if hsq.fused_supported(WORKLOADS[w][i].M, WORKLOADS[w][i].K, WORKLOADS[w][i].r,
                                        WORKLOADS[w][i].group, N=WORKLOADS[w][i].N)]

@@ -41,25 +41,34 @@ struct Fp4Args {
   uint64_t limit_ns;
 };
 
+// Tile 128 tokens x BN outputs; a stage is K = 256 (KCS = 4 chunks of K = 64).
+// BN = 256 halves the activation reads per output against BN = 128 (the kernel is
+// bound by reading its operands from L2), but its accumulator then fills half of
+// Tensor Memory, so there is one (NTM = 1) and the epilogue's reads of it are not
+// overlapped with the next tile's MMAs.
+template <int BN_, int NTM_, int STAGES_>
 struct Fp4Cfg {
-  static constexpr int BM = 128, BN = 128;
+  static constexpr int BM = 128, BN = BN_;
   static constexpr int KCS = 4;                        // 64-wide K chunks per stage (128 bytes per row)
-  static constexpr int STAGES = 5;
+  static constexpr int STAGES = STAGES_;
+  static constexpr int BATOMS = BN / 128;              // 128-row scale atoms of the B tile
   static constexpr int A_BYTES = BM * 128;             // 16 KB
-  static constexpr int B_BYTES = BN * 128;             // 16 KB
+  static constexpr int B_BYTES = BN * 128;
   static constexpr int SF_ATOM = 512;                  // 128 rows x 4 scales
   static constexpr int SFA_OFF = A_BYTES + B_BYTES;
-  static constexpr int SFB_OFF = SFA_OFF + KCS * SF_ATOM;
-  static constexpr int STAGE_BYTES = SFB_OFF + KCS * SF_ATOM;  // 36 KB, a multiple of 1024
+  static constexpr int SFB_OFF = SFA_OFF + KCS * SF_ATOM;  // [BATOMS][KCS] atoms
+  static constexpr int STAGE_BYTES = SFB_OFF + BATOMS * KCS * SF_ATOM;  // a multiple of 1024
   static constexpr int NUM_EPI_WARPS = 4;
   static constexpr int THREADS = 32 * (2 + NUM_EPI_WARPS);
-  static constexpr int NTM = 2;                        // TMEM accumulators
+  static constexpr int NTM = NTM_;                     // TMEM accumulators
+  static constexpr int SFC = 4 + 4 * BATOMS;           // TMEM scale columns per K = 64 chunk (A, then B)
   static constexpr int SF_COL0 = NTM * BN;             // scale columns follow the accumulators
-  static constexpr int SF_COLS = KCS * 8;              // per stage: 4 (A) + 4 (B) columns per chunk
+  static constexpr int SF_COLS = KCS * SFC;            // per stage
   static constexpr int TMEM_COLS = 512;
   static constexpr int YST_BYTES = NUM_EPI_WARPS * 4096;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NTM + 1;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + YST_BYTES + NUM_BARS * 8 + 64;
+  static_assert(BN == 128 || BN == 256, "B tile");
   static_assert(STAGE_BYTES % 1024 == 0, "128-byte-swizzled tiles start on 1024-byte boundaries");
   static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -134,13 +143,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const int nc = min(KCS, args.KC - kc0);
           uint8_t* st = stage_base + s * Cfg::STAGE_BYTES;
           // the boxes are counted whole, rows and K beyond the tensors included (zero-filled)
-          mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * nc * Cfg::SF_ATOM);
+          const int batoms = min(Cfg::BATOMS, (args.N - tn * BN + 127) / 128);  // atoms holding weight rows
+          mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + (1 + batoms) * nc * Cfg::SF_ATOM);
           tma_load_2d(st, &tm_a, &full[s], kc0 * 32, tm * BM);
           tma_load_2d(st + Cfg::A_BYTES, &tm_b, &full[s], kc0 * 32, tn * BN);
           bulk_load(st + Cfg::SFA_OFF, args.x_sf + (static_cast<size_t>(tm) * args.KC + kc0) * Cfg::SF_ATOM,
                     nc * Cfg::SF_ATOM, &full[s]);
-          bulk_load(st + Cfg::SFB_OFF, args.w_sf + (static_cast<size_t>(tn) * args.KC + kc0) * Cfg::SF_ATOM,
-                    nc * Cfg::SF_ATOM, &full[s]);
+          // (an atom past the last weight row is not loaded: its scales only reach
+          // accumulator columns past N, which are never stored)
+          for (int j = 0; j < batoms; ++j)
+              bulk_load(st + Cfg::SFB_OFF + j * KCS * Cfg::SF_ATOM,
+                        args.w_sf + (static_cast<size_t>(tn * Cfg::BATOMS + j) * args.KC + kc0) * Cfg::SF_ATOM,
+                        nc * Cfg::SF_ATOM, &full[s]);
           issued = it + 1;
         }
       }
@@ -161,16 +175,21 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           tc_fence_after();
           const int nc = min(KCS, args.KC - ks * KCS);
           const uint32_t st = smem_u32(stage_base + s * Cfg::STAGE_BYTES);
+          // chunk i's scales: A at columns SFC i .. +3, B's atoms j at SFC i + 4 + 4 j .. +3
+          // (B row n at column SFC i + 4 + n / 32)
           const uint32_t sfc = tmem_base + static_cast<uint32_t>(Cfg::SF_COL0 + (it & 1) * Cfg::SF_COLS);
           for (int i = 0; i < nc; ++i) {
-            tmem_cp_sf_atom(sfc + 8 * i, smem_desc_kmajor(st + Cfg::SFA_OFF + i * Cfg::SF_ATOM, 128, 128));
-            tmem_cp_sf_atom(sfc + 8 * i + 4, smem_desc_kmajor(st + Cfg::SFB_OFF + i * Cfg::SF_ATOM, 128, 128));
+            tmem_cp_sf_atom(sfc + Cfg::SFC * i, smem_desc_kmajor(st + Cfg::SFA_OFF + i * Cfg::SF_ATOM, 128, 128));
+#pragma unroll
+            for (int j = 0; j < Cfg::BATOMS; ++j)
+              tmem_cp_sf_atom(sfc + Cfg::SFC * i + 4 + 4 * j,
+                              smem_desc_kmajor(st + Cfg::SFB_OFF + (j * KCS + i) * Cfg::SF_ATOM, 128, 128));
           }
           for (int i = 0; i < nc; ++i) {
             // chunk i is 32 bytes into each 128-byte swizzled row
             mma_fp4_block16(d, smem_desc_kmajor_sw128(st + 32 * i, 1024),
-                            smem_desc_kmajor_sw128(st + Cfg::A_BYTES + 32 * i, 1024), idesc, sfc + 8 * i,
-                            sfc + 8 * i + 4, (ks > 0 || i > 0) ? 1u : 0u);
+                            smem_desc_kmajor_sw128(st + Cfg::A_BYTES + 32 * i, 1024), idesc, sfc + Cfg::SFC * i,
+                            sfc + Cfg::SFC * i + 4, (ks > 0 || i > 0) ? 1u : 0u);
           }
           mma_commit(&empty[s]);
         }
@@ -191,86 +210,92 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int tb = nt % NTM;
       if (!wait_warp(&tfull[tb], (nt / NTM) & 1, wp)) break;
       tc_fence_after();
-      // the whole row of the accumulator (thread = row), then the buffer is free
-      uint32_t v[BN / 16][16];
-#pragma unroll
-      for (int c = 0; c < BN / 16; ++c) tmem_ld16(t_q + static_cast<uint32_t>(tb * BN + 16 * c), v[c]);
-      // wait for the loads; every destination register passes through a wait, so
-      // that no read of them is scheduled before it (later waits return at once)
-#pragma unroll
-      for (int c = 0; c < BN / 16; c += 2) tmem_ld_wait(v[c], v[c + 1]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[tb]);
-
       const int m = tm * BM + q * 32 + lane;
-      const int n0 = tn * BN;
-      // Y = acc * gx gw + b, then + U[m][j] L2[j][:] rank by rank, in place in
-      // the accumulator registers (an 8-column block is all in or all out: N % 8 == 0)
-      auto vf = [&](int c) -> float& { return *reinterpret_cast<float*>(&v[c >> 4][c & 15]); };
-#pragma unroll
-      for (int c8 = 0; c8 < BN / 8; ++c8) {
-        const int n = n0 + 8 * c8;
-        float b[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = 0.f;
-        if (args.bias && n < args.N) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), b);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fadd_rn(__fmul_rn(vf(8 * c8 + e), gg), b[e]);
-      }
-#pragma unroll 1
-      for (int j = 0; j < args.r; ++j) {
-        const float uj = m < args.M ? __ldg(args.U + static_cast<size_t>(m) * args.r + j) : 0.f;
-        const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(j) * args.N + n0;
-#pragma unroll
-        for (int c8 = 0; c8 < BN / 8; ++c8) {
-          if (n0 + 8 * c8 < args.N) {
-            float l[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + 8 * c8)), l);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fmaf_rn(uj, l[e], vf(8 * c8 + e));
-          }
-        }
-      }
-      auto y = [&](int c) { return __uint_as_float(v[c >> 4][c & 15]); };
-      // store: 32 rows x 128 bytes per TMA box, 128-byte swizzled staging
       const int y0 = tm * BM + q * 32;
-      if (!args.out_f32) {
+      // 128 columns at a time (thread = row); after the last part's loads the
+      // accumulator is free for the next tile's MMAs
+#pragma unroll 1
+      for (int part = 0; part < BN / 128; ++part) {
+        const int n0 = tn * BN + part * 128;
+        uint32_t v[8][16];
 #pragma unroll
-        for (int pz = 0; pz < BN / 64; ++pz) {
-          if (lane == 0) bulk_wait_read_all();
+        for (int c = 0; c < 8; ++c) tmem_ld16(t_q + static_cast<uint32_t>(tb * BN + part * 128 + 16 * c), v[c]);
+        // wait for the loads; every destination register passes through a wait, so
+        // that no read of them is scheduled before it (later waits return at once)
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) tmem_ld_wait(v[c], v[c + 1]);
+        if (part == BN / 128 - 1) {
+          tc_fence_before();
           __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);
+        }
+        if (n0 >= args.N) continue;  // warp-uniform
+        // Y = acc * gx gw + b, then + U[m][j] L2[j][:] rank by rank, in place in
+        // the accumulator registers (an 8-column block is all in or all out: N % 8 == 0)
+        auto vf = [&](int c) -> float& { return *reinterpret_cast<float*>(&v[c >> 4][c & 15]); };
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 w;
-            __nv_bfloat162* wb = reinterpret_cast<__nv_bfloat162*>(&w);
+        for (int c8 = 0; c8 < 16; ++c8) {
+          const int n = n0 + 8 * c8;
+          float b[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              wb[e] = __floats2bfloat162_rn(y(64 * pz + 8 * c + 2 * e), y(64 * pz + 8 * c + 2 * e + 1));
-            *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) = w;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && n0 + 64 * pz < args.N && y0 < args.M) {
-            tma_store_2d(&tm_y, stg, n0 + 64 * pz, y0);
-            bulk_commit_group();
+          for (int e = 0; e < 8; ++e) b[e] = 0.f;
+          if (args.bias && n < args.N) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), b);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fadd_rn(__fmul_rn(vf(8 * c8 + e), gg), b[e]);
+        }
+#pragma unroll 1
+        for (int j = 0; j < args.r; ++j) {
+          const float uj = m < args.M ? __ldg(args.U + static_cast<size_t>(m) * args.r + j) : 0.f;
+          const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(j) * args.N + n0;
+#pragma unroll
+          for (int c8 = 0; c8 < 16; ++c8) {
+            if (n0 + 8 * c8 < args.N) {
+              float l[8];
+              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + 8 * c8)), l);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fmaf_rn(uj, l[e], vf(8 * c8 + e));
+            }
           }
         }
-      } else {
+        auto y = [&](int c) { return __uint_as_float(v[c >> 4][c & 15]); };
+        // store: 32 rows x 128 bytes per TMA box, 128-byte swizzled staging
+        if (!args.out_f32) {
 #pragma unroll
-        for (int pz = 0; pz < BN / 32; ++pz) {
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
+          for (int pz = 0; pz < 2; ++pz) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                make_float4(y(32 * pz + 4 * c), y(32 * pz + 4 * c + 1), y(32 * pz + 4 * c + 2),
-                            y(32 * pz + 4 * c + 3));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && n0 + 32 * pz < args.N && y0 < args.M) {
-            tma_store_2d(&tm_y, stg, n0 + 32 * pz, y0);
-            bulk_commit_group();
+            for (int c = 0; c < 8; ++c) {
+              uint4 w;
+              __nv_bfloat162* wb = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                wb[e] = __floats2bfloat162_rn(y(64 * pz + 8 * c + 2 * e), y(64 * pz + 8 * c + 2 * e + 1));
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) = w;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && n0 + 64 * pz < args.N && y0 < args.M) {
+              tma_store_2d(&tm_y, stg, n0 + 64 * pz, y0);
+              bulk_commit_group();
+            }
+          }
+        } else {
+#pragma unroll
+          for (int pz = 0; pz < 4; ++pz) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<float4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_float4(y(32 * pz + 4 * c), y(32 * pz + 4 * c + 1), y(32 * pz + 4 * c + 2),
+                              y(32 * pz + 4 * c + 3));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && n0 + 32 * pz < args.N && y0 < args.M) {
+              tma_store_2d(&tm_y, stg, n0 + 32 * pz, y0);
+              bulk_commit_group();
+            }
           }
         }
       }

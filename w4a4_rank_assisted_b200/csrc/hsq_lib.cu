@@ -934,6 +934,11 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
 }
 
 // ------------------------------------------------------------------ NVFP4 variant
+// Block-scaled GEMM tile: 128 tokens x HSQ_FP4_BN outputs (hsq_fp4.cuh).
+#ifndef HSQ_FP4_BN
+#define HSQ_FP4_BN 128
+#endif
+using CfgFp4 = hsq::Fp4Cfg<HSQ_FP4_BN, HSQ_FP4_BN == 256 ? 1 : 2, HSQ_FP4_BN == 256 ? 3 : 5>;
 static int fp4_kq(int K) { return (K + 63) / 64 * 64; }
 
 size_t hsq_fp4_codes_bytes(int rows, int K) {
@@ -1040,7 +1045,7 @@ hsq_status hsq_fp4_linear_forward(const uint8_t* x_codes, const uint8_t* x_sf, c
       !aligned16(w_gs) || !aligned16(Y) || (U && !aligned16(U)) || (L2_bf16 && !aligned16(L2_bf16)) ||
       (bias_bf16 && !aligned16(bias_bf16)))
     return HSQ_ERR_ALIGNMENT;
-  using Cfg = hsq::Fp4Cfg;
+  using Cfg = CfgFp4;
   const int Kq = fp4_kq(K);
   CUtensorMap tm_a, tm_b, tm_y;
   if (!make_fp4_codes_map(&tm_a, x_codes, M, Kq) || !make_fp4_codes_map(&tm_b, w_codes, N, Kq) ||

@@ -43,6 +43,7 @@ class LayerSpec:
     seed: int = 0
     bias: bool = False  # the stated workloads use a zero bias; tests switch it on
     group: int = 64     # quantization group along K (the pages use 128 for Qwen3-8B)
+    fmt: str = "int4"   # "int4" (the method's groups of 64/128) or "nvfp4" (the DiRotQ page's FP4 setting)
 
 
 @dataclasses.dataclass
@@ -106,11 +107,12 @@ def _sana(r):
             LayerSpec(f"sana_down_r{r}", 1024, 5600, 2240, r, seed=1, **common)]
 
 
-def _flux(r):
-    common = dict(act="outlier", outlier_frac=0.005, outlier_mult=50.0)
-    return [LayerSpec(f"flux_qkv_r{r}", 4608, 3072, 9216, r, seed=0, **common),
-            LayerSpec(f"flux_mlp_up_r{r}", 4608, 3072, 12288, r, seed=1, **common),
-            LayerSpec(f"flux_mlp_down_r{r}", 4608, 12288, 3072, r, seed=2, **common)]
+def _flux(r, fmt="int4"):
+    common = dict(act="outlier", outlier_frac=0.005, outlier_mult=50.0, fmt=fmt)
+    tag = "" if fmt == "int4" else f"_{fmt}"
+    return [LayerSpec(f"flux_qkv_r{r}{tag}", 4608, 3072, 9216, r, seed=0, **common),
+            LayerSpec(f"flux_mlp_up_r{r}{tag}", 4608, 3072, 12288, r, seed=1, **common),
+            LayerSpec(f"flux_mlp_down_r{r}{tag}", 4608, 12288, 3072, r, seed=2, **common)]
 
 
 def _qwen(M, group=64):
@@ -132,6 +134,8 @@ WORKLOADS: Dict[str, List[LayerSpec]] = {
     **{f"qwen3_8b_m{M}": _qwen(M) for M in (1, 16, 128, 1024, 8192)},
     # the pages' own Qwen3-8B setting: groups of 128 (Table 3 and Table 4 captions)
     **{f"qwen3_8b_m{M}_g128": _qwen(M, 128) for M in (1, 16, 128, 1024, 8192)},
+    # the same FLUX.1 block in the NVFP4 variant (E2M1 values, E4M3 scale per 16, fp32 tensor scale)
+    "flux_block_r4_nvfp4": _flux(4, "nvfp4"),
 }
 
 
