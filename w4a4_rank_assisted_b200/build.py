@@ -10,7 +10,10 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
-LIB_PATH = os.path.join(PKG_DIR, "libhsq.so")
+# HSQ_LIBRARY names another build of the same sources (e.g. one compiled with a
+# different tile option) to load instead of the in-tree library.
+LIB_PATH = os.path.abspath(os.environ["HSQ_LIBRARY"]) if os.environ.get("HSQ_LIBRARY") else os.path.join(
+    PKG_DIR, "libhsq.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

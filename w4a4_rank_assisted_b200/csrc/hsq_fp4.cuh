@@ -66,8 +66,12 @@ struct Fp4Cfg {
   static constexpr int SF_COLS = KCS * SFC;            // per stage
   static constexpr int TMEM_COLS = 512;
   static constexpr int YST_BYTES = NUM_EPI_WARPS * 4096;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NTM + 1;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + YST_BYTES + NUM_BARS * 8 + 64;
+  // the epilogue's bias and L2 columns of a tile, [1 + 32][BN] bf16 (row 0 the
+  // bias, rows 1.. the ranks), two buffers
+  static constexpr int LR_ROWS = 33;
+  static constexpr int LR_BYTES = LR_ROWS * BN * 2;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NTM + 1 + 4;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + YST_BYTES + 2 * LR_BYTES + NUM_BARS * 8 + 64;
   static_assert(BN == 128 || BN == 256, "B tile");
   static_assert(STAGE_BYTES % 1024 == 0, "128-byte-swizzled tiles start on 1024-byte boundaries");
   static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM");
@@ -83,12 +87,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   uint8_t* ystage = smem + STAGES * Cfg::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ystage + Cfg::YST_BYTES);
+  __nv_bfloat16* lrs = reinterpret_cast<__nv_bfloat16*>(ystage + Cfg::YST_BYTES);  // [2][LR_ROWS][BN]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ystage + Cfg::YST_BYTES + 2 * Cfg::LR_BYTES);
   uint64_t* full = bars;                 // [STAGES] stage landed
   uint64_t* empty = bars + STAGES;       // [STAGES] stage consumed by the MMAs
   uint64_t* tfull = empty + STAGES;      // [NTM] accumulator complete
   uint64_t* tempty = tfull + NTM;        // [NTM] accumulator drained
   uint64_t* final_bar = tempty + NTM;    // teardown: all MMAs done
+  uint64_t* lrfull = final_bar + 1;      // [2] a tile's bias and L2 columns landed
+  uint64_t* lrempty = lrfull + 2;        // [2] ... and read by every epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* tail_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -109,6 +116,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(&tempty[b], Cfg::NUM_EPI_WARPS);
     }
     mbar_init(final_bar, 1);
+    mbar_init(&lrfull[0], 1);
+    mbar_init(&lrfull[1], 1);
+    mbar_init(&lrempty[0], Cfg::NUM_EPI_WARPS);
+    mbar_init(&lrempty[1], Cfg::NUM_EPI_WARPS);
     *abort_flag = 0;
     *tail_flag = 0;
     fence_mbar_init();
@@ -128,6 +139,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   grid_dep_wait();  // codes, scales, U come from the preceding kernels
 
   uint32_t issued = 0;  // producer: stages issued (for the teardown)
+  uint32_t lr_issued[2] = {0u, 0u}, lr_done[2] = {0u, 0u};  // epilogue: bias/L2 copies issued / waited per buffer
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -204,11 +216,31 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const uint32_t t_q = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const float gg = __fmul_rn(__ldg(args.x_gs), __ldg(args.w_gs));
     uint8_t* stg = ystage + ew * 4096;
+    // A tile's bias and L2 columns are bulk-copied into shared memory two tiles
+    // ahead (buffer nt & 1), so the epilogue's math reads no global memory.
+    const bool lr_issuer = ew == 0 && lane == 0;
+    auto issue_lr = [&](int t, int b) {
+      const int n0 = (t / args.tiles_m) * BN;
+      const uint32_t cb = static_cast<uint32_t>(min(BN, args.N - n0)) * 2u;  // N % 8 == 0: a multiple of 16
+      mbar_arrive_expect_tx(&lrfull[b], cb * static_cast<uint32_t>(args.r + (args.bias ? 1 : 0)));
+      __nv_bfloat16* dst = lrs + b * Cfg::LR_ROWS * BN;
+      if (args.bias) bulk_load(dst, args.bias + n0, cb, &lrfull[b]);
+      for (int j = 0; j < args.r; ++j)
+        bulk_load(dst + (1 + j) * BN, args.L2 + static_cast<size_t>(j) * args.N + n0, cb, &lrfull[b]);
+      ++lr_issued[b];
+    };
+    if (lr_issuer) {
+      if (blockIdx.x < tiles) issue_lr(blockIdx.x, 0);
+      if (blockIdx.x + gridDim.x < tiles) issue_lr(blockIdx.x + gridDim.x, 1);
+    }
     uint32_t nt = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++nt) {
       const int tm = t % args.tiles_m, tn = t / args.tiles_m;
       const int tb = nt % NTM;
       if (!wait_warp(&tfull[tb], (nt / NTM) & 1, wp)) break;
+      if (!wait_warp(&lrfull[nt & 1], (nt >> 1) & 1, wp)) break;
+      ++lr_done[nt & 1];
+      const __nv_bfloat16* lrb = lrs + (nt & 1) * Cfg::LR_ROWS * BN;
       tc_fence_after();
       const int m = tm * BM + q * 32 + lane;
       const int y0 = tm * BM + q * 32;
@@ -232,29 +264,29 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (n0 >= args.N) continue;  // warp-uniform
         // Y = acc * gx gw + b, then + U[m][j] L2[j][:] rank by rank, in place in
         // the accumulator registers (an 8-column block is all in or all out: N % 8 == 0)
+        // (the columns of the shared bias / L2 rows past N hold stale values: they
+        // only reach outputs past N, which are never stored)
         auto vf = [&](int c) -> float& { return *reinterpret_cast<float*>(&v[c >> 4][c & 15]); };
+        const __nv_bfloat16* lrp = lrb + part * 128;
 #pragma unroll
         for (int c8 = 0; c8 < 16; ++c8) {
-          const int n = n0 + 8 * c8;
           float b[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) b[e] = 0.f;
-          if (args.bias && n < args.N) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(args.bias + n)), b);
+          if (args.bias) bf16x8_to_f32(*reinterpret_cast<const uint4*>(lrp + 8 * c8), b);
 #pragma unroll
           for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fadd_rn(__fmul_rn(vf(8 * c8 + e), gg), b[e]);
         }
 #pragma unroll 1
         for (int j = 0; j < args.r; ++j) {
           const float uj = m < args.M ? __ldg(args.U + static_cast<size_t>(m) * args.r + j) : 0.f;
-          const __nv_bfloat16* l2 = args.L2 + static_cast<size_t>(j) * args.N + n0;
+          const __nv_bfloat16* l2 = lrp + (1 + j) * BN;
 #pragma unroll
           for (int c8 = 0; c8 < 16; ++c8) {
-            if (n0 + 8 * c8 < args.N) {
-              float l[8];
-              bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(l2 + 8 * c8)), l);
+            float l[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(l2 + 8 * c8), l);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fmaf_rn(uj, l[e], vf(8 * c8 + e));
-            }
+            for (int e = 0; e < 8; ++e) vf(8 * c8 + e) = __fmaf_rn(uj, l[e], vf(8 * c8 + e));
           }
         }
         auto y = [&](int c) { return __uint_as_float(v[c >> 4][c & 15]); };
@@ -299,6 +331,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         }
       }
+      // this warp is done with the tile's bias / L2 buffer; once all four are,
+      // it is refilled for the tile two ahead
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lrempty[nt & 1]);
+      if (lr_issuer && t + 2 * static_cast<int>(gridDim.x) < tiles) {
+        if (!wait_one(&lrempty[nt & 1], (nt >> 1) & 1, wp)) break;
+        issue_lr(t + 2 * gridDim.x, nt & 1);
+      }
     }
     if (lane == 0) bulk_wait_all();
   }
@@ -315,6 +355,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     if (warp == 1 && lane == 0) {
       mma_commit(final_bar);  // arrives once every MMA issued above has completed
       wait_one(final_bar, 0, tail);
+    }
+    if (warp == 2 && lane == 0) {
+      // and the bias / L2 copies not yet waited for
+      for (int b = 0; b < 2; ++b)
+        if (lr_issued[b] > lr_done[b]) wait_one(&lrfull[b], (lr_issued[b] - 1) & 1, tail);
     }
     __syncthreads();
   }

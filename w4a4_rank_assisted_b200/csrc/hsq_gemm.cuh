@@ -55,6 +55,12 @@
 
 #include "hsq_device.cuh"
 
+// Drain: hand a TMEM partial buffer back to the MMA warp right after its last
+// load (1) or after the stage's math (0).
+#ifndef HSQ_EARLY_RELEASE
+#define HSQ_EARLY_RELEASE 0
+#endif
+
 // Registers per thread left to the producer / MMA / helper warpgroups of
 // blocks of up to 512 threads (the rest go to the drain warpgroups).
 #ifndef HSQ_REGS_LOW_SMALL
@@ -893,9 +899,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         };
         auto wait_chunk = [&](uint32_t (&dst)[2][4 * CHB]) { tmem_ld_wait(dst[0], dst[1]); };
+        // With HSQ_EARLY_RELEASE the TMEM buffer is handed back to the MMA warp as
+        // soon as the stage's last load has landed, before that chunk's math.
+        auto release_tmem = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) mbar_arrive(&tempty[tb]);
+            else mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[tb]), 0u));  // the MMA issuer's barrier
+          }
+        };
         if constexpr (Cfg::PIPE) {
           issue(0, vbuf[0]);
           wait_chunk(vbuf[0]);
+          if (HSQ_EARLY_RELEASE && nbt == 1) release_tmem();
         }
         float2 rs2[4];
 #pragma unroll
@@ -908,6 +925,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           } else {
             issue(bi, cur);
             wait_chunk(cur);
+            if (HSQ_EARLY_RELEASE && bi + 1 == nbt) release_tmem();
           }
           if (cc == 0) {
             // the four rows' scales of group g+j, times the factor that undoes the
@@ -933,16 +951,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
           }
           if constexpr (Cfg::PIPE) {
-            if (bi + 1 < nbt) wait_chunk(vbuf[(bi + 1) & 1]);
+            if (bi + 1 < nbt) {
+              wait_chunk(vbuf[(bi + 1) & 1]);
+              if (HSQ_EARLY_RELEASE && bi + 2 == nbt) release_tmem();
+            }
           }
         }
-        tc_fence_before();
+        if (!HSQ_EARLY_RELEASE) release_tmem();
         __syncwarp();
-        if (lane == 0) {
-          if (leader) mbar_arrive(&tempty[tb]);
-          else mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[tb]), 0u));  // the MMA issuer's barrier
-          mbar_arrive(&sempty[ss]);
-        }
+        if (lane == 0) mbar_arrive(&sempty[ss]);
       }
       if (!ok) break;
 

@@ -344,14 +344,14 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kp, in
 }
 
 // 2-D map over NVFP4 codes [rows][Kq/2] bytes for the block-scaled kernel: box =
-// 128 bytes (a stage's K = 256) x 128 rows, 128-byte swizzle (the layout its
-// MMA descriptors read).
-bool make_fp4_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kq) {
+// 128 bytes (a stage's K = 256) x box_rows rows (the tile's), 128-byte swizzle
+// (the layout its MMA descriptors read).
+bool make_fp4_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kq, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Kq / 2), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Kq / 2)};
-  const cuuint32_t box[2] = {128u, 128u};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1048,7 +1048,7 @@ hsq_status hsq_fp4_linear_forward(const uint8_t* x_codes, const uint8_t* x_sf, c
   using Cfg = CfgFp4;
   const int Kq = fp4_kq(K);
   CUtensorMap tm_a, tm_b, tm_y;
-  if (!make_fp4_codes_map(&tm_a, x_codes, M, Kq) || !make_fp4_codes_map(&tm_b, w_codes, N, Kq) ||
+  if (!make_fp4_codes_map(&tm_a, x_codes, M, Kq, Cfg::BM) || !make_fp4_codes_map(&tm_b, w_codes, N, Kq, Cfg::BN) ||
       !make_y_map(&tm_y, Y, M, N, out == HSQ_OUT_F32))
     return HSQ_ERR_CUDA;
   hsq::Fp4Args a{};

@@ -197,11 +197,10 @@ __global__ void __launch_bounds__(256) nvfp4_act_amax_kernel(const __nv_bfloat16
   grid_dep_wait();  // X may come from the preceding kernel
   const int lane = lane_id();
   const size_t groups = static_cast<size_t>(M) * (K / 8);
-  // block b takes a contiguous run of 8-element groups, requested into L2 at once
+  // block b takes a contiguous run of 8-element groups
   const size_t per_block = (groups + gridDim.x - 1) / gridDim.x;
   const size_t g0 = static_cast<size_t>(blockIdx.x) * per_block;
   const size_t g1 = min(groups, g0 + per_block);
-  if (threadIdx.x == 0 && g1 > g0) prefetch_l2_bulk(X + g0 * 8, static_cast<uint32_t>((g1 - g0) * 16));
   float amax = 0.f;
   for (size_t base = g0 + (threadIdx.x >> 5) * 32; base < g1; base += (blockDim.x / 32) * 32) {
     const size_t i = base + lane;
@@ -368,12 +367,6 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
   using C = ActCfg<R, SMALL>;
   constexpr int SUB = C::SUB, NW = C::NW, RB = C::RB, NSUB = C::NSUB;
   grid_dep_wait();  // X (and for FP4 the absmax) may come from the preceding kernel
-  if (threadIdx.x == 0) {
-    // the block's rows are contiguous: request all of them into L2 at once, so
-    // that the whole of X streams from HBM while the warps work through it
-    const int r0 = blockIdx.x * RB, nr = min(RB, M - r0);
-    if (nr > 0) prefetch_l2_bulk(X + static_cast<size_t>(r0) * K, static_cast<uint32_t>(nr) * K * 2u);
-  }
   float g = 0.f, sixg = 0.f;
   if constexpr (FP4) {
     g = nvfp4_tensor_scale(gs[1]);

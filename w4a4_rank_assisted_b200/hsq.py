@@ -373,6 +373,10 @@ class Fp4Linear:
         hsq_fp4_pack_weights(W.contiguous(), self.s, self.L1, self.L2, N, K, r, self.w_codes, self.w_sf,
                              self.w_gs, stream=stream)
 
+    def workspace(self, M: int) -> None:
+        """The NVFP4 forward needs no workspace."""
+        return None
+
 
 class Fp4ActBuffers:
     """Per-forward buffers of the NVFP4 activation step for M tokens."""
