@@ -224,7 +224,7 @@ struct GemmCfg {
   // 8-column blocks per TMEM load of the drain (2 or 4): one load and one wait
   // cover 16 * CHB columns of both half quadrants
   static constexpr int CHB = CHB_;
-  static_assert(CHB == 2 || CHB == 4, "drain chunk");
+  static_assert(CHB == 2 || CHB == 4 || CHB == 8, "drain chunk");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(CW % (8 * CHB_) == 0, "drain chunks");
   static_assert(TMEM_NEED <= 512, "TMEM");
@@ -893,12 +893,22 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if constexpr (CHB == 2) {
             tmem_ld_q8(t_q + col, dst[0]);
             tmem_ld_q8(t_q + (16u << 16) + col, dst[1]);
-          } else {
+          } else if constexpr (CHB == 4) {
             tmem_ld_q16(t_q + col, dst[0]);
             tmem_ld_q16(t_q + (16u << 16) + col, dst[1]);
+          } else {
+            tmem_ld_q32(t_q + col, dst[0]);
+            tmem_ld_q32(t_q + (16u << 16) + col, dst[1]);
           }
         };
-        auto wait_chunk = [&](uint32_t (&dst)[2][4 * CHB]) { tmem_ld_wait(dst[0], dst[1]); };
+        auto wait_chunk = [&](uint32_t (&dst)[2][4 * CHB]) {
+          if constexpr (CHB == 8) {
+            tmem_ld_wait(dst[0]);  // (one wait covers both loads; the second passes its registers through)
+            tmem_ld_wait(dst[1]);
+          } else {
+            tmem_ld_wait(dst[0], dst[1]);
+          }
+        };
         // With HSQ_EARLY_RELEASE the TMEM buffer is handed back to the MMA warp as
         // soon as the stage's last load has landed, before that chunk's math.
         auto release_tmem = [&]() {

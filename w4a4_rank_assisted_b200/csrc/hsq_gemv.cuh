@@ -83,6 +83,8 @@ inline GemvLayout gemv_layout(int MT, int Kp, int G, int rows_per_block, size_t 
   const size_t fixed = gemv_align16(static_cast<size_t>(G) * rows_per_block * 4) +
                        gemv_align16(static_cast<size_t>(MT) * Kp) + gemv_align16(static_cast<size_t>(G) * MT * 4) +
                        gemv_align16(MT * 4 * 4) + gemv_align16((kGemvThreads / 32) * MT * 4 * 4);
+  // the block's scales are one TMA box: at most 256 along each dimension
+  if (rows_per_block > 256 || G > 256) return L;
   L.rs = rowbytes >= kGemvStageBytes ? 1 : kGemvStageBytes / rowbytes;
   if (L.rs > rows_per_block) L.rs = rows_per_block;
   const size_t stage = static_cast<size_t>(L.rs) * rowbytes;
@@ -114,7 +116,8 @@ __device__ __forceinline__ void gemv_compute_sync() { named_bar_sync(1, kGemvCom
 // lane holds 32 codes, so 2 for groups of 64 and 4 for groups of 128); RF: -1
 // reads the activation step's outputs, 0/1/2/4 is the fused form of that rank.
 template <int MT, int LPG, int RF = -1>
-__global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    w4a4_gemv_kernel(const __grid_constant__ CUtensorMap tm_sw, const GemvArgs a) {
   extern __shared__ __align__(16) uint8_t gemv_smem[];
   const int W4 = a.Kp / 8;  // packed 32-bit words per row
   const int rowbytes = a.Kp / 2;
@@ -153,14 +156,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) w4a4_gemv_kernel(const GemvAr
     // ------------------------------------------------------------ weight stream
     // The packed weights and their scales are never written by the kernel just
     // before this one, so they are requested before waiting for it: the block's
-    // scales (one contiguous run per group: RB is a multiple of 4 and so is ld),
+    // scales as one 2-D box of [G][RB] floats (rows past the matrix read as 0),
     // then its rows, a stage of rs contiguous rows per bulk copy, as far ahead as
     // the ring allows.
     if (lane == 0) {
-      const uint32_t sbytes = static_cast<uint32_t>(min(RB, a.ldw - n0)) * 4u;
-      mbar_arrive_expect_tx(sfull, sbytes * static_cast<uint32_t>(a.G));
-      for (int g = 0; g < a.G; ++g)
-        bulk_load(sws + static_cast<size_t>(g) * RB, a.w_scales + static_cast<size_t>(g) * a.ldw + n0, sbytes, sfull);
+      prefetch_tensormap(&tm_sw);
+      mbar_arrive_expect_tx(sfull, static_cast<uint32_t>(RB) * a.G * 4u);
+      tma_load_2d(sws, &tm_sw, sfull, n0, 0);
       for (int it = 0; it < nst; ++it) {
         const int s = it % a.stages;
         if (it >= a.stages && !wait_one(&empty[s], ((it / a.stages) & 1) ^ 1, wp)) break;

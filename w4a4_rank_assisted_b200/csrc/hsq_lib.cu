@@ -58,11 +58,17 @@ constexpr int kMaxRank = 32;
 #ifndef HSQ_LARGE_PIPE
 #define HSQ_LARGE_PIPE -1
 #endif
-using CfgLarge64 = hsq::GemmCfg<256, HSQ_LARGE_DH, HSQ_PAIR ? 8 : HSQ_LARGE_STAGES, false, 1, 3, 2, 2,
-                                HSQ_PAIR ? 12 : HSQ_LARGE_STAGES + 4, true, HSQ_LARGE_PIPE, true, HSQ_LARGE_CHB,
-                                1, HSQ_PAIR != 0>;
-using CfgLarge128 = hsq::GemmCfg<256, HSQ_LARGE_DH, HSQ_PAIR ? 4 : HSQ_LARGE128_STAGES, false, 1, 3, 2, 2,
-                                 HSQ_PAIR ? 8 : HSQ_LARGE128_STAGES + 4, true,
+#ifndef HSQ_LARGE_BN
+#define HSQ_LARGE_BN 256
+#endif
+#ifndef HSQ_LARGE_NTM
+#define HSQ_LARGE_NTM 2
+#endif
+using CfgLarge64 = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_PAIR ? 8 : HSQ_LARGE_STAGES, false, 1, 3,
+                                HSQ_LARGE_NTM, 2, HSQ_PAIR ? 12 : HSQ_LARGE_STAGES + 4, true, HSQ_LARGE_PIPE, true,
+                                HSQ_LARGE_CHB, 1, HSQ_PAIR != 0>;
+using CfgLarge128 = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_PAIR ? 4 : HSQ_LARGE128_STAGES, false, 1, 3,
+                                 HSQ_LARGE_NTM, 2, HSQ_PAIR ? 8 : HSQ_LARGE128_STAGES + 4, true,
                                  HSQ_LARGE_PIPE, true, HSQ_LARGE_CHB, 2, HSQ_PAIR != 0>;
 // 64 < M <= 256, groups of 64 ("mid"): tokens x outputs tiles of 128 x 256 that
 // unpack both packed operands in shared memory (6 warps) instead of expanding
@@ -358,6 +364,20 @@ bool make_fp4_codes_map(CUtensorMap* map, const uint8_t* codes, int rows, int Kq
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over a group-major scale matrix [G][ld] fp32 for the weight stream: box
+// = box_rows rows x G groups (one block's scales in one copy).
+bool make_scales_map(CUtensorMap* map, const float* scales, int ld, int G, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(G)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(G)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(scales), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Pre-expanded E4M3 tiles (large tiles with CTA pairs) viewed as rows of 256
 // bytes; one box of 32 rows is one 8 KB block of 128 rows x 64 codes.
 bool make_e8_map(CUtensorMap* map, const uint8_t* base, size_t bytes) {
@@ -459,10 +479,12 @@ hsq_status launch_gemv(const Plan& p, hsq::GemvArgs a, cudaStream_t st) {
   a.rs = L.rs; a.stages = L.stages;
   a.off_sws = L.off_sws; a.off_x = L.off_x; a.off_sxs = L.off_sxs; a.off_us = L.off_us; a.off_bars = L.off_bars;
   a.limit_ns = wait_limit_ns();
+  CUtensorMap tm_sw;
+  if (!make_scales_map(&tm_sw, a.w_scales, a.ldw, a.G, a.rows_per_block)) return HSQ_ERR_CUDA;
   // starts early: its weight copies do not depend on the preceding kernel, and
   // it waits for the activation step before reading its codes
-  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG, RF>, dim3(p.grid), dim3(hsq::kGemvThreads), L.bytes, st, a) !=
-      cudaSuccess)
+  if (launch_pdl(true, hsq::w4a4_gemv_kernel<MT, LPG, RF>, dim3(p.grid), dim3(hsq::kGemvThreads), L.bytes, st,
+                 tm_sw, a) != cudaSuccess)
     return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
@@ -936,7 +958,7 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
 // ------------------------------------------------------------------ NVFP4 variant
 // Block-scaled GEMM tile: 128 tokens x HSQ_FP4_BN outputs (hsq_fp4.cuh).
 #ifndef HSQ_FP4_BN
-#define HSQ_FP4_BN 128
+#define HSQ_FP4_BN 256
 #endif
 using CfgFp4 = hsq::Fp4Cfg<HSQ_FP4_BN, HSQ_FP4_BN == 256 ? 1 : 2, HSQ_FP4_BN == 256 ? 3 : 5>;
 static int fp4_kq(int K) { return (K + 63) / 64 * 64; }

@@ -214,6 +214,8 @@ def stream_smem_fits(M: int, N: int, K: int, group: int = GROUP, nsm: Optional[i
     Kp = G * group
     T = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8
     RB = (-(-N // nsm) + 3) // 4 * 4
+    if RB > 256 or G > 256:  # the block's scales are one copy of at most 256 x 256
+        return False
     rowbytes = Kp // 2
     rs = min(RB, 1 if rowbytes >= 16384 else 16384 // rowbytes)
     fixed = _a16(G * RB * 4) + _a16(T * Kp) + _a16(G * T * 4) + _a16(T * 16) + _a16(16 * T * 16)
