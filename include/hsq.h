@@ -186,8 +186,9 @@ hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_sca
  *   shared memory holds the rows' widened codes, the block's weight scales and a
  *   ring of weight rows: T (Kp + 4 G + 272) + 4 G RB + S rs Kp/2 + 1024 bytes
  *   <= 227 KiB, T = M rounded up to 1, 2 or 4, RB = ceil(N / SMs) rounded up
- *   to 4 (the rows of one block), rs = min(RB, max(1, 32768 / Kp)) rows per
- *   ring stage and S = 2 stages (1 when one stage holds all RB rows), with
+ *   to 4 (the rows of one block), rs rows per ring stage (about half the
+ *   block's rows, at least 16 KiB of them, at most half of what the ring can
+ *   hold) and S = 2 stages (1 when one stage holds all RB rows), with
  *   RB <= 256 and G <= 256; e.g. K <= 16384 for groups of 64 and K <= 29696
  *   for groups of 128 at M = 4, N = 12288 on 148 SMs.
  * Other shapes return HSQ_ERR_UNSUPPORTED before anything is launched (use the

@@ -58,7 +58,9 @@ struct Fp4Cfg {
   static constexpr int SFA_OFF = A_BYTES + B_BYTES;
   static constexpr int SFB_OFF = SFA_OFF + KCS * SF_ATOM;  // [BATOMS][KCS] atoms
   static constexpr int STAGE_BYTES = SFB_OFF + BATOMS * KCS * SF_ATOM;  // a multiple of 1024
-  static constexpr int NUM_EPI_WARPS = 4;
+  // epilogue: four warps (one per TMEM lane quadrant) for each 128 columns of the tile
+  static constexpr int EPI_PARTS = BN / 128;
+  static constexpr int NUM_EPI_WARPS = 4 * EPI_PARTS;
   static constexpr int THREADS = 32 * (2 + NUM_EPI_WARPS);
   static constexpr int NTM = NTM_;                     // TMEM accumulators
   static constexpr int SFC = 4 + 4 * BATOMS;           // TMEM scale columns per K = 64 chunk (A, then B)
@@ -70,8 +72,10 @@ struct Fp4Cfg {
   // bias, rows 1.. the ranks), two buffers
   static constexpr int LR_ROWS = 33;
   static constexpr int LR_BYTES = LR_ROWS * BN * 2;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NTM + 1 + 4;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + YST_BYTES + 2 * LR_BYTES + NUM_BARS * 8 + 64;
+  static constexpr int LR_BUFS = NTM;  // a tile's copy is issued LR_BUFS tiles ahead
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NTM + 1 + 2 * LR_BUFS;
+  static constexpr int SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + YST_BYTES + LR_BUFS * LR_BYTES + NUM_BARS * 8 + 64;
   static_assert(BN == 128 || BN == 256, "B tile");
   static_assert(STAGE_BYTES % 1024 == 0, "128-byte-swizzled tiles start on 1024-byte boundaries");
   static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM");
@@ -88,14 +92,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint8_t* stage_base = smem;
   uint8_t* ystage = smem + STAGES * Cfg::STAGE_BYTES;
   __nv_bfloat16* lrs = reinterpret_cast<__nv_bfloat16*>(ystage + Cfg::YST_BYTES);  // [2][LR_ROWS][BN]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ystage + Cfg::YST_BYTES + 2 * Cfg::LR_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ystage + Cfg::YST_BYTES + Cfg::LR_BUFS * Cfg::LR_BYTES);
   uint64_t* full = bars;                 // [STAGES] stage landed
   uint64_t* empty = bars + STAGES;       // [STAGES] stage consumed by the MMAs
   uint64_t* tfull = empty + STAGES;      // [NTM] accumulator complete
   uint64_t* tempty = tfull + NTM;        // [NTM] accumulator drained
   uint64_t* final_bar = tempty + NTM;    // teardown: all MMAs done
-  uint64_t* lrfull = final_bar + 1;      // [2] a tile's bias and L2 columns landed
-  uint64_t* lrempty = lrfull + 2;        // [2] ... and read by every epilogue warp
+  uint64_t* lrfull = final_bar + 1;      // [LR_BUFS] a tile's bias and L2 columns landed
+  uint64_t* lrempty = lrfull + Cfg::LR_BUFS;  // [LR_BUFS] ... and read by every epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* tail_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -116,10 +120,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(&tempty[b], Cfg::NUM_EPI_WARPS);
     }
     mbar_init(final_bar, 1);
-    mbar_init(&lrfull[0], 1);
-    mbar_init(&lrfull[1], 1);
-    mbar_init(&lrempty[0], Cfg::NUM_EPI_WARPS);
-    mbar_init(&lrempty[1], Cfg::NUM_EPI_WARPS);
+    for (int b = 0; b < Cfg::LR_BUFS; ++b) {
+      mbar_init(&lrfull[b], 1);
+      mbar_init(&lrempty[b], Cfg::NUM_EPI_WARPS);
+    }
     *abort_flag = 0;
     *tail_flag = 0;
     fence_mbar_init();
@@ -213,11 +217,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant of this warp
     const int ew = warp - 2;
+    const int part = ew >> 2;  // the tile's 128-column part this warp drains
     const uint32_t t_q = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const float gg = __fmul_rn(__ldg(args.x_gs), __ldg(args.w_gs));
     uint8_t* stg = ystage + ew * 4096;
-    // A tile's bias and L2 columns are bulk-copied into shared memory two tiles
-    // ahead (buffer nt & 1), so the epilogue's math reads no global memory.
+    // A tile's bias and L2 columns are bulk-copied into shared memory LR_BUFS
+    // tiles ahead (buffer nt % LR_BUFS), so the epilogue's math reads no global memory.
     const bool lr_issuer = ew == 0 && lane == 0;
     auto issue_lr = [&](int t, int b) {
       const int n0 = (t / args.tiles_m) * BN;
@@ -229,25 +234,24 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         bulk_load(dst + (1 + j) * BN, args.L2 + static_cast<size_t>(j) * args.N + n0, cb, &lrfull[b]);
       ++lr_issued[b];
     };
-    if (lr_issuer) {
-      if (blockIdx.x < tiles) issue_lr(blockIdx.x, 0);
-      if (blockIdx.x + gridDim.x < tiles) issue_lr(blockIdx.x + gridDim.x, 1);
-    }
+    if (lr_issuer)
+      for (int b = 0; b < Cfg::LR_BUFS; ++b)
+        if (blockIdx.x + b * static_cast<int>(gridDim.x) < tiles) issue_lr(blockIdx.x + b * gridDim.x, b);
     uint32_t nt = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++nt) {
       const int tm = t % args.tiles_m, tn = t / args.tiles_m;
       const int tb = nt % NTM;
       if (!wait_warp(&tfull[tb], (nt / NTM) & 1, wp)) break;
-      if (!wait_warp(&lrfull[nt & 1], (nt >> 1) & 1, wp)) break;
-      ++lr_done[nt & 1];
-      const __nv_bfloat16* lrb = lrs + (nt & 1) * Cfg::LR_ROWS * BN;
+      const int lb = nt % Cfg::LR_BUFS;
+      if (!wait_warp(&lrfull[lb], (nt / Cfg::LR_BUFS) & 1, wp)) break;
+      ++lr_done[lb];
+      const __nv_bfloat16* lrb = lrs + lb * Cfg::LR_ROWS * BN;
       tc_fence_after();
       const int m = tm * BM + q * 32 + lane;
       const int y0 = tm * BM + q * 32;
-      // 128 columns at a time (thread = row); after the last part's loads the
-      // accumulator is free for the next tile's MMAs
-#pragma unroll 1
-      for (int part = 0; part < BN / 128; ++part) {
+      // this warp's 128 columns (thread = row); once every epilogue warp has its
+      // part in registers the accumulator is free for the next tile's MMAs
+      {
         const int n0 = tn * BN + part * 128;
         uint32_t v[8][16];
 #pragma unroll
@@ -256,12 +260,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         // that no read of them is scheduled before it (later waits return at once)
 #pragma unroll
         for (int c = 0; c < 8; c += 2) tmem_ld_wait(v[c], v[c + 1]);
-        if (part == BN / 128 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[tb]);
-        }
-        if (n0 >= args.N) continue;  // warp-uniform
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+        if (n0 < args.N) {  // warp-uniform
         // Y = acc * gx gw + b, then + U[m][j] L2[j][:] rank by rank, in place in
         // the accumulator registers (an 8-column block is all in or all out: N % 8 == 0)
         // (the columns of the shared bias / L2 rows past N hold stale values: they
@@ -330,14 +332,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
           }
         }
+        }  // n0 < N
       }
-      // this warp is done with the tile's bias / L2 buffer; once all four are,
-      // it is refilled for the tile two ahead
+      // this warp is done with the tile's bias / L2 buffer; once all are, it is
+      // refilled for the tile LR_BUFS ahead
       __syncwarp();
-      if (lane == 0) mbar_arrive(&lrempty[nt & 1]);
-      if (lr_issuer && t + 2 * static_cast<int>(gridDim.x) < tiles) {
-        if (!wait_one(&lrempty[nt & 1], (nt >> 1) & 1, wp)) break;
-        issue_lr(t + 2 * gridDim.x, nt & 1);
+      if (lane == 0) mbar_arrive(&lrempty[lb]);
+      if (lr_issuer && t + Cfg::LR_BUFS * static_cast<int>(gridDim.x) < tiles) {
+        if (!wait_one(&lrempty[lb], (nt / Cfg::LR_BUFS) & 1, wp)) break;
+        issue_lr(t + Cfg::LR_BUFS * gridDim.x, lb);
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -358,7 +361,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     if (warp == 2 && lane == 0) {
       // and the bias / L2 copies not yet waited for
-      for (int b = 0; b < 2; ++b)
+      for (int b = 0; b < Cfg::LR_BUFS; ++b)
         if (lr_issued[b] > lr_done[b]) wait_one(&lrfull[b], (lr_issued[b] - 1) & 1, tail);
     }
     __syncthreads();

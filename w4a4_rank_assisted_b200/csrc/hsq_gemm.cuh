@@ -55,6 +55,10 @@
 
 #include "hsq_device.cuh"
 
+#ifndef HSQ_ONE_PHASE
+#define HSQ_ONE_PHASE 1
+#endif
+
 // Drain: hand a TMEM partial buffer back to the MMA warp right after its last
 // load (1) or after the stage's math (0).
 #ifndef HSQ_EARLY_RELEASE
@@ -207,6 +211,16 @@ struct GemmCfg {
   static_assert(!PAIR || (PRE && LR_MMA), "CTA pairs: pre-expanded tokens x outputs tiles");
   static_assert(!PAIR || A_E8_BLK == 8192 && B_E8_BLK == 8192, "CTA pairs: one 32 x 256-byte TMA box per block");
   static_assert(!PRE || (F8 && !SWAP && GPS == 1), "pre-expanded operands: E4M3, tokens x outputs, one group a stage");
+  // One barrier phase per pipeline step (pre-expanded, single-CTA tiles): the
+  // group's scales are copied on the operand stage's barrier, and the MMA's one
+  // commit per step both frees the stage and tells the drain the partial is
+  // ready.  (Each phase that asynchronous copies or tcgen05.commit complete costs
+  // a CTA a fixed ~800 cycles on B200, whatever the bytes; two phases per step
+  // instead of four halve that.)  Safe for STAGES >= 3: the drain, which waits on
+  // the step's stage barriers, can lag the producer by at most STAGES - 1 + NTM
+  // steps, so no stage barrier runs a phase ahead of it.
+  static constexpr bool ONE_PHASE = HSQ_ONE_PHASE && PRE && !PAIR;
+  static_assert(!ONE_PHASE || (STAGES >= 3 && NTM <= STAGES - 1), "one phase per step: ring depth");
   // Tokens x outputs tiles write Y with TMA stores: each drain warp stages a
   // 32-row x 128-byte box (128-byte swizzle) in its own 4 KB buffer.
   static constexpr bool TMA_STORE = !SWAP;
@@ -522,7 +536,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             for (int i = 0; i < BN / 4; ++i) scw[(Cfg::CS_OFF / 16) + i] = make_float4(1.f, 1.f, 1.f, 1.f);
             const float lo = 1.0f / 262144.0f;
             for (int i = 0; i < BM / 4; ++i) scw[(Cfg::RS_OFF / 16) + i] = make_float4(lo, lo, lo, lo);
-            mbar_arrive(&sfull[ss]);
+            if (!Cfg::ONE_PHASE) mbar_arrive(&sfull[ss]);  // (ONE_PHASE: released with the stage's arrival below)
             if (leader) mbar_arrive(&full[s]);  // pairs: only the MMA issuer's barrier counts
             issued = it + 1;
             continue;
@@ -545,8 +559,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                                2 * (blk * args.rg_c + (c0 + static_cast<int>(crank) * Cfg::B_ROWS) / 8));
             }
           } else if constexpr (Cfg::PRE) {
-            // MMA-ready E4M3 tiles: one contiguous block per operand
-            mbar_arrive_expect_tx(&full[s], Cfg::A_E8 + Cfg::B_E8);
+            // MMA-ready E4M3 tiles: one contiguous block per operand (and, with
+            // ONE_PHASE, the group's scales on the same barrier)
+            mbar_arrive_expect_tx(&full[s], Cfg::A_E8 + Cfg::B_E8 + (Cfg::ONE_PHASE ? ng * (cs_bytes + rs_bytes) : 0u));
 #pragma unroll
             for (int b = 0; b < Cfg::BPG; ++b) {
               const size_t blk = static_cast<size_t>(g) * Cfg::BPG + b;
@@ -562,13 +577,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
             tma_load_2d(st + Cfg::A_PACK, &tm_col, &full[s], g * Cfg::BPG * 32, c0);
           }
-          mbar_arrive_expect_tx(&sfull[ss], ng * (cs_bytes + rs_bytes));
+          uint64_t* sbar = Cfg::ONE_PHASE ? &full[s] : &sfull[ss];
+          if (!Cfg::ONE_PHASE) mbar_arrive_expect_tx(&sfull[ss], ng * (cs_bytes + rs_bytes));
           for (int j = 0; j < ng; ++j) {
             bulk_load(sc + Cfg::CS_OFF + j * Cfg::CS_BYTES,
-                      args.scales_c + static_cast<size_t>(g + j) * args.ld_c + c0, cs_bytes, &sfull[ss]);
+                      args.scales_c + static_cast<size_t>(g + j) * args.ld_c + c0, cs_bytes, sbar);
             if (rs_bytes)
               bulk_load(sc + Cfg::RS_OFF + j * Cfg::RS_BYTES,
-                        args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, &sfull[ss]);
+                        args.scales_r + static_cast<size_t>(g + j) * args.ld_r + r0, rs_bytes, sbar);
           }
           issued = it + 1;
         }
@@ -635,7 +651,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
           }
           commit_both(&empty[s]);
-          commit_both(&tfull[tb]);
+          if (!Cfg::ONE_PHASE) commit_both(&tfull[tb]);
         }
       }
     } else if (!Cfg::PRE && lane == 0) {
@@ -877,7 +893,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int ng = GPS == 1 ? 1 : min(GPS, g1 - g);
         const int ss = it % Cfg::SSLOTS;
         const int tb = it % NTM;
-        if (!wait2_warp(&tfull[tb], (it / NTM) & 1, &sfull[ss], (it / Cfg::SSLOTS) & 1, wp)) { ok = false; break; }
+        if (Cfg::ONE_PHASE) {
+          // the step's MMAs are complete (so its stage, scales included, had landed)
+          if (!wait_warp(&empty[it % STAGES], (it / STAGES) & 1, wp)) { ok = false; break; }
+        } else if (!wait2_warp(&tfull[tb], (it / NTM) & 1, &sfull[ss], (it / Cfg::SSLOTS) & 1, wp)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const float* cs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::CS_OFF);
         const float* rs_stage = reinterpret_cast<const float*>(sc_base + ss * Cfg::SSLOT_BYTES + Cfg::RS_OFF);
@@ -1129,8 +1151,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       if (leader)
         for (uint32_t i = first; i < issued; ++i) wait_one(&full[i % STAGES], (i / STAGES) & 1, tail);
       const uint32_t sfirst = issued > static_cast<uint32_t>(Cfg::SSLOTS) ? issued - Cfg::SSLOTS : 0u;
-      for (uint32_t i = sfirst; i < issued; ++i)
-        wait_one(&sfull[i % Cfg::SSLOTS], (i / Cfg::SSLOTS) & 1, tail);
+      if (!Cfg::ONE_PHASE)  // (with ONE_PHASE the scales land on the stage barriers waited above)
+        for (uint32_t i = sfirst; i < issued; ++i)
+          wait_one(&sfull[i % Cfg::SSLOTS], (i / Cfg::SSLOTS) & 1, tail);
     }
     if (warp == 1 && lane == 0 && leader) {
       // arrives once every MMA issued above has completed (pairs: the even CTA issues them)

@@ -59,7 +59,7 @@ constexpr int kGemvThreads = 512;
 constexpr int kGemvComputeWarps = kGemvThreads / 32 - 1;
 // 16-byte weight chunks a lane reads from the ring per batch
 constexpr int kGemvBatch = 4;
-// bytes of one ring stage (whole rows; at least one row)
+// smallest ring stage (whole rows; at least one row)
 constexpr int kGemvStageBytes = 16384;
 
 // Shared-memory layout of the weight stream for MT tokens, Kp codes per row, G
@@ -85,12 +85,19 @@ inline GemvLayout gemv_layout(int MT, int Kp, int G, int rows_per_block, size_t 
                        gemv_align16(MT * 4 * 4) + gemv_align16((kGemvThreads / 32) * MT * 4 * 4);
   // the block's scales are one TMA box: at most 256 along each dimension
   if (rows_per_block > 256 || G > 256) return L;
-  L.rs = rowbytes >= kGemvStageBytes ? 1 : kGemvStageBytes / rowbytes;
+  // Few, large stages: every stage is one bulk copy whose completion costs the
+  // block a fixed ~800 cycles whatever its size, so the block's rows come in
+  // about two copies (half of them each, or half the ring when that is smaller).
+  const size_t budget = smem_max > fixed + 1024 ? smem_max - fixed - 1024 : 0;  // 1024: barriers, rounding
+  size_t target = static_cast<size_t>(rows_per_block) * rowbytes / 2;
+  if (target > budget / 2) target = budget / 2;
+  if (target < static_cast<size_t>(kGemvStageBytes)) target = kGemvStageBytes;
+  L.rs = static_cast<int>(target / rowbytes);
+  if (L.rs < 1) L.rs = 1;
   if (L.rs > rows_per_block) L.rs = rows_per_block;
   const size_t stage = static_cast<size_t>(L.rs) * rowbytes;
   const int need = (rows_per_block + L.rs - 1) / L.rs;  // stages the block's rows fill
-  int st = 0;
-  if (smem_max > fixed + 1024) st = static_cast<int>((smem_max - fixed - 1024) / stage);  // 1024: barriers, rounding
+  int st = static_cast<int>(budget / stage);
   if (st > need) st = need;
   if (st > 32) st = 32;
   L.stages = (st >= 2 || (st >= 1 && need == 1)) ? st : 0;

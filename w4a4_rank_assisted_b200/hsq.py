@@ -208,7 +208,7 @@ def stream_smem_fits(M: int, N: int, K: int, group: int = GROUP, nsm: Optional[i
     hsq_linear_forward_fused (no library call, so it can be asked without a GPU).
     T = M rounded up to 1, 2, 4 or 8; RB = rows per block = ceil(N / SMs) rounded
     up to 4; a ring of at least two stages (one if one stage holds all RB rows)
-    of min(RB, max(1, 16384 // (Kp/2))) rows."""
+    of rs rows, rs = max(1, max(16384, min(RB Kp/4, budget/2)) // (Kp/2))."""
     nsm = nsm or _sm_count()
     G = -(-K // group)
     Kp = G * group
@@ -217,10 +217,12 @@ def stream_smem_fits(M: int, N: int, K: int, group: int = GROUP, nsm: Optional[i
     if RB > 256 or G > 256:  # the block's scales are one copy of at most 256 x 256
         return False
     rowbytes = Kp // 2
-    rs = min(RB, 1 if rowbytes >= 16384 else 16384 // rowbytes)
     fixed = _a16(G * RB * 4) + _a16(T * Kp) + _a16(G * T * 4) + _a16(T * 16) + _a16(16 * T * 16)
+    budget = max(0, 227 * 1024 - fixed - 1024)
+    target = max(16384, min(RB * rowbytes // 2, budget // 2))
+    rs = min(RB, max(1, target // rowbytes))
     min_stages = 1 if -(-RB // rs) == 1 else 2
-    return fixed + 1024 + min_stages * rs * rowbytes <= 227 * 1024
+    return min_stages * rs * rowbytes <= budget
 
 
 def fused_supported(M: int, K: int, r: int, group: int = GROUP, N: int = 8, nsm: Optional[int] = None) -> bool:
