@@ -56,7 +56,7 @@
 #include "hsq_device.cuh"
 
 #ifndef HSQ_ONE_PHASE
-#define HSQ_ONE_PHASE 1
+#define HSQ_ONE_PHASE 0
 #endif
 
 // Drain: hand a TMEM partial buffer back to the MMA warp right after its last
