@@ -73,6 +73,8 @@ SMALL_SHAPES = [
     (200, 224, 1160, 4),
     (256, 1152, 1152, 4),
     (300, 640, 512, 32),
+    (8, 12288, 4096, 4),     # weight stream whose ring reuses its slots, partial last stage, ragged last block
+    (8, 16384, 2048, 2),     # ... four stages through two slots
     (16, 4096, 2048, 4),     # stream-K, decode tile
     (24, 4096, 2048, 4),     # stream-K, decode tile of 32 tokens
     (128, 2048, 1024, 4),    # stream-K, large tile

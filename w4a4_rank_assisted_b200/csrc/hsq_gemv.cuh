@@ -61,6 +61,14 @@ constexpr int kGemvComputeWarps = kGemvThreads / 32 - 1;
 constexpr int kGemvBatch = 4;
 // smallest ring stage (whole rows; at least one row)
 constexpr int kGemvStageBytes = 16384;
+// most shared memory the ring may take, and into how many stages a block's rows
+// are cut at most (before the ring's size limits them)
+#ifndef HSQ_GEMV_RING_KB
+#define HSQ_GEMV_RING_KB 224
+#endif
+#ifndef HSQ_GEMV_SPLIT
+#define HSQ_GEMV_SPLIT 2
+#endif
 
 // Shared-memory layout of the weight stream for MT tokens, Kp codes per row, G
 // scale groups and rows_per_block rows: the weight ring (stages of rs rows),
@@ -88,8 +96,9 @@ inline GemvLayout gemv_layout(int MT, int Kp, int G, int rows_per_block, size_t 
   // Few, large stages: every stage is one bulk copy whose completion costs the
   // block a fixed ~800 cycles whatever its size, so the block's rows come in
   // about two copies (half of them each, or half the ring when that is smaller).
-  const size_t budget = smem_max > fixed + 1024 ? smem_max - fixed - 1024 : 0;  // 1024: barriers, rounding
-  size_t target = static_cast<size_t>(rows_per_block) * rowbytes / 2;
+  size_t budget = smem_max > fixed + 1024 ? smem_max - fixed - 1024 : 0;  // 1024: barriers, rounding
+  if (budget > static_cast<size_t>(HSQ_GEMV_RING_KB) * 1024) budget = static_cast<size_t>(HSQ_GEMV_RING_KB) * 1024;
+  size_t target = static_cast<size_t>(rows_per_block) * rowbytes / HSQ_GEMV_SPLIT;
   if (target > budget / 2) target = budget / 2;
   if (target < static_cast<size_t>(kGemvStageBytes)) target = kGemvStageBytes;
   L.rs = static_cast<int>(target / rowbytes);
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], a.rs);  // one arrival per row
+      mbar_init(&empty[s], kGemvComputeWarps);  // every compute warp arrives once per stage
     }
     mbar_init(sfull, 1);
     *abort_flag = 0;
@@ -295,13 +304,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 
     // the block's weight scales
     bool ok = wait_warp(sfull, 0, wp);
-    // rows cw, cw + 15, ... of the block, each read from the ring: its chunks'
+    // Rows cw, cw + 15, ... of the block, each read from the ring: its chunks'
     // group partials (dp4a of int8 16*q, exact), scaled, into acc; at the row's
     // end the low-rank branch (lane j adds U[m][j] L2[j][n]), the warp's sum, the
-    // bias, Y
-    for (int i = cw; ok && i < nrows; i += kGemvComputeWarps) {
-      const int it = i / a.rs, s = it % a.stages;
+    // bias, Y.  Every warp waits for every stage in order and arrives on its
+    // release once, also for stages that hold none of its rows: a parity wait is
+    // only sound if the waiter has seen the slot's previous use land and the
+    // slot cannot be refilled twice before the waiter looks (with the ring
+    // reusing slots, a warp that skipped a phase could pass a wait one use early,
+    // or miss a use and wait for one two ahead).
+    for (int it = 0; ok && it < nst; ++it) {
+      const int s = it % a.stages;
       if (!wait_warp(&full[s], (it / a.stages) & 1, wp)) { ok = false; break; }
+      const int r0 = it * a.rs, r1 = min(nrows, r0 + a.rs);
+      for (int i = r0 + (cw - r0 % kGemvComputeWarps + kGemvComputeWarps) % kGemvComputeWarps; i < r1;
+           i += kGemvComputeWarps) {
       const uint4* wrow = reinterpret_cast<const uint4*>(ring + (static_cast<size_t>(s) * a.rs + (i - it * a.rs)) * rowbytes);
       const int n = n0 + i;
       float acc[MT];
@@ -349,8 +366,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           }
         }
       }
-      __syncwarp();  // every lane's ring reads of the row are done
-      if (lane == 0) mbar_arrive(&empty[s]);
       if (lane < a.r) {
         const float l2 = __bfloat162float(a.L2[static_cast<size_t>(lane) * a.N + n]);
 #pragma unroll
@@ -371,6 +386,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           else static_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(y);
         }
       }
+      }  // rows of this stage
+      __syncwarp();  // every lane's ring reads of the stage are done
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
   }
 
