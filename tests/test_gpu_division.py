@@ -34,11 +34,11 @@ def _run(X, s):
     return act, xc, xs
 
 
-def test_every_bf16_value_through_its_group_scale():
+@pytest.mark.parametrize("K", [4096, 512])  # 512: enough rows for the many-row kernel
+def test_every_bf16_value_through_its_group_scale(K):
     """One nonzero element per 64-group: the group's scale is fl(|fl(x/s)|/7),
     so a smoothed value off by one ulp would change the scale."""
     vals = _all_finite_bf16()
-    K = 4096
     G = K // 64
     M = -(-len(vals) // G)
     X = np.zeros((M, K), dtype=np.float32)
@@ -53,10 +53,11 @@ def test_every_bf16_value_through_its_group_scale():
     assert np.array_equal(to_np(act.x_codes), xc)
 
 
-def test_code_rounding_near_half_integers():
+@pytest.mark.parametrize("M", [512, 4400])  # 4400: the many-row kernel
+def test_code_rounding_near_half_integers(M):
     """Groups whose elements sit at and around k + 1/2 steps of the group scale."""
     rng = np.random.default_rng(1)
-    K, M = 1024, 512
+    K = 1024
     X = np.zeros((M, K), dtype=np.float32)
     G = K // 64
     for m in range(M):
@@ -70,6 +71,40 @@ def test_code_rounding_near_half_integers():
             blk[1:] = (k + frac) * sc
             X[m, g * 64:(g + 1) * 64] = blk
     s = np.ones(K, dtype=np.float32)
+    act, xc, xs = _run(X, s)
+    assert np.array_equal(to_np(act.x_scales), pad_scales(xs, hsq.hsq_scales_ld(M)))
+    assert np.array_equal(to_np(act.x_codes), xc)
+
+
+def test_extreme_values_and_smoothing_factors():
+    """Rows that mix a normal group absmax with bf16 subnormals and values below
+    2^-100, groups of such tiny values only, values above 2^100, all-zero groups,
+    and channels whose smoothing factor lies outside [2^-24, 2^24] (in the last
+    256-channel chunk only): every code and scale must still equal what the
+    oracle's IEEE quotients give."""
+    rng = np.random.default_rng(2)
+    K, M = 1024, 4400  # enough rows for the many-row kernel
+    G = K // 64
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    tiny = np.array([2.0 ** -133, 2.0 ** -126, 2.0 ** -110, 2.0 ** -101, 2.0 ** -100, 3 * 2.0 ** -105],
+                    dtype=np.float32)
+    sign = lambda n: rng.choice(np.array([-1.0, 1.0], dtype=np.float32), n)
+    for m in range(M):
+        kind = m % 5
+        if kind == 0:    # a normal absmax with tiny elements beside it
+            idx = rng.choice(768, 40, replace=False)
+            X[m, idx] = rng.choice(tiny, 40) * sign(40)
+        elif kind == 1:  # one group of tiny values only
+            g = rng.integers(12)
+            X[m, g * 64:(g + 1) * 64] = rng.choice(tiny, 64) * sign(64)
+        elif kind == 2:  # values above 2^100
+            idx = rng.choice(768, 3, replace=False)
+            X[m, idx] = (2.0 ** rng.uniform(100.0, 120.0, 3)).astype(np.float32) * sign(3)
+        elif kind == 3:  # an all-zero group
+            g = rng.integers(G)
+            X[m, g * 64:(g + 1) * 64] = 0.0
+    s = np.exp(rng.uniform(np.log(0.05), np.log(50.0), K)).astype(np.float32)
+    s[900:904] = np.array([2.0 ** -30, 2.0 ** -25, 2.0 ** 25, 2.0 ** 30], dtype=np.float32)
     act, xc, xs = _run(X, s)
     assert np.array_equal(to_np(act.x_scales), pad_scales(xs, hsq.hsq_scales_ld(M)))
     assert np.array_equal(to_np(act.x_codes), xc)

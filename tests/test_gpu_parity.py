@@ -86,6 +86,10 @@ SMALL_SHAPES = [
     (40, 328, 264, 8),       # few rows, rank 8, ragged last chunk
     (33, 328, 128, 7),       # generic odd rank, few rows
     (150, 584, 136, 5),      # generic odd rank, ragged rows and last chunk
+    (4150, 1160, 136, 4),    # many-row activation kernel: ragged last block, lanes past the padded K
+    (4150, 264, 136, 0),     # ... no low-rank branch
+    (4200, 520, 136, 1),     # ... rank 1
+    (4150, 2056, 136, 2),    # ... rank 2, a last chunk of 8 channels
     # M <= 8: the CUDA-core weight stream
     (2, 640, 264, 32),
     (3, 1152, 1160, 0),
@@ -119,6 +123,8 @@ SHAPES_G128 = [
     (300, 640, 512, 32),
     (6, 640, 264, 16),       # the CUDA-core weight stream, four lanes per group
     (8, 1024, 1160, 4),
+    (4150, 1160, 136, 2),    # many-row activation kernel
+    (4160, 392, 136, 4),     # ... K = 392 pads to 512
 ]
 
 

@@ -142,6 +142,15 @@ cudaError_t launch_pdl(bool allow, void (*kernel)(KArgs...), dim3 grid, dim3 blo
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The row-owning activation kernel for many rows (0: always the sub-block kernel).
+#ifndef HSQ_ACT_ROWS
+#define HSQ_ACT_ROWS 1
+#endif
+// ... from this many rows per SM on
+#ifndef HSQ_ACT_ROWS16_MIN
+#define HSQ_ACT_ROWS16_MIN 28
+#endif
+
 thread_local int t_debug_flags = 0;
 thread_local int t_debug_limit_ms = 0;
 
@@ -532,6 +541,31 @@ BlasSlot g_blas[kMaxDevices];
 
 }  // namespace
 
+// The many-row activation kernel: its X ring is dynamic shared memory (set once
+// per device and instantiation).
+template <int R, int GL, int NW, int SUB>
+cudaError_t launch_act_rows(const __nv_bfloat16* X, const float* s, const __nv_bfloat16* L1, int M, int K, int Kp,
+                            int ld, uint8_t* codes, float* scales, float* U, cudaStream_t st) {
+  using C = hsq::ActRowsCfg<NW, SUB>;
+  constexpr int kSmem = C::STAGES * C::STAGE_BYTES;
+  static std::mutex mu;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      const cudaError_t e = cudaFuncSetAttribute(hsq::quantize_act_rows_kernel<R, GL, NW, SUB>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
+  return launch_pdl(true, hsq::quantize_act_rows_kernel<R, GL, NW, SUB>, dim3((M + C::RB - 1) / C::RB),
+                    dim3(NW * 32), static_cast<size_t>(kSmem), st, X, s, L1, M, K, Kp, ld, codes, scales, U,
+                    wait_limit_ns());
+}
+
 extern "C" {
 
 size_t hsq_lowrank_workspace_bytes(int N, int K, int r) {
@@ -739,13 +773,30 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
     case 32: HSQ_ACT_LAUNCH(32, SM); break; \
     default: HSQ_ACT_LAUNCH(-1, SM); break; \
   }
+#define HSQ_ACT_ROWS_LAUNCH(RV, NW, SUB)                                                                  \
+  lerr = (group == 128 ? launch_act_rows<RV, 16, NW, SUB>(X, s, L1, M, K, Kp, ld, x_codes, x_scales, U, stream) \
+                       : launch_act_rows<RV, 8, NW, SUB>(X, s, L1, M, K, Kp, ld, x_codes, x_scales, U, stream))
+#define HSQ_ACT_ROWS_RANKS(NW, SUB)               \
+  switch (r) {                                    \
+    case 0: HSQ_ACT_ROWS_LAUNCH(0, NW, SUB); break; \
+    case 1: HSQ_ACT_ROWS_LAUNCH(1, NW, SUB); break; \
+    case 2: HSQ_ACT_ROWS_LAUNCH(2, NW, SUB); break; \
+    default: HSQ_ACT_ROWS_LAUNCH(4, NW, SUB); break; \
+  }
   cudaError_t lerr = cudaSuccess;
-  // few rows: one block per sub-block with 32 warps spread over K; else 8 warps x 2 sub-blocks
+  // few rows: one block per sub-block with 32 warps spread over K; many rows
+  // (enough for two 16-row blocks per SM, nearly) and ranks 0, 1, 2, 4: the
+  // row-owning kernel; else 8 warps x 2 sub-blocks
+  const bool rows_kernel = HSQ_ACT_ROWS && (r <= 2 || r == 4) && M >= HSQ_ACT_ROWS16_MIN * device_sm_count();
   if (M <= 64) {
     HSQ_ACT_RANKS(true)
+  } else if (rows_kernel) {
+    HSQ_ACT_ROWS_RANKS(8, 2)
   } else {
     HSQ_ACT_RANKS(false)
   }
+#undef HSQ_ACT_ROWS_RANKS
+#undef HSQ_ACT_ROWS_LAUNCH
 #undef HSQ_ACT_RANKS
 #undef HSQ_ACT_LAUNCH
   return (lerr == cudaSuccess && cudaGetLastError() == cudaSuccess) ? HSQ_OK : HSQ_ERR_CUDA;

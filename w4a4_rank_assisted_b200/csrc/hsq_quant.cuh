@@ -574,4 +574,382 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
   }
 }
 
+// ---------------------------------------------------------------------------
+// The activation step for many rows and ranks 0..4 (the same outputs as
+// quantize_act_kernel, fewer instructions per element).
+//
+// A block of NW warps owns RB = NW * SUB consecutive rows; warp w owns rows
+// w*SUB .. w*SUB+SUB-1 of them across all of K, so U needs no reduction across
+// warps.  K is walked in chunks of 256 channels:
+//   * each warp streams its own row pieces (512 bytes per row and chunk) into a
+//     ring of STAGES shared-memory stages with 16-byte asynchronous copies, one
+//     per lane, STAGES chunks ahead of its compute (the copies zero-fill past K
+//     and past the last row);
+//   * the chunk's per-channel tables -- RN(1/s), -s and the L1 rows as fp32 --
+//     sit in a ring of TS slots; every warp builds its 256/NW channels of chunk
+//     c + TD while it computes chunk c (the global loads issued two chunks
+//     earlier) and arrives on the slot's `tfull` mbarrier; a warp done with a
+//     chunk arrives on the slot's `tempty` mbarrier, which the builders of the
+//     slot's next chunk wait for.  Warps are never held in lockstep: a warp
+//     may run up to TS - TD chunks ahead of the slowest one.
+// Lane l handles channels 8l .. 8l+7 of a row; the SUB rows of a warp are
+// processed side by side.  Arithmetic on channel pairs uses the packed fp32x2
+// instructions: X_hat = x / s as a product with RN(1/s) and Markstein's
+// correction, the rank products accumulated per channel parity, the codes as a
+// product with RN(1/scale), its correction and the round-to-integer addition.
+// The correction gives the IEEE quotient when the dividend, divisor and
+// quotient are normal; instead of testing every element, a group takes it only
+// when s lies in [2^-24, 2^24] for the chunk and the group's absmax (a
+// NaN-propagating maximum) lies in [2^-60, 2^75]:
+//   * such a group's elements with 2^-100 <= |x| <= 2^100 are exact;
+//   * smaller elements have |X_hat| < 2^-75, far below half a code step
+//     (scale >= 2^-63), so code 0 on both sides and no effect on the absmax;
+//   * larger elements make the absmax exceed 2^75 (or NaN), so the group is
+//     not taken;
+// otherwise the warp redoes the chunk's rows with IEEE divisions (quantize8).
+// ---------------------------------------------------------------------------
+template <int NW, int SUB>
+struct ActRowsCfg {
+  static constexpr int RB = NW * SUB;
+  static constexpr int STAGES = 4;  // X ring depth (chunks)
+  static constexpr int TS = 4;      // table slots
+  static constexpr int TD = 2;      // tables are built this many chunks ahead
+  static constexpr int STAGE_BYTES = RB * 512;
+};
+
+// Shared-memory float4 slot of logical slot q in a lane's block of S slots
+// (S = 1, 2, 4 or 8), XOR-swizzled so that the 8 lanes of each quarter-warp
+// phase of a 128-bit load hit 8 different 16-byte bank groups.
+template <int S>
+__device__ __forceinline__ int swz_slot(int lane, int q) {
+  return q ^ ((lane / (8 / S)) & (S - 1));
+}
+
+// max that propagates NaN (PTX max.NaN.f32).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// NaN-propagating absmax of a lane's 8 values (a depth-3 tree).
+__device__ __forceinline__ float absmax8_nan(const float (&v)[8]) {
+  const float a = fmax_nan(fmax_nan(fabsf(v[0]), fabsf(v[1])), fmax_nan(fabsf(v[2]), fabsf(v[3])));
+  const float b = fmax_nan(fmax_nan(fabsf(v[4]), fabsf(v[5])), fmax_nan(fabsf(v[6]), fabsf(v[7])));
+  return fmax_nan(a, b);
+}
+
+// 16-byte asynchronous global -> shared copy; bytes past `src_bytes` (0 or 16)
+// are zero-filled.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Sum over e of (0x4B400000 << 4e) modulo 2^32: the exponent bits that the
+// round-to-integer additions leave in the nibble-packing sum below.
+__host__ __device__ constexpr uint32_t int4_pack_bias() {
+  uint32_t b = 0;
+  for (int e = 0; e < 8; ++e) b += 0x4B400000u << (4 * e);
+  return b;
+}
+
+// Codes of 8 values of a group whose absmax `amax` lies in [2^-60, 2^75]
+// (every lane of the group passes the same amax): scale = RN(amax / 7) by
+// Markstein's correction against RN(1/7); each code RN(v / scale) by the
+// correction against RN(1/scale), then rounded to an integer by adding
+// 1.5 * 2^23 + 8, which leaves code + 8 (in 1..15) in the low mantissa bits.
+// The 8 sums are packed by shifts and adds; the exponent bits they drag along
+// add up to one constant (int4_pack_bias), and XOR 8 per nibble turns code + 8
+// into the code's 4-bit two's complement.
+__device__ __forceinline__ uint32_t quantize8_int4_ranged(const float (&v)[8], float amax, float& scale) {
+  constexpr float kInv7 = 1.0f / 7.0f;
+  const float q = __fmul_rn(amax, kInv7);
+  scale = __fmaf_rn(__fmaf_rn(-q, 7.0f, amax), kInv7, q);
+  const float z = __frcp_rn(scale);
+  const float ns = -scale;
+  constexpr float kRound = 12582920.0f;  // 1.5 * 2^23 + 8
+  uint32_t b[8];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    float q0, q1, r0, r1, t0, t1;
+    fmul2(q0, q1, v[2 * p], v[2 * p + 1], z, z);
+    ffma2(r0, r1, q0, q1, ns, ns, v[2 * p], v[2 * p + 1]);
+    ffma2(t0, t1, r0, r1, z, z, q0, q1);
+    fadd2(t0, t1, t0, t1, kRound, kRound);
+    b[2 * p] = __float_as_uint(t0);
+    b[2 * p + 1] = __float_as_uint(t1);
+  }
+  const uint32_t p01 = (b[1] << 4) + b[0], p23 = (b[3] << 4) + b[2];
+  const uint32_t p45 = (b[5] << 4) + b[4], p67 = (b[7] << 4) + b[6];
+  const uint32_t acc = (((p67 << 8) + p45) << 16) + ((p23 << 8) + p01);
+  return (acc - int4_pack_bias()) ^ 0x88888888u;
+}
+
+template <int R, int GL, int NW, int SUB>
+__global__ void __launch_bounds__(NW * 32, 16 / NW)
+    quantize_act_rows_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
+                             const __nv_bfloat16* __restrict__ L1, int M, int K, int Kp, int ld,
+                             uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U,
+                             uint64_t limit_ns) {
+  static_assert(R >= 0 && R <= 4 && R != 3, "ranks 0, 1, 2 and 4");
+  static_assert(NW <= 8, "one byte per warp in an 8-byte flag word");
+  using C = ActRowsCfg<NW, SUB>;
+  constexpr int RB = C::RB, STAGES = C::STAGES, TS = C::TS, TD = C::TD, NT = NW * 32;
+  constexpr int CPT = 256 / NT;          // table channels built per thread
+  constexpr int RT = R > 0 ? R : 1;
+  constexpr int LS = 2 * RT;             // float4 slots of a lane's L1 block (8 channels x R)
+  constexpr int PW = RT > 1 ? RT / 2 : 1;
+  extern __shared__ __align__(128) uint8_t ring[];  // STAGES x STAGE_BYTES (dynamic)
+  // per lane (8 channels): 4 slots (z_2p, z_2p+1, -s_2p, -s_2p+1), swizzled
+  __shared__ __align__(16) float tzs[TS][32 * 16];
+  // per lane: slot data L1[2p][j], L1[2p+1][j] at ((p R + j) 2 + h), swizzled
+  __shared__ __align__(16) float tl1[R > 0 ? TS : 1][R > 0 ? 32 * 8 * RT : 4];
+  __shared__ __align__(8) uint8_t tbad[TS][8];  // per warp: some s of its channels out of range
+  __shared__ __align__(8) uint64_t tfull[TS], tempty[TS];
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = lane_id();
+  const int mw = blockIdx.x * RB + warp * SUB;  // this warp's first row
+  const int nchunks = (Kp + 255) >> 8;
+  if (tid == 0) {
+#pragma unroll
+    for (int t = 0; t < TS; ++t) {
+      mbar_init(&tfull[t], NW);
+      mbar_init(&tempty[t], NW);
+      *reinterpret_cast<uint2*>(tbad[t]) = make_uint2(0u, 0u);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dep_wait();  // X may come from the preceding kernel
+  const bool early = gridDim.x <= 64;
+  if (early && tid == 0) grid_dep_launch();
+  const WaitPolicy wp{limit_ns, &abort_flag};
+
+  // this warp's row pieces of chunk c into stage c % STAGES (one commit group
+  // per chunk, empty past the last chunk, so that group counts stay uniform)
+  auto issue = [&](int c) {
+    if (c < nchunks) {
+      const int k0 = c * 256 + lane * 8;
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) {
+        const int m = mw + i;
+        const bool in = m < M && k0 < K;
+        cp_async16(ring + (c % STAGES) * C::STAGE_BYTES + (warp * SUB + i) * 512 + lane * 16,
+                   in ? static_cast<const void*>(X + static_cast<size_t>(m) * K + k0) : static_cast<const void*>(X),
+                   in ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // the table inputs of this thread's channels; queue slot d holds chunk c+TD+d
+  // during iteration c
+  float ps[2][CPT];
+  uint32_t pl[2][CPT][PW];
+  auto fetch = [&](int c, float (&fs)[CPT], uint32_t (&fl)[CPT][PW]) {
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) {
+      const int k = c * 256 + tid + q * NT;
+      const bool in = c < nchunks && k < K;
+      fs[q] = in ? __ldg(s + k) : 1.f;
+      if constexpr (R == 4) {
+        const uint2 v = in ? __ldg(reinterpret_cast<const uint2*>(L1 + static_cast<size_t>(k) * 4))
+                           : make_uint2(0u, 0u);
+        fl[q][0] = v.x;
+        fl[q][1] = v.y;
+      } else if constexpr (R == 2) {
+        fl[q][0] = in ? __ldg(reinterpret_cast<const unsigned int*>(L1 + static_cast<size_t>(k) * 2)) : 0u;
+      } else if constexpr (R == 1) {
+        fl[q][0] = in ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(L1 + k))) : 0u;
+      } else {
+        fl[q][0] = 0u;
+      }
+    }
+  };
+  // this warp's channels of chunk cb's tables into slot cb % TS (after the
+  // slot's previous chunk is released); returns false on a timeout
+  auto build = [&](int cb) -> bool {
+    const int t = cb % TS;
+    if (cb >= TS && !wait_warp(&tempty[t], ((cb / TS) - 1) & 1, wp)) return false;
+    bool bad = false;
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) {
+      const int ch = tid + q * NT;          // channel within the chunk
+      const int ln = ch >> 3, e = ch & 7;   // consuming lane, its channel
+      const float sv = ps[0][q];
+      bad |= !(sv >= 0x1p-24f && sv <= 0x1p24f);
+      float* zb = &tzs[t][ln * 16];
+      const int p = e >> 1, h = e & 1;
+      zb[swz_slot<4>(ln, p) * 4 + h] = __frcp_rn(sv);
+      zb[swz_slot<4>(ln, p) * 4 + 2 + h] = -sv;
+      if constexpr (R > 0) {
+        float* lb = &tl1[t][ln * 8 * RT];
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+          const uint32_t w = pl[0][q][j >> 1];
+          const float f = __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
+          const int idx = (p * R + j) * 2 + h;
+          lb[swz_slot<LS>(ln, idx >> 2) * 4 + (idx & 3)] = f;
+        }
+      }
+    }
+    const bool anybad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      tbad[t][warp] = anybad ? 1 : 0;
+      mbar_arrive(&tfull[t]);  // release: this warp's table writes
+    }
+    return true;
+  };
+  auto advance = [&](int cnext) {  // shift the queue, fetch chunk cnext into its tail
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) {
+      ps[0][q] = ps[1][q];
+#pragma unroll
+      for (int h = 0; h < PW; ++h) pl[0][q][h] = pl[1][q][h];
+    }
+    fetch(cnext, ps[1], pl[1]);
+  };
+
+  // prologue: X chunks 0..STAGES-1 in flight, tables of chunks 0..TD-1 built,
+  // the queue holding chunks TD and TD+1
+  bool ok = true;
+#pragma unroll
+  for (int c = 0; c < STAGES; ++c) issue(c);
+  fetch(0, ps[0], pl[0]);
+  fetch(1, ps[1], pl[1]);
+#pragma unroll
+  for (int c = 0; c < TD; ++c) {
+    if (c < nchunks) ok = ok && build(c);
+    advance(c + 2);
+  }
+
+  float2 acc[SUB][RT];
+#pragma unroll
+  for (int i = 0; i < SUB; ++i)
+#pragma unroll
+    for (int j = 0; j < RT; ++j) acc[i][j] = make_float2(0.f, 0.f);
+
+  for (int c = 0; ok && c < nchunks; ++c) {
+    const int t = c % TS;
+    if (c + TD < nchunks) {
+      if (!build(c + TD)) { ok = false; break; }
+    }
+    advance(c + TD + 2);
+    if (!wait_warp(&tfull[t], (c / TS) & 1, wp)) { ok = false; break; }
+    cp_async_wait<STAGES - 1>();  // this lane's copies of chunk c have landed
+    __syncwarp();                 // ... and every other lane's
+    if (mw < M) {
+      const uint2 bw = *reinterpret_cast<const uint2*>(tbad[t]);
+      const bool sbad = (bw.x | bw.y) != 0u;
+      const int k0 = c * 256 + lane * 8;
+      const bool real = k0 < K, in_k = k0 < Kp;
+      float zz[8], ns[8];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float4 v = *reinterpret_cast<const float4*>(&tzs[t][lane * 16 + swz_slot<4>(lane, p) * 4]);
+        zz[2 * p] = v.x; zz[2 * p + 1] = v.y; ns[2 * p] = v.z; ns[2 * p + 1] = v.w;
+      }
+      const uint8_t* stage = ring + (c % STAGES) * C::STAGE_BYTES + warp * SUB * 512 + lane * 16;
+      float xh[SUB][8], amax[SUB];
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(stage + i * 512);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float x0 = __uint_as_float(w[p] << 16), x1 = __uint_as_float(w[p] & 0xffff0000u);
+          float q0, q1, r0, r1;
+          fmul2(q0, q1, x0, x1, zz[2 * p], zz[2 * p + 1]);
+          ffma2(r0, r1, q0, q1, ns[2 * p], ns[2 * p + 1], x0, x1);
+          ffma2(xh[i][2 * p], xh[i][2 * p + 1], r0, r1, zz[2 * p], zz[2 * p + 1], q0, q1);
+        }
+        amax[i] = absmax8_nan(xh[i]);
+      }
+#pragma unroll
+      for (int o = 1; o < GL; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) amax[i] = fmax_nan(amax[i], __shfl_xor_sync(0xffffffffu, amax[i], o));
+      bool bad = false;
+#pragma unroll
+      for (int i = 0; i < SUB; ++i)
+        bad |= (mw + i < M) && in_k && (sbad || !(amax[i] >= 0x1p-60f && amax[i] <= 0x1p75f));
+      uint32_t packed[SUB];
+      float sc[SUB];
+      if (__any_sync(0xffffffffu, bad)) {
+        // the exact path: IEEE quotients (-ns = s; padding lanes read zeros)
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) {
+          float x[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(stage + i * 512), x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xh[i][e] = real ? __fdiv_rn(x[e], -ns[e]) : 0.f;
+          packed[i] = quantize8<GL>(xh[i], sc[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) packed[i] = quantize8_int4_ranged(xh[i], amax[i], sc[i]);
+      }
+      if constexpr (R > 0) {
+        float lp[8 * RT];
+#pragma unroll
+        for (int q = 0; q < LS; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(&tl1[t][lane * 8 * RT + swz_slot<LS>(lane, q) * 4]);
+          lp[4 * q] = v.x; lp[4 * q + 1] = v.y; lp[4 * q + 2] = v.z; lp[4 * q + 3] = v.w;
+        }
+#pragma unroll
+        for (int i = 0; i < SUB; ++i)
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int j = 0; j < R; ++j)
+              ffma2(acc[i][j].x, acc[i][j].y, xh[i][2 * p], xh[i][2 * p + 1], lp[(p * R + j) * 2],
+                    lp[(p * R + j) * 2 + 1], acc[i][j].x, acc[i][j].y);
+      }
+      if (in_k) {
+#pragma unroll
+        for (int i = 0; i < SUB; ++i)
+          if (mw + i < M)
+            *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(mw + i) * (Kp / 2) + k0 / 2) = packed[i];
+        if ((lane & (GL - 1)) == 0) {
+          float* srow = scales + static_cast<size_t>(k0 / (8 * GL)) * ld;
+          if (SUB == 2 && mw + 1 < M) {
+            *reinterpret_cast<float2*>(srow + mw) = make_float2(sc[0], sc[SUB - 1]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < SUB; ++i)
+              if (mw + i < M) srow[mw + i] = sc[i];
+          }
+          if (M - 1 < mw + SUB)
+            for (int p = M; p < ld; ++p) srow[p] = 0.f;  // padding of the group-major layout
+        }
+      }
+    }
+    __syncwarp();  // every lane is done with stage c % STAGES and table slot t
+    if (lane == 0) mbar_arrive(&tempty[t]);
+    issue(c + STAGES);
+  }
+  cp_async_wait<0>();  // no copy outlives the block
+  if (!early && tid == 0) grid_dep_launch();
+
+  if constexpr (R > 0) {
+#pragma unroll
+    for (int i = 0; i < SUB; ++i)
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        float v = acc[i][j].x + acc[i][j].y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && ok && mw + i < M) U[static_cast<size_t>(mw + i) * R + j] = v;
+      }
+  }
+}
+
 }  // namespace hsq
