@@ -181,16 +181,34 @@ hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_sca
 /*
  * Activation step and forward in one launch, for decode-sized inputs: the
  * same results as hsq_quantize_act followed by hsq_linear_forward (the same
- * codes, scales and U, which are kept on chip and not written out), for
- *   M <= 4 tokens, rank r in {0, 1, 2, 4}, and K small enough that one block's
- *   shared memory holds the rows' widened codes, the block's weight scales and a
- *   ring of weight rows: T (Kp + 4 G + 272) + 4 G RB + S rs Kp/2 + 1024 bytes
- *   <= 227 KiB, T = M rounded up to 1, 2 or 4, RB = ceil(N / SMs) rounded up
- *   to 4 (the rows of one block), rs rows per ring stage (about half the
- *   block's rows, at least 16 KiB of them, at most half of what the ring can
- *   hold) and S = 2 stages (1 when one stage holds all RB rows), with
- *   RB <= 256 and G <= 256; e.g. K <= 16384 for groups of 64 and K <= 29696
- *   for groups of 128 at M = 4, N = 12288 on 148 SMs.
+ * codes and scales; U up to its fp32 summation order), for up to 16 tokens and
+ * any rank r <= 32.  Two forms, chosen from the shape (hsq_fused_form tells
+ * which without launching anything):
+ *   1. the weight stream, each block repeating the activation step with the
+ *      codes kept on chip (nothing of the step goes through HBM), for
+ *      M <= 4 tokens, rank r in {0, 1, 2, 4}, and K small enough that one
+ *      block's shared memory holds the rows' widened codes, the block's weight
+ *      scales and a ring of weight rows: T (Kp + 4 G + 272) + 4 G RB +
+ *      S rs Kp/2 + 1024 bytes <= 227 KiB, T = M rounded up to 1, 2 or 4,
+ *      RB = ceil(N / SMs) rounded up to 4 (the rows of one block), rs rows per
+ *      ring stage (about half the block's rows, at least 16 KiB of them, at
+ *      most half of what the ring can hold) and S = 2 stages (1 when one stage
+ *      holds all RB rows), with RB <= 256 and G <= 256; e.g. K <= 16384 for
+ *      groups of 64 and K <= 29696 for groups of 128 at M = 4, N = 12288 on
+ *      148 SMs;
+ *   2. otherwise, for M <= 16: the 16-token tensor-core decode tiles, launched
+ *      cooperatively (every CTA resident at once), whose CTAs first share out
+ *      the activation step -- (token, 256-channel) pieces, written to a
+ *      library-owned device array -- then meet at a grid barrier (time-limited:
+ *      a barrier that does not gather sets HSQ_ERR_TIMEOUT in the device status
+ *      and the launch does no GEMM work), sum U per CTA in a fixed order and
+ *      run the decode-tile GEMM on those codes.  The array is 8 MiB: the
+ *      shape's stream-K partials (about 16 KiB per SM), its codes M Kp/2, its
+ *      scales, U partials and copies must fit it (K up to about 500000 at
+ *      M = 16).  As with hsq_linear_forward_noalloc, all calls share that one
+ *      array: calls whose kernels overlap on the GPU (different streams, no
+ *      ordering between them) race; the first call on a device looks up the
+ *      array's address (once per device), so make it before any stream capture.
  * Other shapes return HSQ_ERR_UNSUPPORTED before anything is launched (use the
  * two calls).  The pages do not name this fusion; it is the step before the
  * path (activations quantized online) moved into the path's first kernel.
@@ -203,6 +221,14 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
                                     const void* L2_bf16, const void* bias_bf16,
                                     int M, int N, int K, int r, int group,
                                     void* Y, hsq_out_dtype out, cudaStream_t stream);
+
+/*
+ * The form hsq_linear_forward_fused takes for this shape on the current device:
+ * 0 = none (the call returns HSQ_ERR_UNSUPPORTED, or INVALID_ARG for an invalid
+ * shape), 1 = the weight stream, 2 = the cooperative decode tiles.  Host
+ * arithmetic only: launches nothing, and with no device present assumes 148 SMs.
+ */
+int hsq_fused_form(int M, int N, int K, int r, int group);
 
 /*
  * Pack-time helper: plain truncated-SVD initialisation of the low-rank pair

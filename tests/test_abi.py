@@ -90,26 +90,47 @@ def test_fused_forward_argument_validation():
         return f(a["X"], a["s"], a["L1"], a["wc"], a["ws"], a["L2"], a["b"], a["M"], a["N"], a["K"], a["r"],
                  a["g"], a["Y"], a["out"], None)
 
-    assert call(M=5) == hsq.HSQ_ERR_UNSUPPORTED          # more than 4 tokens: the two-call path
-    assert call(r=3) == hsq.HSQ_ERR_UNSUPPORTED
-    assert call(r=8) == hsq.HSQ_ERR_UNSUPPORTED
-    assert call(M=4, K=65536) == hsq.HSQ_ERR_UNSUPPORTED  # the rows' codes do not fit one block
+    # (only shapes the library rejects before launching are called: fake
+    # pointers must never reach a launch)
+    assert call(M=17) == hsq.HSQ_ERR_UNSUPPORTED         # more than 16 tokens: the two-call path
+    assert call(r=33) == hsq.HSQ_ERR_UNSUPPORTED
+    assert call(M=16, K=1 << 20) == hsq.HSQ_ERR_UNSUPPORTED  # the codes alone overflow the library's array
     assert call(g=96) == hsq.HSQ_ERR_UNSUPPORTED
     assert call(M=0) == hsq.HSQ_ERR_INVALID_ARG
     assert call(X=None) == hsq.HSQ_ERR_INVALID_ARG
     assert call(L1=None) == hsq.HSQ_ERR_INVALID_ARG      # r > 0 needs L1 and L2
     assert call(r=0) == hsq.HSQ_ERR_INVALID_ARG          # r == 0 wants L1 == L2 == NULL
     assert call(X=MIS) == hsq.HSQ_ERR_ALIGNMENT
-    assert hsq.fused_supported(1, 4096, 4, N=12288) and not hsq.fused_supported(5, 4096, 4, N=12288)
-    # the Python restatement of the shared-memory limit agrees with the library at its edge
+
+
+def test_fused_form_query_and_its_python_restatement():
+    """hsq_fused_form (host arithmetic, no launch) against fused_supported and
+    the weight stream's shared-memory restatement, on both sides of each limit."""
+    form = hsq.hsq_fused_form
+    assert form(1, 12288, 4096, 4, 64) == 1 and form(4, 12288, 4096, 2, 128) == 1
+    assert form(5, 12288, 4096, 4, 64) == 2 and form(16, 4096, 12288, 4, 64) == 2
+    assert form(2, 4096, 4096, 8, 64) == 2 and form(16, 4096, 4096, 32, 128) == 2
+    assert form(17, 4096, 4096, 4, 64) == 0 and form(16, 64, 1 << 20, 4, 64) == 0
+    assert form(4, 4096, 4096, 33, 64) == 0 and form(4, 4096, 4100, 4, 64) == 0
+    if hsq._sm_count() != 148:
+        return
+    # the weight stream's shared-memory limit, at its edge
     for N, M in ((4096, 4), (12288, 1), (12288, 4)):
         lo, hi = 64, 1 << 17
-        while hi - lo > 64:  # the largest K (a multiple of 64) the restatement accepts
+        while hi - lo > 64:  # the largest K (a multiple of 64) the restatement gives the stream
             mid = (lo + hi) // 2 // 64 * 64
-            lo, hi = (mid, hi) if hsq.fused_supported(M, mid, 4, N=N, nsm=148) else (lo, mid)
-        # (only the rejected side is called: fake pointers must never reach a launch)
-        if hsq._sm_count() == 148:
-            assert call(M=M, N=N, K=lo + 64) == hsq.HSQ_ERR_UNSUPPORTED
+            lo, hi = (mid, hi) if hsq.stream_smem_fits(M, N, mid, 64, nsm=148) else (lo, mid)
+        assert form(M, N, lo, 4, 64) == 1 and form(M, N, lo + 64, 4, 64) == 2
+    # the decode tiles' array limit, at its edge (K where the codes fill it)
+    for N, M, r, g in ((4096, 16, 4, 64), (12288, 9, 32, 128), (128, 16, 0, 64)):
+        lo, hi = 64, 1 << 20
+        while hi - lo > 64:
+            mid = (lo + hi) // 2 // 64 * 64
+            lo, hi = (mid, hi) if hsq.fused_supported(M, mid, r, g, N=N, nsm=148) else (lo, mid)
+        assert form(M, N, lo, r, g) == 2 and form(M, N, lo + 64, r, g) == 0
+    for M, K, r, g, N in ((1, 4096, 4, 64, 12288), (3, 1152, 8, 64, 520), (16, 4096, 4, 64, 12288),
+                          (12, 200, 7, 64, 136), (16, 1024, 16, 128, 264)):
+        assert hsq.fused_supported(M, K, r, g, N=N, nsm=148) == (form(M, N, K, r, g) != 0)
 
 
 def test_lowrank_helper_argument_validation():

@@ -145,6 +145,17 @@ FUSED_SHAPES = [
     (4, 1152, 520, 0, 64),
     (1, 1024, 264, 4, 128),
     (4, 384, 136, 2, 128),
+    # the decode-tile form (cooperative launch, the step shared out over the grid)
+    (5, 640, 264, 2, 64),      # from 5 tokens
+    (8, 4096, 1160, 4, 64),
+    (16, 1152, 520, 0, 64),    # no low-rank branch
+    (16, 2048, 2048, 32, 64),  # largest rank
+    (12, 200, 136, 7, 64),     # K = 200 pads to 256, an odd rank
+    (3, 1152, 520, 8, 64),     # a rank the weight stream's form does not take
+    (1, 2048, 4096, 32, 64),   # one token, rank 32
+    (16, 12288, 1024, 4, 64),  # stream-K over many stages
+    (16, 1024, 264, 16, 128),
+    (9, 384, 136, 2, 128),
 ]
 
 
@@ -160,10 +171,12 @@ def test_fused_forward_matches_oracle_and_two_calls(M, K, N, r, group, out):
     ref = oracle_layer(layer.X, layer.W, layer.s, layer.L1 if r else None, layer.L2 if r else None, layer.bias,
                        group=group)
     check_y(to_np(Yf), ref["Y"], out == hsq.HSQ_OUT_F32, f"fused {M}x{K}x{N} r{r} g{group}")
-    # the same codes and scales, and U up to its fp32 summation order
+    # the same codes and scales; U and the group sums up to their fp32 summation
+    # order (from 5 tokens the two calls run the weight stream or other decode
+    # tiles), so bf16 outputs may differ by the one rounding of the output: an ulp
     a, b = to_np(Yf).astype(np.float64), to_np(Y2).astype(np.float64)
     rms = np.sqrt(np.mean(ref["Y"] ** 2))
-    tol = 1e-5 * rms if out == hsq.HSQ_OUT_F32 else 1e-5 * rms + np.abs(b) * 2.0 ** -8
+    tol = 1e-5 * rms if out == hsq.HSQ_OUT_F32 else 1e-5 * rms + O.bf16_ulp(np.maximum(np.abs(a), np.abs(b)))
     assert np.all(np.abs(a - b) <= tol), "fused forward differs from the two calls"
 
 
@@ -249,6 +262,33 @@ def test_forced_timeout_reports_status_and_library_recovers():
     hsq.forward(pl, layer.X.to(DEV), act, Y, workspace=ws, out=hsq.HSQ_OUT_F32)
     assert hsq.hsq_get_device_status() == hsq.HSQ_OK
     assert torch.equal(Y, Y_ok)
+
+
+def test_fused_decode_tiles_repeat_bit_exact_and_recover_from_a_timeout():
+    """The decode-tile form of the single launch: its grid barrier and stream-K
+    counters are back at zero after every call (also after a forced timeout),
+    so repeated calls give the same bits."""
+    layer = make_layer(_spec(16, 4096, 2048, 8, seed=5))
+    assert hsq.hsq_fused_form(16, 2048, 4096, 8, 64) == 2
+    pl, act, Y2, ws = _run_gpu(layer)
+    X = layer.X.to(DEV)
+    Y = torch.empty_like(Y2)
+    hsq.forward_fused(pl, X, Y, out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    Y0 = Y.clone()
+    for _ in range(3):
+        hsq.forward_fused(pl, X, Y, out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y0)
+    hsq.hsq_debug_force_timeout(1, 30)  # the producer issues nothing: the drain's waits run out
+    hsq.forward_fused(pl, X, Y, out=hsq.HSQ_OUT_F32)
+    assert hsq.hsq_get_device_status() == hsq.HSQ_ERR_TIMEOUT
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    hsq.forward_fused(pl, X, Y, out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    assert torch.equal(Y, Y0)
 
 
 def test_invalid_arguments_launch_nothing():

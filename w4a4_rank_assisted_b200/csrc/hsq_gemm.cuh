@@ -54,6 +54,7 @@
 #pragma once
 
 #include "hsq_device.cuh"
+#include "hsq_quant.cuh"
 
 #ifndef HSQ_ONE_PHASE
 #define HSQ_ONE_PHASE 0
@@ -109,11 +110,26 @@ struct GemmArgs {
   const uint8_t* xe;      // pre-expanded row operand (kernels with PRE): [G][rg_r][4][8][16] E4M3
   const uint8_t* we;      // pre-expanded col operand: [G][rg_c][4][8][16]
   int rg_r, rg_c;         // 8-row groups of each (rows padded to whole tiles)
+  // Kernels with FUSED (decode tiles): the activation step runs inside the
+  // kernel.  Its input, and scratch for its codes [M][Kp/2] (which tm_col maps),
+  // its scales [G][ld_c] (= scales_c), the per-chunk U partials [M][nchunks][r],
+  // one copy of U per CTA [grid][M][r] and the grid barrier's two counters; the
+  // stream-K counters (fx_zero_words words) are cleared before the barrier.
+  const __nv_bfloat16* fx_X;   // [M][fx_K]
+  const float* fx_s;           // [fx_K]
+  const __nv_bfloat16* fx_L1;  // [fx_K][r]
+  int fx_K, fx_Kp, fx_group;
+  uint8_t* fx_codes;
+  float* fx_scales;
+  float* fx_upart;
+  float* fx_U;
+  unsigned* fx_bar;
+  int fx_zero_words;
 };
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
           int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false, int CHB_ = 2,
-          int BPG_ = 1, bool PAIR_ = false>
+          int BPG_ = 1, bool PAIR_ = false, bool FUSED_ = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -150,6 +166,10 @@ struct GemmCfg {
   // its own Tensor Memory.  Per CTA and step the operand bytes drop from
   // (128 + BN) to (128 + BN/2) rows' worth, the drain work stays the same.
   static constexpr bool PAIR = PAIR_;
+  // The activation step inside the kernel (decode tiles; launched cooperatively):
+  // see fused_act_phase.
+  static constexpr bool FUSED = FUSED_;
+  static_assert(!FUSED || (SWAP && !PRE && !PAIR), "fused activation step: decode tiles");
   static constexpr int PM = PAIR ? 2 : 1;      // CTAs per tile
   static constexpr int TILE_M = BM * PM;       // tokens per tile
   static constexpr int B_ROWS = BN / PM;       // col-operand rows held by one CTA
@@ -401,6 +421,117 @@ __device__ __forceinline__ bool next_unit(const GemmArgs& a, int k, Unit& u) {
   return true;
 }
 
+// The activation step inside a decode-tile launch (kernels with FUSED).  Every
+// warp of the grid takes (token, 256-channel chunk) items gw, gw + W, ... and
+// computes them as the activation kernel does -- X_hat = X/s, the group absmax,
+// codes and scales, with the same helpers, so the same bits -- writing codes
+// and scales to the scratch and the chunk's U partial, summed over the warp's
+// lanes, to fx_upart.  The stream-K counters are cleared on the way.  Every
+// thread calls it.
+template <int GL>
+__device__ __forceinline__ void fused_act_phase(const GemmArgs& a) {
+  const int lane = lane_id();
+  const int nw = static_cast<int>(blockDim.x >> 5);
+  const int gw = static_cast<int>(blockIdx.x) * nw + static_cast<int>(threadIdx.x >> 5);
+  const int W = static_cast<int>(gridDim.x) * nw;
+  for (int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x); i < a.fx_zero_words;
+       i += static_cast<int>(gridDim.x * blockDim.x))
+    a.ws_counters[i] = 0u;
+  const int M = a.M, K = a.fx_K, Kp = a.fx_Kp, r = a.r;
+  const int nchk = (Kp + 255) >> 8;
+  for (int item = gw; item < M * nchk; item += W) {
+    const int m = item / nchk, c = item - m * nchk;  // warp-uniform
+    const int k0 = c * 256 + lane * 8;
+    const bool real = k0 < K, in_k = k0 < Kp;  // K % 8 == 0: a lane's 8 channels are all real or all padding
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    float sv[8], sz[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sv[e] = 1.f;
+    if (real) {
+      raw = __ldg(reinterpret_cast<const uint4*>(a.fx_X + static_cast<size_t>(m) * K + k0));
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(a.fx_s + k0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(a.fx_s + k0 + 4));
+      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+      sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sz[e] = __frcp_rn(sv[e]);
+    float xh[8];
+    smooth8(raw, sv, sz, real, xh);
+    float sc;
+    const uint32_t packed = quantize8_fast<GL>(xh, sc);
+    if (in_k) {
+      *reinterpret_cast<uint32_t*>(a.fx_codes + static_cast<size_t>(m) * (Kp / 2) + k0 / 2) = packed;
+      if ((lane & (GL - 1)) == 0) {
+        float* srow = a.fx_scales + static_cast<size_t>(k0 / (8 * GL)) * a.ld_c;
+        srow[m] = sc;
+        if (m == M - 1)
+          for (int p = M; p < a.ld_c; ++p) srow[p] = 0.f;  // padding of the group-major layout
+      }
+    }
+    for (int j0 = 0; j0 < r; j0 += 8) {  // the chunk's U partial, 8 ranks at a time
+      float u[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) u[jj] = 0.f;
+      if (real) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const __nv_bfloat16* row = a.fx_L1 + static_cast<size_t>(k0 + e) * r + j0;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            if (j0 + jj < r) u[jj] = fmaf(xh[e], __bfloat162float(__ldg(row + jj)), u[jj]);
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) u[jj] += __shfl_xor_sync(0xffffffffu, u[jj], o);
+      if (lane == 0)
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+          if (j0 + jj < r) a.fx_upart[(static_cast<size_t>(m) * nchk + c) * r + j0 + jj] = u[jj];
+    }
+  }
+}
+
+// Grid-wide barrier of a cooperative launch (every CTA resident), with a time
+// limit.  Counters bar[0] (arrivals) and bar[1] (departures) are zero between
+// launches: the last CTA to leave clears both, after a timeout too.  Every
+// thread calls it; it returns false, with the timeout status raised and the
+// CTA's abort flag set, if the grid did not gather in time.  Writes made before
+// it are visible after it to every CTA, to the async proxy (TMA and bulk copies
+// issued by thread 0) as well.
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, uint64_t limit_ns, volatile int* abort, int* s_ok) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");  // this thread's writes, for async-proxy readers
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    atomicAdd(&bar[0], 1u);
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (v >= gridDim.x) break;
+      __nanosleep(128);
+      if (global_timer_ns() - t0 > limit_ns) {
+        ok = 0;
+        *abort = 1;
+        atomicOr(&g_status, kStatusTimeout);
+        break;
+      }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    if (atomicAdd(&bar[1], 1u) == gridDim.x - 1) {  // every CTA has left the wait
+      atomicExch(&bar[0], 0u);
+      atomicExch(&bar[1], 0u);
+    }
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_row, const __grid_constant__ CUtensorMap tm_col,
@@ -484,31 +615,69 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   // every warp but the producer reads or writes global memory only after the
   // preceding kernel is complete (U, L2, bias, Y, the workspace)
-  if (warp != 0) grid_dep_wait();
+  if (!Cfg::FUSED && warp != 0) grid_dep_wait();
 
   uint32_t issued = 0;  // producer: stages issued (for the teardown drain)
+  uint32_t npre = 0;    // producer: weight tiles requested before the preceding kernel completed
+  // Weights x tokens tiles: the weight tiles of the first STAGES steps are
+  // requested before waiting for the preceding kernel (the packed weights are
+  // never written by the kernel just before this one: the packing kernel does
+  // not let its successor start early).  Their token halves follow once the
+  // tokens' codes exist.
+  auto prefetch_weights = [&]() {
+    if constexpr (Cfg::SWAP) {
+      Unit pu;
+      for (int k = 0; npre < static_cast<uint32_t>(STAGES) && next_unit<GPS, PAIR>(args, k, pu); ++k) {
+        const int r0p = (pu.tile % args.tiles_r) * BM;
+        for (int g = pu.g0; g < pu.g1 && npre < static_cast<uint32_t>(STAGES); g += GPS, ++npre) {
+          mbar_arrive_expect_tx(&full[npre], Cfg::A_PACK + Cfg::B_PACK);
+          tma_load_2d(stage_base + npre * Cfg::STAGE_BYTES, &tm_row, &full[npre], g * Cfg::BPG * 32, r0p);
+        }
+      }
+    }
+  };
+  // FUSED: the activation step, distributed over the grid, then a grid barrier;
+  // U is then summed per CTA (fixed chunk order) into the CTA's own copy.
+  bool fused_ok = true;
+  const float* Uv = args.U;
+  // U: the preceding kernel's (read-only here), or this CTA's own copy (written above)
+  auto load_u = [](const float* p) -> float {
+    if constexpr (Cfg::FUSED) return *p;
+    else return __ldg(p);
+  };
+  if constexpr (Cfg::FUSED) {
+    if (warp == 0 && lane == 0 && !(args.debug_flags & 1)) prefetch_weights();
+    issued = npre;
+    grid_dep_wait();
+    fused_act_phase<(Cfg::BPG == 2 ? 16 : 8)>(args);
+    fused_ok = grid_barrier(args.fx_bar, args.limit_ns, abort_flag, reinterpret_cast<int*>(tmem_slot + 3));
+    if (fused_ok) {
+      const int nchk = (args.fx_Kp + 255) >> 8;
+      float* Uc = args.fx_U + static_cast<size_t>(blockIdx.x) * args.M * args.r;
+      for (int t = threadIdx.x; t < args.M * args.r; t += Cfg::THREADS) {
+        const int m = t / args.r, j = t - (t / args.r) * args.r;
+        float v = 0.f;
+        for (int c = 0; c < nchk; ++c) v += __ldcg(args.fx_upart + (static_cast<size_t>(m) * nchk + c) * args.r + j);
+        Uc[t] = v;
+      }
+      Uv = Uc;
+      __syncthreads();
+    }
+  }
 
-  if (warp == 0) {
+  if (!fused_ok) {
+    // the grid did not gather: no work unit runs; the teardown lets the weight
+    // tiles already requested land
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (Cfg::REALLOC) regs_dealloc<Cfg::REGS_LOW>();
     if (lane == 0 && !(args.debug_flags & 1)) {
-      // Weights x tokens tiles: the weight tiles of the first STAGES steps are
-      // requested before waiting for the preceding kernel (the packed weights
-      // are never written by the kernel just before this one: the packing
-      // kernel does not let its successor start early).  Their activation
-      // halves follow right after the wait, before anything that can give up.
-      uint32_t npre = 0;
-      if constexpr (Cfg::SWAP) {
-        Unit pu;
-        for (int k = 0; npre < static_cast<uint32_t>(STAGES) && next_unit<GPS, PAIR>(args, k, pu); ++k) {
-          const int r0p = (pu.tile % args.tiles_r) * BM;
-          for (int g = pu.g0; g < pu.g1 && npre < static_cast<uint32_t>(STAGES); g += GPS, ++npre) {
-            mbar_arrive_expect_tx(&full[npre], Cfg::A_PACK + Cfg::B_PACK);
-            tma_load_2d(stage_base + npre * Cfg::STAGE_BYTES, &tm_row, &full[npre], g * Cfg::BPG * 32, r0p);
-          }
-        }
+      // (weight tiles first; the token halves follow right after the wait,
+      // before anything that can give up)
+      if constexpr (!Cfg::FUSED) {
+        prefetch_weights();
+        grid_dep_wait();
       }
-      grid_dep_wait();
       grid_dep_launch();
       uint32_t it = 0;
       bool ok = true;
@@ -882,8 +1051,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
               for (int b = 0; b < NBLK; ++b) {
                 const int m = col0 + 8 * b;
-                if (m < args.M) acc2[i * NBLK + b].x = fmaf(__ldg(args.U + static_cast<size_t>(m) * args.r + kk), l2, acc2[i * NBLK + b].x);
-                if (m + 1 < args.M) acc2[i * NBLK + b].y = fmaf(__ldg(args.U + static_cast<size_t>(m + 1) * args.r + kk), l2, acc2[i * NBLK + b].y);
+                if (m < args.M) acc2[i * NBLK + b].x = fmaf(load_u(Uv + static_cast<size_t>(m) * args.r + kk), l2, acc2[i * NBLK + b].x);
+                if (m + 1 < args.M) acc2[i * NBLK + b].y = fmaf(load_u(Uv + static_cast<size_t>(m + 1) * args.r + kk), l2, acc2[i * NBLK + b].y);
               }
             }
           }

@@ -87,6 +87,10 @@ using CfgDec64_64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulator
 using CfgDec16_128 = hsq::GemmCfg<16, 1, 6, true, 2, 2, 4, 10, 10, false, -1, false, 2, 2>;
 using CfgDec32_128 = hsq::GemmCfg<32, 1, 5, true, 2, 2, 2, 10, 9, false, -1, false, 2, 2>;
 using CfgDec64_128 = hsq::GemmCfg<64, 1, 8, true, 1, 2, 2, 6, 12, false, -1, false, 2, 2>;
+// ... and the single-launch forward for up to 16 tokens: the 16-token decode
+// tiles with the activation step inside (cooperative launch)
+using CfgDec16F_64 = hsq::GemmCfg<16, 1, 6, true, 4, 2, 4, 10, 10, false, -1, false, 2, 1, false, true>;
+using CfgDec16F_128 = hsq::GemmCfg<16, 1, 6, true, 2, 2, 4, 10, 10, false, -1, false, 2, 2, false, true>;
 
 #ifndef HSQ_LR_MMA
 #define HSQ_LR_MMA 1  // U L2 + b as a tensor-core step where the kernel supports it
@@ -114,6 +118,28 @@ hsq_status noalloc_scratch(void** out) {
   if (dev < 0 || dev >= kMaxDevices) return HSQ_ERR_UNSUPPORTED;
   NoallocSlot& slot = g_noalloc_slots[dev];
   std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch); });
+  if (slot.err != cudaSuccess || !slot.ptr) return HSQ_ERR_CUDA;
+  *out = slot.ptr;
+  return HSQ_OK;
+}
+
+// Scratch of the single-launch forward's decode-tile form: the grid barrier's
+// counters (the first 256 bytes, zero between launches; nothing else uses them),
+// then per call the stream-K counters and partial tiles, the activation step's
+// codes, scales and U partials, and one copy of U per CTA.
+#ifndef HSQ_FUSED_SCRATCH_BYTES
+#define HSQ_FUSED_SCRATCH_BYTES (8u << 20)
+#endif
+constexpr size_t kFusedScratchBytes = HSQ_FUSED_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_fused_scratch[kFusedScratchBytes];
+NoallocSlot g_fused_slots[kMaxDevices];
+
+hsq_status fused_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HSQ_ERR_UNSUPPORTED;
+  NoallocSlot& slot = g_fused_slots[dev];
+  std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_fused_scratch); });
   if (slot.err != cudaSuccess || !slot.ptr) return HSQ_ERR_CUDA;
   *out = slot.ptr;
   return HSQ_OK;
@@ -260,6 +286,8 @@ int large_workers(int nsm) {
   return n;
 }
 
+void finish_plan(Plan& p, int G, int group, int nsm);
+
 Plan make_plan(int M, int N, int K, int group, int nsm) {
   Plan p{};
   p.group = group;
@@ -297,6 +325,12 @@ Plan make_plan(int M, int N, int K, int group, int nsm) {
     p.tiles_r = (M + CfgLarge64::TILE_M - 1) / CfgLarge64::TILE_M;
     p.tiles_c = (N + p.BN - 1) / p.BN;
   }
+  finish_plan(p, G, group, nsm);
+  return p;
+}
+
+// Work decomposition and workspace sizes of a plan whose kernel and tiles are set.
+void finish_plan(Plan& p, int G, int group, int nsm) {
   const long tiles = static_cast<long>(p.tiles_r) * p.tiles_c;
   p.stages_per_tile = (G + p.gps_stage - 1) / p.gps_stage;
   // Whole tiles per worker (a CTA, or a CTA pair) when they fill the device in
@@ -322,6 +356,18 @@ Plan make_plan(int M, int N, int K, int group, int nsm) {
     p.pre_x_bytes = blocks * p.rg_r * CfgLarge64::E8_SBO;
     p.pre_w_bytes = blocks * p.rg_c * CfgLarge64::E8_SBO;
   }
+}
+
+// The 16-token decode tiles for any M <= 16 (the single-launch forward).
+Plan make_dec16_plan(int M, int N, int K, int group, int nsm) {
+  Plan p{};
+  p.group = group;
+  p.swap = true;
+  p.kind = kDec16;
+  group == 128 ? plan_from<CfgDec16F_128>(p) : plan_from<CfgDec16F_64>(p);
+  p.tiles_r = (N + 127) / 128;
+  p.tiles_c = (M + p.BN - 1) / p.BN;
+  finish_plan(p, groups_of(K, group), group, nsm);
   return p;
 }
 static_assert(CfgLarge64::PRE && CfgLarge128::PRE && CfgLarge64::BN == CfgLarge128::BN &&
@@ -466,6 +512,49 @@ hsq_status launch_gemm(const Plan& p, const CUtensorMap& tr, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
+// The single-launch forward on 16-token decode tiles: the kernel runs the
+// activation step itself, spread over its CTAs, and then waits at a grid
+// barrier, so every CTA must be resident at once -- a cooperative launch, after
+// the occupancy check.
+template <class Cfg>
+hsq_status launch_gemm_fused(const Plan& p, const CUtensorMap& tr, const CUtensorMap& tc, const hsq::GemmArgs& a,
+                             cudaStream_t st) {
+  static_assert(Cfg::FUSED && !Cfg::REALLOC, "fused decode tiles");
+  static std::mutex mu;
+  static int max_blocks[64] = {0};  // resident CTAs per SM, per device (0: not asked yet)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSQ_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return HSQ_ERR_UNSUPPORTED;
+  int nb = 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (max_blocks[dev] == 0) {
+      if (cudaFuncSetAttribute(hsq::w4a4_gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::SMEM_BYTES) != cudaSuccess)
+        return HSQ_ERR_CUDA;
+      int b = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, hsq::w4a4_gemm_kernel<Cfg>, Cfg::THREADS,
+                                                        Cfg::SMEM_BYTES) != cudaSuccess)
+        return HSQ_ERR_CUDA;
+      max_blocks[dev] = b > 0 ? b : -1;
+    }
+    nb = max_blocks[dev];
+  }
+  if (nb <= 0 || p.grid > nb * device_sm_count()) return HSQ_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, hsq::w4a4_gemm_kernel<Cfg>, tr, tc, tr, a) != cudaSuccess) return HSQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
 // `a` has the shape, rows_per_block and pointers set; the ring layout and the
 // wait limit are filled in here.
 template <int MT, int LPG, int RF = -1>
@@ -564,6 +653,103 @@ cudaError_t launch_act_rows(const __nv_bfloat16* X, const float* s, const __nv_b
   return launch_pdl(true, hsq::quantize_act_rows_kernel<R, GL, NW, SUB>, dim3((M + C::RB - 1) / C::RB),
                     dim3(NW * 32), static_cast<size_t>(kSmem), st, X, s, L1, M, K, Kp, ld, codes, scales, U,
                     wait_limit_ns());
+}
+
+// hsq_linear_forward_fused for the shapes the weight stream's fused form does
+// not take (5..16 tokens, or ranks other than 0, 1, 2, 4): 16-token decode
+// tiles with the activation step inside, scratch from g_fused_scratch.
+// Scratch layout of the decode-tile form (byte offsets into g_fused_scratch).
+struct FusedLayout {
+  Plan p;
+  size_t o_cnt, o_part, o_codes, o_sc, o_up, o_u, total;
+};
+FusedLayout fused_dec16_layout(int M, int N, int K, int r, int group, int nsm) {
+  FusedLayout L{};
+  const int G = groups_of(K, group), Kp = G * group;
+  L.p = make_dec16_plan(M, N, K, group, nsm);
+  const int ldx = scales_ld(M), nchk = (Kp + 255) / 256, rr = std::max(r, 1);
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t off = 256;  // [0, 256): the grid barrier's counters
+  L.o_cnt = off;
+  off = up(off + L.p.counters_bytes);
+  L.o_part = off;
+  off = up(off + L.p.partial_bytes);
+  L.o_codes = off;
+  off = up(off + static_cast<size_t>(M) * (Kp / 2));
+  L.o_sc = off;
+  off = up(off + static_cast<size_t>(G) * ldx * 4);
+  L.o_up = off;
+  off = up(off + static_cast<size_t>(M) * nchk * rr * 4);
+  L.o_u = off;
+  off = up(off + static_cast<size_t>(L.p.grid) * M * rr * 4);
+  L.total = off;
+  return L;
+}
+
+// Which form hsq_linear_forward_fused takes (0: none), from the shape alone.
+int fused_form(int M, int N, int K, int r, int group, int nsm) {
+  if (group != 64 && group != 128) return 0;
+  if (M < 1 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim || r < 0 || r > kMaxRank) return 0;
+  if (K % 8 != 0 || N % 8 != 0) return 0;
+  const int G = groups_of(K, group), Kp = G * group;
+  if (M <= 4 && (r == 0 || r == 1 || r == 2 || r == 4) && gemv_plan_layout(M, N, Kp, G, nsm).stages >= 1) return 1;
+  if (M <= 16 && fused_dec16_layout(M, N, K, r, group, nsm).total <= kFusedScratchBytes) return 2;
+  return 0;
+}
+
+hsq_status forward_fused_dec16(const void* X_bf16, const float* s, const void* L1_bf16, const uint8_t* w_codes,
+                               const float* w_scales, const void* L2_bf16, const void* bias_bf16, int M, int N, int K,
+                               int r, int group, void* Y, hsq_out_dtype out, cudaStream_t stream) {
+  const int G = groups_of(K, group), Kp = G * group, nsm = device_sm_count();
+  const FusedLayout FL = fused_dec16_layout(M, N, K, r, group, nsm);
+  const Plan& p = FL.p;
+  const int ldx = scales_ld(M), ldw = scales_ld(N);
+  const size_t o_cnt = FL.o_cnt, o_part = FL.o_part, o_codes = FL.o_codes, o_sc = FL.o_sc, o_up = FL.o_up,
+               o_u = FL.o_u;
+  if (FL.total > kFusedScratchBytes) return HSQ_ERR_UNSUPPORTED;
+  void* scr = nullptr;
+  hsq_status st = fused_scratch(&scr);
+  if (st != HSQ_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(scr);
+
+  hsq::GemmArgs a{};
+  CUtensorMap tm_row, tm_col;
+  a.scales_r = w_scales; a.ld_r = ldw; a.rows_r = N;
+  a.scales_c = reinterpret_cast<float*>(base + o_sc); a.ld_c = ldx; a.rows_c = M;
+  if (!make_codes_map(&tm_row, w_codes, N, Kp, 128, p.bps_stage) ||
+      !make_codes_map(&tm_col, base + o_codes, M, Kp, p.BN, p.bps_stage))
+    return HSQ_ERR_CUDA;
+  a.U = nullptr;  // the kernel's own
+  a.L2 = static_cast<const __nv_bfloat16*>(L2_bf16);
+  a.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+  a.Y = Y;
+  a.out_f32 = out == HSQ_OUT_F32 ? 1 : 0;
+  a.M = M; a.N = N; a.G = G; a.r = r;
+  a.tiles_r = p.tiles_r; a.tiles_c = p.tiles_c;
+  a.stages_per_tile = p.stages_per_tile; a.stream_len = p.stream_len;
+  if (p.stream_len > 0) {
+    a.ws_counters = reinterpret_cast<unsigned*>(base + o_cnt);
+    a.ws_partials = reinterpret_cast<float*>(base + o_part);
+    a.fx_zero_words = static_cast<int>(p.counters_bytes / 4);
+  }
+  a.fx_X = static_cast<const __nv_bfloat16*>(X_bf16);
+  a.fx_s = s;
+  a.fx_L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
+  a.fx_K = K; a.fx_Kp = Kp; a.fx_group = group;
+  a.fx_codes = base + o_codes;
+  a.fx_scales = reinterpret_cast<float*>(base + o_sc);
+  a.fx_upart = reinterpret_cast<float*>(base + o_up);
+  a.fx_U = reinterpret_cast<float*>(base + o_u);
+  a.fx_bar = reinterpret_cast<unsigned*>(base);
+  a.lr_mma = 0;
+  a.limit_ns = wait_limit_ns();
+  if (t_debug_flags) {
+    a.debug_flags = t_debug_flags;
+    a.limit_ns = static_cast<uint64_t>(t_debug_limit_ms > 0 ? t_debug_limit_ms : 50) * 1000000ull;
+    t_debug_flags = 0;
+  }
+  return group == 128 ? launch_gemm_fused<CfgDec16F_128>(p, tm_row, tm_col, a, stream)
+                      : launch_gemm_fused<CfgDec16F_64>(p, tm_row, tm_col, a, stream);
 }
 
 extern "C" {
@@ -970,8 +1156,14 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
   const int G = groups_of(K, group), Kp = G * group;
   const int mt = gemv_mt(M);
   const int nsm = device_sm_count();
-  if (M > 4 || !(r == 0 || r == 1 || r == 2 || r == 4) || gemv_plan_layout(M, N, Kp, G, nsm).stages < 1)
-    return HSQ_ERR_UNSUPPORTED;
+  // up to 4 tokens at ranks 0, 1, 2, 4 with the block's rows in shared memory:
+  // the weight stream, each block repeating the activation step; else up to 16
+  // tokens: the decode tiles, the step spread over the grid
+  const int form = fused_form(M, N, K, r, group, nsm);
+  if (form == 0) return HSQ_ERR_UNSUPPORTED;
+  if (form == 2)
+    return forward_fused_dec16(X_bf16, s, L1_bf16, w_codes, w_scales, L2_bf16, bias_bf16, M, N, K, r, group, Y, out,
+                               stream);
   Plan p{};
   p.kind = kGemv;
   p.tiles_r = gemv_rows_per_block(N, nsm);
@@ -1005,6 +1197,8 @@ hsq_status hsq_linear_forward_fused(const void* X_bf16, const float* s, const vo
 #undef HSQ_FUSED_R
 #undef HSQ_FUSED
 }
+
+int hsq_fused_form(int M, int N, int K, int r, int group) { return fused_form(M, N, K, r, group, device_sm_count()); }
 
 // ------------------------------------------------------------------ NVFP4 variant
 // Block-scaled GEMM tile: 128 tokens x HSQ_FP4_BN outputs (hsq_fp4.cuh).

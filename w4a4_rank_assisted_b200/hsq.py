@@ -35,7 +35,7 @@ EXPORTED = (
     "hsq_num_groups", "hsq_codes_bytes", "hsq_scales_ld", "hsq_scales_bytes",
     "hsq_workspace_bytes", "hsq_pack_weights", "hsq_quantize_act",
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
-    "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused",
+    "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused", "hsq_fused_form",
     "hsq_lowrank_workspace_bytes", "hsq_lowrank_init",
     "hsq_fp4_codes_bytes", "hsq_fp4_scales_bytes", "hsq_fp4_pack_weights", "hsq_fp4_quantize_act",
     "hsq_fp4_linear_forward",
@@ -82,6 +82,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_linear_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
     lib.hsq_linear_forward_fused.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]
     lib.hsq_linear_forward_fused.restype = i
+    lib.hsq_fused_form.argtypes = [i, i, i, i, i]
+    lib.hsq_fused_form.restype = i
     lib.hsq_lowrank_workspace_bytes.argtypes = [i, i, i]; lib.hsq_lowrank_workspace_bytes.restype = sz
     lib.hsq_lowrank_init.argtypes = [vp, vp, i, i, i, i, c.c_ulonglong, vp, vp, vp, sz, vp]
     lib.hsq_lowrank_init.restype = i
@@ -225,12 +227,54 @@ def stream_smem_fits(M: int, N: int, K: int, group: int = GROUP, nsm: Optional[i
     return min_stages * rs * rowbytes <= budget
 
 
+def _dec16_scratch_bytes(M: int, N: int, K: int, r: int, group: int, nsm: int) -> int:
+    """Bytes of the library's array that the decode-tile form of
+    hsq_linear_forward_fused uses for this shape (restated from the planner: the
+    barrier's 256 bytes, stream-K counters and partials, codes, scales, U
+    partials and per-CTA copies of U, each rounded up to 256)."""
+    up = lambda v: -(-v // 256) * 256
+    G = -(-K // group)
+    Kp = G * group
+    gps = 4 if group == 64 else 2          # scale groups per pipeline stage
+    tiles = -(-N // 128)                   # 128 weight rows x 16 tokens
+    S = -(-G // gps)
+    waves = -(-tiles // nsm)
+    fill = tiles / (waves * nsm)
+    total = tiles * S
+    if (tiles >= nsm and fill >= 0.9) or total <= nsm or total >= (1 << 30):
+        grid = min(tiles, nsm)
+    else:
+        sl = -(-total // nsm)
+        grid = -(-total // sl)
+    counters = up(tiles * 4 * 4)
+    partials = grid * 2 * 16 * 128 * 4
+    ldx = (M + 3) // 4 * 4
+    rr = max(r, 1)
+    nchk = -(-Kp // 256)
+    off = 256
+    for b in (counters, partials, M * (Kp // 2), G * ldx * 4, M * nchk * rr * 4, grid * M * rr * 4):
+        off = up(off + b)
+    return off
+
+
+FUSED_SCRATCH_BYTES = 8 << 20
+
+
 def fused_supported(M: int, K: int, r: int, group: int = GROUP, N: int = 8, nsm: Optional[int] = None) -> bool:
     """Whether hsq_linear_forward_fused takes this shape (the limits stated in
-    include/hsq.h: M <= 4, r in {0, 1, 2, 4}, and the stream's shared memory)."""
-    if M < 1 or M > 4 or r not in (0, 1, 2, 4) or group not in (64, 128):
+    include/hsq.h, restated without a library call so it can be asked without a
+    GPU): the weight stream for M <= 4, r in {0, 1, 2, 4} and a block's shared
+    memory, else the decode tiles for M <= 16, r <= 32 and the library's array."""
+    if M < 1 or M > 16 or r < 0 or r > 32 or group not in (64, 128) or K % 8 or N % 8:
         return False
-    return stream_smem_fits(M, N, K, group, nsm)
+    nsm = nsm or _sm_count()
+    if M <= 4 and r in (0, 1, 2, 4) and stream_smem_fits(M, N, K, group, nsm):
+        return True
+    return _dec16_scratch_bytes(M, N, K, r, group, nsm) <= FUSED_SCRATCH_BYTES
+
+
+def hsq_fused_form(M: int, N: int, K: int, r: int, group: int = GROUP) -> int:
+    return int(load().hsq_fused_form(M, N, K, r, group))
 
 
 def hsq_lowrank_workspace_bytes(N: int, K: int, r: int) -> int:
