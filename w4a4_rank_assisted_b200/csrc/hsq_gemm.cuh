@@ -432,7 +432,8 @@ template <int GL>
 __device__ __forceinline__ void fused_act_phase(const GemmArgs& a) {
   const int lane = lane_id();
   const int nw = static_cast<int>(blockDim.x >> 5);
-  const int gw = static_cast<int>(blockIdx.x) * nw + static_cast<int>(threadIdx.x >> 5);
+  // items spread over the CTAs first (warp w of CTA b is global warp w * grid + b)
+  const int gw = static_cast<int>(threadIdx.x >> 5) * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
   const int W = static_cast<int>(gridDim.x) * nw;
   for (int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x); i < a.fx_zero_words;
        i += static_cast<int>(gridDim.x * blockDim.x))
@@ -477,9 +478,16 @@ __device__ __forceinline__ void fused_act_phase(const GemmArgs& a) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const __nv_bfloat16* row = a.fx_L1 + static_cast<size_t>(k0 + e) * r + j0;
+          if (r % 8 == 0) {  // ranks j0 .. j0+7 of channel k0+e: one 16-byte load
+            float f[8];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(row)), f);
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj)
-            if (j0 + jj < r) u[jj] = fmaf(xh[e], __bfloat162float(__ldg(row + jj)), u[jj]);
+            for (int jj = 0; jj < 8; ++jj) u[jj] = fmaf(xh[e], f[jj], u[jj]);
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              if (j0 + jj < r) u[jj] = fmaf(xh[e], __bfloat162float(__ldg(row + jj)), u[jj]);
+          }
         }
       }
 #pragma unroll
@@ -637,7 +645,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   };
   // FUSED: the activation step, distributed over the grid, then a grid barrier;
-  // U is then summed per CTA (fixed chunk order) into the CTA's own copy.
+  // the drain warps then sum U (fixed chunk order) into the CTA's own copy while
+  // the pipeline fills.
   bool fused_ok = true;
   const float* Uv = args.U;
   // U: the preceding kernel's (read-only here), or this CTA's own copy (written above)
@@ -651,18 +660,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     grid_dep_wait();
     fused_act_phase<(Cfg::BPG == 2 ? 16 : 8)>(args);
     fused_ok = grid_barrier(args.fx_bar, args.limit_ns, abort_flag, reinterpret_cast<int*>(tmem_slot + 3));
-    if (fused_ok) {
-      const int nchk = (args.fx_Kp + 255) >> 8;
-      float* Uc = args.fx_U + static_cast<size_t>(blockIdx.x) * args.M * args.r;
-      for (int t = threadIdx.x; t < args.M * args.r; t += Cfg::THREADS) {
-        const int m = t / args.r, j = t - (t / args.r) * args.r;
-        float v = 0.f;
-        for (int c = 0; c < nchk; ++c) v += __ldcg(args.fx_upart + (static_cast<size_t>(m) * nchk + c) * args.r + j);
-        Uc[t] = v;
-      }
-      Uv = Uc;
-      __syncthreads();
-    }
+    Uv = args.fx_U + static_cast<size_t>(blockIdx.x) * args.M * args.r;  // summed by the drain warps
   }
 
   if (!fused_ok) {
@@ -982,6 +980,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ------------------------------------------------------------ drain + epilogue
     if (Cfg::REALLOC) regs_alloc<Cfg::REGS_HIGH>();
     const int dw = warp - (2 + Cfg::NUM_UNPACK_WARPS);
+    if constexpr (Cfg::FUSED) {
+      // this CTA's copy of U: the chunks' partials in a fixed order; the drain
+      // warps alone read it (named barrier 1 over them)
+      const int nchk = (args.fx_Kp + 255) >> 8;
+      float* Uc = const_cast<float*>(Uv);
+      for (int t = dw * 32 + lane; t < args.M * args.r; t += 32 * Cfg::NUM_DRAIN_WARPS) {
+        const int m = t / args.r, j = t - (t / args.r) * args.r;
+        float v = 0.f;
+        for (int c = 0; c < nchk; ++c) v += __ldcg(args.fx_upart + (static_cast<size_t>(m) * nchk + c) * args.r + j);
+        Uc[t] = v;
+      }
+      named_bar_sync(1, 32 * Cfg::NUM_DRAIN_WARPS);
+    }
     const int q = warp & 3;            // TMEM lane quadrant
     const int h = dw >> 2;             // column slice
     const int qd = lane >> 2, qc = lane & 3;

@@ -148,6 +148,9 @@ hsq_status fused_scratch(void** out) {
 #ifndef HSQ_PDL
 #define HSQ_PDL 1  // launch with programmatic stream serialization (see grid_dep_wait)
 #endif
+#ifndef HSQ_FUSED_PDL
+#define HSQ_FUSED_PDL 1  // ... the cooperative decode tiles too, where the driver accepts it
+#endif
 
 // Launch `kernel` so that it may start while the preceding kernel in the stream
 // is still running; the kernel itself waits (grid_dep_wait) before touching
@@ -546,10 +549,26 @@ hsq_status launch_gemm_fused(const Plan& p, const CUtensorMap& tr, const CUtenso
   cfg.blockDim = dim3(Cfg::THREADS);
   cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  // with an early start where the driver takes one (the kernel requests only
+  // weight tiles before its grid_dep_wait), else without
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
+  static int pdl_ok[64] = {0};  // 0: untried, 1: accepted, -1: refused
+  if (HSQ_PDL && HSQ_FUSED_PDL && pdl_ok[dev] >= 0) {
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, hsq::w4a4_gemm_kernel<Cfg>, tr, tc, tr, a);
+    if (e == cudaSuccess) {
+      pdl_ok[dev] = 1;
+      return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+    }
+    if (pdl_ok[dev] == 1) return HSQ_ERR_CUDA;
+    (void)cudaGetLastError();  // refused at the first try: launch without the early start from now on
+    pdl_ok[dev] = -1;
+  }
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, hsq::w4a4_gemm_kernel<Cfg>, tr, tc, tr, a) != cudaSuccess) return HSQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
