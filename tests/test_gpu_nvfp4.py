@@ -112,6 +112,11 @@ SHAPES = [
     (64, 2048, 384, 32),   # largest rank
     (300, 640, 512, 0),    # no low-rank branch
     (97, 192, 136, 15),
+    # the many-row activation kernel in its NVFP4 form
+    (4150, 1160, 136, 4),  # ragged last block of rows, K pads to 1216
+    (4150, 264, 136, 0),
+    (4200, 520, 136, 1),
+    (4160, 392, 264, 2),
 ]
 
 
@@ -123,8 +128,9 @@ def test_nvfp4_layer_matches_oracle(M, K, N, r, out):
     _check(layer, pl, act, Y, out, f"nvfp4 {M}x{K}x{N} r{r}")
 
 
-def test_nvfp4_zero_token_zero_block_and_zero_input():
-    layer = make_layer(_spec(40, 192, 128, 4, seed=9))
+@pytest.mark.parametrize("M", [40, 4160])  # 4160: the many-row activation kernel
+def test_nvfp4_zero_token_zero_block_and_zero_input(M):
+    layer = make_layer(_spec(M, 192, 128, 4, seed=9))
     X = layer.X.clone()
     X[3] = 0            # an all-zero token: every block scale 0, codes 0
     X[7, 16:32] = 0     # one all-zero 16-value block
@@ -159,3 +165,39 @@ def test_nvfp4_full_size_flux_mlp_up_sampled_rows():
     assert np.array_equal(f(act.x_codes)[rows], packed_codes(xc[rows], spec.K))
     Y_ref = F.nvfp4_linear_forward(xc[rows], xs[rows], xg, U[rows], wc, ws, wg, f(layer.L2), None, spec.K)
     check_y(f(Y)[rows], Y_ref, False, "nvfp4 FLUX MLP up")
+
+
+@pytest.mark.parametrize("huge", [False, True])  # values above 2^100 set g for the whole tensor
+def test_nvfp4_extreme_values_and_smoothing_factors(huge):
+    """Blocks that mix a normal absmax with bf16 subnormals and values below
+    2^-100, blocks of such tiny values only, values above 2^100, and channels
+    whose smoothing factor lies outside [2^-24, 2^24] (last 256-channel chunk
+    only), at enough rows for the many-row kernel: codes, E4M3 scales and the
+    tensor scale bit for bit."""
+    rng = np.random.default_rng(4)
+    M, K, N, r = 4400, 1024, 128, 4
+    layer = make_layer(_spec(M, K, N, r, seed=13))
+    X = layer.X.float().numpy()
+    tiny = np.array([2.0 ** -133, 2.0 ** -126, 2.0 ** -110, 2.0 ** -101, 2.0 ** -100], dtype=np.float32)
+    sign = lambda n: rng.choice(np.array([-1.0, 1.0], dtype=np.float32), n)
+    for m in range(0, M, 7):
+        kind = (m // 7) % 4
+        if kind == 0:
+            idx = rng.choice(768, 30, replace=False)
+            X[m, idx] = rng.choice(tiny, 30) * sign(30)
+        elif kind == 1:
+            b = rng.integers(48)
+            X[m, b * 16:(b + 1) * 16] = rng.choice(tiny, 16) * sign(16)
+        elif kind == 2 and huge:
+            idx = rng.choice(768, 2, replace=False)
+            X[m, idx] = (2.0 ** rng.uniform(100.0, 110.0, 2)).astype(np.float32) * sign(2)
+    s = layer.s.float().numpy().copy()
+    s[900:904] = np.array([2.0 ** -30, 2.0 ** -25, 2.0 ** 25, 2.0 ** 30], dtype=np.float32)
+    layer.X = torch.tensor(X).to(torch.bfloat16)
+    layer.s = torch.tensor(s)
+    pl, act, Y = _run(layer, hsq.HSQ_OUT_F32)
+    f = to_np
+    xc, xs, xg, U = F.nvfp4_quantize_act(f(layer.X), f(layer.s), f(layer.L1))
+    assert np.float32(f(act.x_gs)[0]) == xg
+    assert np.array_equal(f(act.x_codes), packed_codes(xc, K))
+    assert np.array_equal(f(act.x_sf), sf_atoms(xs, M, K))

@@ -651,9 +651,9 @@ BlasSlot g_blas[kMaxDevices];
 
 // The many-row activation kernel: its X ring is dynamic shared memory (set once
 // per device and instantiation).
-template <int R, int GL, int NW, int SUB>
+template <int R, int GL, int NW, int SUB, bool FP4 = false>
 cudaError_t launch_act_rows(const __nv_bfloat16* X, const float* s, const __nv_bfloat16* L1, int M, int K, int Kp,
-                            int ld, uint8_t* codes, float* scales, float* U, cudaStream_t st) {
+                            int ld, uint8_t* codes, float* scales, float* U, cudaStream_t st, float* gs = nullptr) {
   using C = hsq::ActRowsCfg<NW, SUB>;
   constexpr int kSmem = C::STAGES * C::STAGE_BYTES;
   static std::mutex mu;
@@ -663,15 +663,15 @@ cudaError_t launch_act_rows(const __nv_bfloat16* X, const float* s, const __nv_b
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(hsq::quantize_act_rows_kernel<R, GL, NW, SUB>,
+      const cudaError_t e = cudaFuncSetAttribute(hsq::quantize_act_rows_kernel<R, GL, NW, SUB, FP4>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
       if (e != cudaSuccess) return e;
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
   }
-  return launch_pdl(true, hsq::quantize_act_rows_kernel<R, GL, NW, SUB>, dim3((M + C::RB - 1) / C::RB),
+  return launch_pdl(!FP4, hsq::quantize_act_rows_kernel<R, GL, NW, SUB, FP4>, dim3((M + C::RB - 1) / C::RB),
                     dim3(NW * 32), static_cast<size_t>(kSmem), st, X, s, L1, M, K, Kp, ld, codes, scales, U,
-                    wait_limit_ns());
+                    wait_limit_ns(), gs);
 }
 
 // hsq_linear_forward_fused for the shapes the weight stream's fused form does
@@ -1281,10 +1281,11 @@ hsq_status hsq_fp4_quantize_act(const void* X_bf16, const float* s, const void* 
   const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
   float* sf = reinterpret_cast<float*>(x_sf);
   if (cudaMemsetAsync(x_gs, 0, 2 * sizeof(float), stream) != cudaSuccess) return HSQ_ERR_CUDA;
-  const long groups = static_cast<long>(M) * (K / 8);
-  const int ablocks = static_cast<int>(std::min<long>(4l * device_sm_count(), (groups + 255) / 256));
-  if (launch_pdl(false, hsq::nvfp4_act_amax_kernel, dim3(ablocks), dim3(256), 0, stream, X, s, M, K, x_gs) !=
-      cudaSuccess)
+  // the tensor absmax from column maxima: about four blocks of rows per SM
+  const int nsm = device_sm_count();
+  const int rpb = std::max(1, (M + 4 * nsm - 1) / (4 * nsm));
+  if (launch_pdl(false, hsq::nvfp4_act_colmax_kernel, dim3((M + rpb - 1) / rpb), dim3(128), 0, stream, X, s, M, K,
+                 rpb, x_gs) != cudaSuccess)
     return HSQ_ERR_CUDA;
   cudaError_t lerr = cudaSuccess;
 #define HSQ_FP4_ACT(RV, SM)                                                                                \
@@ -1305,6 +1306,14 @@ hsq_status hsq_fp4_quantize_act(const void* X_bf16, const float* s, const void* 
   }
   if (M <= 64) {
     HSQ_FP4_RANKS(true)
+  } else if (HSQ_ACT_ROWS && (r <= 2 || r == 4) && M >= HSQ_ACT_ROWS16_MIN * nsm) {
+    // many rows: the row-owning kernel in its NVFP4 form
+    switch (r) {
+      case 0: lerr = launch_act_rows<0, 2, 8, 2, true>(X, s, L1, M, K, Kq, 0, x_codes, sf, U, stream, x_gs); break;
+      case 1: lerr = launch_act_rows<1, 2, 8, 2, true>(X, s, L1, M, K, Kq, 0, x_codes, sf, U, stream, x_gs); break;
+      case 2: lerr = launch_act_rows<2, 2, 8, 2, true>(X, s, L1, M, K, Kq, 0, x_codes, sf, U, stream, x_gs); break;
+      default: lerr = launch_act_rows<4, 2, 8, 2, true>(X, s, L1, M, K, Kq, 0, x_codes, sf, U, stream, x_gs); break;
+    }
   } else {
     HSQ_FP4_RANKS(false)
   }

@@ -229,6 +229,44 @@ __global__ void __launch_bounds__(256) nvfp4_act_amax_kernel(const __nv_bfloat16
   if (lane == 0 && amax > 0.f) atomicMax(reinterpret_cast<unsigned int*>(gs + 1), __float_as_uint(amax));
 }
 
+// The same absmax from column maxima: max over (m, k) of RN(|x[m,k]| / s[k]) is
+// max over k of RN(max_m |x[m,k]| / s[k]), because a correctly rounded quotient
+// does not decrease as its dividend grows (s > 0).  Block b takes a run of rows;
+// each thread keeps the packed bf16 maxima of |x| over those rows for its 8
+// channels at a time, then divides them by s (IEEE) and folds the block's
+// maximum into gs[1] as nvfp4_act_amax_kernel does.
+__global__ void __launch_bounds__(128) nvfp4_act_colmax_kernel(const __nv_bfloat16* __restrict__ X,
+                                                               const float* __restrict__ s, int M, int K,
+                                                               int rows_per_block, float* gs) {
+  grid_dep_wait();  // X may come from the preceding kernel
+  const int m0 = blockIdx.x * rows_per_block, m1 = min(M, m0 + rows_per_block);
+  float amax = 0.f;
+  for (int cg = threadIdx.x; cg < K / 8; cg += blockDim.x) {
+    __nv_bfloat162 mx[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mx[i] = __floats2bfloat162_rn(0.f, 0.f);
+    const uint4* col = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m0) * K) + cg;
+    for (int m = m0; m < m1; ++m, col += K / 8) {
+      const uint4 raw = __ldg(col);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = __hmax2(mx[i], __habs2(h[i]));
+    }
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + cg * 8));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + cg * 8 + 4));
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(mx[i]);
+      amax = fmaxf(amax, __fdiv_rn(f.x, sv[2 * i]));
+      amax = fmaxf(amax, __fdiv_rn(f.y, sv[2 * i + 1]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0 && amax > 0.f) atomicMax(reinterpret_cast<unsigned int*>(gs + 1), __float_as_uint(amax));
+}
+
 // ---------------------------------------------------------------------------
 // Weight packing (offline): R[n,k] = fp32(W[n,k]*s[k] - sum_j L1[k,j]*L2[j,n]),
 // the sum in fp64 for j = 0..r-1 with every multiply and add rounded on its own
@@ -691,12 +729,44 @@ __device__ __forceinline__ uint32_t quantize8_int4_ranged(const float (&v)[8], f
   return (acc - int4_pack_bias()) ^ 0x88888888u;
 }
 
-template <int R, int GL, int NW, int SUB>
+// NVFP4 codes of a lane's 8 values (half of a 16-value block; both lanes of the
+// block pass the same bmax, which lies in [2^-60, 2^75]), g > 0, z6 = RN(1/sixg):
+// sf = E4M3(RN(bmax / sixg)), the quotient by Markstein's correction; the codes
+// E2M1(RN(v / fp32(b g))) by the correction against RN(1 / fp32(b g)).
+__device__ __forceinline__ uint32_t quantize8_nvfp4_ranged(const float (&v)[8], float bmax, float g, float sixg,
+                                                           float z6, uint32_t& sf) {
+  const float q = __fmul_rn(bmax, z6);
+  sf = f32_to_e4m3_rn_sat(__fmaf_rn(__fmaf_rn(-q, sixg, bmax), z6, q));
+  const float denom = __fmul_rn(e4m3_to_f32(sf), g);
+  if (denom == 0.f) return 0u;
+  const float z = __frcp_rn(denom);
+  const float nd = -denom;
+  float t[8];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    float q0, q1, r0, r1;
+    fmul2(q0, q1, v[2 * p], v[2 * p + 1], z, z);
+    ffma2(r0, r1, q0, q1, nd, nd, v[2 * p], v[2 * p + 1]);
+    ffma2(t[2 * p], t[2 * p + 1], r0, r1, z, z, q0, q1);
+  }
+  return f32x8_to_e2m1(t);
+}
+
+// FP4 = true: the NVFP4 form (GL = 2 lanes per 16-value block; `scales` taken
+// as the bytes of the NVFP4 scale layout, `ld` unused; g from the absmax in
+// gs[1], written to gs[0] by the first block).  A block takes the fast path when
+// its absmax lies in [2^-60, 2^75]: the block scale is then E4M3(RN(bmax / 6g))
+// with the quotient by Markstein's correction against RN(1/(6g)) (a quotient
+// too small to be normal rounds to E4M3 zero either way), the divisor
+// fp32(b g) is 0 or at least bmax / 12, so elements below 2^-100 give
+// quotients far below 1/4 (E2M1 code 0 on both sides), and the codes are the
+// E2M1 rounding of the corrected quotients.
+template <int R, int GL, int NW, int SUB, bool FP4 = false>
 __global__ void __launch_bounds__(NW * 32, 16 / NW)
     quantize_act_rows_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
                              const __nv_bfloat16* __restrict__ L1, int M, int K, int Kp, int ld,
                              uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U,
-                             uint64_t limit_ns) {
+                             uint64_t limit_ns, float* gs = nullptr) {
   static_assert(R >= 0 && R <= 4 && R != 3, "ranks 0, 1, 2 and 4");
   static_assert(NW <= 8, "one byte per warp in an 8-byte flag word");
   using C = ActRowsCfg<NW, SUB>;
@@ -728,7 +798,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     fence_mbar_init();
   }
   __syncthreads();
-  grid_dep_wait();  // X may come from the preceding kernel
+  grid_dep_wait();  // X (and for FP4 the absmax) may come from the preceding kernel
+  float g = 0.f, sixg = 0.f, z6 = 0.f;
+  if constexpr (FP4) {
+    g = nvfp4_tensor_scale(gs[1]);
+    sixg = __fmul_rn(6.0f, g);
+    z6 = sixg > 0.f ? __frcp_rn(sixg) : 0.f;
+    if (blockIdx.x == 0 && tid == 0) gs[0] = g;
+  }
   const bool early = gridDim.x <= 64;
   if (early && tid == 0) grid_dep_launch();
   const WaitPolicy wp{limit_ns, &abort_flag};
@@ -882,7 +959,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
       for (int i = 0; i < SUB; ++i)
         bad |= (mw + i < M) && in_k && (sbad || !(amax[i] >= 0x1p-60f && amax[i] <= 0x1p75f));
       uint32_t packed[SUB];
-      float sc[SUB];
+      float sc[SUB];      // INT4: the group scales
+      uint32_t sfb[SUB];  // FP4: the E4M3 block scales
       if (__any_sync(0xffffffffu, bad)) {
         // the exact path: IEEE quotients (-ns = s; padding lanes read zeros)
 #pragma unroll
@@ -891,11 +969,15 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
           bf16x8_to_f32(*reinterpret_cast<const uint4*>(stage + i * 512), x);
 #pragma unroll
           for (int e = 0; e < 8; ++e) xh[i][e] = real ? __fdiv_rn(x[e], -ns[e]) : 0.f;
-          packed[i] = quantize8<GL>(xh[i], sc[i]);
+          if constexpr (FP4) packed[i] = quantize8_nvfp4(xh[i], g, sixg, sfb[i]);
+          else packed[i] = quantize8<GL>(xh[i], sc[i]);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < SUB; ++i) packed[i] = quantize8_int4_ranged(xh[i], amax[i], sc[i]);
+        for (int i = 0; i < SUB; ++i) {
+          if constexpr (FP4) packed[i] = quantize8_nvfp4_ranged(xh[i], amax[i], g, sixg, z6, sfb[i]);
+          else packed[i] = quantize8_int4_ranged(xh[i], amax[i], sc[i]);
+        }
       }
       if constexpr (R > 0) {
         float lp[8 * RT];
@@ -913,7 +995,19 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
               ffma2(acc[i][j].x, acc[i][j].y, xh[i][2 * p], xh[i][2 * p + 1], lp[(p * R + j) * 2],
                     lp[(p * R + j) * 2 + 1], acc[i][j].x, acc[i][j].y);
       }
-      if (in_k) {
+      if constexpr (FP4) {
+        // the four block scales of each 64-wide chunk: one word on lane 8p
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) {
+          const uint32_t word = gather_sf_word(sfb[i]);
+          if (in_k && mw + i < M) {
+            *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(mw + i) * (Kp / 2) + k0 / 2) = packed[i];
+            if ((lane & 7) == 0)
+              *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(scales) +
+                                           nvfp4_sf_word_offset(mw + i, k0 / 64, Kp / 64)) = word;
+          }
+        }
+      } else if (in_k) {
 #pragma unroll
         for (int i = 0; i < SUB; ++i)
           if (mw + i < M)
