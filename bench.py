@@ -334,7 +334,10 @@ def _sources_sha() -> str:
 # DRAM read + write bytes per launch of the dominant kernel (mean over the
 # step's layers) from one ncu capture, keyed by workload, with the hash of the
 # CUDA sources it was captured from; any other build reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # w4a4_gemm_kernel, FLUX.1 block: 85.6 / 121.7 / 228.2 MB for qkv / MLP up / MLP down
+    "flux_block_r4": ("19d684b9c0ecec1b", 145172565.0),
+}
 
 
 class Workload:
@@ -580,7 +583,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    W = Workload(hsq, specs, dev, host_buffers=True)
+    W = Workload(hsq, specs, dev, host_buffers=True, fused=False if args.no_fused else None)
     layers = W.layers
     W.prepare_steps(args.warmup)
 
@@ -621,6 +624,8 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             stream.wait_event(ev)
             if W.fused:
                 hsq.forward_fused(L["pl"], L["X"], L["Y"], stream=stream)
+            elif W.fp4:
+                hsq.fp4_forward(L["pl"], L["X"], L["act"], L["Y"], stream=stream)
             else:
                 hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
             done = torch.cuda.Event()
@@ -730,6 +735,8 @@ def main():
     ap.add_argument("--workload", default="flux_block_r4", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-size sub-measurements")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="time the two calls (activation step, forward) even where the single launch applies")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3
