@@ -335,8 +335,8 @@ def _sources_sha() -> str:
 # step's layers) from one ncu capture, keyed by workload, with the hash of the
 # CUDA sources it was captured from; any other build reports null.
 NCU_TRAFFIC = {
-    # w4a4_gemm_kernel, FLUX.1 block: 85.6 / 121.7 / 228.2 MB for qkv / MLP up / MLP down
-    "flux_block_r4": ("19d684b9c0ecec1b", 145172565.0),
+    # w4a4_gemm_kernel, FLUX.1 block: 86.5 / 121.6 / 233.7 MB for qkv / MLP up / MLP down
+    "flux_block_r4": ("5bfd2a685728f47c", 147274666.7),
 }
 
 
@@ -359,6 +359,8 @@ class Workload:
                     act = hsq.Fp4ActBuffers(spec.M, spec.K, spec.r, dev)
                 else:
                     pl = hsq.PackedLinear(d(lay.W), d(lay.s), L1, L2, None, group=spec.group)
+                    if self.expands(spec):
+                        pl.expand()  # the weights' E4M3 copy, made once (offline), as a deployment would
                     act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
                 Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
                 out.append(dict(spec=spec, pl=pl, X=d(lay.X), act=act, Y=Y, ws=pl.workspace(spec.M)))
@@ -405,6 +407,13 @@ class Workload:
             a, pl = L["act"], L["pl"]
             self.hsq.hsq_fp4_linear_forward(a.x_codes, a.x_sf, a.x_gs, a.U, pl.w_codes, pl.w_sf, pl.w_gs, pl.L2, None,
                                             s.M, s.N, s.K, s.r, L["Y"], stream=st)
+            return
+        if L["pl"].w_e4m3 is not None:
+            self.hsq.hsq_linear_forward_pre(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
+                                            L["pl"].w_scales, L["pl"].w_e4m3, L["pl"].L2, None, s.M, s.N, s.K, s.r,
+                                            L["Y"], workspace=L["ws"],
+                                            ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
+                                            group=s.group, stream=st)
             return
         self.hsq.hsq_linear_forward(L["act"].x_codes, L["act"].x_scales, L["act"].U, L["pl"].w_codes,
                                     L["pl"].w_scales, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
@@ -476,14 +485,14 @@ class Workload:
             elif s.fmt == "nvfp4":
                 n += 2 + (1 if s.M % 128 else 0) + 1
             else:
-                n += 1 + (3 if self.expands(s) else 1)
+                n += 1 + (2 if self.expands(s) else 1)
         return n
 
     @staticmethod
     def expands(s):
-        """hsq_linear_forward expands both code matrices to E4M3 tiles ahead of
-        the GEMM (two more launches) for more than 256 tokens, or more than 64 at
-        groups of 128."""
+        """For more than 256 tokens, or more than 64 at groups of 128, the GEMM
+        reads E4M3-expanded operands: the weights' copy is made once at load
+        (PackedLinear.expand), the activations' per call (one more launch)."""
         return s.fmt == "int4" and (s.M > 256 or (s.M > 64 and s.group == 128))
 
     def kernel_times(self):
@@ -512,7 +521,7 @@ class Workload:
                     call = lambda i, st: self.launch_gemm(self.replicas[i % self.nrep][li], st)
                     d["gemm_kernel_us"], _ = time_kernel_nodes(call, self.gstream, "w4a4_gemm_kernel", reps)
                     e_us, e_n = time_kernel_nodes(call, self.gstream, "expand_e4m3_kernel", reps)
-                    d["expand_us"] = e_us * e_n  # both launches of one call
+                    d["expand_us"] = e_us * e_n  # the call's expansion launches
                 else:
                     d["gemm_kernel_us"] = d["call_us"]
             out.append(d)
@@ -611,17 +620,29 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     copy_in = torch.cuda.Stream(device=dev)
     copy_out = torch.cuda.Stream(device=dev)
 
+    # Steps are pipelined as a serving loop would run them: a layer's next input
+    # copy waits only until its compute has read X, and its next compute only
+    # until its previous Y is on the host, so one step's output copies overlap
+    # the next step's input copies (both PCIe directions busy).  Every step still
+    # copies all its inputs in and all its outputs out inside the timed region,
+    # which ends once the last step's outputs are on the host.
+    nl = len(layers)
+    x_free, y_free = [None] * nl, [None] * nl
+
     def step_e2e():
-        copy_in.wait_stream(stream)  # the previous step is done with the input buffers
         arrived = []
-        with torch.cuda.stream(copy_in):
-            for L in layers:
+        for i, L in enumerate(layers):
+            if x_free[i] is not None:
+                copy_in.wait_event(x_free[i])
+            with torch.cuda.stream(copy_in):
                 L["X"].copy_(L["X_host"], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(copy_in)
-                arrived.append(ev)
-        for L, ev in zip(layers, arrived):
+            ev = torch.cuda.Event()
+            ev.record(copy_in)
+            arrived.append(ev)
+        for i, (L, ev) in enumerate(zip(layers, arrived)):
             stream.wait_event(ev)
+            if y_free[i] is not None:
+                stream.wait_event(y_free[i])
             if W.fused:
                 hsq.forward_fused(L["pl"], L["X"], L["Y"], stream=stream)
             elif W.fp4:
@@ -630,10 +651,13 @@ def run_gpu(args, specs, wl_name, rank, world, local):
                 hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
             done = torch.cuda.Event()
             done.record(stream)
+            x_free[i] = done
             copy_out.wait_event(done)
             with torch.cuda.stream(copy_out):
                 L["Y_host"].copy_(L["Y"], non_blocking=True)
-        stream.wait_stream(copy_out)  # outputs on the host before the step counts as done
+            out_done = torch.cuda.Event()
+            out_done.record(copy_out)
+            y_free[i] = out_done
 
     for _ in range(max(1, args.warmup // 2)):
         step_e2e()
@@ -641,8 +665,12 @@ def run_gpu(args, specs, wl_name, rank, world, local):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    copy_in.wait_stream(stream)
+    copy_out.wait_stream(stream)
     for _ in range(args.steps):
         step_e2e()
+    stream.wait_stream(copy_out)  # the last step's outputs are on the host
+    stream.wait_stream(copy_in)
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)

@@ -135,6 +135,37 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
                               void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * The weights' expanded copy, for hsq_linear_forward_pre.  Where the GEMM reads
+ * pre-expanded operands -- M > 256, or M > 64 with groups of 128 -- a forward
+ * first rewrites both code matrices into E4M3 tiles (one byte per code, the
+ * layout the tensor cores read).  The weights' part of that never changes
+ * between calls, so it can be done once, after hsq_pack_weights:
+ *   hsq_weights_e4m3_bytes(N, K, group): bytes of the copy, Kp x (N rounded up
+ *     to 256); 0 for an invalid shape;
+ *   hsq_expand_weights: writes the copy from w_codes (asynchronous on stream).
+ * A memory-for-speed trade of the library (Kp N bytes more per layer); the
+ * method's stored format stays the packed INT4 codes.
+ */
+size_t hsq_weights_e4m3_bytes(int N, int K, int group);
+hsq_status hsq_expand_weights(const uint8_t* w_codes, int N, int K, int group, uint8_t* w_e4m3,
+                              cudaStream_t stream);
+
+/*
+ * hsq_linear_forward with the weights' expanded copy w_e4m3 (required): where
+ * the GEMM reads pre-expanded operands it takes the weights from w_e4m3
+ * instead of expanding w_codes again, and the workspace needs only
+ * hsq_workspace_bytes_pre(M, N, K, r) bytes; elsewhere w_e4m3 is unused.  The
+ * results are the same bits as hsq_linear_forward's.
+ */
+size_t hsq_workspace_bytes_pre(int M, int N, int K, int r);
+hsq_status hsq_linear_forward_pre(const uint8_t* x_codes, const float* x_scales, const float* U,
+                                  const uint8_t* w_codes, const float* w_scales, const uint8_t* w_e4m3,
+                                  const void* L2_bf16, const void* bias_bf16,
+                                  int M, int N, int K, int r, int group,
+                                  void* Y, hsq_out_dtype out,
+                                  void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Bytes of the library's built-in scratch array used by
  * hsq_linear_forward_noalloc (16 MiB).  Every GPU on which the library is
  * loaded holds this array for the life of the process.

@@ -103,6 +103,31 @@ def test_fused_forward_argument_validation():
     assert call(X=MIS) == hsq.HSQ_ERR_ALIGNMENT
 
 
+def test_expanded_weights_calls_validate_and_size():
+    """The weights' E4M3 copy: its size (Kp x N rounded up to 256), and the
+    argument checks of the expansion and of the forward that reads it (only
+    calls rejected before any launch are made: fake pointers)."""
+    lib = hsq.load()
+    assert hsq.hsq_weights_e4m3_bytes(300, 200, 64) == 512 * 256
+    assert hsq.hsq_weights_e4m3_bytes(12288, 3072, 64) == 12288 * 3072
+    assert hsq.hsq_weights_e4m3_bytes(100, 200, 128) == 256 * 256
+    assert hsq.hsq_weights_e4m3_bytes(0, 64, 64) == 0 and hsq.hsq_weights_e4m3_bytes(64, 64, 96) == 0
+    ex = lib.hsq_expand_weights
+    assert ex(None, 64, 64, 64, A, None) == hsq.HSQ_ERR_INVALID_ARG
+    assert ex(A, 64, 64, 64, MIS, None) == hsq.HSQ_ERR_ALIGNMENT
+    assert ex(A, 64, 64, 96, A, None) == hsq.HSQ_ERR_UNSUPPORTED
+    pre = lib.hsq_linear_forward_pre
+    args = [A, A, A, A, A, A, A, None, 300, 64, 64, 4, 64, A, 0, A, 1 << 30, None]
+    call = lambda **kw: pre(*[kw.get(str(i), a) for i, a in enumerate(args)])
+    assert call(**{"5": None}) == hsq.HSQ_ERR_INVALID_ARG   # the expanded copy is required
+    assert call(**{"5": MIS}) == hsq.HSQ_ERR_ALIGNMENT
+    assert call(**{"0": None}) == hsq.HSQ_ERR_INVALID_ARG
+    # the workspace without the weights' part is smaller wherever the copy is used
+    for M, N, K in ((300, 512, 640), (4608, 12288, 3072)):
+        assert hsq.hsq_workspace_bytes_pre(M, N, K, 4) < hsq.hsq_workspace_bytes(M, N, K, 4)
+    assert hsq.hsq_workspace_bytes_pre(16, 2048, 4096, 4) == hsq.hsq_workspace_bytes(16, 2048, 4096, 4)
+
+
 def test_fused_form_query_and_its_python_restatement():
     """hsq_fused_form (host arithmetic, no launch) against fused_supported and
     the weight stream's shared-memory restatement, on both sides of each limit."""

@@ -291,6 +291,26 @@ def test_fused_decode_tiles_repeat_bit_exact_and_recover_from_a_timeout():
     assert torch.equal(Y, Y0)
 
 
+@pytest.mark.parametrize("M,K,N,r,group", [
+    (300, 640, 512, 32, 64),    # tokens x outputs tiles with expanded operands
+    (4150, 1160, 136, 4, 64),
+    (130, 320, 264, 15, 128),   # groups of 128 expand from 65 tokens
+    (16, 4096, 2048, 4, 64),    # decode tiles: the copy is not used
+])
+def test_expanded_weight_copy_gives_the_same_bits(M, K, N, r, group):
+    """hsq_linear_forward_pre with the weights' E4M3 copy (hsq_expand_weights,
+    made once) against hsq_linear_forward, which expands them on every call."""
+    layer = make_layer(_spec(M, K, N, r, seed=17 * M + K + N + r + group))
+    pl, act, Y, ws = _run_gpu(layer, hsq.HSQ_OUT_F32, group=group)
+    pl.expand()
+    assert pl.w_e4m3.numel() == hsq.hsq_weights_e4m3_bytes(N, K, group)
+    Y2 = torch.empty_like(Y)
+    hsq.forward(pl, layer.X.to(DEV), act, Y2, workspace=pl.workspace(M), out=hsq.HSQ_OUT_F32)
+    torch.cuda.synchronize()
+    assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+    assert torch.equal(Y, Y2)
+
+
 def test_invalid_arguments_launch_nothing():
     layer = make_layer(_spec(8, 128, 64, 4, seed=1))
     pl, act, Y, ws = _run_gpu(layer)

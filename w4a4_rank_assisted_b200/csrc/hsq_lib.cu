@@ -81,7 +81,16 @@ using CfgMid64 = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 6, 10, true, -1, false,
 // M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; packed codes
 // unpacked in shared memory (the drain is light, so more warps unpack); four
 // 64-blocks per stage either way
-using CfgDec16_64 = hsq::GemmCfg<16, 1, 6, true, 4, 2, 4, 10>;
+#ifndef HSQ_DEC16_STAGES
+#define HSQ_DEC16_STAGES 6
+#endif
+#ifndef HSQ_DEC16_GPS
+#define HSQ_DEC16_GPS 4
+#endif
+#ifndef HSQ_DEC16_UNPACK
+#define HSQ_DEC16_UNPACK 6
+#endif
+using CfgDec16_64 = hsq::GemmCfg<16, 1, HSQ_DEC16_STAGES, true, HSQ_DEC16_GPS, 2, 4, HSQ_DEC16_UNPACK>;
 using CfgDec32_64 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, 10>;
 using CfgDec64_64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
 using CfgDec16_128 = hsq::GemmCfg<16, 1, 6, true, 2, 2, 4, 10, 10, false, -1, false, 2, 2>;
@@ -1007,10 +1016,13 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   return (lerr == cudaSuccess && cudaGetLastError() == cudaSuccess) ? HSQ_OK : HSQ_ERR_CUDA;
 }
 
-hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, const float* U, const uint8_t* w_codes,
-                              const float* w_scales, const void* L2_bf16, const void* bias_bf16, int M, int N, int K,
-                              int r, int group, void* Y, hsq_out_dtype out, void* workspace, size_t ws_bytes,
-                              cudaStream_t stream) {
+// hsq_linear_forward and hsq_linear_forward_pre: w_e4m3, when not null, is the
+// weights' expanded copy (hsq_expand_weights), used where the GEMM reads
+// pre-expanded operands instead of expanding w_codes into the workspace.
+static hsq_status forward_impl(const uint8_t* x_codes, const float* x_scales, const float* U, const uint8_t* w_codes,
+                               const float* w_scales, const uint8_t* w_e4m3, const void* L2_bf16,
+                               const void* bias_bf16, int M, int N, int K, int r, int group, void* Y,
+                               hsq_out_dtype out, void* workspace, size_t ws_bytes, cudaStream_t stream) {
   hsq_status st = check_common(M, K, r, group);
   if (st != HSQ_OK) return st;
   if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
@@ -1020,12 +1032,16 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   if ((r > 0) != (L2_bf16 != nullptr) || (r > 0) != (U != nullptr)) return HSQ_ERR_INVALID_ARG;
   if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
       !aligned16(Y) || (U && !aligned16(U)) || (L2_bf16 && !aligned16(L2_bf16)) ||
-      (bias_bf16 && !aligned16(bias_bf16)) || (workspace && !aligned16(workspace)))
+      (bias_bf16 && !aligned16(bias_bf16)) || (workspace && !aligned16(workspace)) ||
+      (w_e4m3 && !aligned16(w_e4m3)))
     return HSQ_ERR_ALIGNMENT;
 
   const int G = groups_of(K, group), Kp = G * group;
   const Plan p = make_plan(M, N, K, group, device_sm_count());
-  if (p.ws_bytes() > 0 && (!workspace || ws_bytes < p.ws_bytes())) return HSQ_ERR_INVALID_ARG;
+  // with the weights' expanded copy the workspace ends before the expanded weights
+  const bool w_pre = w_e4m3 && p.pre_w_bytes > 0;
+  const size_t ws_need = w_pre ? p.pre_w_offset() : p.ws_bytes();
+  if (ws_need > 0 && (!workspace || ws_bytes < ws_need)) return HSQ_ERR_INVALID_ARG;
   if (p.kind == kGemv) {
     hsq::GemvArgs ga{};
     ga.x_codes = x_codes; ga.x_scales = x_scales; ga.ldx = scales_ld(M);
@@ -1078,12 +1094,12 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
   if (p.pre_x_bytes > 0) {
     // expand both code matrices into MMA-ready E4M3 tiles (rows padded to whole tiles)
     uint8_t* xe = static_cast<uint8_t*>(workspace) + p.pre_x_offset();
-    uint8_t* we = static_cast<uint8_t*>(workspace) + p.pre_w_offset();
+    uint8_t* we = w_pre ? const_cast<uint8_t*>(w_e4m3) : static_cast<uint8_t*>(workspace) + p.pre_w_offset();
     const int blocks = 4 * device_sm_count();
     if (launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, x_codes, M, Kp, p.rg_r * 8,
                    xe) != cudaSuccess ||
-        launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, w_codes, N, Kp, p.rg_c * 8,
-                   we) != cudaSuccess)
+        (!w_pre && launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, w_codes, N, Kp,
+                              p.rg_c * 8, we) != cudaSuccess))
       return HSQ_ERR_CUDA;
     a.xe = xe;
     a.we = we;
@@ -1127,6 +1143,56 @@ hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, con
                   : launch_gemm<CfgDec64_64>(p, tm_row, tm_col, tm_y, a, stream);
   }
   return HSQ_ERR_INVALID_ARG;
+}
+
+hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, const float* U, const uint8_t* w_codes,
+                              const float* w_scales, const void* L2_bf16, const void* bias_bf16, int M, int N, int K,
+                              int r, int group, void* Y, hsq_out_dtype out, void* workspace, size_t ws_bytes,
+                              cudaStream_t stream) {
+  return forward_impl(x_codes, x_scales, U, w_codes, w_scales, nullptr, L2_bf16, bias_bf16, M, N, K, r, group, Y, out,
+                      workspace, ws_bytes, stream);
+}
+
+hsq_status hsq_linear_forward_pre(const uint8_t* x_codes, const float* x_scales, const float* U,
+                                  const uint8_t* w_codes, const float* w_scales, const uint8_t* w_e4m3,
+                                  const void* L2_bf16, const void* bias_bf16, int M, int N, int K, int r, int group,
+                                  void* Y, hsq_out_dtype out, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!w_e4m3) return HSQ_ERR_INVALID_ARG;
+  return forward_impl(x_codes, x_scales, U, w_codes, w_scales, w_e4m3, L2_bf16, bias_bf16, M, N, K, r, group, Y, out,
+                      workspace, ws_bytes, stream);
+}
+
+size_t hsq_weights_e4m3_bytes(int N, int K, int group) {
+  if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim || (group != 64 && group != 128)) return 0;
+  const size_t rows_pad = static_cast<size_t>((N + CfgLarge64::BN - 1) / CfgLarge64::BN) * CfgLarge64::BN;
+  return rows_pad * static_cast<size_t>(groups_of(K, group) * group);
+}
+
+hsq_status hsq_expand_weights(const uint8_t* w_codes, int N, int K, int group, uint8_t* w_e4m3,
+                              cudaStream_t stream) {
+  hsq_status st = check_common(N, K, 0, group);
+  if (st != HSQ_OK) return st;
+  if (!w_codes || !w_e4m3) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(w_codes) || !aligned16(w_e4m3)) return HSQ_ERR_ALIGNMENT;
+  const int Kp = groups_of(K, group) * group;
+  const int rows_pad = (N + CfgLarge64::BN - 1) / CfgLarge64::BN * CfgLarge64::BN;
+  const int blocks = 4 * device_sm_count();
+  if (launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, w_codes, N, Kp, rows_pad,
+                 w_e4m3) != cudaSuccess)
+    return HSQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HSQ_OK : HSQ_ERR_CUDA;
+}
+
+size_t hsq_workspace_bytes_pre(int M, int N, int K, int r) {
+  (void)r;
+  if (M < 1 || N < 1 || K < 1) return 0;
+  const int nsm = device_sm_count();
+  size_t need = 0;
+  for (int group : {64, 128}) {
+    const Plan p = make_plan(M, N, K, group, nsm);
+    need = std::max(need, p.pre_w_bytes > 0 ? p.pre_w_offset() : p.ws_bytes());
+  }
+  return need;
 }
 
 hsq_status hsq_linear_forward_noalloc(const uint8_t* x_codes, const float* x_scales, const float* U,
@@ -1281,9 +1347,11 @@ hsq_status hsq_fp4_quantize_act(const void* X_bf16, const float* s, const void* 
   const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
   float* sf = reinterpret_cast<float*>(x_sf);
   if (cudaMemsetAsync(x_gs, 0, 2 * sizeof(float), stream) != cudaSuccess) return HSQ_ERR_CUDA;
-  // the tensor absmax from column maxima: about four blocks of rows per SM
+  // the tensor absmax from column maxima: about four blocks of rows per SM,
+  // rows per block a multiple of 8 once there are enough (eight loads in flight)
   const int nsm = device_sm_count();
-  const int rpb = std::max(1, (M + 4 * nsm - 1) / (4 * nsm));
+  int rpb = std::max(1, (M + 4 * nsm - 1) / (4 * nsm));
+  if (rpb > 4) rpb = (rpb + 7) / 8 * 8;
   if (launch_pdl(false, hsq::nvfp4_act_colmax_kernel, dim3((M + rpb - 1) / rpb), dim3(128), 0, stream, X, s, M, K,
                  rpb, x_gs) != cudaSuccess)
     return HSQ_ERR_CUDA;

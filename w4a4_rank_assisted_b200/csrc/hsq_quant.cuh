@@ -246,7 +246,20 @@ __global__ void __launch_bounds__(128) nvfp4_act_colmax_kernel(const __nv_bfloat
 #pragma unroll
     for (int i = 0; i < 4; ++i) mx[i] = __floats2bfloat162_rn(0.f, 0.f);
     const uint4* col = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m0) * K) + cg;
-    for (int m = m0; m < m1; ++m, col += K / 8) {
+    const size_t stride = K / 8;
+    int m = m0;
+    for (; m + 8 <= m1; m += 8, col += 8 * stride) {  // eight independent loads in flight
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) raw[j] = __ldg(col + j * stride);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[i] = __hmax2(mx[i], __habs2(h[i]));
+      }
+    }
+    for (; m < m1; ++m, col += stride) {
       const uint4 raw = __ldg(col);
       const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll

@@ -36,6 +36,7 @@ EXPORTED = (
     "hsq_workspace_bytes", "hsq_pack_weights", "hsq_quantize_act",
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
     "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused", "hsq_fused_form",
+    "hsq_weights_e4m3_bytes", "hsq_expand_weights", "hsq_workspace_bytes_pre", "hsq_linear_forward_pre",
     "hsq_lowrank_workspace_bytes", "hsq_lowrank_init",
     "hsq_fp4_codes_bytes", "hsq_fp4_scales_bytes", "hsq_fp4_pack_weights", "hsq_fp4_quantize_act",
     "hsq_fp4_linear_forward",
@@ -84,6 +85,14 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_linear_forward_fused.restype = i
     lib.hsq_fused_form.argtypes = [i, i, i, i, i]
     lib.hsq_fused_form.restype = i
+    lib.hsq_weights_e4m3_bytes.argtypes = [i, i, i]
+    lib.hsq_weights_e4m3_bytes.restype = ctypes.c_size_t
+    lib.hsq_expand_weights.argtypes = [vp, i, i, i, vp, vp]
+    lib.hsq_expand_weights.restype = i
+    lib.hsq_workspace_bytes_pre.argtypes = [i, i, i, i]
+    lib.hsq_workspace_bytes_pre.restype = ctypes.c_size_t
+    lib.hsq_linear_forward_pre.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, ctypes.c_size_t, vp]
+    lib.hsq_linear_forward_pre.restype = i
     lib.hsq_lowrank_workspace_bytes.argtypes = [i, i, i]; lib.hsq_lowrank_workspace_bytes.restype = sz
     lib.hsq_lowrank_init.argtypes = [vp, vp, i, i, i, i, c.c_ulonglong, vp, vp, vp, sz, vp]
     lib.hsq_lowrank_init.restype = i
@@ -182,6 +191,28 @@ def hsq_linear_forward_noalloc(x_codes, x_scales, U, w_codes, w_scales, L2, bias
                                              _ptr(w_scales), _ptr(L2), _ptr(bias), M, N, K, r, group,
                                              _ptr(Y), int(out), _stream(stream)),
            "hsq_linear_forward_noalloc")
+
+
+def hsq_weights_e4m3_bytes(N: int, K: int, group: int = GROUP) -> int:
+    return int(load().hsq_weights_e4m3_bytes(N, K, group))
+
+
+def hsq_expand_weights(w_codes, N, K, w_e4m3, group=GROUP, stream=None) -> None:
+    _check(load().hsq_expand_weights(_ptr(w_codes), N, K, group, _ptr(w_e4m3), _stream(stream)),
+           "hsq_expand_weights")
+
+
+def hsq_workspace_bytes_pre(M: int, N: int, K: int, r: int) -> int:
+    return int(load().hsq_workspace_bytes_pre(M, N, K, r))
+
+
+def hsq_linear_forward_pre(x_codes, x_scales, U, w_codes, w_scales, w_e4m3, L2, bias, M, N, K, r, Y,
+                           out: int = HSQ_OUT_BF16, workspace=None, ws_bytes: int = 0,
+                           group=GROUP, stream=None) -> None:
+    _check(load().hsq_linear_forward_pre(_ptr(x_codes), _ptr(x_scales), _ptr(U), _ptr(w_codes),
+                                         _ptr(w_scales), _ptr(w_e4m3), _ptr(L2), _ptr(bias), M, N, K, r, group,
+                                         _ptr(Y), int(out), _ptr(workspace), int(ws_bytes),
+                                         _stream(stream)), "hsq_linear_forward_pre")
 
 
 def hsq_linear_forward_fused(X, s, L1, w_codes, w_scales, L2, bias, M, N, K, r, Y,
@@ -327,11 +358,21 @@ class PackedLinear:
         self.bias = None if bias is None else bias.contiguous()
         self.w_codes = alloc_codes(N, K, dev, group)
         self.w_scales = alloc_scales(N, K, dev, group)
+        self.w_e4m3 = None  # the weights' expanded copy, once expand() has run
         hsq_pack_weights(W.contiguous(), self.s, self.L1, self.L2, N, K, r,
                          self.w_codes, self.w_scales, group=group, stream=stream)
 
+    def expand(self, stream=None) -> None:
+        """Keep the weights' E4M3-expanded copy (hsq_expand_weights): forwards
+        with many tokens then skip re-expanding the weights on every call."""
+        if self.w_e4m3 is None:
+            self.w_e4m3 = torch.empty(hsq_weights_e4m3_bytes(self.N, self.K, self.group), dtype=torch.uint8,
+                                      device=self.w_codes.device)
+            hsq_expand_weights(self.w_codes, self.N, self.K, self.w_e4m3, group=self.group, stream=stream)
+
     def workspace(self, M: int) -> Optional[torch.Tensor]:
-        n = hsq_workspace_bytes(M, self.N, self.K, self.r)
+        n = (hsq_workspace_bytes(M, self.N, self.K, self.r) if self.w_e4m3 is None
+             else hsq_workspace_bytes_pre(M, self.N, self.K, self.r))
         if n == 0:
             return None
         return torch.zeros(n, dtype=torch.uint8, device=self.w_codes.device)
@@ -366,9 +407,14 @@ def forward(layer: PackedLinear, X: torch.Tensor, act: ActBuffers, Y: torch.Tens
     hsq_quantize_act(X, layer.s, layer.L1, M, layer.K, layer.r, act.x_codes, act.x_scales, act.U,
                      group=layer.group, stream=stream)
     ws_bytes = 0 if workspace is None else workspace.numel()
-    hsq_linear_forward(act.x_codes, act.x_scales, act.U, layer.w_codes, layer.w_scales, layer.L2,
-                       layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace,
-                       ws_bytes=ws_bytes, group=layer.group, stream=stream)
+    if layer.w_e4m3 is not None:
+        hsq_linear_forward_pre(act.x_codes, act.x_scales, act.U, layer.w_codes, layer.w_scales, layer.w_e4m3,
+                               layer.L2, layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace,
+                               ws_bytes=ws_bytes, group=layer.group, stream=stream)
+    else:
+        hsq_linear_forward(act.x_codes, act.x_scales, act.U, layer.w_codes, layer.w_scales, layer.L2,
+                           layer.bias, M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace,
+                           ws_bytes=ws_bytes, group=layer.group, stream=stream)
     return Y
 
 
