@@ -90,7 +90,14 @@ using CfgMid64 = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 6, 10, true, -1, false,
 #ifndef HSQ_DEC16_UNPACK
 #define HSQ_DEC16_UNPACK 6
 #endif
-using CfgDec16_64 = hsq::GemmCfg<16, 1, HSQ_DEC16_STAGES, true, HSQ_DEC16_GPS, 2, 4, HSQ_DEC16_UNPACK>;
+#ifndef HSQ_DEC16_NI8
+#define HSQ_DEC16_NI8 2
+#endif
+#ifndef HSQ_DEC16_NTM
+#define HSQ_DEC16_NTM 4
+#endif
+using CfgDec16_64 = hsq::GemmCfg<16, 1, HSQ_DEC16_STAGES, true, HSQ_DEC16_GPS, HSQ_DEC16_NI8, HSQ_DEC16_NTM,
+                                 HSQ_DEC16_UNPACK>;
 using CfgDec32_64 = hsq::GemmCfg<32, 1, 5, true, 4, 2, 2, 10>;
 using CfgDec64_64 = hsq::GemmCfg<64, 1, 8, true, 2, 2, 2, 6>;  // 64 accumulators: keep registers
 using CfgDec16_128 = hsq::GemmCfg<16, 1, 6, true, 2, 2, 4, 10, 10, false, -1, false, 2, 2>;
@@ -187,6 +194,10 @@ cudaError_t launch_pdl(bool allow, void (*kernel)(KArgs...), dim3 grid, dim3 blo
 // ... from this many rows per SM on
 #ifndef HSQ_ACT_ROWS16_MIN
 #define HSQ_ACT_ROWS16_MIN 28
+#endif
+// ... with this many rows per warp (8 warps per block)
+#ifndef HSQ_ACT_ROWS_SUB
+#define HSQ_ACT_ROWS_SUB 2
 #endif
 
 thread_local int t_debug_flags = 0;
@@ -1005,7 +1016,7 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   if (M <= 64) {
     HSQ_ACT_RANKS(true)
   } else if (rows_kernel) {
-    HSQ_ACT_ROWS_RANKS(8, 2)
+    HSQ_ACT_ROWS_RANKS(8, HSQ_ACT_ROWS_SUB)
   } else {
     HSQ_ACT_RANKS(false)
   }
