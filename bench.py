@@ -2,9 +2,11 @@
 """Benchmark of the rank-r W4A4 linear layer (H-SVDQuant forward) on B200.
 
 One step = one pass of the hot path over one batch: for every linear of the
-workload, the fused activation step (hsq_quantize_act) followed by the INT4
-GEMM + low-rank/bias epilogue (hsq_linear_forward), weights pre-packed (packing
-is offline).  Default workload: the FLUX.1 double-stream block linears
+workload, the fused activation step followed by the INT4 GEMM + low-rank/bias
+epilogue, as one hsq_linear_forward_x call (X in, Y out; the same bits as
+hsq_quantize_act + hsq_linear_forward), or one hsq_linear_forward_fused launch
+at decode sizes; weights pre-packed, and for many tokens their E4M3 copy made
+once, offline (packing is offline).  Default workload: the FLUX.1 double-stream block linears
 (M = 4608 tokens; QKV 3072->9216, MLP up 3072->12288, MLP down 12288->3072;
 rank 4; group-64 INT4), synthetic seeded inputs.
 
@@ -115,8 +117,14 @@ def time_kernel_nodes(launch, stream, name_part: str, calls: int, repeats: int =
         n = _cu(cu.cuGraphGetNodes(graph, 0))[1]
         nodes = _cu(cu.cuGraphGetNodes(graph, n))[0]
         key = lambda nd: int(nd)
-        deps = {key(nd): {key(d) for d in _cu(cu.cuGraphNodeGetDependencies(
-            nd, _cu(cu.cuGraphNodeGetDependencies(nd, 0))[1]))[0]} for nd in nodes}
+
+        def node_deps(nd):
+            # with edge data: a call whose kernels start early has programmatic edges,
+            # which the plain query refuses to report
+            n_d = _cu(cu.cuGraphNodeGetDependencies_v2(nd, 0))[2]
+            return _cu(cu.cuGraphNodeGetDependencies_v2(nd, n_d))[0] if n_d else []
+
+        deps = {key(nd): {key(d) for d in node_deps(nd)} for nd in nodes}
         order, placed = [], set()
         while len(order) < len(nodes):  # launch order (the capture is a chain)
             for nd in nodes:
@@ -139,7 +147,7 @@ def time_kernel_nodes(launch, stream, name_part: str, calls: int, repeats: int =
             else:
                 _cu(cu.cuGraphDestroyNode(nd))
         for a, b in zip(kept[:-1], kept[1:]):  # chain the kept nodes (edges not already there)
-            have = _cu(cu.cuGraphNodeGetDependencies(b, _cu(cu.cuGraphNodeGetDependencies(b, 0))[1]))[0]
+            have = node_deps(b)
             if int(a) not in {int(x) for x in have}:
                 _cu(cu.cuGraphAddDependencies(graph, [a], [b], 1))
         exe = _cu(cu.cuGraphInstantiate(graph, 0))
@@ -159,6 +167,10 @@ def time_kernel_nodes(launch, stream, name_part: str, calls: int, repeats: int =
     if not kept:
         raise RuntimeError(f"no kernel named like {name_part!r} in the call")
     return e0.elapsed_time(e1) * 1e3 / (repeats * len(kept)), len(kept) / calls
+
+
+def _sms() -> int:
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
 
 
 class ClockSampler:
@@ -363,7 +375,8 @@ class Workload:
                         pl.expand()  # the weights' E4M3 copy, made once (offline), as a deployment would
                     act = hsq.ActBuffers(spec.M, spec.K, spec.r, dev, group=spec.group)
                 Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
-                out.append(dict(spec=spec, pl=pl, X=d(lay.X), act=act, Y=Y, ws=pl.workspace(spec.M)))
+                wsx = pl.workspace_x(spec.M) if spec.fmt == "int4" else None
+                out.append(dict(spec=spec, pl=pl, X=d(lay.X), act=act, Y=Y, ws=pl.workspace(spec.M), wsx=wsx))
             return out
 
         self.layers = build_layers()
@@ -420,6 +433,13 @@ class Workload:
                                     workspace=L["ws"], ws_bytes=0 if L["ws"] is None else L["ws"].numel(),
                                     group=s.group, stream=st)
 
+    def launch_x(self, L, st):
+        """The activation step and the forward in one call (hsq_linear_forward_x)."""
+        s = L["spec"]
+        self.hsq.hsq_linear_forward_x(L["X"], L["pl"].s, L["pl"].L1, L["pl"].w_codes, L["pl"].w_scales,
+                                      L["pl"].w_e4m3, L["pl"].L2, None, s.M, s.N, s.K, s.r, L["Y"],
+                                      workspace=L["wsx"], ws_bytes=L["wsx"].numel(), group=s.group, stream=st)
+
     def launch_fused(self, L, st):
         s = L["spec"]
         self.hsq.hsq_linear_forward_fused(L["X"], L["pl"].s, L["pl"].L1, L["pl"].w_codes, L["pl"].w_scales,
@@ -429,6 +449,8 @@ class Workload:
         for L in self.replicas[rep]:
             if self.fused:
                 self.launch_fused(L, st)
+            elif L["spec"].fmt == "int4":
+                self.launch_x(L, st)
             else:
                 self.launch_act(L, st)
                 self.launch_gemm(L, st)
@@ -485,8 +507,16 @@ class Workload:
             elif s.fmt == "nvfp4":
                 n += 2 + (1 if s.M % 128 else 0) + 1
             else:
-                n += 1 + (2 if self.expands(s) else 1)
+                n += 2 + (0 if not self.expands(s) else
+                          (1 if s.M % 128 else 0) if self.x_tiles(s) else 1)
         return n
+
+    @staticmethod
+    def x_tiles(s):
+        """hsq_linear_forward_x's activation kernel writes the GEMM's E4M3 tiles
+        itself (no expansion launch; a pad-zeroing launch when M is not a
+        multiple of 128): many rows, ranks 0, 1, 2, 4."""
+        return s.M >= 28 * _sms() and s.r in (0, 1, 2, 4)
 
     @staticmethod
     def expands(s):
@@ -514,16 +544,19 @@ class Workload:
                 d["call_us"] = per_call(self.launch_fused)
                 d["gemm_kernel_us"] = d["call_us"]
                 d["act_us"] = 0.0
+            elif L["spec"].fmt == "int4":
+                # one call (activation step + forward): its kernels timed apart
+                d["call_us"] = per_call(self.launch_x)
+                call = lambda i, st: self.launch_x(self.replicas[i % self.nrep][li], st)
+                d["gemm_kernel_us"], _ = time_kernel_nodes(call, self.gstream, "w4a4_gem", reps)
+                d["act_us"], _ = time_kernel_nodes(call, self.gstream, "quantize_act", reps)
+                if self.expands(L["spec"]) and (L["spec"].M % 128 or not self.x_tiles(L["spec"])):
+                    e_us, e_n = time_kernel_nodes(call, self.gstream, "e4m3", reps)
+                    d["expand_us"] = e_us * e_n  # expansion or pad-zeroing launches of one call
             else:
                 d["call_us"] = per_call(self.launch_gemm)
                 d["act_us"] = per_call(self.launch_act)
-                if self.expands(L["spec"]):
-                    call = lambda i, st: self.launch_gemm(self.replicas[i % self.nrep][li], st)
-                    d["gemm_kernel_us"], _ = time_kernel_nodes(call, self.gstream, "w4a4_gemm_kernel", reps)
-                    e_us, e_n = time_kernel_nodes(call, self.gstream, "expand_e4m3_kernel", reps)
-                    d["expand_us"] = e_us * e_n  # the call's expansion launches
-                else:
-                    d["gemm_kernel_us"] = d["call_us"]
+                d["gemm_kernel_us"] = d["call_us"]
             out.append(d)
         return out
 
@@ -648,7 +681,7 @@ def run_gpu(args, specs, wl_name, rank, world, local):
             elif W.fp4:
                 hsq.fp4_forward(L["pl"], L["X"], L["act"], L["Y"], stream=stream)
             else:
-                hsq.forward(L["pl"], L["X"], L["act"], L["Y"], workspace=L["ws"], stream=stream)
+                hsq.forward_x(L["pl"], L["X"], L["Y"], L["wsx"], stream=stream)
             done = torch.cuda.Event()
             done.record(stream)
             x_free[i] = done

@@ -125,7 +125,9 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
  *   Y out [M][N], bf16 (HSQ_OUT_BF16, round-to-nearest-even) or fp32 (HSQ_OUT_F32)
  *   workspace / ws_bytes: scratch of at least hsq_workspace_bytes(M,N,K,r) bytes
  *     (may be NULL when that is 0); calls that share a workspace must not run
- *     concurrently.
+ *     concurrently.  Before its first use the workspace must hold zeros (its
+ *     split-K counters); every call leaves them at zero again, so one
+ *     zero-filled buffer serves any number of calls.
  */
 hsq_status hsq_linear_forward(const uint8_t* x_codes, const float* x_scales, const float* U,
                               const uint8_t* w_codes, const float* w_scales,
@@ -164,6 +166,30 @@ hsq_status hsq_linear_forward_pre(const uint8_t* x_codes, const float* x_scales,
                                   int M, int N, int K, int r, int group,
                                   void* Y, hsq_out_dtype out,
                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * The activation step and the forward in one call (X in, Y out), for callers
+ * that do not need the activation codes themselves: the same Y, bit for bit,
+ * as hsq_quantize_act followed by hsq_linear_forward (w_e4m3 NULL) or
+ * hsq_linear_forward_pre (w_e4m3 from hsq_expand_weights).  Where the GEMM
+ * reads expanded operands and the many-row activation kernel applies (M at
+ * least 28 per SM, r in {0, 1, 2, 4}), that kernel writes the activations'
+ * E4M3 tiles itself, so no packed codes are written and no expansion runs;
+ * elsewhere the call is those two steps.  The activation step's scales and U
+ * live in the workspace:
+ *   hsq_workspace_bytes_x(M, N, K, r, group, with_w_e4m3): its bytes (0 for an
+ *     invalid shape); with_w_e4m3 != 0 when w_e4m3 will be passed.
+ *   X_bf16, s, L1_bf16 as for hsq_quantize_act; the rest as for
+ *   hsq_linear_forward; workspace is required, and need not hold zeros (the
+ *   call clears its split-K counters itself).
+ */
+size_t hsq_workspace_bytes_x(int M, int N, int K, int r, int group, int with_w_e4m3);
+hsq_status hsq_linear_forward_x(const void* X_bf16, const float* s, const void* L1_bf16,
+                                const uint8_t* w_codes, const float* w_scales, const uint8_t* w_e4m3,
+                                const void* L2_bf16, const void* bias_bf16,
+                                int M, int N, int K, int r, int group,
+                                void* Y, hsq_out_dtype out,
+                                void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * Bytes of the library's built-in scratch array used by

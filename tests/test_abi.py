@@ -128,6 +128,25 @@ def test_expanded_weights_calls_validate_and_size():
     assert hsq.hsq_workspace_bytes_pre(16, 2048, 4096, 4) == hsq.hsq_workspace_bytes(16, 2048, 4096, 4)
 
 
+def test_forward_x_validates_before_launching():
+    """hsq_linear_forward_x: workspace required and large enough, alignment of
+    every pointer; all checked before anything is launched (fake pointers)."""
+    lib = hsq.load()
+    fx = lib.hsq_linear_forward_x
+    need = hsq.hsq_workspace_bytes_x(4608, 12288, 3072, 4, 64, True)
+    assert need > 0
+    assert hsq.hsq_workspace_bytes_x(4608, 12288, 3072, 4, 64, False) > need  # plus the weights' expansion
+    assert hsq.hsq_workspace_bytes_x(0, 64, 64, 4, 64, True) == 0
+    args = [A, A, A, A, A, A, A, None, 4608, 12288, 3072, 4, 64, A, 0, A, need, None]
+    call = lambda **kw: fx(*[kw.get(str(i), a) for i, a in enumerate(args)])
+    assert call(**{"15": None}) == hsq.HSQ_ERR_INVALID_ARG       # no workspace
+    assert call(**{"16": need - 1}) == hsq.HSQ_ERR_INVALID_ARG   # too small
+    assert call(**{"5": MIS}) == hsq.HSQ_ERR_ALIGNMENT
+    assert call(**{"0": MIS}) == hsq.HSQ_ERR_ALIGNMENT
+    assert call(**{"2": None}) == hsq.HSQ_ERR_INVALID_ARG        # r > 0 needs L1
+    assert call(**{"12": 96}) == hsq.HSQ_ERR_UNSUPPORTED
+
+
 def test_fused_form_query_and_its_python_restatement():
     """hsq_fused_form (host arithmetic, no launch) against fused_supported and
     the weight stream's shared-memory restatement, on both sides of each limit."""

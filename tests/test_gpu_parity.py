@@ -311,6 +311,38 @@ def test_expanded_weight_copy_gives_the_same_bits(M, K, N, r, group):
     assert torch.equal(Y, Y2)
 
 
+@pytest.mark.parametrize("M,K,N,r,group", [
+    (4150, 1160, 136, 4, 64),   # the activation kernel writes the GEMM's E4M3 tiles (padding rows, padded K)
+    (4150, 1160, 136, 2, 128),
+    (4160, 392, 264, 0, 64),
+    (4200, 520, 136, 1, 64),
+    (4150, 1160, 136, 8, 64),   # rank 8: the two steps, with the expansion kernel
+    (300, 640, 512, 32, 64),    # few rows: the two steps
+    (16, 4096, 2048, 4, 64),    # decode tiles
+])
+def test_forward_x_gives_the_bits_of_the_two_calls(M, K, N, r, group):
+    """hsq_linear_forward_x (X in, Y out), with and without the weights' E4M3
+    copy, against hsq_quantize_act + hsq_linear_forward: the same bits, also on
+    a workspace first filled with 0xFF bytes (E4M3 NaN patterns), which the
+    padding rows of the activations' tiles must not keep."""
+    layer = make_layer(_spec(M, K, N, r, seed=19 * M + K + N + r + group))
+    pl, act, Y, ws = _run_gpu(layer, hsq.HSQ_OUT_F32, group=group)
+    X = layer.X.to(DEV)
+    for expanded in (False, True):
+        if expanded:
+            pl.expand()
+        wsx = pl.workspace_x(M)
+        wsx.fill_(0xFF)
+        Yx = torch.full_like(Y, float("nan"))
+        hsq.forward_x(pl, X, Yx, wsx, out=hsq.HSQ_OUT_F32)
+        torch.cuda.synchronize()
+        assert hsq.hsq_get_device_status() == hsq.HSQ_OK
+        assert torch.equal(Yx, Y), f"forward_x (weights' copy: {expanded}) differs from the two calls"
+        hsq.forward_x(pl, X, Yx, wsx, out=hsq.HSQ_OUT_F32)  # again, on the same workspace
+        torch.cuda.synchronize()
+        assert torch.equal(Yx, Y)
+
+
 def test_invalid_arguments_launch_nothing():
     layer = make_layer(_spec(8, 128, 64, 4, seed=1))
     pl, act, Y, ws = _run_gpu(layer)

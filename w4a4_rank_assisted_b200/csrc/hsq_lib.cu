@@ -673,7 +673,8 @@ BlasSlot g_blas[kMaxDevices];
 // per device and instantiation).
 template <int R, int GL, int NW, int SUB, bool FP4 = false>
 cudaError_t launch_act_rows(const __nv_bfloat16* X, const float* s, const __nv_bfloat16* L1, int M, int K, int Kp,
-                            int ld, uint8_t* codes, float* scales, float* U, cudaStream_t st, float* gs = nullptr) {
+                            int ld, uint8_t* codes, float* scales, float* U, cudaStream_t st, float* gs = nullptr,
+                            uint8_t* xe = nullptr, int xe_rg = 0, unsigned* zc = nullptr, int zc_words = 0) {
   using C = hsq::ActRowsCfg<NW, SUB>;
   constexpr int kSmem = C::STAGES * C::STAGE_BYTES;
   static std::mutex mu;
@@ -691,7 +692,7 @@ cudaError_t launch_act_rows(const __nv_bfloat16* X, const float* s, const __nv_b
   }
   return launch_pdl(!FP4, hsq::quantize_act_rows_kernel<R, GL, NW, SUB, FP4>, dim3((M + C::RB - 1) / C::RB),
                     dim3(NW * 32), static_cast<size_t>(kSmem), st, X, s, L1, M, K, Kp, ld, codes, scales, U,
-                    wait_limit_ns(), gs);
+                    wait_limit_ns(), gs, xe, xe_rg, zc, zc_words);
 }
 
 // hsq_linear_forward_fused for the shapes the weight stream's fused form does
@@ -966,8 +967,20 @@ hsq_status hsq_pack_weights(const void* W_bf16, const float* s, const void* L1_b
   return HSQ_OK;
 }
 
+// hsq_quantize_act, optionally also clearing zc_words words at zc (the split-K
+// counters of the GEMM that follows, for hsq_linear_forward_x).
+static hsq_status quantize_act_impl(const void* X_bf16, const float* s, const void* L1_bf16, int M, int K, int r,
+                                    int group, uint8_t* x_codes, float* x_scales, float* U, cudaStream_t stream,
+                                    unsigned* zc, int zc_words);
+
 hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_bf16, int M, int K, int r,
                             int group, uint8_t* x_codes, float* x_scales, float* U, cudaStream_t stream) {
+  return quantize_act_impl(X_bf16, s, L1_bf16, M, K, r, group, x_codes, x_scales, U, stream, nullptr, 0);
+}
+
+static hsq_status quantize_act_impl(const void* X_bf16, const float* s, const void* L1_bf16, int M, int K, int r,
+                                    int group, uint8_t* x_codes, float* x_scales, float* U, cudaStream_t stream,
+                                    unsigned* zc, int zc_words) {
   hsq_status st = check_common(M, K, r, group);
   if (st != HSQ_OK) return st;
   if (!X_bf16 || !s || !x_codes || !x_scales) return HSQ_ERR_INVALID_ARG;
@@ -982,11 +995,11 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
   lerr = (group == 128 ? launch_pdl(true, hsq::quantize_act_kernel<RV, SM, 16>,                             \
                                     dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),     \
                                     dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, \
-                                    x_codes, x_scales, U, static_cast<float*>(nullptr))                    \
+                                    x_codes, x_scales, U, static_cast<float*>(nullptr), zc, zc_words)      \
                        : launch_pdl(true, hsq::quantize_act_kernel<RV, SM, 8>,                              \
                                     dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),     \
                                     dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kp, ld, \
-                                    x_codes, x_scales, U, static_cast<float*>(nullptr)))
+                                    x_codes, x_scales, U, static_cast<float*>(nullptr), zc, zc_words))
 #define HSQ_ACT_RANKS(SM)                   \
   switch (r) {                              \
     case 0: HSQ_ACT_LAUNCH(0, SM); break;   \
@@ -999,8 +1012,10 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
     default: HSQ_ACT_LAUNCH(-1, SM); break; \
   }
 #define HSQ_ACT_ROWS_LAUNCH(RV, NW, SUB)                                                                  \
-  lerr = (group == 128 ? launch_act_rows<RV, 16, NW, SUB>(X, s, L1, M, K, Kp, ld, x_codes, x_scales, U, stream) \
-                       : launch_act_rows<RV, 8, NW, SUB>(X, s, L1, M, K, Kp, ld, x_codes, x_scales, U, stream))
+  lerr = (group == 128 ? launch_act_rows<RV, 16, NW, SUB>(X, s, L1, M, K, Kp, ld, x_codes, x_scales, U, stream,    \
+                                                          nullptr, nullptr, 0, zc, zc_words)                   \
+                       : launch_act_rows<RV, 8, NW, SUB>(X, s, L1, M, K, Kp, ld, x_codes, x_scales, U, stream,     \
+                                                         nullptr, nullptr, 0, zc, zc_words))
 #define HSQ_ACT_ROWS_RANKS(NW, SUB)               \
   switch (r) {                                    \
     case 0: HSQ_ACT_ROWS_LAUNCH(0, NW, SUB); break; \
@@ -1030,10 +1045,13 @@ hsq_status hsq_quantize_act(const void* X_bf16, const float* s, const void* L1_b
 // hsq_linear_forward and hsq_linear_forward_pre: w_e4m3, when not null, is the
 // weights' expanded copy (hsq_expand_weights), used where the GEMM reads
 // pre-expanded operands instead of expanding w_codes into the workspace.
+// x_expanded: the activations' E4M3 tiles are already in the workspace (written
+// by the activation kernel of hsq_linear_forward_x); x_codes is then unused.
 static hsq_status forward_impl(const uint8_t* x_codes, const float* x_scales, const float* U, const uint8_t* w_codes,
                                const float* w_scales, const uint8_t* w_e4m3, const void* L2_bf16,
                                const void* bias_bf16, int M, int N, int K, int r, int group, void* Y,
-                               hsq_out_dtype out, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+                               hsq_out_dtype out, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                               bool x_expanded = false) {
   hsq_status st = check_common(M, K, r, group);
   if (st != HSQ_OK) return st;
   if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
@@ -1107,8 +1125,8 @@ static hsq_status forward_impl(const uint8_t* x_codes, const float* x_scales, co
     uint8_t* xe = static_cast<uint8_t*>(workspace) + p.pre_x_offset();
     uint8_t* we = w_pre ? const_cast<uint8_t*>(w_e4m3) : static_cast<uint8_t*>(workspace) + p.pre_w_offset();
     const int blocks = 4 * device_sm_count();
-    if (launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, x_codes, M, Kp, p.rg_r * 8,
-                   xe) != cudaSuccess ||
+    if ((!x_expanded && launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, x_codes, M,
+                                   Kp, p.rg_r * 8, xe) != cudaSuccess) ||
         (!w_pre && launch_pdl(false, hsq::expand_e4m3_kernel, dim3(blocks), dim3(256), 0, stream, w_codes, N, Kp,
                               p.rg_c * 8, we) != cudaSuccess))
       return HSQ_ERR_CUDA;
@@ -1171,6 +1189,99 @@ hsq_status hsq_linear_forward_pre(const uint8_t* x_codes, const float* x_scales,
   if (!w_e4m3) return HSQ_ERR_INVALID_ARG;
   return forward_impl(x_codes, x_scales, U, w_codes, w_scales, w_e4m3, L2_bf16, bias_bf16, M, N, K, r, group, Y, out,
                       workspace, ws_bytes, stream);
+}
+
+// hsq_linear_forward_x's workspace: the GEMM's part first, then the activation
+// step's outputs (packed codes only where the GEMM does not take expanded tiles
+// from the activation kernel), scales and U.
+struct XLayout {
+  Plan p;
+  bool expanded;  // the activation kernel writes the GEMM's E4M3 tiles itself
+  size_t gemm, o_codes, o_scales, o_u, total;
+};
+static XLayout x_layout(int M, int N, int K, int r, int group, int nsm, bool w_pre) {
+  XLayout L{};
+  L.p = make_plan(M, N, K, group, nsm);
+  const int G = groups_of(K, group), Kp = G * group;
+  L.expanded = L.p.pre_x_bytes > 0 && HSQ_ACT_ROWS && (r <= 2 || r == 4) && M >= HSQ_ACT_ROWS16_MIN * nsm;
+  L.gemm = (w_pre && L.p.pre_w_bytes > 0) ? L.p.pre_w_offset() : L.p.ws_bytes();
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t off = up(L.gemm);
+  L.o_codes = off;
+  if (!L.expanded) off = up(off + static_cast<size_t>(M) * (Kp / 2));
+  L.o_scales = off;
+  off = up(off + static_cast<size_t>(G) * scales_ld(M) * 4);
+  L.o_u = off;
+  off = up(off + static_cast<size_t>(M) * std::max(r, 1) * 4);
+  L.total = off;
+  return L;
+}
+
+size_t hsq_workspace_bytes_x(int M, int N, int K, int r, int group, int with_w_e4m3) {
+  if (check_common(M, K, r, group) != HSQ_OK || N < 1 || N > kMaxDim) return 0;
+  return x_layout(M, N, K, r, group, device_sm_count(), with_w_e4m3 != 0).total;
+}
+
+hsq_status hsq_linear_forward_x(const void* X_bf16, const float* s, const void* L1_bf16, const uint8_t* w_codes,
+                                const float* w_scales, const uint8_t* w_e4m3, const void* L2_bf16,
+                                const void* bias_bf16, int M, int N, int K, int r, int group, void* Y,
+                                hsq_out_dtype out, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  hsq_status st = check_common(M, K, r, group);
+  if (st != HSQ_OK) return st;
+  if (N < 1 || N > kMaxDim) return HSQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return HSQ_ERR_UNSUPPORTED;
+  if (out != HSQ_OUT_BF16 && out != HSQ_OUT_F32) return HSQ_ERR_INVALID_ARG;
+  if (!X_bf16 || !s || !w_codes || !w_scales || !Y || !workspace) return HSQ_ERR_INVALID_ARG;
+  if ((r > 0) != (L1_bf16 != nullptr) || (r > 0) != (L2_bf16 != nullptr)) return HSQ_ERR_INVALID_ARG;
+  if (!aligned16(X_bf16) || !aligned16(s) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(Y) ||
+      !aligned16(workspace) || (w_e4m3 && !aligned16(w_e4m3)) || (L1_bf16 && !aligned16(L1_bf16)) ||
+      (L2_bf16 && !aligned16(L2_bf16)) || (bias_bf16 && !aligned16(bias_bf16)))
+    return HSQ_ERR_ALIGNMENT;
+  const int nsm = device_sm_count();
+  const XLayout L = x_layout(M, N, K, r, group, nsm, w_e4m3 != nullptr);
+  if (ws_bytes < L.total) return HSQ_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(base + L.o_scales);
+  float* U = r > 0 ? reinterpret_cast<float*>(base + L.o_u) : nullptr;
+  // the split-K counters start at zero whatever the workspace held: the
+  // activation kernel clears them (after the preceding kernel, before the GEMM)
+  unsigned* zc = (L.p.kind != kGemv && L.p.stream_len > 0) ? static_cast<unsigned*>(workspace) : nullptr;
+  const int zc_words = zc ? static_cast<int>(L.p.counters_bytes / 4) : 0;
+  if (!L.expanded) {
+    st = quantize_act_impl(X_bf16, s, L1_bf16, M, K, r, group, base + L.o_codes, xs, U, stream, zc, zc_words);
+    if (st != HSQ_OK) return st;
+    return forward_impl(base + L.o_codes, xs, U, w_codes, w_scales, w_e4m3, L2_bf16, bias_bf16, M, N, K, r, group,
+                        Y, out, workspace, L.gemm, stream);
+  }
+  // the activation kernel writes the GEMM's E4M3 tiles (padding rows zeroed first)
+  const int G = groups_of(K, group), Kp = G * group, ld = scales_ld(M);
+  const int rows_pad = L.p.rg_r * 8;
+  uint8_t* xe = base + L.p.pre_x_offset();
+  if (rows_pad > M) {
+    const size_t n = static_cast<size_t>(Kp / 64) * (rows_pad - M) * 4;
+    const int blocks = static_cast<int>(std::min<size_t>(4 * nsm, (n + 255) / 256));
+    if (launch_pdl(true, hsq::zero_e4m3_rows_kernel, dim3(blocks), dim3(256), 0, stream, xe, M, rows_pad, Kp) !=
+        cudaSuccess)
+      return HSQ_ERR_CUDA;
+  }
+  const auto* X = static_cast<const __nv_bfloat16*>(X_bf16);
+  const auto* L1 = static_cast<const __nv_bfloat16*>(L1_bf16);
+  cudaError_t lerr = cudaSuccess;
+#define HSQ_X_ACT(RV)                                                                                          \
+  lerr = group == 128 ? launch_act_rows<RV, 16, 8, HSQ_ACT_ROWS_SUB>(X, s, L1, M, K, Kp, ld, nullptr, xs, U, stream, \
+                                                                    nullptr, xe, L.p.rg_r, zc, zc_words)        \
+                      : launch_act_rows<RV, 8, 8, HSQ_ACT_ROWS_SUB>(X, s, L1, M, K, Kp, ld, nullptr, xs, U, stream,  \
+                                                                   nullptr, xe, L.p.rg_r, zc, zc_words)
+  switch (r) {
+    case 0: HSQ_X_ACT(0); break;
+    case 1: HSQ_X_ACT(1); break;
+    case 2: HSQ_X_ACT(2); break;
+    default: HSQ_X_ACT(4); break;
+  }
+#undef HSQ_X_ACT
+  if (lerr != cudaSuccess || cudaGetLastError() != cudaSuccess) return HSQ_ERR_CUDA;
+  return forward_impl(xe, xs, U, w_codes, w_scales, w_e4m3, L2_bf16, bias_bf16, M, N, K, r, group, Y, out, workspace,
+                      L.gemm, stream, true);
 }
 
 size_t hsq_weights_e4m3_bytes(int N, int K, int group) {
@@ -1371,7 +1482,7 @@ hsq_status hsq_fp4_quantize_act(const void* X_bf16, const float* s, const void* 
   lerr = launch_pdl(false, hsq::quantize_act_kernel<RV, SM, 2, true>,                                      \
                     dim3((M + hsq::ActCfg<RV, SM>::RB - 1) / hsq::ActCfg<RV, SM>::RB),                     \
                     dim3(hsq::ActCfg<RV, SM>::NW * 32), 0, stream, X, s, L1, M, K, r, Kq, 0, x_codes, sf, U, \
-                    x_gs)
+                    x_gs, static_cast<unsigned*>(nullptr), 0)
 #define HSQ_FP4_RANKS(SM)                  \
   switch (r) {                             \
     case 0: HSQ_FP4_ACT(0, SM); break;     \

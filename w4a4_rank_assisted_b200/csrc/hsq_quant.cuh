@@ -280,6 +280,24 @@ __global__ void __launch_bounds__(128) nvfp4_act_colmax_kernel(const __nv_bfloat
   if ((threadIdx.x & 31) == 0 && amax > 0.f) atomicMax(reinterpret_cast<unsigned int*>(gs + 1), __float_as_uint(amax));
 }
 
+// Rows [rows, rows_pad) of an E4M3 tile layout (that of expand_e4m3_kernel:
+// [Kp/64][rows_pad/8][4 chunks][8 rows][16 B]) set to zero codes: one thread per
+// (64-block, padding row, chunk), 16 bytes each.
+__global__ void zero_e4m3_rows_kernel(uint8_t* __restrict__ xe, int rows, int rows_pad, int Kp) {
+  grid_dep_wait();
+  const int pad = rows_pad - rows;
+  const size_t total = static_cast<size_t>(Kp / 64) * pad * 4;
+  for (size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int chunk = static_cast<int>(t & 3);
+    const int row = rows + static_cast<int>((t >> 2) % pad);
+    const size_t blk = (t >> 2) / pad;
+    *reinterpret_cast<uint4*>(xe + ((blk * (rows_pad / 8) + (row >> 3)) * 4 + chunk) * 128 + (row & 7) * 16) =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (threadIdx.x == 0) grid_dep_launch();
+}
+
 // ---------------------------------------------------------------------------
 // Weight packing (offline): R[n,k] = fp32(W[n,k]*s[k] - sum_j L1[k,j]*L2[j,n]),
 // the sum in fp64 for j = 0..r-1 with every multiply and add rounded on its own
@@ -414,10 +432,14 @@ __global__ void __launch_bounds__(ActCfg<R, SMALL>::NW * 32)
     quantize_act_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
                         const __nv_bfloat16* __restrict__ L1, int M, int K, int r, int Kp, int ld,
                         uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U,
-                        float* gs = nullptr) {
+                        float* gs = nullptr, unsigned* zc = nullptr, int zc_words = 0) {
   using C = ActCfg<R, SMALL>;
   constexpr int SUB = C::SUB, NW = C::NW, RB = C::RB, NSUB = C::NSUB;
   grid_dep_wait();  // X (and for FP4 the absmax) may come from the preceding kernel
+  // the next GEMM's split-K counters, when asked (the preceding kernel is done with them)
+  for (int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x); i < zc_words;
+       i += static_cast<int>(gridDim.x * blockDim.x))
+    zc[i] = 0u;
   float g = 0.f, sixg = 0.f;
   if constexpr (FP4) {
     g = nvfp4_tensor_scale(gs[1]);
@@ -779,7 +801,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     quantize_act_rows_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ s,
                              const __nv_bfloat16* __restrict__ L1, int M, int K, int Kp, int ld,
                              uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ U,
-                             uint64_t limit_ns, float* gs = nullptr) {
+                             uint64_t limit_ns, float* gs = nullptr, uint8_t* __restrict__ xe = nullptr,
+                             int xe_rg = 0, unsigned* zc = nullptr, int zc_words = 0) {
   static_assert(R >= 0 && R <= 4 && R != 3, "ranks 0, 1, 2 and 4");
   static_assert(NW <= 8, "one byte per warp in an 8-byte flag word");
   using C = ActRowsCfg<NW, SUB>;
@@ -812,6 +835,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
   }
   __syncthreads();
   grid_dep_wait();  // X (and for FP4 the absmax) may come from the preceding kernel
+  // the next GEMM's split-K counters, when asked (the preceding kernel is done with them)
+  for (int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x); i < zc_words;
+       i += static_cast<int>(gridDim.x * blockDim.x))
+    zc[i] = 0u;
   float g = 0.f, sixg = 0.f, z6 = 0.f;
   if constexpr (FP4) {
     g = nvfp4_tensor_scale(gs[1]);
@@ -1021,10 +1048,32 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
           }
         }
       } else if (in_k) {
+        if (xe) {
+          // the GEMM's E4M3 tile layout instead of packed codes: lane l's 8 codes
+          // are codes 8(l % 8) .. +7 of 64-block k0/64; even codes go to chunk
+          // 2h, odd ones to chunk 2h+1 (h = (l % 8) / 4), bytes 4(l % 4) .. +3
+          // of the row's 16-byte slot (the layout of expand_e4m3_kernel)
+          const int h = (lane & 7) >> 2;
+          const size_t blk = static_cast<size_t>(k0 >> 6);
 #pragma unroll
-        for (int i = 0; i < SUB; ++i)
-          if (mw + i < M)
-            *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(mw + i) * (Kp / 2) + k0 / 2) = packed[i];
+          for (int i = 0; i < SUB; ++i) {
+            const int m = mw + i;
+            if (m >= M) break;
+            const uint32_t w = packed[i];
+            const uint32_t sg = w & 0x88888888u, one = sg >> 3;
+            const uint32_t sm = (w ^ (sg - one)) + one;  // sign-magnitude nibbles (codes are never -8)
+            const uint32_t lo = (sm & 0x07070707u) | ((sm << 4) & 0x80808080u);
+            const uint32_t hi = ((sm >> 4) & 0x07070707u) | (sm & 0x80808080u);
+            uint8_t* dst = xe + ((blk * xe_rg + (m >> 3)) * 4 + 2 * h) * 128 + (m & 7) * 16 + 4 * (lane & 3);
+            *reinterpret_cast<uint32_t*>(dst) = lo;
+            *reinterpret_cast<uint32_t*>(dst + 128) = hi;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < SUB; ++i)
+            if (mw + i < M)
+              *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(mw + i) * (Kp / 2) + k0 / 2) = packed[i];
+        }
         if ((lane & (GL - 1)) == 0) {
           float* srow = scales + static_cast<size_t>(k0 / (8 * GL)) * ld;
           if (SUB == 2 && mw + 1 < M) {

@@ -37,6 +37,7 @@ EXPORTED = (
     "hsq_linear_forward", "hsq_status_string", "hsq_get_device_status",
     "hsq_debug_force_timeout", "hsq_linear_forward_noalloc", "hsq_linear_forward_fused", "hsq_fused_form",
     "hsq_weights_e4m3_bytes", "hsq_expand_weights", "hsq_workspace_bytes_pre", "hsq_linear_forward_pre",
+    "hsq_workspace_bytes_x", "hsq_linear_forward_x",
     "hsq_lowrank_workspace_bytes", "hsq_lowrank_init",
     "hsq_fp4_codes_bytes", "hsq_fp4_scales_bytes", "hsq_fp4_pack_weights", "hsq_fp4_quantize_act",
     "hsq_fp4_linear_forward",
@@ -93,6 +94,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.hsq_workspace_bytes_pre.restype = ctypes.c_size_t
     lib.hsq_linear_forward_pre.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, ctypes.c_size_t, vp]
     lib.hsq_linear_forward_pre.restype = i
+    lib.hsq_workspace_bytes_x.argtypes = [i, i, i, i, i, i]
+    lib.hsq_workspace_bytes_x.restype = ctypes.c_size_t
+    lib.hsq_linear_forward_x.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp, ctypes.c_size_t, vp]
+    lib.hsq_linear_forward_x.restype = i
     lib.hsq_lowrank_workspace_bytes.argtypes = [i, i, i]; lib.hsq_lowrank_workspace_bytes.restype = sz
     lib.hsq_lowrank_init.argtypes = [vp, vp, i, i, i, i, c.c_ulonglong, vp, vp, vp, sz, vp]
     lib.hsq_lowrank_init.restype = i
@@ -213,6 +218,18 @@ def hsq_linear_forward_pre(x_codes, x_scales, U, w_codes, w_scales, w_e4m3, L2, 
                                          _ptr(w_scales), _ptr(w_e4m3), _ptr(L2), _ptr(bias), M, N, K, r, group,
                                          _ptr(Y), int(out), _ptr(workspace), int(ws_bytes),
                                          _stream(stream)), "hsq_linear_forward_pre")
+
+
+def hsq_workspace_bytes_x(M: int, N: int, K: int, r: int, group: int = GROUP, with_w_e4m3: bool = True) -> int:
+    return int(load().hsq_workspace_bytes_x(M, N, K, r, group, 1 if with_w_e4m3 else 0))
+
+
+def hsq_linear_forward_x(X, s, L1, w_codes, w_scales, w_e4m3, L2, bias, M, N, K, r, Y,
+                         out: int = HSQ_OUT_BF16, workspace=None, ws_bytes: int = 0,
+                         group=GROUP, stream=None) -> None:
+    _check(load().hsq_linear_forward_x(_ptr(X), _ptr(s), _ptr(L1), _ptr(w_codes), _ptr(w_scales), _ptr(w_e4m3),
+                                       _ptr(L2), _ptr(bias), M, N, K, r, group, _ptr(Y), int(out),
+                                       _ptr(workspace), int(ws_bytes), _stream(stream)), "hsq_linear_forward_x")
 
 
 def hsq_linear_forward_fused(X, s, L1, w_codes, w_scales, L2, bias, M, N, K, r, Y,
@@ -370,6 +387,11 @@ class PackedLinear:
                                       device=self.w_codes.device)
             hsq_expand_weights(self.w_codes, self.N, self.K, self.w_e4m3, group=self.group, stream=stream)
 
+    def workspace_x(self, M: int) -> torch.Tensor:
+        """Workspace of forward_x for M tokens."""
+        n = hsq_workspace_bytes_x(M, self.N, self.K, self.r, self.group, self.w_e4m3 is not None)
+        return torch.zeros(max(n, 16), dtype=torch.uint8, device=self.w_codes.device)
+
     def workspace(self, M: int) -> Optional[torch.Tensor]:
         n = (hsq_workspace_bytes(M, self.N, self.K, self.r) if self.w_e4m3 is None
              else hsq_workspace_bytes_pre(M, self.N, self.K, self.r))
@@ -395,6 +417,17 @@ def forward_fused(layer: PackedLinear, X: torch.Tensor, Y: torch.Tensor, out: in
     hsq_linear_forward_fused(X, layer.s, layer.L1, layer.w_codes, layer.w_scales, layer.L2, layer.bias,
                              X.shape[0], layer.N, layer.K, layer.r, Y, out=out, group=layer.group,
                              stream=stream)
+    return Y
+
+
+def forward_x(layer: PackedLinear, X: torch.Tensor, Y: torch.Tensor, workspace: torch.Tensor,
+              out: int = HSQ_OUT_BF16, stream=None) -> torch.Tensor:
+    """The activation step and the forward in one call (hsq_linear_forward_x);
+    `workspace` of at least layer.workspace_x(M) bytes."""
+    M = X.shape[0]
+    hsq_linear_forward_x(X, layer.s, layer.L1, layer.w_codes, layer.w_scales, layer.w_e4m3, layer.L2, layer.bias,
+                         M, layer.N, layer.K, layer.r, Y, out=out, workspace=workspace, ws_bytes=workspace.numel(),
+                         group=layer.group, stream=stream)
     return Y
 
 
