@@ -516,7 +516,7 @@ class Workload:
         """hsq_linear_forward_x's activation kernel writes the GEMM's E4M3 tiles
         itself (no expansion launch; a pad-zeroing launch when M is not a
         multiple of 128): many rows, ranks 0, 1, 2, 4."""
-        return s.M >= 28 * _sms() and s.r in (0, 1, 2, 4)
+        return s.M >= 24 * _sms() and s.r in (0, 1, 2, 4)
 
     @staticmethod
     def expands(s):

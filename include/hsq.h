@@ -173,7 +173,7 @@ hsq_status hsq_linear_forward_pre(const uint8_t* x_codes, const float* x_scales,
  * as hsq_quantize_act followed by hsq_linear_forward (w_e4m3 NULL) or
  * hsq_linear_forward_pre (w_e4m3 from hsq_expand_weights).  Where the GEMM
  * reads expanded operands and the many-row activation kernel applies (M at
- * least 28 per SM, r in {0, 1, 2, 4}), that kernel writes the activations'
+ * least 24 per SM, r in {0, 1, 2, 4}), that kernel writes the activations'
  * E4M3 tiles itself, so no packed codes are written and no expansion runs;
  * elsewhere the call is those two steps.  The activation step's scales and U
  * live in the workspace:

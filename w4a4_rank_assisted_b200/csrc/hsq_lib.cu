@@ -193,7 +193,7 @@ cudaError_t launch_pdl(bool allow, void (*kernel)(KArgs...), dim3 grid, dim3 blo
 #endif
 // ... from this many rows per SM on
 #ifndef HSQ_ACT_ROWS16_MIN
-#define HSQ_ACT_ROWS16_MIN 28
+#define HSQ_ACT_ROWS16_MIN 24
 #endif
 // ... with this many rows per warp (8 warps per block)
 #ifndef HSQ_ACT_ROWS_SUB
@@ -1025,7 +1025,7 @@ static hsq_status quantize_act_impl(const void* X_bf16, const float* s, const vo
   }
   cudaError_t lerr = cudaSuccess;
   // few rows: one block per sub-block with 32 warps spread over K; many rows
-  // (enough for two 16-row blocks per SM, nearly) and ranks 0, 1, 2, 4: the
+  // (from 24 per SM: one and a half 16-row blocks per SM) and ranks 0, 1, 2, 4: the
   // row-owning kernel; else 8 warps x 2 sub-blocks
   const bool rows_kernel = HSQ_ACT_ROWS && (r <= 2 || r == 4) && M >= HSQ_ACT_ROWS16_MIN * device_sm_count();
   if (M <= 64) {
