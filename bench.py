@@ -347,8 +347,8 @@ def _sources_sha() -> str:
 # step's layers) from one ncu capture, keyed by workload, with the hash of the
 # CUDA sources it was captured from; any other build reports null.
 NCU_TRAFFIC = {
-    # w4a4_gemm_kernel, FLUX.1 block: 87.0 / 121.8 / 235.5 MB for qkv / MLP up / MLP down
-    "flux_block_r4": ("363db09ca01444c1", 148082090.7),
+    # w4a4_gemm_kernel, FLUX.1 block: 86.5 / 121.9 / 236.4 MB for qkv / MLP up / MLP down
+    "flux_block_r4": ("cda07b5ebc605b3d", 148257109.3),
 }
 
 
