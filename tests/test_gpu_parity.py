@@ -81,6 +81,10 @@ SMALL_SHAPES = [
     (130, 320, 264, 15),     # largest rank of one tensor-core low-rank step
     (97, 192, 136, 16),      # two low-rank steps
     (96, 256, 200, 31),      # three low-rank steps, the last with one rank
+    (300, 640, 512, 16),     # large tiles, two low-rank steps (one rank in the second)
+    (520, 384, 776, 17),     # ... two ranks in the second: the many-rank kernels
+    (200, 320, 264, 17),     # mid tiles, the many-rank kernels
+    (2048, 128, 2560, 32),   # more tiles than SMs: later tiles' low-rank steps built ahead
     (129, 128, 256, 0),      # no low-rank pair: the step carries the bias alone
     (70, 200, 136, 8),       # rank 8: eight L1 rows per warp load, chunk of 200 channels
     (40, 328, 264, 8),       # few rows, rank 8, ragged last chunk
@@ -121,6 +125,7 @@ SHAPES_G128 = [
     (200, 1024, 1160, 4),
     (128, 2048, 1024, 4),    # large tile, split-K or whole tiles
     (300, 640, 512, 32),
+    (520, 640, 392, 20),     # the many-rank kernels, two low-rank steps
     (6, 640, 264, 16),       # the CUDA-core weight stream, four lanes per group
     (8, 1024, 1160, 4),
     (4150, 1160, 136, 2),    # many-row activation kernel

@@ -129,7 +129,7 @@ struct GemmArgs {
 
 template <int BN_, int DH_, int STAGES_, bool SWAP_, int GPS_, int NI8_, int NTM_, int UNPACK_WARPS_ = 6,
           int SSLOTS_ = STAGES_ + 4, bool F8_ = false, int PIPE_ = -1, bool PRE_ = false, int CHB_ = 2,
-          int BPG_ = 1, bool PAIR_ = false, bool FUSED_ = false>
+          int BPG_ = 1, bool PAIR_ = false, bool FUSED_ = false, bool LRFAST_ = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
@@ -228,6 +228,11 @@ struct GemmCfg {
   static_assert(!LR_MMA || PRE || (BM + BN) / 8 * LR_SBO <= I8_BYTES, "low-rank operands fit an int8 buffer");
   // with pre-expanded operands the low-rank operands get a buffer of their own
   static constexpr int LR_BYTES = (PRE && LR_MMA) ? (BM + B_ROWS) / 8 * LR_SBO : 0;
+  // Build the low-rank steps with build_lr_operands_mlp (the host takes these
+  // kernels for ranks above LR_MAX_RANK; a separate instantiation, so that the
+  // kernels for lower ranks keep their code unchanged)
+  static constexpr bool LRFAST = LRFAST_;
+  static_assert(!LRFAST || LR_MMA, "many-rank builder: kernels with low-rank steps");
   static_assert(!PAIR || (PRE && LR_MMA), "CTA pairs: pre-expanded tokens x outputs tiles");
   static_assert(!PAIR || A_E8_BLK == 8192 && B_E8_BLK == 8192, "CTA pairs: one 32 x 256-byte TMA box per block");
   static_assert(!PRE || (F8 && !SWAP && GPS == 1), "pre-expanded operands: E4M3, tokens x outputs, one group a stage");
@@ -371,6 +376,104 @@ __device__ __forceinline__ void build_lr_operands(const GemmArgs& a, int r0, int
 #pragma unroll
       for (int e = 0; e < 4; ++e) wb[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
       *reinterpret_cast<uint4*>(base + c * 128) = w;
+    }
+  }
+}
+
+// The same operands, built for ranks above LR_MAX_RANK (kernels with LRFAST).
+// Those take two or three low-rank steps per tile, and every step after the
+// first is built while the MMA issuer waits for it (one operand buffer), so
+// the build's latency is paid per tile.  Here a row's loads (its ranks of U or
+// of L2, and its bias) are all issued before any is used, at clamped in-range
+// addresses, so they are in flight together: a step takes a few memory round
+// trips instead of one per rank.  The bits are those of build_lr_operands.
+template <class Cfg>
+__device__ __forceinline__ void build_lr_operands_mlp(const GemmArgs& a, int r0, int c0, int chunk, uint8_t* dst, int t0,
+                                                  int nt) {
+  constexpr int BM = Cfg::BM, BNR = Cfg::B_ROWS, K = Cfg::LR_K, R = Cfg::LR_MAX_RANK;
+  static_assert(K == 32 && R <= 15, "one step: four 16-byte K-chunks of four ranks each, the last with the bias");
+  const int rk0 = R * chunk;                               // first rank of this step
+  const int nr = a.r > rk0 ? min(R, a.r - rk0) : 0;        // ranks in this step
+  auto store_chunk = [](uint8_t* p, const float (&f)[8]) {
+    uint4 w;
+    __nv_bfloat162* wb = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) wb[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+    *reinterpret_cast<uint4*>(p) = w;
+  };
+  // token rows: [hi lo] pairs of U
+  for (int t = t0; t < BM; t += nt) {
+    const int m = r0 + t;
+    const bool valid = m < a.M;
+    float u[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j) u[j] = 0.f;
+    if (nr > 0) {
+      const float* up = a.U + static_cast<size_t>(min(m, a.M - 1)) * a.r + rk0;
+#pragma unroll
+      for (int j = 0; j < R; ++j) u[j] = __ldg(up + min(j, nr - 1));
+    }
+    uint8_t* base = dst + (t >> 3) * Cfg::LR_SBO + (t & 7) * 16;
+#pragma unroll
+    for (int c = 0; c < K / 8; ++c) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * c + e;
+        if (j < R && j < nr && valid) {
+          f[2 * e] = __bfloat162float(__float2bfloat16_rn(u[j]));
+          f[2 * e + 1] = u[j] - f[2 * e];  // exact; rounded to bf16 in the store
+        }
+      }
+      if (c == K / 8 - 1 && chunk == 0 && valid) f[6] = 1.f;  // ones against the bias
+      store_chunk(base + c * 128, f);
+    }
+  }
+  // output rows: L2 twice, and the bias; two rows per pass where few warps build
+  // (more would spill under the builders' register budget)
+  constexpr int P = Cfg::NUM_UNPACK_WARPS <= 2 ? 2 : 1;
+  for (int t = t0; t < BNR; t += P * nt) {
+    unsigned short l[P][R], bb[P];
+    bool valid[P];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const int row = t + p * nt;
+      const int n = c0 + row;
+      valid[p] = row < BNR && n < a.N;
+      const int nc = min(n, a.N - 1);
+#pragma unroll
+      for (int j = 0; j < R; ++j) l[p][j] = 0;
+      if (nr > 0) {
+#pragma unroll
+        for (int j = 0; j < R; ++j)
+          l[p][j] = __ldg(reinterpret_cast<const unsigned short*>(a.L2) + static_cast<size_t>(rk0 + min(j, nr - 1)) * a.N + nc);
+      }
+      bb[p] = (chunk == 0 && a.bias) ? __ldg(reinterpret_cast<const unsigned short*>(a.bias) + nc) : 0;
+    }
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const int row = t + p * nt;
+      if (!(row < BNR)) continue;
+      uint8_t* base = dst + (BM / 8) * Cfg::LR_SBO + (row >> 3) * Cfg::LR_SBO + (row & 7) * 16;
+#pragma unroll
+      for (int c = 0; c < K / 8; ++c) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * c + e;
+          if (j < R && j < nr && valid[p]) {
+            const float v = __bfloat162float(__ushort_as_bfloat16(l[p][j]));
+            f[2 * e] = v;
+            f[2 * e + 1] = v;
+          }
+        }
+        if (c == K / 8 - 1 && chunk == 0 && valid[p]) f[6] = __bfloat162float(__ushort_as_bfloat16(bb[p]));
+        store_chunk(base + c * 128, f);
+      }
     }
   }
 }
@@ -894,9 +997,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (!wait_warp(lrempty, (nlr & 1) ^ 1, wp)) { ok = false; break; }
           // chunks as constants, so that each build unrolls over a fixed rank range
           constexpr int LT = 32 * Cfg::NUM_UNPACK_WARPS;
-          if (chunk == 0) build_lr_operands<Cfg>(args, lr0, lc0, 0, lr_buf, ut, LT);
-          else if (chunk == 1) build_lr_operands<Cfg>(args, lr0, lc0, 1, lr_buf, ut, LT);
-          else build_lr_operands<Cfg>(args, lr0, lc0, 2, lr_buf, ut, LT);
+          if constexpr (Cfg::LRFAST) {
+            if (chunk == 0) build_lr_operands_mlp<Cfg>(args, lr0, lc0, 0, lr_buf, ut, LT);
+            else if (chunk == 1) build_lr_operands_mlp<Cfg>(args, lr0, lc0, 1, lr_buf, ut, LT);
+            else build_lr_operands_mlp<Cfg>(args, lr0, lc0, 2, lr_buf, ut, LT);
+          } else {
+            if (chunk == 0) build_lr_operands<Cfg>(args, lr0, lc0, 0, lr_buf, ut, LT);
+            else if (chunk == 1) build_lr_operands<Cfg>(args, lr0, lc0, 1, lr_buf, ut, LT);
+            else build_lr_operands<Cfg>(args, lr0, lc0, 2, lr_buf, ut, LT);
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -947,9 +1056,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           if (Cfg::LR_MMA && g < g0) {
             const int tr = un.tile % args.tiles_r, tc = un.tile / args.tiles_r;
             const int chunk = (g - (g0 - GPS * args.lr_mma)) / GPS;
-            if (chunk == 0) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 0, dst, ut, NT);
-            else if (chunk == 1) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 1, dst, ut, NT);
-            else build_lr_operands<Cfg>(args, tr * BM, tc * BN, 2, dst, ut, NT);
+            if constexpr (Cfg::LRFAST) {
+              if (chunk == 0) build_lr_operands_mlp<Cfg>(args, tr * BM, tc * BN, 0, dst, ut, NT);
+              else if (chunk == 1) build_lr_operands_mlp<Cfg>(args, tr * BM, tc * BN, 1, dst, ut, NT);
+              else build_lr_operands_mlp<Cfg>(args, tr * BM, tc * BN, 2, dst, ut, NT);
+            } else {
+              if (chunk == 0) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 0, dst, ut, NT);
+              else if (chunk == 1) build_lr_operands<Cfg>(args, tr * BM, tc * BN, 1, dst, ut, NT);
+              else build_lr_operands<Cfg>(args, tr * BM, tc * BN, 2, dst, ut, NT);
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {

@@ -78,6 +78,23 @@ using CfgLarge128 = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_PAIR ? 4 : HSQ_
 #define HSQ_MID_MAX_M 256
 #endif
 using CfgMid64 = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 6, 10, true, -1, false, 2, 1>;
+// The same tiles for ranks above one low-rank step (LR_MAX_RANK): the steps after
+// a tile's first are built on the MMA issuer's path, by the many-rank builder.
+using CfgLarge64R = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_PAIR ? 8 : HSQ_LARGE_STAGES, false, 1, 3,
+                                 HSQ_LARGE_NTM, 2, HSQ_PAIR ? 12 : HSQ_LARGE_STAGES + 4, true, HSQ_LARGE_PIPE, true,
+                                 HSQ_LARGE_CHB, 1, HSQ_PAIR != 0, false, true>;
+using CfgLarge128R = hsq::GemmCfg<HSQ_LARGE_BN, HSQ_LARGE_DH, HSQ_PAIR ? 4 : HSQ_LARGE128_STAGES, false, 1, 3,
+                                  HSQ_LARGE_NTM, 2, HSQ_PAIR ? 8 : HSQ_LARGE128_STAGES + 4, true,
+                                  HSQ_LARGE_PIPE, true, HSQ_LARGE_CHB, 2, HSQ_PAIR != 0, false, true>;
+using CfgMid64R = hsq::GemmCfg<256, 2, 6, false, 1, 3, 2, 6, 10, true, -1, false, 2, 1, false, false, true>;
+// Which kernels a rank takes.  The many-rank builder pays for itself once the
+// second low-rank step holds two ranks or more.  Measured on FLUX MLP up
+// (M = 4608, K = 3072, N = 12288): 463 vs 468 us at r = 16 (one rank in the
+// second step: the previous builder is faster), 779 vs 528 us at r = 32.
+static bool many_rank_kernel(int r) { return r > CfgLarge64::LR_MAX_RANK + 1; }
+static_assert(CfgLarge64R::SMEM_BYTES == CfgLarge64::SMEM_BYTES && CfgLarge128R::SMEM_BYTES == CfgLarge128::SMEM_BYTES &&
+                  CfgMid64R::SMEM_BYTES == CfgMid64::SMEM_BYTES && CfgLarge64R::THREADS == CfgLarge64::THREADS,
+              "many-rank kernels: the same tiles");
 // M <= 64: roles swapped, 128 weight rows x 16/32/64 tokens; packed codes
 // unpacked in shared memory (the drain is light, so more warps unpack); four
 // 64-blocks per stage either way
@@ -1157,9 +1174,13 @@ static hsq_status forward_impl(const uint8_t* x_codes, const float* x_scales, co
   const bool g128 = group == 128;
   switch (p.kind) {
     case kLarge:
+      if (many_rank_kernel(r))
+        return g128 ? launch_gemm<CfgLarge128R>(p, tm_row, tm_col, tm_y, a, stream)
+                    : launch_gemm<CfgLarge64R>(p, tm_row, tm_col, tm_y, a, stream);
       return g128 ? launch_gemm<CfgLarge128>(p, tm_row, tm_col, tm_y, a, stream)
                   : launch_gemm<CfgLarge64>(p, tm_row, tm_col, tm_y, a, stream);
     case kMid:
+      if (many_rank_kernel(r)) return launch_gemm<CfgMid64R>(p, tm_row, tm_col, tm_y, a, stream);
       return launch_gemm<CfgMid64>(p, tm_row, tm_col, tm_y, a, stream);
     case kDec16:
       return g128 ? launch_gemm<CfgDec16_128>(p, tm_row, tm_col, tm_y, a, stream)
