@@ -67,6 +67,7 @@ def layer_gemm_bytes(spec):
     Kp = gs * G
     return (M * Kp // 2 + 4 * M * G + 4 * M * r      # x codes, scales, U
             + N * Kp // 2 + 4 * N * G + 2 * r * N    # w codes, scales, L2
+            + (2 * N if spec.bias else 0)            # bias (bf16; the stated workloads have none)
             + 2 * M * N)                             # Y (bf16)
 
 
@@ -77,7 +78,8 @@ def layer_fused_bytes(spec):
     M, N, K, r, gs = spec.M, spec.N, spec.K, spec.r, spec.group
     G = -(-K // gs)
     Kp = gs * G
-    return 2 * M * K + 4 * K + 2 * K * r + N * Kp // 2 + 4 * N * G + 2 * r * N + 2 * M * N
+    return (2 * M * K + 4 * K + 2 * K * r + N * Kp // 2 + 4 * N * G + 2 * r * N + (2 * N if spec.bias else 0)
+            + 2 * M * N)
 
 
 def layer_act_bytes(spec):
